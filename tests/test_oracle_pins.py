@@ -1,0 +1,361 @@
+"""Pins of the CPU oracle against things other than itself (CPU only).
+
+Each check is chosen so that a plausible slip in the oracle (the window edge
+off by one, a dropped scale, transposed operands, a wrong GQA mapping, a
+wrong retire order, a wrong FP8 rounding) fails at least one of them:
+
+* library routines: torch's fp64 scaled_dot_product_attention (with its own
+  GQA expansion), torch's and ml_dtypes' float8_e4m3fn casts;
+* an operational model of delayed eviction written independently of the
+  oracle's inequality (tokens carry a removal step), brute-forced over every
+  flag pattern of short prompts;
+* closed forms: retained counts, uniform mean for zero keys, one-hot values
+  reading off the weights, a single visible key returning its value, the
+  slot recurrence, the page's 6.4x compression at ctx 8192;
+* page figures and format landmarks stored under tests/golden/.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from synth import configs
+from oracle import attention, compaction, fp8, mask, reference, slots
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+PAGE = json.load(open(os.path.join(GOLDEN, "page_figures.json")))
+E4M3 = json.load(open(os.path.join(GOLDEN, "e4m3_spec.json")))
+
+
+# ---------------------------------------------------------------------------
+# independent operational model of delayed eviction
+# ---------------------------------------------------------------------------
+
+def operational_cache_sets(evict, w):
+    """Cache contents after each arrival: a flagged token is given a removal
+    step w after its arrival and is physically dropped when that step comes."""
+    cache = []          # (position, removal step or None)
+    sets = []
+    for t, f in enumerate(evict):
+        cache = [(p, r) for (p, r) in cache if r is None or r > t]
+        cache.append((t, t + w if f else None))
+        sets.append(sorted(p for p, _ in cache))
+    return sets
+
+
+def sdpa(q, K, V, scale, mask_=None):
+    """torch fp64 SDPA for one decode query: q [Hq, D], K/V [n, Hkv, D]."""
+    qt = torch.from_numpy(np.asarray(q, np.float64))[None, :, None, :]
+    Kt = torch.from_numpy(np.asarray(K, np.float64)).permute(1, 0, 2)[None]
+    Vt = torch.from_numpy(np.asarray(V, np.float64)).permute(1, 0, 2)[None]
+    am = None
+    if mask_ is not None:   # [Hkv, n] -> broadcast to each query head of the group
+        g = q.shape[0] // K.shape[1]
+        am = torch.from_numpy(np.repeat(mask_, g, axis=0))[None, :, None, :]
+    out = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=am, scale=scale,
+                                                           enable_gqa=True)
+    return out[0, :, 0, :].numpy()
+
+
+def rand_case(rng, n, Hq=8, Hkv=2, D=16):
+    q = rng.standard_normal((Hq, D))
+    K = rng.standard_normal((n, Hkv, D))
+    V = rng.standard_normal((n, Hkv, D))
+    return q, K, V
+
+
+# ---------------------------------------------------------------------------
+# mask and attention
+# ---------------------------------------------------------------------------
+
+def test_eviction_off_window_gives_full_attention():
+    rng = np.random.default_rng(0)
+    w_off = PAGE["eviction_off_window"]["value"]
+    t = 40
+    q, K, V = rand_case(rng, t + 1)
+    evict = rng.integers(0, 2, size=(t + 1, 2)).astype(np.uint8)
+    got = attention.decode_attention(q, K, V, evict, t, w_off, 0.3)
+    np.testing.assert_allclose(got, sdpa(q, K, V, 0.3), rtol=0, atol=1e-12)
+
+
+def test_no_flags_gives_full_attention_for_any_window():
+    rng = np.random.default_rng(1)
+    t = 33
+    q, K, V = rand_case(rng, t + 1)
+    evict = np.zeros((t + 1, 2), dtype=np.uint8)
+    for w in (1, 2, 7):
+        got = attention.decode_attention(q, K, V, evict, t, w, 0.25)
+        np.testing.assert_allclose(got, sdpa(q, K, V, 0.25), rtol=0, atol=1e-12)
+
+
+def test_all_flags_give_sliding_window_of_w():
+    rng = np.random.default_rng(2)
+    t = 50
+    q, K, V = rand_case(rng, t + 1)
+    evict = np.ones((t + 1, 2), dtype=np.uint8)
+    for w in (1, 3, 8):
+        got = attention.decode_attention(q, K, V, evict, t, w, 0.2)
+        ref = sdpa(q, K[t - w + 1:], V[t - w + 1:], 0.2)
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_page_window_holds_exactly_512_tokens_when_all_flagged():
+    w = PAGE["delay_window"]["value"]
+    t = PAGE["ctx_len"]["value"] - 1
+    evict = np.ones(t + 1, dtype=np.uint8)
+    vis = mask.visible_positions(t, evict, w)
+    assert len(vis) == 512 and vis[0] == t - 511 and vis[-1] == t
+
+
+def test_general_flags_match_sdpa_with_operational_mask():
+    """Random flags: the oracle equals torch SDPA given the cache contents of
+    the operational model as a boolean mask (also pins the GQA mapping, the
+    score scale and the softmax axis)."""
+    rng = np.random.default_rng(3)
+    n, w = 64, 5
+    q, K, V = rand_case(rng, n, Hq=12, Hkv=3, D=8)
+    evict = (rng.random((n, 3)) < 0.7).astype(np.uint8)
+    for t in (0, 4, 5, 17, 63):
+        m = np.zeros((3, t + 1), dtype=bool)
+        for h in range(3):
+            m[h, operational_cache_sets(evict[:t + 1, h], w)[t]] = True
+        got = attention.decode_attention(q, K[:t + 1], V[:t + 1], evict[:t + 1], t, w, 0.37)
+        np.testing.assert_allclose(got, sdpa(q, K[:t + 1], V[:t + 1], 0.37, m), rtol=0, atol=1e-12)
+
+
+def test_zero_keys_give_uniform_mean_of_visible_values():
+    # flags on even positions, w = 3, t = 10: the visible set is the odd
+    # positions plus the last three (8, 9, 10)
+    t, w = 10, 3
+    evict = np.array([1 - (j % 2) for j in range(t + 1)], dtype=np.uint8)
+    expect_vis = [1, 3, 5, 7, 8, 9, 10]
+    rng = np.random.default_rng(4)
+    V = rng.standard_normal((t + 1, 1, 6))
+    K = np.zeros((t + 1, 1, 6))
+    q = rng.standard_normal((2, 6))
+    got = attention.decode_attention(q, K, V, evict[:, None], t, w, 1.0)
+    np.testing.assert_allclose(got, np.tile(V[expect_vis, 0].mean(axis=0), (2, 1)), atol=1e-14)
+
+
+def test_one_hot_values_read_off_attention_weights():
+    rng = np.random.default_rng(5)
+    t, w, D = 11, 4, 12            # D >= t+1 so value j is the unit vector e_j
+    evict = (rng.random(t + 1) < 0.5).astype(np.uint8)
+    K = rng.standard_normal((t + 1, 1, D))
+    V = np.eye(D)[: t + 1][:, None, :]
+    q = rng.standard_normal((1, D))
+    o = attention.decode_attention(q, K, V, evict[:, None], t, w, 0.5)[0]
+    vis = operational_cache_sets(evict, w)[t]
+    s = 0.5 * K[vis, 0] @ q[0]
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    expect = np.zeros(D)
+    expect[vis] = p
+    np.testing.assert_allclose(o, expect, atol=1e-14)
+    hidden = [j for j in range(t + 1) if j not in vis]
+    assert np.all(o[hidden] == 0.0)
+
+
+def test_single_visible_key_returns_its_value_exactly():
+    rng = np.random.default_rng(6)
+    t = 9
+    q, K, V = rand_case(rng, t + 1, Hq=4, Hkv=1, D=8)
+    evict = np.ones((t + 1, 1), dtype=np.uint8)
+    got = attention.decode_attention(q, K, V, evict, t, 1, 0.9)
+    assert np.array_equal(got, np.tile(V[t, 0], (4, 1)))
+
+
+@pytest.mark.parametrize("w", [1, 2, 3, 4])
+def test_brute_force_visible_sets_match_operational_model(w):
+    for P in range(1, 11):
+        for bits in itertools.product((0, 1), repeat=P):
+            evict = np.array(bits, dtype=np.uint8)
+            op = operational_cache_sets(evict, w)
+            for t in range(P):
+                assert list(mask.visible_positions(t, evict, w)) == op[t]
+
+
+# ---------------------------------------------------------------------------
+# compaction and slot bookkeeping
+# ---------------------------------------------------------------------------
+
+def test_prefill_retained_count_closed_form():
+    rng = np.random.default_rng(7)
+    for P, w, p in [(256, 32, 0.85), (1000, 512, 0.9), (300, 512, 0.5), (1, 4, 1.0), (513, 512, 1.0)]:
+        evict = (rng.random(P) < p).astype(np.uint8)
+        kept = compaction.prefill_kept_positions(evict, w)
+        older = max(0, P - w)
+        assert len(kept) == min(P, w) + int((evict[:older] == 0).sum())
+        assert list(kept) == operational_cache_sets(evict, w)[P - 1]
+
+
+def test_prefill_slots_are_ranks_and_ring_holds_last_window():
+    rng = np.random.default_rng(8)
+    P, w = 200, 16
+    evict = (rng.random(P) < 0.8).astype(np.uint8)
+    slot = compaction.prefill_slots(evict, w)
+    pos = sorted(slot)
+    assert [slot[j] for j in pos] == list(range(len(pos)))
+    ring = compaction.prefill_ring(evict, w)
+    for j in range(P - w, P):
+        assert ring[j % w] == (slot[j], int(evict[j]))
+    short = compaction.prefill_ring(evict[:5], w)
+    assert [e is None for e in short] == [False] * 5 + [True] * (w - 5)
+
+
+@pytest.mark.parametrize("P,w,p,steps", [(64, 8, 0.7, 80), (5, 8, 0.9, 30), (40, 1, 1.0, 10),
+                                         (100, 16, 0.0, 20)])
+def test_decode_slots_follow_reuse_recurrence_and_hold_visible_set(P, w, p, steps):
+    """slot(t) = slot(t-w) when token t-w was flagged, else the next new slot;
+    the held positions are exactly the visible set, one slot each."""
+    rng = np.random.default_rng(P * 131 + w)
+    evict = (rng.random(P + steps) < p).astype(np.uint8)
+    store = slots.HeadStore(evict[:P], w)
+    slot_of = dict(compaction.prefill_slots(evict[:P], w))
+    n_slots = len(slot_of)
+    op = operational_cache_sets(evict, w)
+    for t in range(P, P + steps):
+        expect = slot_of[t - w] if (t - w >= 0 and evict[t - w]) else n_slots
+        if expect == n_slots:
+            n_slots += 1
+        s = store.append(t, int(evict[t]))
+        slot_of[t] = s
+        assert s == expect
+        assert store.n_slots == n_slots == store.n_retained
+        assert list(store.positions()) == op[t]
+        assert sorted(store.pos_of_slot) == list(range(store.n_slots))
+        assert len(store.free) == 0
+
+
+def test_llama_workload_compaction_matches_page_compression():
+    """The 6.4x of the pages at ctx 8192 is 1280 kept tokens per head; the
+    Llama-3.2-1B workload (keep 0.10, w 512) has exactly that expectation,
+    and its seeded flags land within binomial error of it."""
+    wl = configs.LLAMA1B_CTX8K
+    P = PAGE["ctx_len"]["value"]
+    assert wl.prompt == P and wl.window == PAGE["delay_window"]["value"]
+    expect = wl.window + wl.p_keep * (P - wl.window)
+    assert abs(expect - P / PAGE["compression_llama_3_2_1b"]["value"]) < 1e-9
+    sigma = np.sqrt((P - wl.window) * wl.p_keep * (1 - wl.p_keep))
+    counts = []
+    for layer in range(wl.n_layers):
+        for h in range(wl.n_kv_heads):
+            flags = reference.head_flags(wl, layer, 0, h, P)
+            counts.append(len(compaction.prefill_kept_positions(flags, wl.window)))
+    counts = np.array(counts)
+    assert np.all(np.abs(counts - expect) < 6 * sigma)
+    assert abs(counts.mean() - expect) < 5 * sigma / np.sqrt(len(counts))
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3 codec
+# ---------------------------------------------------------------------------
+
+ALL_CODES = np.arange(256, dtype=np.uint8)
+
+
+def test_e4m3_golden_landmarks():
+    for code, val in E4M3["codes"].items():
+        got = fp8.e4m3_decode(np.uint8(int(code, 16)))
+        assert got == val and np.signbit(got) == np.signbit(val)
+    for code in E4M3["nan_codes"]:
+        assert np.isnan(fp8.e4m3_decode(np.uint8(int(code, 16))))
+    finite = fp8.e4m3_decode(ALL_CODES)
+    finite = finite[~np.isnan(finite)]
+    assert finite.max() == E4M3["max_finite"]
+    assert np.abs(finite[finite != 0]).min() == E4M3["min_subnormal"]
+
+
+def test_e4m3_decode_matches_torch_and_ml_dtypes():
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    ours = fp8.e4m3_decode(ALL_CODES)
+    tt = torch.from_numpy(ALL_CODES.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ml = ALL_CODES.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    for ref in (tt, ml):
+        assert np.array_equal(np.isnan(ours), np.isnan(ref))
+        ok = ~np.isnan(ours)
+        assert np.array_equal(ours[ok], ref[ok])
+
+
+def test_e4m3_encode_roundtrips_every_finite_code():
+    vals = fp8.e4m3_decode(ALL_CODES)
+    ok = ~np.isnan(vals)
+    assert np.array_equal(fp8.e4m3_encode(vals[ok]), ALL_CODES[ok])
+
+
+def test_e4m3_midpoints_round_to_even_and_match_torch():
+    pos = np.sort(fp8.e4m3_decode(np.arange(0x7F, dtype=np.uint8)))
+    mids = (pos[:-1] + pos[1:]) / 2
+    codes = fp8.e4m3_encode(mids)
+    assert np.all(codes % 2 == 0)                         # even mantissa wins the tie
+    assert np.all((fp8.e4m3_decode(codes) == pos[:-1]) | (fp8.e4m3_decode(codes) == pos[1:]))
+    tt = torch.from_numpy(mids.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, tt)
+    neg = fp8.e4m3_encode(-mids)
+    assert np.array_equal(neg, codes | 0x80)
+
+
+def test_e4m3_encode_matches_torch_on_dense_fp32_grid():
+    x = np.linspace(-448.0, 448.0, 2_000_001, dtype=np.float32)
+    x = np.concatenate([x, np.float32(2.0) ** -np.arange(0, 12, 0.125).astype(np.float32)])
+    tt = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(fp8.e4m3_encode(x), tt)
+
+
+def test_e4m3_saturates_instead_of_nan():
+    big = np.array([448.5, 463.9, 464.0, 470.0, 1e4, 3e38], dtype=np.float32)
+    assert np.all(fp8.e4m3_encode(big) == 0x7E)
+    assert np.all(fp8.e4m3_encode(-big) == 0xFE)
+    assert fp8.e4m3_encode(np.float32(np.nan)) == 0x7F
+
+
+def test_fp8_scale_and_fp32_quotient():
+    assert fp8.fp8_scale(448.0) == 1.0 and fp8.fp8_scale(0.0) == 1.0
+    assert fp8.fp8_scale(1.0) == np.float32(1.0) / np.float32(448.0)
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal(100_000).astype(np.float32)
+    s = fp8.fp8_scale(np.abs(x).max())
+    y = torch.from_numpy(x) / torch.tensor(s, dtype=torch.float32)
+    tt = y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(fp8.quantize(x, s), tt)
+    assert np.abs(fp8.dequantize(fp8.quantize(x, s), s)).max() <= np.abs(x).max()
+
+
+# ---------------------------------------------------------------------------
+# generator sanity (its bit-exact twin on the device is tested on the GPU)
+# ---------------------------------------------------------------------------
+
+def test_splitmix64_reference_sequence():
+    """First outputs of SplitMix64 from state 0 (Vigna's splitmix64.c)."""
+    assert [int(synth.hash64(0, n)) for n in (1, 2, 3)] == [
+        0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+
+
+def test_generator_moments_and_flag_rate():
+    x = synth.normal_f32(5, synth.STREAM_K, 3, 1, np.arange(200_000), 2, 7)
+    assert abs(x.mean()) < 5 / np.sqrt(x.size) and abs(x.var() - 1) < 0.02
+    assert np.abs(x).max() <= 6.0
+    xb = synth.normal(5, synth.STREAM_K, 3, 1, np.arange(1000), 2, 7, "bf16")
+    assert np.array_equal(xb, torch.from_numpy(x[:1000]).to(torch.bfloat16).float().numpy())
+    thr = synth.keep_threshold(0.1)
+    f = synth.evict_flags(5, 0, 0, np.arange(200_000), 0, thr)
+    assert abs((1 - f.mean()) - 0.1) < 5 * np.sqrt(0.09 / f.size)
+
+
+def test_oracle_and_product_do_not_import_each_other():
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for dirpath, _, files in os.walk(os.path.join(root, "oracle")):
+        for f in files:
+            if f.endswith(".py"):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "compact_decode_attention_b200" not in src, f
+    pkg = os.path.join(root, "compact_decode_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f
