@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark: compact-KV DMS decode on B200.
+
+One step = one decode position of the whole hot path over every layer of the
+workload: dms_append_evict_layers (retire / reclaim / append) then
+dms_decode_attn_layers (split-K attention over each head's held rows).
+The default workload is Qwen3-8B attention shapes at ctx 8192 (36 layers,
+32 q / 8 kv heads, head_dim 128, bf16 K/V, window 512, per-head keep
+probability U[0.02, 0.30], seed 2).
+
+value      retained-KV GB/s of the whole step (held K/V bytes read per step,
+           summed over steps and ranks, / max-over-ranks device time)
+roofline   the attention kernel alone: algorithmic bytes / its CUDA-event time
+e2e        the same metric through the Python/C API with pinned host inputs
+           copied in and outputs copied out inside the timed region
+cpu_baseline  the CPU oracle timed on a bounded sample (rank 0, N = 1)
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+(for N > 1 launch with torch.distributed.run; each rank runs a replica).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+from synth import configs  # noqa: E402
+
+METRIC = "compact-KV decode attn: retained-KV GB/s vs HBM peak; decode steps/s at ctx 8K"
+DEFAULT_WORKLOAD = configs.QWEN8B_CTX8K.name
+ATTN_KERNEL_SRC = os.path.join(ROOT, "compact_decode_attention_b200", "csrc", "attn.cu")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_attn_qwen3-8b_ctx8k.md")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(configs.BY_NAME))
+    ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--cpu-heads", type=int, default=72)
+    ap.add_argument("--cpu-steps", type=int, default=30)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# measured peaks, clocks
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read only)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
+               0x1: "gpu_idle"}
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], 0
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.err = str(e)
+        self.period = period_s
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable"}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(wl, t0: int, n_heads: int, n_steps: int, bytes_per_step: float):
+    """Time the oracle (as it stands, one thread) on a sample of (head, step)
+    pairs of the workload; scale to a whole step by the number of heads."""
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    from oracle import attention as oatt
+    from oracle import reference as oref
+    from oracle import slots as oslots
+    H = wl.n_layers * wl.batch * wl.n_kv_heads
+    picks = []
+    rng = np.random.Generator(np.random.PCG64(12345))
+    for i in rng.choice(H, size=min(n_heads, H), replace=False):
+        h = int(i % wl.n_kv_heads)
+        b = int((i // wl.n_kv_heads) % wl.batch)
+        layer = int(i // (wl.n_kv_heads * wl.batch))
+        picks.append((layer, b, h))
+    # untimed: inputs of each sampled head (flags, the rows it may see, queries)
+    prep = []
+    for (layer, b, h) in picks:
+        T = t0 + n_steps
+        flags = oref.head_flags(wl, layer, b, h, T)
+        need = np.unique(np.concatenate([oracle_visible(t, flags, wl.window) for t in (t0, T - 1)]))
+        need = np.unique(np.concatenate([need, np.arange(max(0, t0 - wl.window), T)]))
+        K, V = oref.stored_rows(wl, layer, b, h, need)
+        Kf = np.zeros((T, wl.head_dim))
+        Vf = np.zeros((T, wl.head_dim))
+        Kf[need], Vf[need] = K, V
+        qs = [oref.head_query(wl, layer, b, h, t).astype(np.float64) for t in range(t0, T)]
+        store = oslots.HeadStore(flags[:wl.prompt], wl.window)
+        for t in range(wl.prompt, t0):
+            store.append(t, int(flags[t]))
+        prep.append((flags, Kf, Vf, qs, store))
+    # timed: the oracle's decode step for each sampled head
+    start = time.perf_counter()
+    for (flags, Kf, Vf, qs, store) in prep:
+        for s in range(n_steps):
+            t = t0 + s
+            store.append(t, int(flags[t]))
+            oatt.decode_attention(qs[s], Kf[:t + 1, None, :], Vf[:t + 1, None, :], flags[:t + 1, None],
+                                  t, wl.window)
+    elapsed = time.perf_counter() - start
+    per_head_step = elapsed / (len(prep) * n_steps)
+    step_time = per_head_step * H
+    return {
+        "value": bytes_per_step / step_time / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "sample": (f"{len(prep)} of {H} (layer, seq, kv-head) heads x {n_steps} decode steps from "
+                   f"t={t0}: slot bookkeeping + fp64 masked attention per head, {elapsed:.1f} s; "
+                   f"per-step time = mean head-step time x {H} heads"),
+        "seconds": elapsed, "step_seconds_extrapolated": step_time,
+    }
+
+
+def oracle_visible(t, flags, w):
+    from oracle import mask
+    return mask.visible_positions(t, flags, w)
+
+
+def expected_bytes_per_step(wl):
+    """Expected retained K/V bytes per step from the workload's keep probabilities."""
+    p = wl.keep_probs()
+    n = np.minimum(wl.prompt, wl.window) + p * max(0, wl.prompt - wl.window)
+    return float(n.sum() * wl.batch * 2 * wl.head_dim * wl.kv_elem_bytes())
+
+
+# ---------------------------------------------------------------------------
+# roofline helpers
+# ---------------------------------------------------------------------------
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.dirname(ATTN_KERNEL_SRC))):
+        if f in ("attn.cu", "dms_internal.cuh"):
+            h.update(open(os.path.join(os.path.dirname(ATTN_KERNEL_SRC), f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, when it was taken on the current kernel source; else None."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None, None
+    txt = open(PROFILE_SUMMARY).read()
+    m_src = re.search(r"kernel source hash:\s*([0-9a-f]+)", txt)
+    m_tr = re.search(r"dram bytes per full launch:\s*([0-9.eE+]+)", txt)
+    if not (m_src and m_tr) or m_src.group(1) != attn_source_hash():
+        return None, None
+    return float(m_tr.group(1)), m_src.group(1)
+
+
+# ---------------------------------------------------------------------------
+# the benchmark
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = configs.BY_NAME[args.workload]
+    bps = expected_bytes_per_step(wl)
+    t0 = time.perf_counter()
+    steps = max(1, args.steps)
+    per = max(1, args.cpu_steps // 3)
+    cb = cpu_baseline(wl, wl.prompt + args.warmup, max(8, args.cpu_heads // 3), per, bps)
+    wall = time.perf_counter() - t0
+    line = {
+        "impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": cb["step_seconds_extrapolated"] * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "bytes_per_step": bps},
+        "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": ("the reference arm is the CPU oracle (the pages ship no code); each step is a bounded "
+                 "sample of the workload's decode step, extrapolated by head count"),
+        "wall_s": wall,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from compact_decode_attention_b200 import dms
+    from compact_decode_attention_b200.workload import DeviceWorkload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = configs.BY_NAME[args.workload]
+    W, K, E = args.warmup, args.steps, args.e2e_steps
+    assert W >= 3 and K >= 1
+    dw = DeviceWorkload(wl, W + K + E, device=f"cuda:{local}")
+    dw.prefill()
+    torch.cuda.synchronize()
+
+    L, B, Hkv, D, w, P = wl.n_layers, wl.batch, wl.n_kv_heads, wl.head_dim, wl.window, wl.prompt
+    H = L * B * Hkv
+    row_bytes = 2 * D * wl.kv_elem_bytes()           # K row + V row of one token
+
+    # exact held tokens after each step: +1 per head, -1 per head whose token
+    # t - w carried a flag (flags drawn by the same device generator)
+    fl = dw.flags(0, L, P + 0 - w, W + K + E) if P - w >= 0 else None
+    retired = fl.sum(dim=(0, 1, 3)).cpu().numpy().astype(np.int64) if fl is not None else \
+        np.zeros(W + K + E, np.int64)
+    base = int(dw.pool.stats().retained_tokens)
+    held = base + np.cumsum(H - retired)                  # after step s
+    bytes_step = held.astype(np.float64) * row_bytes
+
+    stream = torch.cuda.current_stream()
+    for s in range(W):
+        dw.step(s)
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: exactly K steps ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    si = dw.step_inputs
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for j in range(K):
+            s = W + j
+            dw.pool.append_evict_layers(0, P + s, si["k"][s], si["v"][s], si["evict"][s])
+            ev[j][0].record(stream)
+            dw.pool.decode_attn_layers(0, si["q"][s], dw.out)
+            ev[j][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = t_start.elapsed_time(t_end)
+    attn_ms = np.array([a.elapsed_time(b) for a, b in ev])
+    st = dw.pool.stats()
+    if st.error_flags:
+        raise SystemExit(f"device error word 0x{st.error_flags:x}")
+
+    my_bytes = float(bytes_step[W:W + K].sum())
+    if world > 1:
+        t = torch.tensor([ms, my_bytes], dtype=torch.float64, device=f"cuda:{local}")
+        mx = t.clone()
+        dist.all_reduce(mx[0:1], op=dist.ReduceOp.MAX)
+        dist.all_reduce(t[1:2], op=dist.ReduceOp.SUM)
+        ms_max, total_bytes = float(mx[0]), float(t[1])
+    else:
+        ms_max, total_bytes = ms, my_bytes
+    value = total_bytes / (ms_max * 1e-3) / 1e9
+
+    # ---- roofline of the attention kernel ----
+    peak, peak_kind = measured_peaks()
+    achieved = float((bytes_step[W:W + K] / (attn_ms * 1e-3)).mean() / 1e9)
+    traffic, _ = profiled_traffic()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "decode_attn_kernel<bf16,128>" if wl.kv_dtype == "bf16" and D == 128 else "decode_attn_kernel",
+                "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "algorithmic_bytes_per_launch": float(bytes_step[W:W + K].mean()),
+                "attn_us_per_launch": float(attn_ms.mean() * 1e3)}
+
+    # ---- end to end: pinned host inputs in, outputs out, inside the timed region ----
+    e2e = None
+    if E > 0:
+        hk = si["k"][W + K:].cpu().pin_memory()
+        hv = si["v"][W + K:].cpu().pin_memory()
+        hq = si["q"][W + K:].cpu().pin_memory()
+        he = si["evict"][W + K:].cpu().pin_memory()
+        ho = torch.empty((E,) + tuple(dw.out.shape), dtype=dw.out.dtype).pin_memory()
+        dk, dv = torch.empty_like(si["k"][0]), torch.empty_like(si["v"][0])
+        dq, de = torch.empty_like(si["q"][0]), torch.empty_like(si["evict"][0])
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for j in range(E):
+            s = W + K + j
+            dk.copy_(hk[j], non_blocking=True)
+            dv.copy_(hv[j], non_blocking=True)
+            dq.copy_(hq[j], non_blocking=True)
+            de.copy_(he[j], non_blocking=True)
+            dw.pool.append_evict_layers(0, P + s, dk, dv, de)
+            dw.pool.decode_attn_layers(0, dq, dw.out)
+            ho[j].copy_(dw.out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=f"cuda:{local}")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        e_bytes = float(bytes_step[W + K:W + K + E].sum()) * world
+        h2d = int(hk[0].numel() * hk.element_size() * 2 + hq[0].numel() * hq.element_size()
+                  + he[0].numel() * he.element_size())
+        d2h = int(dw.out.numel() * dw.out.element_size())
+        e2e = {"value": e_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": E, "ms_per_step": e_ms / E}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, P + W, args.cpu_heads, args.cpu_steps, float(bytes_step[W]))
+        cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.kv_dtype == "bf16" else wl.kv_dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "layers": L, "batch": B, "q_heads": wl.n_q_heads,
+                       "kv_heads": Hkv, "head_dim": D, "prompt": P, "window": w, "kv_dtype": wl.kv_dtype,
+                       "seed": wl.seed, "parallelism": f"replicas x{world}",
+                       "l2": (f"no flush: {bytes_step[W] / 1e6:.0f} MB of held K/V read per step "
+                              f"> 126 MB L2")},
+            "decode_steps_per_s": world * K / (ms_max * 1e-3),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 2 * K, "clocks": clk.summary(),
+            "pool": {"blocks_in_use": int(st.blocks_in_use), "kv_bytes_in_use": int(st.kv_bytes_in_use),
+                     "retained_tokens": int(st.retained_tokens),
+                     "min_retained": int(st.min_retained), "max_retained": int(st.max_retained)},
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,790 @@
+// dms_decode_attn: split-K flash decoding over the compact DMS store.
+//
+// DMS only changes which keys a query sees: each kv-head keeps its own
+// ragged set of tokens (delayed eviction, "NVIDIA veröffentlicht
+// Qwen3-8B-DMS-8x ..." (mindverse), section "Dynamic Memory Sparsification
+// (DMS): Eine innovative Lösung"), and decode is bound by reading that set
+// from memory ("Nvidia DMS ..." (stiva.ai), opening section; FastDMS page:
+// faster decode from less KV).  The kernel therefore streams every held row
+// of every head once and nothing else.
+//
+// Work split (stream-K over blocks): the held rows of all heads of the call,
+// in (layer, sequence, kv-head) order, form U blocks of up to 64 rows.  A
+// persistent grid of G CTAs (one per SM) takes the contiguous ranges
+// [c*U/G, (c+1)*U/G), so every CTA moves the same bytes whatever the head
+// lengths.  A CTA's piece of a head ends in a partial softmax state
+// (m, l, o); a head cut by CTA boundaries is merged by log-sum-exp in the
+// CTA that finishes it last (an atomic ticket -- nobody waits).  Partial id
+// c + i is unique per (CTA c, head i) piece.
+//
+// Inside a CTA: warp 4 is the producer.  It issues one 1-D TMA bulk copy per
+// full block (K tile and V tile are adjacent in the pool, 32 KB for bf16
+// D=128) plus the g query rows of the head, into a ring of NS shared-memory
+// stages paced by mbarriers (expect-tx on "full", one arrive on "empty").
+// Warps 0-3 consume stages round-robin.  Each keeps its own online-softmax
+// state for the current head and computes on tensor cores with the GQA
+// group as the N=8 side of mma.sync m16n8k16 (tokens as M): S^T = K Q^T,
+// then O^T += V^T P^T, P moved from accumulator to operand layout with
+// movmatrix.  The stored rows' 16-byte chunks are XOR-swizzled by row, so
+// ldmatrix reads them without bank conflicts.  FP8-E4M3 rows are decoded to
+// f16 in registers (exact) from a layout that gives each lane its fragment
+// bytes in two 16-byte loads; fp32 rows use CUDA-core FMA.
+//
+// Every wait is bounded (1 s); a timeout sets DMS_DEVERR_TIMEOUT and the CTA
+// drains its in-flight copies and returns.
+#include <math.h>
+
+#include "dms_internal.cuh"
+
+namespace dms {
+
+constexpr int kNCW = 4;                       // consumer warps
+constexpr int kAttnThreads = 32 * (kNCW + 1);
+
+enum { KV_F32 = 0, KV_BF16 = 1, KV_FP8 = 2 };
+
+template <int KV, int D>
+struct AttnTraits {
+  static constexpr int ESZ = KV == KV_F32 ? 4 : KV == KV_BF16 ? 2 : 1;
+  static constexpr int QESZ = KV == KV_F32 ? 4 : 2;  // q / out element bytes
+  static constexpr int ROWB = D * ESZ;
+  static constexpr int TILEB = kBlockTokens * ROWB;
+  static constexpr int QB = 8 * D * QESZ;              // room for 8 query rows
+  static constexpr int STAGEB = 2 * TILEB + QB;
+  static constexpr int NS = KV == KV_F32 ? (D == 128 ? 3 : 4) : (KV == KV_BF16 && D == 128) ? 6 : 8;
+  static constexpr int COMBINE_FLOATS = kNCW * 8 * D + 2 * kNCW * 8;
+  static constexpr int MISC_INTS = 16 + kAttnThreads / 32;
+  static constexpr size_t SMEM = size_t(NS) * STAGEB + COMBINE_FLOATS * 4 + 2 * NS * 8 +
+                                 MISC_INTS * 4;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(STAGEB % 128 == 0, "stage alignment");
+};
+
+struct AttnParams {
+  PoolView v;
+  int l0, nl, batch;
+  const uint8_t* q;   // [nl, batch, Hq, D] q dtype
+  uint8_t* out;       // same layout and dtype
+  float scale_log2;   // sm_scale * log2(e)
+  float* ws_o;        // [(G + Htot) * g * D]
+  float* ws_ml;       // [(G + Htot) * g * 2]
+  int G;
+};
+
+__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ int units_of(int n) { return (n + kBlockTokens - 1) / kBlockTokens; }
+
+// head index i of the call -> pool head id
+__device__ __forceinline__ int pool_head(const AttnParams& p, int i) {
+  const int h = i % p.v.Hkv;
+  const int lb = i / p.v.Hkv;  // li * batch + b
+  return p.v.head(p.l0 + lb / p.batch, lb % p.batch, h);
+}
+
+__device__ __forceinline__ int n_of(const AttnParams& p, int i) { return p.v.n_slots[pool_head(p, i)]; }
+
+// CTA whose unit range holds unit u (U units cut into G ranges).
+__device__ __forceinline__ int cta_of(int64_t u, int64_t U, int G) {
+  return int(((u + 1) * G - 1) / U);
+}
+
+template <int QESZ>
+__device__ __forceinline__ void store_out(uint8_t* out, int64_t idx, float x) {
+  if constexpr (QESZ == 4) {
+    reinterpret_cast<float*>(out)[idx] = x;
+  } else {
+    reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(x);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-warp online-softmax state and unit compute, tensor-core paths
+// ---------------------------------------------------------------------------
+template <int KV, int D>
+struct MmaWarp {
+  static constexpr int KSTEPS = D / 16;  // QK^T k-steps over head_dim
+  static constexpr int MTD = D / 16;     // PV m-tiles over head_dim
+  using T = AttnTraits<KV, D>;
+  float m[2], l[2];
+  float o[MTD][4];
+  uint32_t qf[KSTEPS][2];
+  float scale;  // log2-domain score scale (includes the K scale for FP8)
+  float vscale; // V scale (FP8), else 1
+
+  __device__ __forceinline__ void reset() {
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+#pragma unroll
+    for (int i = 0; i < MTD; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  }
+
+  // Q^T B fragments from the stage's query rows (row n = lane / 4).
+  __device__ __forceinline__ void load_q(const uint8_t* qs, int lane) {
+    const int n = lane >> 2, q2 = (lane & 3) * 2;
+    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(qs) + n * D;
+#pragma unroll
+    for (int kt = 0; kt < KSTEPS; ++kt) {
+      const uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + kt * 16 + q2);
+      const uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + kt * 16 + 8 + q2);
+      if constexpr (KV == KV_FP8) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+        qf[kt][0] = pack_f16x2(a.x, a.y);
+        qf[kt][1] = pack_f16x2(b.x, b.y);
+      } else {
+        qf[kt][0] = lo;
+        qf[kt][1] = hi;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                      uint32_t b1) {
+    if constexpr (KV == KV_FP8) mma_f16_16816(d, a, b0, b1);
+    else mma_bf16_16816(d, a, b0, b1);
+  }
+
+  __device__ __forceinline__ void unit(const uint8_t* stage, int rows, int lane) {
+    const uint8_t* Ks = stage;
+    const uint8_t* Vs = stage + T::TILEB;
+    const int q = lane & 3, r8 = lane >> 2;
+    float s[4][4];
+    // ---- S^T = K Q^T over the 64 rows (4 m-tiles of 16 tokens) ----
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
+      if (mt * 16 < rows) {
+        if constexpr (KV == KV_BF16) {
+          const uint32_t kbase = smem_u32(Ks);
+          const int row = mt * 16 + (lane & 15);
+#pragma unroll
+          for (int kt = 0; kt < KSTEPS; ++kt) {
+            const int ch = 2 * kt + (lane >> 4);
+            uint32_t a[4];
+            ldmatrix_x4(a, kbase + row * T::ROWB + (swz_chunk(ch, row) << 4));
+            mma(s[mt], a, qf[kt][0], qf[kt][1]);
+          }
+        } else {  // FP8, D = 128: two 16-byte loads per row give all 8 k-steps
+          const int r0 = mt * 16 + r8, r1 = r0 + 8;
+          const uint4 a0lo = *reinterpret_cast<const uint4*>(Ks + r0 * 128 + (((2 * q) ^ (r0 & 7)) << 4));
+          const uint4 a0hi = *reinterpret_cast<const uint4*>(Ks + r0 * 128 + (((2 * q + 1) ^ (r0 & 7)) << 4));
+          const uint4 a1lo = *reinterpret_cast<const uint4*>(Ks + r1 * 128 + (((2 * q) ^ (r1 & 7)) << 4));
+          const uint4 a1hi = *reinterpret_cast<const uint4*>(Ks + r1 * 128 + (((2 * q + 1) ^ (r1 & 7)) << 4));
+          const uint32_t w0[8] = {a0lo.x, a0lo.y, a0lo.z, a0lo.w, a0hi.x, a0hi.y, a0hi.z, a0hi.w};
+          const uint32_t w1[8] = {a1lo.x, a1lo.y, a1lo.z, a1lo.w, a1hi.x, a1hi.y, a1hi.z, a1hi.w};
+#pragma unroll
+          for (int kt = 0; kt < KSTEPS; ++kt) {
+            uint32_t a[4];
+            a[0] = e4m3x2_to_f16x2(uint16_t(w0[kt] & 0xffff));
+            a[1] = e4m3x2_to_f16x2(uint16_t(w1[kt] & 0xffff));
+            a[2] = e4m3x2_to_f16x2(uint16_t(w0[kt] >> 16));
+            a[3] = e4m3x2_to_f16x2(uint16_t(w1[kt] >> 16));
+            mma(s[mt], a, qf[kt][0], qf[kt][1]);
+          }
+        }
+      }
+    }
+    // ---- scale, mask rows past `rows`, online softmax ----
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      const int r0 = mt * 16 + r8;
+      const bool v0 = r0 < rows, v1 = r0 + 8 < rows;
+      s[mt][0] = v0 ? s[mt][0] * scale : -INFINITY;
+      s[mt][1] = v0 ? s[mt][1] * scale : -INFINITY;
+      s[mt][2] = v1 ? s[mt][2] * scale : -INFINITY;
+      s[mt][3] = v1 ? s[mt][3] * scale : -INFINITY;
+      mx0 = fmaxf(mx0, fmaxf(s[mt][0], s[mt][2]));
+      mx1 = fmaxf(mx1, fmaxf(s[mt][1], s[mt][3]));
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+    const float al0 = fast_exp2(m[0] - mn0), al1 = fast_exp2(m[1] - mn1);
+    m[0] = mn0;
+    m[1] = mn1;
+    l[0] *= al0;
+    l[1] *= al1;
+#pragma unroll
+    for (int md = 0; md < MTD; ++md) {
+      o[md][0] *= al0;
+      o[md][1] *= al1;
+      o[md][2] *= al0;
+      o[md][3] *= al1;
+    }
+    uint32_t pb[4][2];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      const float p0 = fast_exp2(s[mt][0] - mn0), p1 = fast_exp2(s[mt][1] - mn1);
+      const float p2 = fast_exp2(s[mt][2] - mn0), p3 = fast_exp2(s[mt][3] - mn1);
+      l[0] += p0 + p2;
+      l[1] += p1 + p3;
+      if constexpr (KV == KV_FP8) {
+        pb[mt][0] = movmatrix_trans(pack_f16x2(p0, p1));
+        pb[mt][1] = movmatrix_trans(pack_f16x2(p2, p3));
+      } else {
+        pb[mt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+        pb[mt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+      }
+    }
+    // ---- O^T += V^T P^T ----
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      if (mt * 16 >= rows) break;
+      const bool partial = mt * 16 + 16 > rows;
+      const int t0 = mt * 16 + 2 * q;
+      const uint32_t m01 = (t0 < rows ? 0x0000ffffu : 0u) | (t0 + 1 < rows ? 0xffff0000u : 0u);
+      const uint32_t m23 = (t0 + 8 < rows ? 0x0000ffffu : 0u) | (t0 + 9 < rows ? 0xffff0000u : 0u);
+      if constexpr (KV == KV_BF16) {
+        const uint32_t vbase = smem_u32(Vs);
+        const int row = mt * 16 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+        for (int md = 0; md < MTD; ++md) {
+          const int ch = 2 * md + ((lane >> 3) & 1);
+          uint32_t a[4];
+          ldmatrix_x4_trans(a, vbase + row * T::ROWB + (swz_chunk(ch, row) << 4));
+          if (partial) {
+            a[0] &= m01;
+            a[1] &= m01;
+            a[2] &= m23;
+            a[3] &= m23;
+          }
+          mma(o[md], a, pb[mt][0], pb[mt][1]);
+        }
+      } else {  // FP8: V^T tile [D][64], 16 bytes per (d row, owner lane)
+#pragma unroll
+        for (int md = 0; md < MTD; ++md) {
+          const int d0 = md * 16 + r8;
+          const uint4 x0 = *reinterpret_cast<const uint4*>(Vs + d0 * 64 + q * 16);
+          const uint4 x1 = *reinterpret_cast<const uint4*>(Vs + (d0 + 8) * 64 + q * 16);
+          const uint32_t w0 = mt == 0 ? x0.x : mt == 1 ? x0.y : mt == 2 ? x0.z : x0.w;
+          const uint32_t w1 = mt == 0 ? x1.x : mt == 1 ? x1.y : mt == 2 ? x1.z : x1.w;
+          uint32_t a[4];
+          a[0] = e4m3x2_to_f16x2(uint16_t(w0 & 0xffff));
+          a[1] = e4m3x2_to_f16x2(uint16_t(w1 & 0xffff));
+          a[2] = e4m3x2_to_f16x2(uint16_t(w0 >> 16));
+          a[3] = e4m3x2_to_f16x2(uint16_t(w1 >> 16));
+          if (partial) {
+            a[0] &= m01;
+            a[1] &= m01;
+            a[2] &= m23;
+            a[3] &= m23;
+          }
+          mma(o[md], a, pb[mt][0], pb[mt][1]);
+        }
+      }
+    }
+  }
+
+  // Write this warp's state for query heads n < g into the combine area.
+  __device__ __forceinline__ void write_state(float* ow, float* mw, float* lw, int g, int lane) {
+    float l0 = l[0], l1 = l[1];
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    const int n0 = (lane & 3) * 2, r8 = lane >> 2;
+#pragma unroll
+    for (int md = 0; md < MTD; ++md) {
+      const int d = md * 16 + r8;
+      if (n0 < g) {
+        ow[n0 * D + d] = o[md][0] * vscale;
+        ow[n0 * D + d + 8] = o[md][2] * vscale;
+      }
+      if (n0 + 1 < g) {
+        ow[(n0 + 1) * D + d] = o[md][1] * vscale;
+        ow[(n0 + 1) * D + d + 8] = o[md][3] * vscale;
+      }
+    }
+    if (r8 == 0) {
+      if (n0 < g) {
+        mw[n0] = m[0];
+        lw[n0] = l0;
+      }
+      if (n0 + 1 < g) {
+        mw[n0 + 1] = m[1];
+        lw[n0 + 1] = l1;
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// fp32 path (CUDA-core FMA; exact fp32 arithmetic, no TF32)
+// ---------------------------------------------------------------------------
+template <int D>
+struct F32Warp {
+  static constexpr int DPL = D / 32;  // output elements per lane per query head
+  using T = AttnTraits<KV_F32, D>;
+  float m[8], l[8];
+  float o[8][DPL];
+  const float* qrow;  // stage query rows (set per unit)
+  float scale, vscale;
+  int g;
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      m[n] = -INFINITY;
+      l[n] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) o[n][e] = 0.f;
+    }
+  }
+  __device__ __forceinline__ void load_q(const uint8_t*, int) {}
+
+  __device__ __forceinline__ float kval(const uint8_t* tile, int r, int d) const {
+    return reinterpret_cast<const float*>(tile + r * T::ROWB + (swz_chunk(d >> 2, r) << 4))[d & 3];
+  }
+
+  __device__ __forceinline__ void unit(const uint8_t* stage, int rows, int lane) {
+    const uint8_t* Ks = stage;
+    const uint8_t* Vs = stage + T::TILEB;
+    const float* qs = reinterpret_cast<const float*>(stage + 2 * T::TILEB);
+    float s[2][8];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int r = lane + 32 * hh;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) s[hh][n] = 0.f;
+      if (r < rows) {
+        for (int d = 0; d < D; ++d) {
+          const float kd = kval(Ks, r, d);
+#pragma unroll
+          for (int n = 0; n < 8; ++n)
+            if (n < g) s[hh][n] = fmaf(qs[n * D + d], kd, s[hh][n]);
+        }
+      }
+#pragma unroll
+      for (int n = 0; n < 8; ++n) s[hh][n] = r < rows ? s[hh][n] * scale : -INFINITY;
+    }
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      if (n >= g) continue;
+      float mx = fmaxf(s[0][n], s[1][n]);
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float mn = fmaxf(m[n], mx);
+      const float al = fast_exp2(m[n] - mn);
+      m[n] = mn;
+      s[0][n] = fast_exp2(s[0][n] - mn);
+      s[1][n] = fast_exp2(s[1][n] - mn);
+      float ps = s[0][n] + s[1][n];
+      for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      l[n] = l[n] * al + ps;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) o[n][e] *= al;
+    }
+    for (int r = 0; r < rows; ++r) {
+      float pr[8];
+#pragma unroll
+      for (int n = 0; n < 8; ++n) pr[n] = __shfl_sync(0xffffffffu, s[r >> 5][n], r & 31);
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) {
+        const float vd = kval(Vs, r, lane + 32 * e);
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+          if (n < g) o[n][e] = fmaf(pr[n], vd, o[n][e]);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void write_state(float* ow, float* mw, float* lw, int gg, int lane) {
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      if (n >= gg) continue;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) ow[n * D + lane + 32 * e] = o[n][e] * vscale;
+      if (lane == 0) {
+        mw[n] = m[n];
+        lw[n] = l[n];
+      }
+    }
+  }
+};
+
+template <int KV, int D>
+struct WarpSel {
+  using type = MmaWarp<KV, D>;
+};
+template <int D>
+struct WarpSel<KV_F32, D> {
+  using type = F32Warp<D>;
+};
+
+// ---------------------------------------------------------------------------
+template <int KV, int D>
+__global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const AttnParams p) {
+  using T = AttnTraits<KV, D>;
+  using W = typename WarpSel<KV, D>::type;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* stages = smem;
+  float* s_ow = reinterpret_cast<float*>(smem + size_t(T::NS) * T::STAGEB);
+  float* s_mw = s_ow + kNCW * 8 * D;
+  float* s_lw = s_mw + kNCW * 8;
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_lw + kNCW * 8);
+  uint64_t* empty = full + T::NS;
+  int* s_misc = reinterpret_cast<int*>(empty + T::NS);
+  volatile int* s_abort = s_misc;        // [0]
+  int* s_scan = s_misc + 16;             // [kAttnThreads / 32]
+
+  const PoolView& v = p.v;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = v.Hq / v.Hkv;
+  const int Htot = p.nl * p.batch * v.Hkv;
+  const int c = blockIdx.x, G = p.G;
+
+  if (tid == 0) {
+    for (int s = 0; s < T::NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    s_misc[0] = 0;
+    fence_mbar_init();
+  }
+  // query rows g..7 of every stage stay zero (padding of the N=8 side)
+  for (int s = 0; s < T::NS; ++s) {
+    uint4* qa = reinterpret_cast<uint4*>(stages + size_t(s) * T::STAGEB + 2 * T::TILEB);
+    for (int i = tid; i < T::QB / 16; i += kAttnThreads) qa[i] = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();  // order these generic writes before later TMA writes
+
+  // ---- find this CTA's unit range: per-thread head ranges + block scan ----
+  const int per = (Htot + kAttnThreads - 1) / kAttnThreads;
+  const int hb = min(Htot, tid * per), he = min(Htot, hb + per);
+  int su = 0;
+  for (int i = hb; i < he; ++i) {
+    const int n = n_of(p, i);
+    su += units_of(n);
+    if (n == 0 && i % G == c) {  // no key at all: define the output as 0
+      const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
+      for (int e = 0; e < g * D; ++e) store_out<T::QESZ>(p.out, orow * D + e, 0.f);
+    }
+  }
+  int incl = su;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) s_scan[warp] = incl;
+  __syncthreads();
+  int wbase = 0, U = 0;
+  for (int k = 0; k < kAttnThreads / 32; ++k) {
+    wbase += k < warp ? s_scan[k] : 0;
+    U += s_scan[k];
+  }
+  const int excl = wbase + incl - su;
+  const int u_beg = int((int64_t(c) * U) / G), u_end = int((int64_t(c + 1) * U) / G);
+  if (u_beg < u_end && u_beg >= excl && u_beg < excl + su) {
+    int pre = excl;
+    for (int i = hb; i < he; ++i) {
+      const int nu = units_of(n_of(p, i));
+      if (u_beg < pre + nu) {
+        s_misc[1] = i;
+        s_misc[2] = pre;
+        break;
+      }
+      pre += nu;
+    }
+  }
+  __syncthreads();
+  if (u_beg >= u_end) return;
+  const int i0 = s_misc[1], p0 = s_misc[2];
+  const int qrow_bytes = g * D * T::QESZ;
+
+  if (warp == kNCW) {
+    // ======================= producer =======================
+    const uint64_t pol = policy_evict_first();   // K/V rows: read once per step
+    const uint64_t qpol = policy_evict_last();   // query rows: re-read per block
+    int k = 0, issued = 0;
+    bool aborted = false;
+    int i = i0, pp = p0, n = n_of(p, i0), nu = units_of(n);
+    for (int ub = u_beg; ub < u_end; ub += 32) {
+      const int u = ub + lane;
+      int mi = i, mp = pp, mn = n, mnu = nu;
+      int blk = 0, rows = 0;
+      if (u < u_end) {
+        while (u >= mp + mnu) {
+          mp += mnu;
+          ++mi;
+          mn = n_of(p, mi);
+          mnu = units_of(mn);
+        }
+        const int bi = u - mp;
+        blk = v.bt[int64_t(pool_head(p, mi)) * v.mbh + bi];
+        rows = min(kBlockTokens, mn - bi * kBlockTokens);
+      }
+      const int cnt = min(32, u_end - ub);
+      for (int j = 0; j < cnt; ++j) {
+        const int jblk = __shfl_sync(0xffffffffu, blk, j);
+        const int jrows = __shfl_sync(0xffffffffu, rows, j);
+        const int ji = __shfl_sync(0xffffffffu, mi, j);
+        if (lane == 0 && !aborted) {
+          const int s = k % T::NS;
+          const uint32_t ph = (k / T::NS) & 1;
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1, s_abort)) {
+            aborted = true;
+            *s_abort = 1;
+            report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
+          } else {
+            uint8_t* st = stages + size_t(s) * T::STAGEB;
+            const uint8_t* src = v.blocks + int64_t(jblk) * v.block_bytes;
+            const uint8_t* qsrc = p.q + int64_t(ji / v.Hkv) * v.Hq * D * T::QESZ +
+                                  int64_t(ji % v.Hkv) * qrow_bytes;
+            const uint32_t kbytes = uint32_t(jrows) * T::ROWB;
+            const bool whole = jrows == kBlockTokens;
+            const uint32_t vbytes = (whole || KV == KV_FP8) ? T::TILEB : kbytes;
+            mbar_arrive_expect_tx(&full[s], kbytes + vbytes + qrow_bytes);
+            if (whole) {
+              bulk_g2s(st, src, 2 * T::TILEB, &full[s], pol);
+            } else {
+              bulk_g2s(st, src, kbytes, &full[s], pol);
+              bulk_g2s(st + T::TILEB, src + T::TILEB, vbytes, &full[s], pol);
+            }
+            bulk_g2s(st + 2 * T::TILEB, qsrc, qrow_bytes, &full[s], qpol);
+            issued = k + 1;
+          }
+        }
+        ++k;
+      }
+      const int last = cnt - 1;
+      i = __shfl_sync(0xffffffffu, mi, last);
+      pp = __shfl_sync(0xffffffffu, mp, last);
+      n = __shfl_sync(0xffffffffu, mn, last);
+      nu = __shfl_sync(0xffffffffu, mnu, last);
+      aborted = __shfl_sync(0xffffffffu, aborted, 0);
+    }
+    // drain: the CTA may not leave while a copy into its shared memory is in flight
+    if (lane == 0) {
+      volatile int never = 0;
+      for (int kk = max(0, issued - T::NS); kk < issued; ++kk)
+        mbar_wait_bounded(&full[kk % T::NS], (kk / T::NS) & 1, &never);
+    }
+    return;
+  }
+
+  // ========================= consumers =========================
+  W st;
+  st.reset();
+  if constexpr (KV == KV_F32) st.g = g;
+  float* my_ow = s_ow + warp * 8 * D;
+  float* my_mw = s_mw + warp * 8;
+  float* my_lw = s_lw + warp * 8;
+  int i = i0, pp = p0, n = n_of(p, i0), nu = units_of(n);
+  bool have_q = false;
+  auto set_head_scales = [&](int head_i) {
+    st.scale = p.scale_log2;
+    st.vscale = 1.f;
+    if constexpr (KV == KV_FP8) {
+      const int hkv = head_i % v.Hkv;
+      const int lyr = p.l0 + (head_i / v.Hkv) / p.batch;
+      st.scale = p.scale_log2 * v.scales[(int64_t(lyr) * v.Hkv + hkv) * 2 + 0];
+      st.vscale = v.scales[(int64_t(lyr) * v.Hkv + hkv) * 2 + 1];
+    }
+  };
+  set_head_scales(i);
+  int k = 0;
+  for (int u = u_beg; u < u_end; ++u, ++k) {
+    while (u >= pp + nu) {
+      pp += nu;
+      ++i;
+      n = n_of(p, i);
+      nu = units_of(n);
+      set_head_scales(i);
+    }
+    const int rows = min(kBlockTokens, n - (u - pp) * kBlockTokens);
+    if (k % kNCW == warp) {
+      const int s = k % T::NS;
+      const uint32_t ph = (k / T::NS) & 1;
+      bool ok = false;
+      if (!*s_abort) {
+        ok = mbar_wait_bounded(&full[s], ph, s_abort);
+        if (!ok && lane == 0) {
+          *s_abort = 1;
+          report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0) && __all_sync(0xffffffffu, ok);
+      if (ok) {
+        const uint8_t* stage = stages + size_t(s) * T::STAGEB;
+        if constexpr (KV == KV_F32) {
+          st.unit(stage, rows, lane);
+        } else {
+          if (!have_q) {
+            st.load_q(stage + 2 * T::TILEB, lane);
+            have_q = true;
+          }
+          st.unit(stage, rows, lane);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // ---- end of this CTA's piece of head i: combine the 4 warps ----
+    if (u + 1 == u_end || u + 1 >= pp + nu) {
+      st.write_state(my_ow, my_mw, my_lw, g, lane);
+      consumer_bar();
+      const int hd = pool_head(p, i);
+      const int cf = cta_of(pp, U, G), cl = cta_of(int64_t(pp) + nu - 1, U, G);
+      const bool whole = cf == cl;
+      const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
+      const int pid = c + i;
+      for (int idx = tid; idx < g * D; idx += 128) {
+        const int nn = idx / D, d = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kNCW; ++w) M = fmaxf(M, s_mw[w * 8 + nn]);
+        float o = 0.f, L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kNCW; ++w) {
+          const float f = fast_exp2(s_mw[w * 8 + nn] - M);
+          o += f * s_ow[(w * 8 + nn) * D + d];
+          L += f * s_lw[w * 8 + nn];
+        }
+        if (whole) {
+          store_out<T::QESZ>(p.out, orow * D + idx, o / L);
+        } else {
+          p.ws_o[(int64_t(pid) * g + nn) * D + d] = o;
+          if (d == 0) {
+            p.ws_ml[(int64_t(pid) * g + nn) * 2 + 0] = M;
+            p.ws_ml[(int64_t(pid) * g + nn) * 2 + 1] = L;
+          }
+        }
+      }
+      if (!whole) {
+        consumer_bar();
+        if (tid == 0) {
+          __threadfence();
+          const int prev = atomicAdd(&v.tickets[hd], 1);
+          s_misc[3] = prev == cl - cf;
+        }
+        consumer_bar();
+        if (s_misc[3]) {
+          __threadfence();
+          for (int idx = tid; idx < g * D; idx += 128) {
+            const int nn = idx / D, d = idx % D;
+            float M = -INFINITY;
+            for (int cc = cf; cc <= cl; ++cc)
+              M = fmaxf(M, __ldcg(&p.ws_ml[(int64_t(cc + i) * g + nn) * 2]));
+            float o = 0.f, L = 0.f;
+            for (int cc = cf; cc <= cl; ++cc) {
+              const int64_t id = int64_t(cc + i) * g + nn;
+              const float f = fast_exp2(__ldcg(&p.ws_ml[id * 2]) - M);
+              o += f * __ldcg(&p.ws_o[id * D + d]);
+              L += f * __ldcg(&p.ws_ml[id * 2 + 1]);
+            }
+            store_out<T::QESZ>(p.out, orow * D + idx, o / L);
+          }
+          if (tid == 0) v.tickets[hd] = 0;
+        }
+      }
+      consumer_bar();
+      st.reset();
+      have_q = false;
+    }
+  }
+}
+
+template <int KV, int D>
+static dms_status launch_attn(const AttnParams& prm, cudaStream_t stream) {
+  using T = AttnTraits<KV, D>;
+  static bool attr_set = false;  // per instantiation; set once per process
+  if (!attr_set) {
+    dms_status st = cuda_status(cudaFuncSetAttribute(decode_attn_kernel<KV, D>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      int(T::SMEM)),
+                                "attn smem attribute");
+    if (st != DMS_OK) return st;
+    attr_set = true;
+  }
+  decode_attn_kernel<KV, D><<<prm.G, kAttnThreads, T::SMEM, stream>>>(prm);
+  return cuda_status(cudaGetLastError(), "decode_attn_kernel");
+}
+
+}  // namespace dms
+
+using namespace dms;
+
+static size_t attn_workspace_bytes(const dms_pool* pool, int n_layers, int batch) {
+  const PoolView& v = pool->view;
+  const int g = v.Hq / v.Hkv;
+  const size_t parts = size_t(pool->sm_count) + size_t(n_layers) * batch * v.Hkv;
+  const size_t o_bytes = (parts * g * v.D * 4 + 255) & ~size_t(255);
+  return o_bytes + parts * g * 2 * 4;
+}
+
+extern "C" dms_status dms_decode_workspace_bytes(const dms_pool* pool, int n_layers, int batch,
+                                                 size_t* bytes) {
+  if (!pool || !bytes || n_layers < 1 || batch < 1) {
+    set_last_error("bad arguments");
+    return DMS_ERR_INVALID_ARG;
+  }
+  *bytes = attn_workspace_bytes(pool, n_layers, batch);
+  return DMS_OK;
+}
+
+extern "C" dms_status dms_decode_attn_layers(dms_pool* pool, int layer0, int n_layers, int batch,
+                                             const void* q, dms_dtype q_dtype, void* out,
+                                             float sm_scale, void* workspace,
+                                             size_t workspace_bytes, cudaStream_t stream) {
+  if (!pool) {
+    set_last_error("null pool");
+    return DMS_ERR_INVALID_ARG;
+  }
+  const PoolView& v = pool->view;
+  if (layer0 < 0 || n_layers < 1 || layer0 + n_layers > v.L || batch < 1 || batch > v.Bmax) {
+    set_last_error("bad layer range / batch (%d+%d, %d)", layer0, n_layers, batch);
+    return DMS_ERR_INVALID_ARG;
+  }
+  if (!q || !out || !workspace) {
+    set_last_error("null q / out / workspace");
+    return DMS_ERR_INVALID_ARG;
+  }
+  const dms_dtype want = v.kv_dtype == DMS_F32 ? DMS_F32 : DMS_BF16;
+  if (q_dtype != want) {
+    set_last_error("q_dtype must be %s for this pool", want == DMS_F32 ? "DMS_F32" : "DMS_BF16");
+    return DMS_ERR_INVALID_ARG;
+  }
+  if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(workspace) & 255)) {
+    set_last_error("q must be 16-byte aligned and workspace 256-byte aligned");
+    return DMS_ERR_INVALID_ARG;
+  }
+  const size_t need = attn_workspace_bytes(pool, n_layers, batch);
+  if (workspace_bytes < need) {
+    set_last_error("workspace has %zu bytes, needs %zu", workspace_bytes, need);
+    return DMS_ERR_CAPACITY;
+  }
+  const int g = v.Hq / v.Hkv;
+  const size_t parts = size_t(pool->sm_count) + size_t(n_layers) * batch * v.Hkv;
+  AttnParams prm;
+  prm.v = v;
+  prm.l0 = layer0;
+  prm.nl = n_layers;
+  prm.batch = batch;
+  prm.q = static_cast<const uint8_t*>(q);
+  prm.out = static_cast<uint8_t*>(out);
+  const float sc = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf(float(v.D));
+  prm.scale_log2 = sc * 1.4426950408889634f;
+  prm.ws_o = static_cast<float*>(workspace);
+  prm.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                       ((parts * g * v.D * 4 + 255) & ~size_t(255)));
+  prm.G = pool->sm_count;
+  if (v.kv_dtype == DMS_BF16) {
+    return v.D == 128 ? launch_attn<KV_BF16, 128>(prm, stream) : launch_attn<KV_BF16, 64>(prm, stream);
+  }
+  if (v.kv_dtype == DMS_FP8_E4M3) return launch_attn<KV_FP8, 128>(prm, stream);
+  return v.D == 128 ? launch_attn<KV_F32, 128>(prm, stream) : launch_attn<KV_F32, 64>(prm, stream);
+}
+
+extern "C" dms_status dms_decode_attn(dms_pool* pool, int layer, int batch, const void* q,
+                                      dms_dtype q_dtype, void* out, float sm_scale,
+                                      void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream) {
+  return dms_decode_attn_layers(pool, layer, 1, batch, q, q_dtype, out, sm_scale, workspace,
+                                workspace_bytes, stream);
+}

@@ -1,0 +1,266 @@
+// Internal definitions shared by the libdms CUDA sources (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "dms.h"
+
+namespace dms {
+
+constexpr int kBlockTokens = 64;     // BT: rows per physical block
+constexpr int kFreeStackCap = 4;     // per-head free slots awaiting reuse
+constexpr int kPrefillChunk = 256;   // prompt tokens per compaction CTA
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // every device wait gives up after 1 s
+
+// Device-side header at the start of the pool buffer.
+struct DevHeader {
+  int32_t next_block;       // bump pointer into the block region
+  int32_t block_stack_top;  // entries on the global free-block stack
+  uint32_t error;           // DMS_DEVERR_* bits
+  int32_t err_layer;        // first failing head, -1 when none
+  int32_t err_seq;
+  int32_t err_head;
+  int32_t prefill_go;       // set by the prefill planner when the layer may be written
+  int32_t pad;
+};
+
+// Everything a kernel needs to address the pool; passed by value.
+struct PoolView {
+  int32_t L, Bmax, Hq, Hkv, D, w, BT, kv_dtype;
+  int32_t mbh;              // block table width (max blocks per head)
+  int32_t free_cap;
+  int32_t n_heads;
+  int32_t n_chunks_max;     // prefill scratch: chunks per (b, h)
+  int64_t max_blocks;
+  int64_t row_bytes;        // D * elem size
+  int64_t tile_bytes;       // BT * row_bytes
+  int64_t block_bytes;      // 2 * tile_bytes
+  uint8_t* blocks;
+  int32_t* bt;
+  int32_t* n_slots;
+  int32_t* n_retained;
+  uint32_t* ring;
+  int32_t* free_top;
+  int32_t* free_stack;
+  int32_t* block_stack;
+  float* scales;            // [L][Hkv][2] (K, V)
+  int32_t* tickets;         // [n_heads] split-K merge tickets (self-resetting)
+  DevHeader* hdr;
+  int32_t* chunk_counts;    // prefill scratch [Bmax][Hkv][n_chunks_max]
+  uint32_t* amax;           // prefill scratch [2][Hkv] (float bits, non-negative)
+  void* stats;              // staging for dms_pool_stats
+
+  __host__ __device__ __forceinline__ int head(int l, int b, int h) const {
+    return (l * Bmax + b) * Hkv + h;
+  }
+};
+
+// ------------------------------------------------------------------------
+// error word
+// ------------------------------------------------------------------------
+__device__ __forceinline__ void report_error(DevHeader* hdr, uint32_t bit, int l, int b, int h) {
+  atomicOr(&hdr->error, bit);
+  if (atomicCAS(&hdr->err_layer, -1, l) == -1) {
+    hdr->err_seq = b;
+    hdr->err_head = h;
+  }
+}
+
+// ------------------------------------------------------------------------
+// stored-row layout
+// ------------------------------------------------------------------------
+// bf16 / fp32 rows: 16-byte chunk c of row r lives at chunk c ^ (r & 7).
+__host__ __device__ __forceinline__ int swz_chunk(int c, int r) { return c ^ (r & 7); }
+
+// FP8 K rows (D = 128): logical element d of row r is stored at byte
+//   chunk' * 16 + (pos & 15),  pos = owner * 32 + kt * 4 + hi * 2 + lo,
+//   owner = (d & 7) >> 1, kt = d >> 4, hi = (d >> 3) & 1, lo = d & 1,
+//   chunk' = (pos >> 4) ^ (r & 7)
+// so that lane (r, owner) of an m16n8k16 A fragment reads its 32 values as
+// two conflict-free 16-byte loads.
+__host__ __device__ __forceinline__ int fp8k_pos(int d) {
+  return (((d & 7) >> 1) << 5) | ((d >> 4) << 2) | (((d >> 3) & 1) << 1) | (d & 1);
+}
+__host__ __device__ __forceinline__ int fp8k_byte(int r, int d) {
+  const int pos = fp8k_pos(d);
+  return r * 128 + ((((pos >> 4) ^ (r & 7)) << 4) | (pos & 15));
+}
+// FP8 V tiles are stored transposed, [D][BT]: token row r of element d sits
+// at byte d * 64 + owner * 16 + kt * 4 + hi * 2 + lo with the same split of
+// the token index r (owner = (r & 7) >> 1, kt = r >> 4, hi = (r >> 3) & 1).
+__host__ __device__ __forceinline__ int fp8v_byte(int r, int d) {
+  return d * 64 + ((((r & 7) >> 1) << 4) | ((r >> 4) << 2) | (((r >> 3) & 1) << 1) | (r & 1));
+}
+
+// ------------------------------------------------------------------------
+// PTX wrappers
+// ------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase of `parity` to complete; gives up after kWaitLimitNs or
+// when *abort becomes non-zero.  Returns false when it gave up.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 1-D bulk copy global -> shared (TMA), completion counted on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                         uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// D += A(16x16, row) * B(16x8, col), bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Same shape with f16 inputs (the FP8 path decodes E4M3 to f16 exactly).
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// 2^x with the hardware approximation (max rel. error ~2^-22).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two E4M3 bytes (low byte = first element) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
+  uint32_t y;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(y) : "h"(x));
+  return y;
+}
+
+// E4M3 code of an fp32 value: round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint8_t f32_to_e4m3(float x) {
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+
+// ------------------------------------------------------------------------
+// host helpers
+// ------------------------------------------------------------------------
+void set_last_error(const char* fmt, ...);
+dms_status cuda_status(cudaError_t e, const char* what);
+int device_sm_count(int device);
+
+}  // namespace dms
+
+// The opaque host handle.
+struct dms_pool {
+  dms_pool_config cfg;
+  dms_pool_layout_t layout;
+  dms::PoolView view;
+  void* base;
+  size_t bytes;
+  int device;
+  int sm_count;
+};

@@ -1,0 +1,293 @@
+"""Python binding of libdms (ctypes): argument marshalling only.
+
+Every function mirrors one C entry point of ``include/dms.h`` /
+``include/dms_synth.h`` under the same name and returns what the C call
+writes.  A non-OK status raises ``DmsError`` carrying the status and the
+library's last error message.  Tensors are passed as raw pointers; PyTorch
+is used only for device memory and streams (``Pool`` allocates the pool
+buffer with it).  Importing this module does not load the library; the first
+call does, and it raises ``DmsLibraryMissing`` when ``libdms.so`` has not
+been built -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdms.so")
+
+DMS_OK, DMS_ERR_INVALID_ARG, DMS_ERR_CAPACITY, DMS_ERR_CUDA, DMS_ERR_UNSUPPORTED, DMS_ERR_DEVICE = range(6)
+DMS_F32, DMS_BF16, DMS_FP8_E4M3 = 0, 1, 2
+
+DEVERR_BLOCKS_EXHAUSTED = 0x1
+DEVERR_HEAD_TABLE_FULL = 0x2
+DEVERR_FREE_STACK_FULL = 0x4
+DEVERR_TIMEOUT = 0x8
+DEVERR_LAYER_NOT_EMPTY = 0x10
+
+BLOCK_TOKENS = 64
+
+
+class DmsLibraryMissing(RuntimeError):
+    pass
+
+
+class DmsError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        self.status = status
+        super().__init__(f"{where}: status {status}: {msg}")
+
+
+class PoolConfig(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int32), ("max_batch", ctypes.c_int32),
+                ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("block_tokens", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
+                ("max_blocks", ctypes.c_int64), ("max_context", ctypes.c_int64)]
+
+
+class PoolLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_uint64) for n in
+                ("header", "blocks", "block_table", "n_slots", "n_retained", "ring", "free_top",
+                 "free_stack", "block_stack", "scales", "tickets", "scratch", "total")] + [
+        ("block_bytes", ctypes.c_int64), ("row_bytes", ctypes.c_int64),
+        ("max_blocks_per_head", ctypes.c_int32), ("free_stack_cap", ctypes.c_int32),
+        ("n_heads", ctypes.c_int32), ("fp8_layout", ctypes.c_int32)]
+
+
+class PoolStats(ctypes.Structure):
+    _fields_ = [("retained_tokens", ctypes.c_int64), ("slots_in_use", ctypes.c_int64),
+                ("min_retained", ctypes.c_int32), ("max_retained", ctypes.c_int32),
+                ("heads_nonempty", ctypes.c_int32), ("pad0", ctypes.c_int32),
+                ("blocks_in_use", ctypes.c_int64), ("blocks_total", ctypes.c_int64),
+                ("kv_bytes_in_use", ctypes.c_int64), ("kv_bytes_retained", ctypes.c_int64),
+                ("error_flags", ctypes.c_uint32), ("error_layer", ctypes.c_int32),
+                ("error_seq", ctypes.c_int32), ("error_head", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_ if f != "pad0"}
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SIGS = {
+    "dms_status_string": (ctypes.c_char_p, [_I]),
+    "dms_last_error": (ctypes.c_char_p, []),
+    "dms_pool_bytes_required": (_I, [ctypes.POINTER(PoolConfig), ctypes.POINTER(ctypes.c_size_t)]),
+    "dms_pool_create": (_I, [ctypes.POINTER(PoolConfig), _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
+    "dms_pool_destroy": (_I, [_P]),
+    "dms_pool_reset": (_I, [_P, _P]),
+    "dms_pool_layout": (_I, [_P, ctypes.POINTER(PoolLayout)]),
+    "dms_compact_prefill": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P]),
+    "dms_append_evict_layers": (_I, [_P, _I, _I, _I, _I64, _P, _P, _I, _P, _P]),
+    "dms_append_evict": (_I, [_P, _I, _I, _I64, _P, _P, _I, _P, _P]),
+    "dms_decode_workspace_bytes": (_I, [_P, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "dms_decode_attn_layers": (_I, [_P, _I, _I, _I, _P, _I, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
+    "dms_decode_attn": (_I, [_P, _I, _I, _P, _I, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
+    "dms_pool_stats": (_I, [_P, ctypes.POINTER(PoolStats), _P]),
+    "dms_synth_normal": (_I, [ctypes.c_uint64, _I, _I, _I, _I, _I64, _I, _I, _I, _I, _P, _P]),
+    "dms_synth_flags": (_I, [ctypes.c_uint64, _I, _I, _I, _I64, _I, _I, _P, _P, _P]),
+}
+EXPORTED = sorted(_SIGS)
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdms.so (once).  Raises DmsLibraryMissing if it is not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise DmsLibraryMissing(
+                f"{LIB_PATH} not built; run `python -m compact_decode_attention_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = h
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != DMS_OK:
+        msg = lib().dms_last_error().decode(errors="replace")
+        raise DmsError(status, where, msg)
+
+
+def dms_status_string(s: int) -> str:
+    return lib().dms_status_string(s).decode()
+
+
+def dms_pool_bytes_required(cfg: PoolConfig) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().dms_pool_bytes_required(ctypes.byref(cfg), ctypes.byref(n)), "dms_pool_bytes_required")
+    return n.value
+
+
+def dms_pool_create(cfg: PoolConfig, dev_buf: int, nbytes: int, stream: int) -> int:
+    h = _P()
+    _check(lib().dms_pool_create(ctypes.byref(cfg), dev_buf, nbytes, stream, ctypes.byref(h)),
+           "dms_pool_create")
+    return h.value
+
+
+def dms_pool_destroy(pool: int):
+    _check(lib().dms_pool_destroy(pool), "dms_pool_destroy")
+
+
+def dms_pool_reset(pool: int, stream: int):
+    _check(lib().dms_pool_reset(pool, stream), "dms_pool_reset")
+
+
+def dms_pool_layout(pool: int) -> PoolLayout:
+    lay = PoolLayout()
+    _check(lib().dms_pool_layout(pool, ctypes.byref(lay)), "dms_pool_layout")
+    return lay
+
+
+def dms_compact_prefill(pool: int, layer: int, batch: int, prompt_len: int, k: int, v: int,
+                        in_dtype: int, evict: int, stream: int):
+    _check(lib().dms_compact_prefill(pool, layer, batch, prompt_len, k, v, in_dtype, evict, stream),
+           "dms_compact_prefill")
+
+
+def dms_append_evict_layers(pool: int, layer0: int, n_layers: int, batch: int, pos: int, k: int,
+                            v: int, in_dtype: int, evict: int, stream: int):
+    _check(lib().dms_append_evict_layers(pool, layer0, n_layers, batch, pos, k, v, in_dtype, evict,
+                                         stream), "dms_append_evict_layers")
+
+
+def dms_append_evict(pool: int, layer: int, batch: int, pos: int, k: int, v: int, in_dtype: int,
+                     evict: int, stream: int):
+    _check(lib().dms_append_evict(pool, layer, batch, pos, k, v, in_dtype, evict, stream),
+           "dms_append_evict")
+
+
+def dms_decode_workspace_bytes(pool: int, n_layers: int, batch: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().dms_decode_workspace_bytes(pool, n_layers, batch, ctypes.byref(n)),
+           "dms_decode_workspace_bytes")
+    return n.value
+
+
+def dms_decode_attn_layers(pool: int, layer0: int, n_layers: int, batch: int, q: int, q_dtype: int,
+                           out: int, sm_scale: float, workspace: int, workspace_bytes: int,
+                           stream: int):
+    _check(lib().dms_decode_attn_layers(pool, layer0, n_layers, batch, q, q_dtype, out, sm_scale,
+                                        workspace, workspace_bytes, stream), "dms_decode_attn_layers")
+
+
+def dms_decode_attn(pool: int, layer: int, batch: int, q: int, q_dtype: int, out: int,
+                    sm_scale: float, workspace: int, workspace_bytes: int, stream: int):
+    _check(lib().dms_decode_attn(pool, layer, batch, q, q_dtype, out, sm_scale, workspace,
+                                 workspace_bytes, stream), "dms_decode_attn")
+
+
+def dms_pool_stats(pool: int, stream: int, check: bool = True) -> PoolStats:
+    st = PoolStats()
+    rc = lib().dms_pool_stats(pool, ctypes.byref(st), stream)
+    if check:
+        _check(rc, "dms_pool_stats")
+    return st
+
+
+def dms_synth_normal(seed: int, stream_id: int, layer0: int, n_layers: int, batch: int, pos0: int,
+                     n_pos: int, n_heads: int, head_dim: int, dtype: int, out: int, stream: int):
+    _check(lib().dms_synth_normal(seed, stream_id, layer0, n_layers, batch, pos0, n_pos, n_heads,
+                                  head_dim, dtype, out, stream), "dms_synth_normal")
+
+
+def dms_synth_flags(seed: int, layer0: int, n_layers: int, batch: int, pos0: int, n_pos: int,
+                    n_heads: int, thr: int, out: int, stream: int):
+    _check(lib().dms_synth_flags(seed, layer0, n_layers, batch, pos0, n_pos, n_heads, thr, out,
+                                 stream), "dms_synth_flags")
+
+
+# ---------------------------------------------------------------------------
+# torch plumbing: device memory and streams only
+# ---------------------------------------------------------------------------
+
+def torch_dtype_code(dtype) -> int:
+    import torch
+    if dtype == torch.float32:
+        return DMS_F32
+    if dtype == torch.bfloat16:
+        return DMS_BF16
+    raise ValueError(f"unsupported dtype {dtype}")
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return int(t.data_ptr())
+
+
+class Pool:
+    """A pool whose buffer is a torch uint8 CUDA tensor (owned by this object)."""
+
+    def __init__(self, n_layers, max_batch, n_q_heads, n_kv_heads, head_dim, window, kv_dtype,
+                 max_blocks, max_context, device="cuda", stream=None):
+        import torch
+        self.cfg = PoolConfig(n_layers, max_batch, n_q_heads, n_kv_heads, head_dim, window,
+                              BLOCK_TOKENS, kv_dtype, max_blocks, max_context)
+        self.nbytes = dms_pool_bytes_required(self.cfg)
+        self.buffer = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        self.handle = dms_pool_create(self.cfg, _ptr(self.buffer), self.nbytes, _stream(stream))
+        self.layout = dms_pool_layout(self.handle)
+        self._ws = {}
+
+    def close(self):
+        if self.handle:
+            dms_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def reset(self, stream=None):
+        dms_pool_reset(self.handle, _stream(stream))
+
+    def compact_prefill(self, layer, k, v, evict, stream=None):
+        B, P = k.shape[0], k.shape[1]
+        dms_compact_prefill(self.handle, layer, B, P, _ptr(k), _ptr(v), torch_dtype_code(k.dtype),
+                            _ptr(evict), _stream(stream))
+
+    def append_evict_layers(self, layer0, pos, k, v, evict, stream=None):
+        nl, B = k.shape[0], k.shape[1]
+        dms_append_evict_layers(self.handle, layer0, nl, B, pos, _ptr(k), _ptr(v),
+                                torch_dtype_code(k.dtype), _ptr(evict), _stream(stream))
+
+    def workspace(self, n_layers, batch, device="cuda"):
+        import torch
+        key = (n_layers, batch)
+        if key not in self._ws:
+            n = dms_decode_workspace_bytes(self.handle, n_layers, batch)
+            self._ws[key] = torch.empty(n, dtype=torch.uint8, device=device)
+        return self._ws[key]
+
+    def decode_attn_layers(self, layer0, q, out, sm_scale=0.0, stream=None):
+        nl, B = q.shape[0], q.shape[1]
+        ws = self.workspace(nl, B, q.device)
+        dms_decode_attn_layers(self.handle, layer0, nl, B, _ptr(q), torch_dtype_code(q.dtype),
+                               _ptr(out), sm_scale, _ptr(ws), ws.numel(), _stream(stream))
+
+    def stats(self, stream=None, check=True) -> PoolStats:
+        return dms_pool_stats(self.handle, _stream(stream), check)
+
+    # raw views of the bookkeeping regions (for tests and tools)
+    def region(self, name, dtype, count):
+        import torch
+        off = getattr(self.layout, name)
+        esz = torch.empty(0, dtype=dtype).element_size()
+        return self.buffer[off: off + count * esz].view(dtype)

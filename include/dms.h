@@ -1,0 +1,235 @@
+/*
+ * dms.h -- C ABI of libdms: compact-KV decode for Dynamic Memory
+ * Sparsification (DMS) on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes
+ * -------------------------
+ * DMS learns, per attention head, which tokens to evict, and evicts them
+ * with a delay: a token flagged for eviction stays visible for a window of w
+ * tokens and is removed afterwards ("NVIDIA veröffentlicht Qwen3-8B-DMS-8x
+ * mit innovativer Speicherkompression für verbesserte Inferenzzeiten"
+ * (mindverse), section "Dynamic Memory Sparsification (DMS): Eine innovative
+ * Lösung", w = 512; "Nvidia DMS: сжатие памяти LLM в 8 раз" (stiva.ai),
+ * section "Ключевое изобретение: delayed eviction").  For the query at
+ * position t, key j of kv-head h is visible unless evict[j,h] and t-j >= w.
+ * FastDMS stores only the visible tokens in a compact KV store that reclaims
+ * the slots of evicted tokens ("FastDMS: vLLM BF16/FP8보다 빠른 6.4x KV
+ * cache 압축" (molayo1419.me), opening paragraphs), with per-layer,
+ * per-head variable token counts instead of fixed pages (same page, table
+ * "What's the catch?", row "PagedAttention / KV memory pool").
+ *
+ * The pool
+ * --------
+ * One caller-provided device buffer holds every (layer, sequence, kv-head)
+ * "head" of the store:
+ *   - physical blocks of BT = block_tokens token rows; block = [K tile
+ *     BT x D][V tile BT x D] in the pool's kv dtype.  A row of bf16/fp32 is
+ *     stored with its 16-byte chunks permuted: chunk c of row r sits at
+ *     chunk c ^ (r & 7) (the shared-memory image the attention kernel
+ *     reads, conflict free).  The FP8 layout is given in dms_pool_layout_t.
+ *   - per head: a block table (logical slot s lives in block
+ *     table[s / BT], row s % BT), n_slots (slots ever handed out),
+ *     n_retained (tokens held), a window ring of w entries
+ *     (slot | flag << 31 for the last w positions; entry t mod w holds
+ *     token t) and a LIFO free-slot stack;
+ *   - a global free-block stack and bump counter, FP8 scales, an error word.
+ * Slots of one head are dense: a retired slot is reused by the same step's
+ * new token, so the held tokens are exactly slots [0, n_slots).
+ *
+ * Conventions
+ * -----------
+ * - Ownership: the caller allocates every device buffer (pool, inputs,
+ *   outputs, workspace) and owns every stream.  libdms never allocates
+ *   device memory; a dms_pool is a small host handle.
+ * - Asynchrony: every call enqueues its kernels on the given stream and
+ *   returns; argument errors are reported at once, device-side errors
+ *   (pool exhausted, table overflow, a wait that timed out) set bits of the
+ *   pool's error word, read back by dms_pool_stats.  No kernel traps or
+ *   waits without a time limit.
+ * - Calls that touch the same layer must be ordered (same stream or
+ *   events).  Pointers are device pointers unless marked host.
+ * - Layouts are row-major, C order.  B = batch (sequences 0..B-1 of the
+ *   pool, B <= max_batch), P = prompt length, Hq / Hkv query / kv heads,
+ *   g = Hq / Hkv (query head hq reads kv head hq / g), D = head_dim.
+ */
+#ifndef DMS_H
+#define DMS_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DMS_OK = 0,
+  DMS_ERR_INVALID_ARG = 1,   /* bad pointer, size, dtype, layer range ... */
+  DMS_ERR_CAPACITY = 2,      /* buffer too small for the requested pool    */
+  DMS_ERR_CUDA = 3,          /* a CUDA runtime call failed                 */
+  DMS_ERR_UNSUPPORTED = 4,   /* valid but not built (e.g. head_dim 96)     */
+  DMS_ERR_DEVICE = 5         /* the pool's device error word is non-zero   */
+} dms_status;
+
+typedef enum { DMS_F32 = 0, DMS_BF16 = 1, DMS_FP8_E4M3 = 2 } dms_dtype;
+
+/* Bits of the device error word (dms_pool_stats_t.error_flags). */
+#define DMS_DEVERR_BLOCKS_EXHAUSTED 0x1u  /* global block pool ran out; write skipped   */
+#define DMS_DEVERR_HEAD_TABLE_FULL  0x2u  /* a head outgrew max_context; write skipped   */
+#define DMS_DEVERR_FREE_STACK_FULL  0x4u  /* per-head free stack overflow                */
+#define DMS_DEVERR_TIMEOUT          0x8u  /* a bounded wait gave up; outputs invalid     */
+#define DMS_DEVERR_LAYER_NOT_EMPTY  0x10u /* prefill into a layer that already holds data */
+
+typedef struct {
+  int32_t n_layers;
+  int32_t max_batch;
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;       /* 64 or 128 */
+  int32_t window;         /* delay window w >= 1 (512 in the pages)        */
+  int32_t block_tokens;   /* BT; 64 is the only value built                */
+  int32_t kv_dtype;       /* dms_dtype of the stored K/V                    */
+  int64_t max_blocks;     /* physical blocks shared by all heads            */
+  int64_t max_context;    /* most tokens one head may hold (table width)    */
+} dms_pool_config;
+
+typedef struct dms_pool dms_pool;  /* opaque host handle */
+
+/* Byte offsets of each region inside the pool buffer, for inspection by
+ * tests and tools (the pool is plain device memory). */
+typedef struct {
+  uint64_t header, blocks, block_table, n_slots, n_retained, ring, free_top,
+           free_stack, block_stack, scales, tickets, scratch, total;
+  int64_t block_bytes;          /* bytes of one block (K tile + V tile)      */
+  int64_t row_bytes;            /* bytes of one stored row (D * elem size)   */
+  int32_t max_blocks_per_head;  /* block table width                         */
+  int32_t free_stack_cap;       /* per-head free stack capacity              */
+  int32_t n_heads;              /* n_layers * max_batch * n_kv_heads         */
+  int32_t fp8_layout;           /* 1: FP8 rows use the permuted layout below */
+} dms_pool_layout_t;
+
+typedef struct {
+  int64_t retained_tokens;      /* sum of n_retained over all heads           */
+  int64_t slots_in_use;         /* sum of n_slots                             */
+  int32_t min_retained;         /* over heads with n_retained > 0             */
+  int32_t max_retained;
+  int32_t heads_nonempty;
+  int32_t pad0;
+  int64_t blocks_in_use;        /* handed out and not returned                */
+  int64_t blocks_total;
+  int64_t kv_bytes_in_use;      /* blocks_in_use * block_bytes                */
+  int64_t kv_bytes_retained;    /* retained_tokens * 2 * row_bytes            */
+  uint32_t error_flags;         /* DMS_DEVERR_* bits                          */
+  int32_t error_layer;          /* first failing head (or -1)                 */
+  int32_t error_seq;
+  int32_t error_head;
+} dms_pool_stats_t;
+
+/* Human-readable name of a status code (static string). */
+const char* dms_status_string(dms_status s);
+
+/* Last host-side error message of the calling thread ("" if none). */
+const char* dms_last_error(void);
+
+/* Bytes of device memory a pool with this configuration needs.  Pure host
+ * computation.  Returns DMS_ERR_INVALID_ARG for an invalid config. */
+dms_status dms_pool_bytes_required(const dms_pool_config* cfg, size_t* bytes);
+
+/* Carve a pool out of dev_buf (caller-owned, >= bytes_required, 256-byte
+ * aligned) and clear its bookkeeping on `stream`.  *out receives a host
+ * handle that must be released with dms_pool_destroy.  The device must be
+ * current.  Source: compact store with slot reclaim and per-head ragged
+ * counts (FastDMS page, opening paragraphs and table "What's the catch?"). */
+dms_status dms_pool_create(const dms_pool_config* cfg, void* dev_buf, size_t bytes,
+                           cudaStream_t stream, dms_pool** out);
+
+/* Free the host handle only (the buffer stays the caller's). */
+dms_status dms_pool_destroy(dms_pool* pool);
+
+/* Clear every head, the block stack and the error word (async on stream). */
+dms_status dms_pool_reset(dms_pool* pool, cudaStream_t stream);
+
+/* Region offsets of the pool buffer. */
+dms_status dms_pool_layout(const dms_pool* pool, dms_pool_layout_t* out);
+
+/* Prefill compaction of one layer (DMS delayed eviction applied at the end
+ * of the prompt, t = P - 1): for every sequence b < batch and kv-head h,
+ * keeps position j iff evict[b,j,h] == 0 or P-1-j < w, writes the kept K/V
+ * rows to slots 0.. in position order, sets n_slots = n_retained = kept
+ * count and fills the window ring with positions max(0,P-w)..P-1.
+ * For an FP8 pool the per-(layer, kv-head) scales become amax/448 over all
+ * P*batch rows of that head (before eviction), K and V separately, and rows
+ * are stored as e4m3(x / scale) (round to nearest even, saturating).
+ *   k, v   [batch, P, Hkv, D]  in_dtype (DMS_F32 or DMS_BF16)
+ *   evict  [batch, P, Hkv]     uint8, non-zero = flagged
+ * The layer must be empty (fresh pool or after dms_pool_reset), else the
+ * device sets DMS_DEVERR_LAYER_NOT_EMPTY and writes nothing.  in_dtype
+ * must equal kv_dtype, or be F32/BF16 for an FP8 pool.
+ * Source: compaction = the compact store of the FastDMS page; eviction
+ * before FP8 quantisation = the same page's FP8 paragraph. */
+dms_status dms_compact_prefill(dms_pool* pool, int layer, int batch, int prompt_len,
+                               const void* k, const void* v, dms_dtype in_dtype,
+                               const uint8_t* evict, cudaStream_t stream);
+
+/* One decode step at position `pos` (= t) for layers [layer0, layer0 +
+ * n_layers): for every (layer, b, h): if t >= w and token t-w was flagged,
+ * its slot goes onto the head's free stack (delayed eviction retires it);
+ * token t takes the top free slot, else slot n_slots (a new block when the
+ * slot starts one); its K/V row is written (FP8: with the prefill scale,
+ * saturating); ring[t mod w] = slot | flag << 31.
+ *   k, v   [n_layers, batch, Hkv, D]  in_dtype
+ *   evict  [n_layers, batch, Hkv]     uint8
+ * Positions must increase by one per step from the prompt length.
+ * Source: delayed eviction (mindverse page, section "Dynamic Memory
+ * Sparsification (DMS): Eine innovative Lösung"), slot reclaim (FastDMS
+ * page, opening paragraphs). */
+dms_status dms_append_evict_layers(dms_pool* pool, int layer0, int n_layers, int batch,
+                                   int64_t pos, const void* k, const void* v,
+                                   dms_dtype in_dtype, const uint8_t* evict,
+                                   cudaStream_t stream);
+
+/* Single-layer form of dms_append_evict_layers (k, v [batch, Hkv, D]). */
+dms_status dms_append_evict(dms_pool* pool, int layer, int batch, int64_t pos,
+                            const void* k, const void* v, dms_dtype in_dtype,
+                            const uint8_t* evict, cudaStream_t stream);
+
+/* Workspace bytes dms_decode_attn_layers needs for n_layers x batch. */
+dms_status dms_decode_workspace_bytes(const dms_pool* pool, int n_layers, int batch,
+                                      size_t* bytes);
+
+/* Decode attention over the compact store for layers [layer0, layer0 +
+ * n_layers): out[l,b,hq] = softmax(sm_scale * q[l,b,hq] . K_h^T) V_h over
+ * the n_slots held rows of kv-head h = hq / g (the query's own token
+ * included, appended before this call).  Split-K flash decoding: the held
+ * rows of all heads form one list of BT-row blocks that is cut evenly over
+ * a persistent grid; partial softmax states are merged by log-sum-exp.
+ *   q, out     [n_layers, batch, Hq, D]  q_dtype (DMS_BF16 or DMS_F32;
+ *              F32 only for an F32 pool); out has q's dtype
+ *   sm_scale   <= 0 selects 1/sqrt(D)
+ *   workspace  >= dms_decode_workspace_bytes, 256-byte aligned; no
+ *              initialisation needed; must not be shared by concurrent calls
+ * Source: attention over each head's retained tokens only (mindverse page,
+ * DMS section; FastDMS page, speed claim at 8K context). */
+dms_status dms_decode_attn_layers(dms_pool* pool, int layer0, int n_layers, int batch,
+                                  const void* q, dms_dtype q_dtype, void* out, float sm_scale,
+                                  void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream);
+
+/* Single-layer form of dms_decode_attn_layers (q, out [batch, Hq, D]). */
+dms_status dms_decode_attn(dms_pool* pool, int layer, int batch, const void* q,
+                           dms_dtype q_dtype, void* out, float sm_scale, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream);
+
+/* Reduce the pool's counters on the device and copy them to *out (host).
+ * Synchronises `stream`.  Returns DMS_ERR_DEVICE when the error word is
+ * non-zero (*out is filled either way).  Source: real allocator memory,
+ * not theoretical KV bytes (FastDMS page, paragraph before the memory
+ * table). */
+dms_status dms_pool_stats(dms_pool* pool, dms_pool_stats_t* out, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DMS_H */
