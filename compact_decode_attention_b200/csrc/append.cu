@@ -29,13 +29,34 @@ __device__ __forceinline__ float in_to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
 
-constexpr int kAppendThreads = 1024;
+constexpr int kAppendThreads = 512;
+constexpr int kAppendRegChunks = 20;   // 16-byte input chunks a thread can hold
 
 template <typename InT, bool FP8>
 __global__ void __launch_bounds__(kAppendThreads)
     append_evict_kernel(PoolView v, int l0, int nl, int batch, int64_t pos, const InT* k,
                         const InT* vv, const uint8_t* evict) {
   extern __shared__ int s_dyn[];
+  // Rows of the new tokens: chunk c of head hh is K chunk c (c < nch) or V
+  // chunk c - nch.  When they fit in registers they are loaded first, so the
+  // loads overlap the bookkeeping below instead of following it.
+  const int nch = int(v.row_bytes >> 4);
+  const int H_ = nl * batch * v.Hkv;
+  const int total_chunks = H_ * 2 * nch;
+  const bool preload = !FP8 && total_chunks <= int(blockDim.x) * kAppendRegChunks;
+  uint4 reg[kAppendRegChunks];
+  if (preload) {
+#pragma unroll
+    for (int r = 0; r < kAppendRegChunks; ++r) {
+      const int c = threadIdx.x + r * blockDim.x;
+      if (c < total_chunks) {
+        const int hh = c / (2 * nch), cc = c % (2 * nch);
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(cc < nch ? k : vv) +
+                             int64_t(hh) * v.row_bytes + (cc % nch) * 16;
+        reg[r] = *reinterpret_cast<const uint4*>(src);
+      }
+    }
+  }
   const int H = nl * batch * v.Hkv;
   int* s_slot = s_dyn;          // [H] slot of the new token (-1: failed)
   int* s_blk = s_dyn + H;       // [H] physical block of that slot
@@ -157,8 +178,21 @@ __global__ void __launch_bounds__(kAppendThreads)
   }
 
   // ---- 4. write the rows ---------------------------------------------------
-  if constexpr (!FP8) {
-    const int nch = int(v.row_bytes >> 4);
+  if (preload) {
+#pragma unroll
+    for (int r = 0; r < kAppendRegChunks; ++r) {
+      const int c = threadIdx.x + r * blockDim.x;
+      if (c < total_chunks) {
+        const int hh = c / (2 * nch), cc = c % (2 * nch);
+        const int slot = s_slot[hh];
+        if (slot < 0) continue;
+        const int row = slot % v.BT;
+        uint8_t* dst = v.blocks + int64_t(s_blk[hh]) * v.block_bytes + (cc < nch ? 0 : v.tile_bytes) +
+                       int64_t(row) * v.row_bytes + swz_chunk(cc % nch, row) * 16;
+        *reinterpret_cast<uint4*>(dst) = reg[r];
+      }
+    }
+  } else if constexpr (!FP8) {
     for (int i = tid; i < H * nch; i += blockDim.x) {
       const int hh = i / nch, c = i % nch;
       const int slot = s_slot[hh];
@@ -249,8 +283,7 @@ extern "C" dms_status dms_append_evict_layers(dms_pool* pool, int layer0, int n_
     set_last_error("too many heads (%d) for one append call; split the layer range", H);
     return DMS_ERR_UNSUPPORTED;
   }
-  int threads = ((H + 31) / 32) * 32;
-  threads = threads < 128 ? 128 : threads > kAppendThreads ? kAppendThreads : threads;
+  const int threads = kAppendThreads;
   dms_status st = DMS_OK;
 #define DMS_LAUNCH_APPEND(T, F)                                                                    \
   do {                                                                                             \

@@ -11,8 +11,8 @@
 // Work split (stream-K over blocks): the held rows of all heads of the call,
 // in (layer, sequence, kv-head) order, form U blocks of up to 64 rows.  A
 // persistent grid of G CTAs (one per SM) takes the contiguous ranges
-// [c*U/G, (c+1)*U/G), so every CTA moves the same bytes whatever the head
-// lengths.  A CTA's piece of a head ends in a partial softmax state
+// [c*U/G', (c+1)*U/G') with G' = min(G, U), so every CTA moves the same
+// bytes whatever the head lengths.  A CTA's piece of a head ends in a partial softmax state
 // (m, l, o); a head cut by CTA boundaries is merged by log-sum-exp in the
 // CTA that finishes it last (an atomic ticket -- nobody waits).  Partial id
 // c + i is unique per (CTA c, head i) piece.
@@ -479,7 +479,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const Attn
     U += s_scan[k];
   }
   const int excl = wbase + incl - su;
-  const int u_beg = int((int64_t(c) * U) / G), u_end = int((int64_t(c + 1) * U) / G);
+  // with fewer blocks than CTAs only the first U CTAs take one block each,
+  // so that every CTA in [0, Geff) has a non-empty range
+  const int Geff = min(G, U);
+  if (c >= Geff) return;
+  const int u_beg = int((int64_t(c) * U) / Geff), u_end = int((int64_t(c + 1) * U) / Geff);
   if (u_beg < u_end && u_beg >= excl && u_beg < excl + su) {
     int pre = excl;
     for (int i = hb; i < he; ++i) {
@@ -493,7 +497,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const Attn
     }
   }
   __syncthreads();
-  if (u_beg >= u_end) return;
   const int i0 = s_misc[1], p0 = s_misc[2];
   const int qrow_bytes = g * D * T::QESZ;
 
@@ -630,7 +633,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const Attn
       st.write_state(my_ow, my_mw, my_lw, g, lane);
       consumer_bar();
       const int hd = pool_head(p, i);
-      const int cf = cta_of(pp, U, G), cl = cta_of(int64_t(pp) + nu - 1, U, G);
+      const int cf = cta_of(pp, U, Geff), cl = cta_of(int64_t(pp) + nu - 1, U, Geff);
       const bool whole = cf == cl;
       const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
       const int pid = c + i;

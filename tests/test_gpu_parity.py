@@ -242,10 +242,13 @@ def test_blocks_exhausted_is_reported_and_nothing_written():
     assert np.all(read_state(pool)["n_slots"] == 0)
 
 
-def test_head_table_full_is_reported():
+def test_position_past_max_context_is_rejected():
+    """A head cannot outgrow its block table: positions at or past max_context
+    are refused on the host (the device check behind it is never reached)."""
     K, V, flags, Q = make_inputs(2, 1, 64, 2, 4, 1, 64, "bf16", p_keep=1.0)
-    pool, _ = run_small(K, V, flags, Q, 64, 128, "bf16", max_context=64)
-    assert pool.stats(check=False).error_flags & dms.DEVERR_HEAD_TABLE_FULL
+    with pytest.raises(dms.DmsError) as e:
+        run_small(K, V, flags, Q, 64, 128, "bf16", max_context=64)
+    assert e.value.status == dms.DMS_ERR_INVALID_ARG
 
 
 def test_prefill_into_filled_layer_is_refused():
