@@ -791,3 +791,121 @@ extern "C" dms_status dms_decode_attn(dms_pool* pool, int layer, int batch, cons
   return dms_decode_attn_layers(pool, layer, 1, batch, q, q_dtype, out, sm_scale, workspace,
                                 workspace_bytes, stream);
 }
+
+// ---------------------------------------------------------------------------
+// Decode attention for callers that cannot allocate device memory.
+//
+// Some callers have no way to obtain a workspace: a serving engine that has
+// already handed every free byte of HBM to its KV pool, a plugin whose host
+// framework exposes no device allocator, or a latency-critical path where
+// cudaMalloc's device-wide synchronisation would stall other streams.  This
+// entry point gives them the split-K scratch from a fixed array compiled into
+// the library instead of a caller buffer.
+//
+// The array is kStaticWorkspaceBytes (16 MiB) of global memory on every GPU
+// that loads the library, held until the process exits.  Host code cannot
+// hand the array's name to a kernel (in host code it names a host-side
+// stand-in, not device memory), so the first call on each device looks up
+// its device address with cudaGetSymbolAddress while that device is current
+// and caches it; make that first call before any stream capture.  Every call
+// on a device shares the one array, which keeps the previous call's partial
+// results: nothing in it has to start at zero (each launch writes every
+// partial it later reads, and the merge tickets live in the pool), but calls
+// whose kernels overlap on the GPU race on it and must be ordered.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace dms {
+
+constexpr size_t kStaticWorkspaceBytes = size_t(16) << 20;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+static std::mutex g_static_ws_mutex;
+static void* g_static_ws_addr[kMaxDevices] = {};
+
+// Device address of g_static_workspace on the current device (looked up once).
+static dms_status static_workspace_address(int device, void** addr) {
+  if (device < 0 || device >= kMaxDevices) {
+    set_last_error("device %d out of range for the fixed workspace table", device);
+    return DMS_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (!g_static_ws_addr[device]) {
+    void* p = nullptr;
+    dms_status st = cuda_status(cudaGetSymbolAddress(&p, g_static_workspace),
+                                "cudaGetSymbolAddress(g_static_workspace)");
+    if (st != DMS_OK) return st;
+    g_static_ws_addr[device] = p;
+  }
+  *addr = g_static_ws_addr[device];
+  return DMS_OK;
+}
+
+}  // namespace dms
+
+extern "C" dms_status dms_decode_attn_layers_noalloc(dms_pool* pool, int layer0, int n_layers,
+                                                     int batch, const void* q, dms_dtype q_dtype,
+                                                     void* out, float sm_scale,
+                                                     cudaStream_t stream) {
+  if (!pool) {
+    set_last_error("null pool");
+    return DMS_ERR_INVALID_ARG;
+  }
+  const PoolView& v = pool->view;
+  if (layer0 < 0 || n_layers < 1 || layer0 + n_layers > v.L || batch < 1 || batch > v.Bmax) {
+    set_last_error("bad layer range / batch (%d+%d, %d)", layer0, n_layers, batch);
+    return DMS_ERR_INVALID_ARG;
+  }
+  if (!q || !out) {
+    set_last_error("null q / out");
+    return DMS_ERR_INVALID_ARG;
+  }
+  const dms_dtype want = v.kv_dtype == DMS_F32 ? DMS_F32 : DMS_BF16;
+  if (q_dtype != want) {
+    set_last_error("q_dtype must be %s for this pool", want == DMS_F32 ? "DMS_F32" : "DMS_BF16");
+    return DMS_ERR_INVALID_ARG;
+  }
+  if (reinterpret_cast<uintptr_t>(q) & 15) {
+    set_last_error("q must be 16-byte aligned");
+    return DMS_ERR_INVALID_ARG;
+  }
+  const size_t need = attn_workspace_bytes(pool, n_layers, batch);
+  if (need > kStaticWorkspaceBytes) {
+    set_last_error("this call needs %zu bytes of scratch; the fixed workspace holds %zu "
+                   "(use dms_decode_attn_layers with a caller workspace, or fewer layers)",
+                   need, kStaticWorkspaceBytes);
+    return DMS_ERR_CAPACITY;
+  }
+  int dev = -1;
+  dms_status st = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != DMS_OK) return st;
+  if (dev != pool->device) {
+    set_last_error("current device %d is not the pool's device %d", dev, pool->device);
+    return DMS_ERR_INVALID_ARG;
+  }
+  void* ws = nullptr;
+  st = static_workspace_address(dev, &ws);
+  if (st != DMS_OK) return st;
+  const int g = v.Hq / v.Hkv;
+  const size_t parts = size_t(pool->sm_count) + size_t(n_layers) * batch * v.Hkv;
+  AttnParams prm;
+  prm.v = v;
+  prm.l0 = layer0;
+  prm.nl = n_layers;
+  prm.batch = batch;
+  prm.q = static_cast<const uint8_t*>(q);
+  prm.out = static_cast<uint8_t*>(out);
+  const float sc = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf(float(v.D));
+  prm.scale_log2 = sc * 1.4426950408889634f;
+  prm.ws_o = static_cast<float*>(ws);
+  prm.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                       ((parts * g * v.D * 4 + 255) & ~size_t(255)));
+  prm.G = pool->sm_count;
+  if (v.kv_dtype == DMS_BF16) {
+    return v.D == 128 ? launch_attn<KV_BF16, 128>(prm, stream) : launch_attn<KV_BF16, 64>(prm, stream);
+  }
+  if (v.kv_dtype == DMS_FP8_E4M3) return launch_attn<KV_FP8, 128>(prm, stream);
+  return v.D == 128 ? launch_attn<KV_F32, 128>(prm, stream) : launch_attn<KV_F32, 64>(prm, stream);
+}

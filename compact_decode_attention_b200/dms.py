@@ -86,6 +86,7 @@ _SIGS = {
     "dms_decode_workspace_bytes": (_I, [_P, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
     "dms_decode_attn_layers": (_I, [_P, _I, _I, _I, _P, _I, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
     "dms_decode_attn": (_I, [_P, _I, _I, _P, _I, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
+    "dms_decode_attn_layers_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, ctypes.c_float, _P]),
     "dms_pool_stats": (_I, [_P, ctypes.POINTER(PoolStats), _P]),
     "dms_synth_normal": (_I, [ctypes.c_uint64, _I, _I, _I, _I, _I64, _I, _I, _I, _I, _P, _P]),
     "dms_synth_flags": (_I, [ctypes.c_uint64, _I, _I, _I, _I64, _I, _I, _P, _P, _P]),
@@ -184,6 +185,12 @@ def dms_decode_attn(pool: int, layer: int, batch: int, q: int, q_dtype: int, out
                     sm_scale: float, workspace: int, workspace_bytes: int, stream: int):
     _check(lib().dms_decode_attn(pool, layer, batch, q, q_dtype, out, sm_scale, workspace,
                                  workspace_bytes, stream), "dms_decode_attn")
+
+
+def dms_decode_attn_layers_noalloc(pool: int, layer0: int, n_layers: int, batch: int, q: int,
+                                   q_dtype: int, out: int, sm_scale: float, stream: int):
+    _check(lib().dms_decode_attn_layers_noalloc(pool, layer0, n_layers, batch, q, q_dtype, out,
+                                                sm_scale, stream), "dms_decode_attn_layers_noalloc")
 
 
 def dms_pool_stats(pool: int, stream: int, check: bool = True) -> PoolStats:

@@ -221,6 +221,21 @@ dms_status dms_decode_attn(dms_pool* pool, int layer, int batch, const void* q,
                            dms_dtype q_dtype, void* out, float sm_scale, void* workspace,
                            size_t workspace_bytes, cudaStream_t stream);
 
+/* dms_decode_attn_layers for callers that cannot allocate device memory
+ * (an engine that gave all free HBM to its KV pool, a plugin without access
+ * to an allocator, a path that must not pay cudaMalloc's synchronisation).
+ * The pages have no counterpart: this is a library convenience.  The
+ * split-K scratch comes from a fixed 16 MiB array in the library's device
+ * globals (present on every GPU that loads the library until exit) instead
+ * of a caller workspace; calls needing more return DMS_ERR_CAPACITY.  The
+ * first call on a device looks up the array's device address (make it
+ * before any stream capture).  All calls on a device share the array:
+ * nothing in it must start at zero, but calls whose kernels overlap on the
+ * GPU race and must be ordered.  The current device must be the pool's. */
+dms_status dms_decode_attn_layers_noalloc(dms_pool* pool, int layer0, int n_layers, int batch,
+                                          const void* q, dms_dtype q_dtype, void* out,
+                                          float sm_scale, cudaStream_t stream);
+
 /* Reduce the pool's counters on the device and copy them to *out (host).
  * Synchronises `stream`.  Returns DMS_ERR_DEVICE when the error word is
  * non-zero (*out is filled either way).  Source: real allocator memory,
