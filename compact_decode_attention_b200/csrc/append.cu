@@ -101,7 +101,11 @@ __global__ void __launch_bounds__(kAppendThreads)
     s_slot[i] = slot;
     s_need[i] = need;
     // counters are committed in step 3 once the block (if any) is secured
+    if (slot >= 0 && !DMS_CHECK(hd >= 0 && hd < v.n_heads && slot < v.mbh * v.BT, v.hdr, 101, hd, slot))
+      slot = -1;
     s_blk[i] = slot < 0 ? -1 : (need ? -2 : v.bt[int64_t(hd) * v.mbh + slot / v.BT]);
+    if (slot >= 0 && !need && !DMS_CHECK(s_blk[i] >= 0 && s_blk[i] < v.max_blocks, v.hdr, 102, hd, s_blk[i]))
+      slot = -1, s_slot[i] = -1;
     if (slot >= 0) {
       v.free_top[hd] = ft;
       // n_slots / n_retained written below
@@ -162,6 +166,10 @@ __global__ void __launch_bounds__(kAppendThreads)
       }
       const int a = s_need[i] - 1;
       const int id = a < stack_top ? v.block_stack[stack_top - 1 - a] : next + (a - stack_top);
+      if (!DMS_CHECK(id >= 0 && id < v.max_blocks, v.hdr, 103, hd, id)) {
+        s_slot[i] = -1;
+        continue;
+      }
       v.bt[int64_t(hd) * v.mbh + slot / v.BT] = id;
       s_blk[i] = id;
     }

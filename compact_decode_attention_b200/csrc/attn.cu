@@ -38,11 +38,14 @@
 
 namespace dms {
 
-constexpr int kNCW = 4;                       // consumer warps
-constexpr int kAttnThreads = 32 * (kNCW + 1);
-
 enum { KV_F32 = 0, KV_BF16 = 1, KV_FP8 = 2 };
 
+// Stage ownership: unit k goes to stage k % NS and to consumer warp k % NCW.
+// NS must be a multiple of NCW so that every stage always belongs to the same
+// warp.  A parity wait only tells "this phase" from "the previous one"; if a
+// stage were shared by two warps, one of them could start waiting two phases
+// ahead of the barrier, see the older phase of the same parity as complete,
+// and read (and release) a stage whose copy is still landing.
 template <int KV, int D>
 struct AttnTraits {
   static constexpr int ESZ = KV == KV_F32 ? 4 : KV == KV_BF16 ? 2 : 1;
@@ -51,11 +54,17 @@ struct AttnTraits {
   static constexpr int TILEB = kBlockTokens * ROWB;
   static constexpr int QB = 8 * D * QESZ;              // room for 8 query rows
   static constexpr int STAGEB = 2 * TILEB + QB;
+  // 34 KB stages for bf16 D=128: 6 stages over 3 consumer warps (2 each);
+  // fp32 D=128 (68 KB stages): 3 stages, 3 warps; the others 8 (or 4) over 4.
+  static constexpr bool BIG = (KV == KV_BF16 && D == 128) || (KV == KV_F32 && D == 128);
+  static constexpr int NCW = BIG ? 3 : 4;              // consumer warps
   static constexpr int NS = KV == KV_F32 ? (D == 128 ? 3 : 4) : (KV == KV_BF16 && D == 128) ? 6 : 8;
-  static constexpr int COMBINE_FLOATS = kNCW * 8 * D + 2 * kNCW * 8;
-  static constexpr int MISC_INTS = 16 + kAttnThreads / 32;
+  static constexpr int THREADS = 32 * (NCW + 1);       // + one producer warp
+  static constexpr int COMBINE_FLOATS = NCW * 8 * D + 2 * NCW * 8;
+  static constexpr int MISC_INTS = 16 + THREADS / 32;
   static constexpr size_t SMEM = size_t(NS) * STAGEB + COMBINE_FLOATS * 4 + 2 * NS * 8 +
                                  MISC_INTS * 4;
+  static_assert(NS % NCW == 0, "each stage must always belong to the same consumer warp");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(STAGEB % 128 == 0, "stage alignment");
 };
@@ -71,7 +80,11 @@ struct AttnParams {
   int G;
 };
 
-__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier 1 among the consumer warps only (the producer never joins it).
+template <int NCW>
+__device__ __forceinline__ void consumer_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * NCW) : "memory");
+}
 
 __device__ __forceinline__ int units_of(int n) { return (n + kBlockTokens - 1) / kBlockTokens; }
 
@@ -418,9 +431,13 @@ struct WarpSel<KV_F32, D> {
 
 // ---------------------------------------------------------------------------
 template <int KV, int D>
-__global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
+    decode_attn_kernel(const AttnParams p) {
   using T = AttnTraits<KV, D>;
   using W = typename WarpSel<KV, D>::type;
+  constexpr int kNCW = T::NCW;
+  constexpr int kAttnThreads = T::THREADS;
+  constexpr int kCons = 32 * kNCW;   // consumer threads
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* stages = smem;
   float* s_ow = reinterpret_cast<float*>(smem + size_t(T::NS) * T::STAGEB);
@@ -519,7 +536,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const Attn
           mnu = units_of(mn);
         }
         const int bi = u - mp;
-        blk = v.bt[int64_t(pool_head(p, mi)) * v.mbh + bi];
+        if (DMS_CHECK(mi < Htot && bi < v.mbh, v.hdr, 301, mi, bi))
+          blk = v.bt[int64_t(pool_head(p, mi)) * v.mbh + bi];
         rows = min(kBlockTokens, mn - bi * kBlockTokens);
       }
       const int cnt = min(32, u_end - ub);
@@ -530,10 +548,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const Attn
         if (lane == 0 && !aborted) {
           const int s = k % T::NS;
           const uint32_t ph = (k / T::NS) & 1;
-          if (!mbar_wait_bounded(&empty[s], ph ^ 1, s_abort)) {
+          if (!DMS_CHECK(jblk >= 0 && jblk < v.max_blocks && jrows >= 1 && jrows <= kBlockTokens &&
+                             ji >= 0 && ji < Htot, v.hdr, 302, jblk, jrows)) {
             aborted = true;
             *s_abort = 1;
-            report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
+          } else if (!mbar_wait_bounded(&empty[s], ph ^ 1, s_abort) || *s_abort) {
+            aborted = true;
+            if (!*s_abort) report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
+            *s_abort = 1;
           } else {
             uint8_t* st = stages + size_t(s) * T::STAGEB;
             const uint8_t* src = v.blocks + int64_t(jblk) * v.block_bytes;
@@ -612,7 +634,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const Attn
           report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0) && __all_sync(0xffffffffu, ok);
+      ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         const uint8_t* stage = stages + size_t(s) * T::STAGEB;
         if constexpr (KV == KV_F32) {
@@ -625,19 +647,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const Attn
           st.unit(stage, rows, lane);
         }
       }
+      // release the stage only after its copy was seen complete; after an
+      // abort the producer issues nothing more and drains what it issued
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      if (ok && lane == 0) mbar_arrive(&empty[s]);
     }
     // ---- end of this CTA's piece of head i: combine the 4 warps ----
     if (u + 1 == u_end || u + 1 >= pp + nu) {
       st.write_state(my_ow, my_mw, my_lw, g, lane);
-      consumer_bar();
+      consumer_bar<kNCW>();
       const int hd = pool_head(p, i);
       const int cf = cta_of(pp, U, Geff), cl = cta_of(int64_t(pp) + nu - 1, U, Geff);
       const bool whole = cf == cl;
       const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
       const int pid = c + i;
-      for (int idx = tid; idx < g * D; idx += 128) {
+      DMS_CHECK(i < Htot && pid < G + Htot && cf >= 0 && cl < Geff, v.hdr, 303, i, pid);
+      for (int idx = tid; idx < g * D; idx += kCons) {
         const int nn = idx / D, d = idx % D;
         float M = -INFINITY;
 #pragma unroll
@@ -660,16 +685,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const Attn
         }
       }
       if (!whole) {
-        consumer_bar();
+        consumer_bar<kNCW>();
         if (tid == 0) {
           __threadfence();
           const int prev = atomicAdd(&v.tickets[hd], 1);
           s_misc[3] = prev == cl - cf;
         }
-        consumer_bar();
+        consumer_bar<kNCW>();
         if (s_misc[3]) {
           __threadfence();
-          for (int idx = tid; idx < g * D; idx += 128) {
+          for (int idx = tid; idx < g * D; idx += kCons) {
             const int nn = idx / D, d = idx % D;
             float M = -INFINITY;
             for (int cc = cf; cc <= cl; ++cc)
@@ -686,7 +711,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) decode_attn_kernel(const Attn
           if (tid == 0) v.tickets[hd] = 0;
         }
       }
-      consumer_bar();
+      consumer_bar<kNCW>();
       st.reset();
       have_q = false;
     }
@@ -705,7 +730,7 @@ static dms_status launch_attn(const AttnParams& prm, cudaStream_t stream) {
     if (st != DMS_OK) return st;
     attr_set = true;
   }
-  decode_attn_kernel<KV, D><<<prm.G, kAttnThreads, T::SMEM, stream>>>(prm);
+  decode_attn_kernel<KV, D><<<prm.G, T::THREADS, T::SMEM, stream>>>(prm);
   return cuda_status(cudaGetLastError(), "decode_attn_kernel");
 }
 

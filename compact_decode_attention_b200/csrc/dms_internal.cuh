@@ -70,6 +70,16 @@ __device__ __forceinline__ void report_error(DevHeader* hdr, uint32_t bit, int l
   }
 }
 
+// Bounds checks of DMS_DEBUG builds: a failed check records DMS_DEVERR_BOUNDS
+// with (site, a, b) in the error fields and evaluates to false, so the caller
+// skips the access.  Release builds compile the check away.
+#ifdef DMS_DEBUG
+#define DMS_CHECK(cond, hdr, site, a, b) \
+  ((cond) ? true : (report_error((hdr), DMS_DEVERR_BOUNDS, (site), int(a), int(b)), false))
+#else
+#define DMS_CHECK(cond, hdr, site, a, b) true
+#endif
+
 // ------------------------------------------------------------------------
 // stored-row layout
 // ------------------------------------------------------------------------

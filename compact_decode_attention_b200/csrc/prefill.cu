@@ -263,6 +263,9 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
         const int jj = chunk * kPrefillChunk + s_kept[kk];
         const int slot = base + kk;
         const int row = slot % v.BT;
+        if (!DMS_CHECK(slot < v.mbh * v.BT && table[slot / v.BT] >= 0 &&
+                       table[slot / v.BT] < v.max_blocks, v.hdr, 201, hd, slot))
+          continue;
         uint8_t* blk = v.blocks + int64_t(table[slot / v.BT]) * v.block_bytes;
         const int64_t src_off = ((int64_t(b) * P + jj) * v.Hkv + h) * v.row_bytes + c * 16;
         const int64_t dst_off = int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;

@@ -15,7 +15,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdms.so")
+# DMS_LIBRARY=debug selects libdms_debug.so (device bounds checks, DMS_DEBUG)
+LIB_PATH = os.path.join(_HERE, "libdms_debug.so" if os.environ.get("DMS_LIBRARY") == "debug"
+                        else "libdms.so")
 
 DMS_OK, DMS_ERR_INVALID_ARG, DMS_ERR_CAPACITY, DMS_ERR_CUDA, DMS_ERR_UNSUPPORTED, DMS_ERR_DEVICE = range(6)
 DMS_F32, DMS_BF16, DMS_FP8_E4M3 = 0, 1, 2
@@ -25,6 +27,7 @@ DEVERR_HEAD_TABLE_FULL = 0x2
 DEVERR_FREE_STACK_FULL = 0x4
 DEVERR_TIMEOUT = 0x8
 DEVERR_LAYER_NOT_EMPTY = 0x10
+DEVERR_BOUNDS = 0x20
 
 BLOCK_TOKENS = 64
 

@@ -80,6 +80,7 @@ typedef enum { DMS_F32 = 0, DMS_BF16 = 1, DMS_FP8_E4M3 = 2 } dms_dtype;
 #define DMS_DEVERR_FREE_STACK_FULL  0x4u  /* per-head free stack overflow                */
 #define DMS_DEVERR_TIMEOUT          0x8u  /* a bounded wait gave up; outputs invalid     */
 #define DMS_DEVERR_LAYER_NOT_EMPTY  0x10u /* prefill into a layer that already holds data */
+#define DMS_DEVERR_BOUNDS           0x20u /* DMS_DEBUG builds: an index failed its check  */
 
 typedef struct {
   int32_t n_layers;
