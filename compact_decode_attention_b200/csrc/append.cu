@@ -12,10 +12,14 @@
 // opening paragraphs).  Otherwise the token takes slot n_slots, opening a
 // new block when that slot starts one.
 //
-// One CTA does the bookkeeping of every head of the call so that new blocks
-// are handed out by a prefix sum in (layer, sequence, head) order: the
-// physical block ids are a deterministic function of the inputs.  The same
-// CTA then writes the rows (16-byte chunks spread over all threads).
+// One warp per head: the per-head state it needs (counters, last block, the
+// ring entry and the physical row of the token leaving the window) is read
+// with independent loads, so the kernel waits on memory about once before
+// its stores, and the rows are written by as many SMs as there are heads / 8.
+// A new block comes from an atomic bump of the block counter: the logical
+// state (slots, counts, rings, stored bytes) is a deterministic function of
+// the inputs; which physical block a head gets during decode is not (prefill
+// hands blocks out by a prefix sum and is deterministic).
 #include "dms_internal.cuh"
 
 namespace dms {
@@ -29,212 +33,132 @@ __device__ __forceinline__ float in_to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
 
-constexpr int kAppendThreads = 512;
-constexpr int kAppendRegChunks = 20;   // 16-byte input chunks a thread can hold
+constexpr int kAppendHeadsPerCta = 8;            // one warp per head
+constexpr int kAppendThreads = 32 * kAppendHeadsPerCta;
 
+// One warp per (layer, sequence, kv-head).  Lane 0 does the bookkeeping; all
+// lanes load the new K/V row first (it does not depend on the bookkeeping)
+// and store it once the destination is known.
 template <typename InT, bool FP8>
 __global__ void __launch_bounds__(kAppendThreads)
     append_evict_kernel(PoolView v, int l0, int nl, int batch, int64_t pos, const InT* k,
                         const InT* vv, const uint8_t* evict) {
-  extern __shared__ int s_dyn[];
-  // Rows of the new tokens: chunk c of head hh is K chunk c (c < nch) or V
-  // chunk c - nch.  When they fit in registers they are loaded first, so the
-  // loads overlap the bookkeeping below instead of following it.
-  const int nch = int(v.row_bytes >> 4);
-  const int H_ = nl * batch * v.Hkv;
-  const int total_chunks = H_ * 2 * nch;
-  const bool preload = !FP8 && total_chunks <= int(blockDim.x) * kAppendRegChunks;
-  uint4 reg[kAppendRegChunks];
-  if (preload) {
-#pragma unroll
-    for (int r = 0; r < kAppendRegChunks; ++r) {
-      const int c = threadIdx.x + r * blockDim.x;
-      if (c < total_chunks) {
-        const int hh = c / (2 * nch), cc = c % (2 * nch);
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(cc < nch ? k : vv) +
-                             int64_t(hh) * v.row_bytes + (cc % nch) * 16;
-        reg[r] = *reinterpret_cast<const uint4*>(src);
-      }
-    }
-  }
+  // the new rows and the pool state may have been written by the kernel
+  // before this one; once they are visible, let the next kernel (decode
+  // attention) be scheduled
+  pdl_wait_prerequisites();
+  pdl_launch_dependents();
   const int H = nl * batch * v.Hkv;
-  int* s_slot = s_dyn;          // [H] slot of the new token (-1: failed)
-  int* s_blk = s_dyn + H;       // [H] physical block of that slot
-  int* s_need = s_dyn + 2 * H;  // [H] 1 when the slot opens a new block
-  __shared__ int s_warp[32];
-  __shared__ int s_total, s_fail_blocks;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kAppendHeadsPerCta + (threadIdx.x >> 5);
+  if (i >= H) return;
+  const int h = i % v.Hkv, b = (i / v.Hkv) % batch, l = l0 + i / (v.Hkv * batch);
+  const int hd = v.head(l, b, h);
   const int t = int(pos);
-  const int ring_idx = t % v.w;
+  const int64_t ri = int64_t(hd) * v.w + t % v.w;
 
-  // ---- 1. retire the token leaving the window, pick the slot -------------
-  for (int i = tid; i < H; i += blockDim.x) {
-    const int h = i % v.Hkv, b = (i / v.Hkv) % batch, l = l0 + i / (v.Hkv * batch);
-    const int hd = v.head(l, b, h);
-    int ns = v.n_slots[hd], nr = v.n_retained[hd], ft = v.free_top[hd];
-    int* stack = v.free_stack + int64_t(hd) * v.free_cap;
-    if (t >= v.w) {
-      const uint32_t e = v.ring[int64_t(hd) * v.w + ring_idx];
-      if (e >> 31) {
-        if (ft < v.free_cap) {
-          stack[ft++] = int(e & 0x7fffffffu);
-          nr -= 1;
-        } else {
-          report_error(v.hdr, DMS_DEVERR_FREE_STACK_FULL, l, b, h);
-        }
-      }
-    }
-    int slot, need = 0;
-    if (ft > 0) {
-      slot = stack[--ft];
-    } else {
-      slot = ns;
-      need = (slot % v.BT) == 0;
-      if (slot / v.BT >= v.mbh) {
-        report_error(v.hdr, DMS_DEVERR_HEAD_TABLE_FULL, l, b, h);
-        slot = -1;
-        need = 0;
-      } else {
-        ns += 1;
-      }
-    }
-    s_slot[i] = slot;
-    s_need[i] = need;
-    // counters are committed in step 3 once the block (if any) is secured
-    if (slot >= 0 && !DMS_CHECK(hd >= 0 && hd < v.n_heads && slot < v.mbh * v.BT, v.hdr, 101, hd, slot))
-      slot = -1;
-    s_blk[i] = slot < 0 ? -1 : (need ? -2 : v.bt[int64_t(hd) * v.mbh + slot / v.BT]);
-    if (slot >= 0 && !need && !DMS_CHECK(s_blk[i] >= 0 && s_blk[i] < v.max_blocks, v.hdr, 102, hd, s_blk[i]))
-      slot = -1, s_slot[i] = -1;
-    if (slot >= 0) {
-      v.free_top[hd] = ft;
-      // n_slots / n_retained written below
-      s_dyn[3 * H + i] = ns;
-      s_dyn[4 * H + i] = nr + 1;
-    }
-  }
-  __syncthreads();
-
-  // ---- 2. exclusive prefix of new blocks in (layer, seq, head) order ------
-  {
-    int running = 0;
-    for (int i0 = 0; i0 < H; i0 += blockDim.x) {
-      const int i = i0 + tid;
-      const int x = i < H ? s_need[i] : 0;
-      int incl = x;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (lane == 31) s_warp[warp] = incl;
-      __syncthreads();
-      if (warp == 0) {
-        int tt = lane < nwarps ? s_warp[lane] : 0;
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, tt, o);
-          if (lane >= o) tt += y;
-        }
-        s_warp[lane] = tt;
-      }
-      __syncthreads();
-      if (i < H) s_need[i] = x ? running + (warp ? s_warp[warp - 1] : 0) + incl - x + 1 : 0;
-      running += s_warp[nwarps - 1];
-      __syncthreads();
-    }
-    if (tid == 0) {
-      s_total = running;
-      const int stack = v.hdr->block_stack_top;
-      const int64_t avail = int64_t(stack) + (v.max_blocks - v.hdr->next_block);
-      s_fail_blocks = running > avail;
-      if (s_fail_blocks) report_error(v.hdr, DMS_DEVERR_BLOCKS_EXHAUSTED, l0, -1, -1);
-    }
-    __syncthreads();
-  }
-
-  // ---- 3. commit: new blocks, counters, ring -------------------------------
-  const int stack_top = v.hdr->block_stack_top;
-  const int next = v.hdr->next_block;
-  for (int i = tid; i < H; i += blockDim.x) {
-    const int h = i % v.Hkv, b = (i / v.Hkv) % batch, l = l0 + i / (v.Hkv * batch);
-    const int hd = v.head(l, b, h);
-    int slot = s_slot[i];
-    if (slot < 0) continue;
-    if (s_need[i]) {
-      if (s_fail_blocks) {
-        s_slot[i] = -1;
-        continue;
-      }
-      const int a = s_need[i] - 1;
-      const int id = a < stack_top ? v.block_stack[stack_top - 1 - a] : next + (a - stack_top);
-      if (!DMS_CHECK(id >= 0 && id < v.max_blocks, v.hdr, 103, hd, id)) {
-        s_slot[i] = -1;
-        continue;
-      }
-      v.bt[int64_t(hd) * v.mbh + slot / v.BT] = id;
-      s_blk[i] = id;
-    }
-    v.n_slots[hd] = s_dyn[3 * H + i];
-    v.n_retained[hd] = s_dyn[4 * H + i];
-    const uint8_t f = evict[i];  // [nl, batch, Hkv] flattened like i
-    v.ring[int64_t(hd) * v.w + ring_idx] = uint32_t(slot) | (uint32_t(f != 0) << 31);
-  }
-  __syncthreads();
-  if (tid == 0 && !s_fail_blocks) {
-    const int total = s_total;
-    v.hdr->block_stack_top = stack_top > total ? stack_top - total : 0;
-    v.hdr->next_block = next + (total > stack_top ? total - stack_top : 0);
-  }
-
-  // ---- 4. write the rows ---------------------------------------------------
-  if (preload) {
+  // ---- new rows into registers (bf16/fp32: 16-byte chunks, K then V) ----
+  const int nch = int(v.row_bytes >> 4);       // chunks per row: 8, 16 or 32
+  constexpr int kMaxPerLane = 2;               // 2 * 32 chunks per lane pair covers fp32 D=128
+  uint4 chunk[kMaxPerLane];
+  if constexpr (!FP8) {
 #pragma unroll
-    for (int r = 0; r < kAppendRegChunks; ++r) {
-      const int c = threadIdx.x + r * blockDim.x;
-      if (c < total_chunks) {
-        const int hh = c / (2 * nch), cc = c % (2 * nch);
-        const int slot = s_slot[hh];
-        if (slot < 0) continue;
-        const int row = slot % v.BT;
-        uint8_t* dst = v.blocks + int64_t(s_blk[hh]) * v.block_bytes + (cc < nch ? 0 : v.tile_bytes) +
-                       int64_t(row) * v.row_bytes + swz_chunk(cc % nch, row) * 16;
-        *reinterpret_cast<uint4*>(dst) = reg[r];
+    for (int r = 0; r < kMaxPerLane; ++r) {
+      const int c = lane + 32 * r;
+      if (c < 2 * nch) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(c < nch ? k : vv) +
+                             int64_t(i) * v.row_bytes + (c % nch) * 16;
+        chunk[r] = *reinterpret_cast<const uint4*>(src);
       }
     }
-  } else if constexpr (!FP8) {
-    for (int i = tid; i < H * nch; i += blockDim.x) {
-      const int hh = i / nch, c = i % nch;
-      const int slot = s_slot[hh];
-      if (slot < 0) continue;
-      const int row = slot % v.BT;
-      uint8_t* blk = v.blocks + int64_t(s_blk[hh]) * v.block_bytes;
-      const int64_t src = int64_t(hh) * v.row_bytes + c * 16;
-      const int64_t dst = int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;
-      *reinterpret_cast<uint4*>(blk + dst) =
-          *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(k) + src);
-      *reinterpret_cast<uint4*>(blk + v.tile_bytes + dst) =
-          *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vv) + src);
+  }
+
+  // ---- bookkeeping (lane 0; all its loads are independent) ----
+  int slot = -1, prow = -1, opened = 0;
+  if (lane == 0) {
+    int ns = v.n_slots[hd], nr = v.n_retained[hd], ft = v.free_top[hd];
+    const int lb = v.last_block[hd];
+    const uint32_t e = v.ring[ri];
+    const int er = v.ring_row[ri];
+    const uint32_t flag = evict[i] != 0;     // [nl, batch, Hkv] flattened like i
+    if (t >= v.w && (e >> 31)) {
+      // DMS delayed eviction retires token t - w; its slot is pushed on the
+      // head's LIFO free stack and popped right back by the new token, so
+      // the pair is done in registers and the row comes from the row ring
+      if (ft < v.free_cap) {
+        slot = int(e & 0x7fffffffu);
+        prow = er;
+        nr -= 1;
+      } else {
+        report_error(v.hdr, DMS_DEVERR_FREE_STACK_FULL, l, b, h);
+      }
+    } else if (ft > 0) {      // a slot freed earlier and not reused yet
+      ft -= 1;
+      slot = v.free_stack[int64_t(hd) * v.free_cap + ft];
+      prow = v.bt[int64_t(hd) * v.mbh + slot / v.BT] * v.BT + slot % v.BT;
+    } else if (ns / v.BT < v.mbh) {
+      slot = ns;
+      ns += 1;
+      if (slot % v.BT == 0) {  // the slot opens a new block: bump the block counter
+        const int id = atomicAdd(&v.hdr->next_block, 1);
+        if (id < v.max_blocks) {
+          v.bt[int64_t(hd) * v.mbh + slot / v.BT] = id;
+          v.last_block[hd] = id;
+          prow = id * v.BT;
+          opened = 1;
+        } else {
+          report_error(v.hdr, DMS_DEVERR_BLOCKS_EXHAUSTED, l, b, h);
+          slot = -1;
+        }
+      } else {
+        prow = lb * v.BT + slot % v.BT;
+      }
+    } else {
+      report_error(v.hdr, DMS_DEVERR_HEAD_TABLE_FULL, l, b, h);
+    }
+    if (slot >= 0 && !DMS_CHECK(prow >= 0 && prow < v.max_blocks * v.BT, v.hdr, 101, hd, prow))
+      slot = -1;
+    if (slot >= 0) {
+      v.n_slots[hd] = ns;
+      v.n_retained[hd] = nr + 1;
+      v.free_top[hd] = ft;
+      v.ring[ri] = uint32_t(slot) | (flag << 31);
+      v.ring_row[ri] = prow;
+    }
+  }
+  slot = __shfl_sync(0xffffffffu, slot, 0);
+  prow = __shfl_sync(0xffffffffu, prow, 0);
+  opened = __shfl_sync(0xffffffffu, opened, 0);
+  if (slot < 0) return;
+  const int row = prow % v.BT;
+  uint8_t* blk = v.blocks + int64_t(prow / v.BT) * v.block_bytes;
+
+  // ---- store the row ----
+  if constexpr (!FP8) {
+#pragma unroll
+    for (int r = 0; r < kMaxPerLane; ++r) {
+      const int c = lane + 32 * r;
+      if (c < 2 * nch) {
+        uint8_t* dst = blk + (c < nch ? 0 : v.tile_bytes) + int64_t(row) * v.row_bytes +
+                       swz_chunk(c % nch, row) * 16;
+        *reinterpret_cast<uint4*>(dst) = chunk[r];
+      }
     }
   } else {
-    // a new block's transposed V tile is cleared first so that token columns
-    // not yet written decode to 0 (the attention kernel reads whole V tiles)
-    for (int i = tid; i < H * 512; i += blockDim.x) {
-      const int hh = i >> 9;
-      if (s_slot[hh] < 0 || s_need[hh] == 0) continue;  // only blocks opened by this step
-      uint8_t* blk = v.blocks + int64_t(s_blk[hh]) * v.block_bytes;
-      reinterpret_cast<uint4*>(blk + v.tile_bytes)[i & 511] = make_uint4(0, 0, 0, 0);
+    // a block opened by this step gets its transposed V tile cleared first,
+    // so token columns not yet written decode to 0 (the attention kernel
+    // reads whole V tiles)
+    if (opened) {
+      uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);
+      for (int c = lane; c < int(v.tile_bytes / 16); c += 32) tile[c] = make_uint4(0, 0, 0, 0);
+      __syncwarp();
     }
-    __syncthreads();
-    for (int i = tid; i < H * 8; i += blockDim.x) {
-      const int hh = i >> 3, lc = i & 7;
-      const int slot = s_slot[hh];
-      if (slot < 0) continue;
-      const int h = hh % v.Hkv, l = l0 + hh / (v.Hkv * batch);
-      const float sK = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 0];
-      const float sV = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 1];
-      const int row = slot % v.BT;
-      uint8_t* blk = v.blocks + int64_t(s_blk[hh]) * v.block_bytes;
-      const InT* srck = k + int64_t(hh) * v.D;
-      const InT* srcv = vv + int64_t(hh) * v.D;
+    const float sK = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 0];
+    const float sV = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 1];
+    const InT* srck = k + int64_t(i) * v.D;
+    const InT* srcv = vv + int64_t(i) * v.D;
+    if (lane < 8) {            // K: lane lc fills 16-byte chunk lc of the permuted row
+      const int lc = lane;
       uint8_t codes[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -244,11 +168,11 @@ __global__ void __launch_bounds__(kAppendThreads)
       }
       *reinterpret_cast<uint4*>(blk + row * 128 + ((lc ^ (row & 7)) << 4)) =
           *reinterpret_cast<const uint4*>(codes);
+    }
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int d = lc * 16 + e;
-        blk[v.tile_bytes + fp8v_byte(row, d)] = f32_to_e4m3(__fdiv_rn(in_to_f32(srcv[d]), sV));
-      }
+    for (int e = 0; e < 4; ++e) {  // V: 4 elements per lane into the transposed tile
+      const int d = lane * 4 + e;
+      blk[v.tile_bytes + fp8v_byte(row, d)] = f32_to_e4m3(__fdiv_rn(in_to_f32(srcv[d]), sV));
     }
   }
 }
@@ -286,24 +210,13 @@ extern "C" dms_status dms_append_evict_layers(dms_pool* pool, int layer0, int n_
     return DMS_ERR_INVALID_ARG;
   }
   const int H = n_layers * batch * pv.Hkv;
-  const size_t smem = sizeof(int) * 5 * size_t(H);
-  if (smem > 200 * 1024) {
-    set_last_error("too many heads (%d) for one append call; split the layer range", H);
-    return DMS_ERR_UNSUPPORTED;
-  }
-  const int threads = kAppendThreads;
+  const dim3 grid((H + kAppendHeadsPerCta - 1) / kAppendHeadsPerCta);
   dms_status st = DMS_OK;
-#define DMS_LAUNCH_APPEND(T, F)                                                                    \
-  do {                                                                                             \
-    auto fn = append_evict_kernel<T, F>;                                                           \
-    if (smem > 48 * 1024) {                                                                        \
-      st = cuda_status(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
-                                            int(smem)), "append smem attribute");                  \
-      if (st != DMS_OK) return st;                                                                 \
-    }                                                                                              \
-    fn<<<1, threads, smem, stream>>>(pv, layer0, n_layers, batch, pos, static_cast<const T*>(k),   \
-                                     static_cast<const T*>(v), evict);                            \
-  } while (0)
+#define DMS_LAUNCH_APPEND(T, F)                                                                   \
+  st = cuda_status(launch_pdl(append_evict_kernel<T, F>, grid, dim3(kAppendThreads), 0, stream,  \
+                              pv, layer0, n_layers, batch, pos, static_cast<const T*>(k),         \
+                              static_cast<const T*>(v), evict),                                   \
+                   "append_evict_kernel")
   if (in_dtype == DMS_BF16) {
     if (fp8) DMS_LAUNCH_APPEND(__nv_bfloat16, true);
     else DMS_LAUNCH_APPEND(__nv_bfloat16, false);
@@ -312,7 +225,7 @@ extern "C" dms_status dms_append_evict_layers(dms_pool* pool, int layer0, int n_
     else DMS_LAUNCH_APPEND(float, false);
   }
 #undef DMS_LAUNCH_APPEND
-  return cuda_status(cudaGetLastError(), "append_evict_kernel");
+  return st;
 }
 
 extern "C" dms_status dms_append_evict(dms_pool* pool, int layer, int batch, int64_t pos,

@@ -470,6 +470,11 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   }
   fence_proxy_async_smem();  // order these generic writes before later TMA writes
 
+  // everything above only touched shared memory; the pool state and the
+  // queries may come from the kernel before this one (append/evict)
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
+
   // ---- find this CTA's unit range: per-thread head ranges + block scan ----
   const int per = (Htot + kAttnThreads - 1) / kAttnThreads;
   const int hb = min(Htot, tid * per), he = min(Htot, hb + per);
@@ -730,8 +735,9 @@ static dms_status launch_attn(const AttnParams& prm, cudaStream_t stream) {
     if (st != DMS_OK) return st;
     attr_set = true;
   }
-  decode_attn_kernel<KV, D><<<prm.G, T::THREADS, T::SMEM, stream>>>(prm);
-  return cuda_status(cudaGetLastError(), "decode_attn_kernel");
+  return cuda_status(launch_pdl(decode_attn_kernel<KV, D>, dim3(prm.G), dim3(T::THREADS), T::SMEM,
+                                stream, prm),
+                     "decode_attn_kernel");
 }
 
 }  // namespace dms

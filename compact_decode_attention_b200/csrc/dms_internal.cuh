@@ -7,6 +7,8 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "dms.h"
 
 namespace dms {
@@ -43,7 +45,9 @@ struct PoolView {
   int32_t* bt;
   int32_t* n_slots;
   int32_t* n_retained;
-  uint32_t* ring;
+  uint32_t* ring;           // [n_heads][w] slot | flag << 31
+  int32_t* ring_row;        // [n_heads][w] physical row (block * BT + row) of that slot
+  int32_t* last_block;      // [n_heads] block of slot n_slots - 1 (-1 when empty)
   int32_t* free_top;
   int32_t* free_stack;
   int32_t* block_stack;
@@ -227,6 +231,16 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Programmatic dependent launch: let the next kernel of the stream be
+// scheduled now / wait until every kernel this one depends on has finished
+// and its writes are visible.  Both are no-ops without the launch attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prerequisites() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // 2^x with the hardware approximation (max rel. error ~2^-22).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -259,6 +273,22 @@ __device__ __forceinline__ uint8_t f32_to_e4m3(float x) {
 // host helpers
 // ------------------------------------------------------------------------
 void set_last_error(const char* fmt, ...);
+// Launch with programmatic stream serialisation (PDL) allowed.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 dms_status cuda_status(cudaError_t e, const char* what);
 int device_sm_count(int device);
 

@@ -81,8 +81,8 @@ static dms_status plan_layout(const dms_pool_config* c, dms_pool_layout_t* lay) 
     set_last_error("block_tokens must be %d", kBlockTokens);
     return DMS_ERR_UNSUPPORTED;
   }
-  if (c->max_blocks >= (int64_t(1) << 31) || c->max_context >= (int64_t(1) << 24)) {
-    set_last_error("max_blocks must be < 2^31 and max_context < 2^24");
+  if (c->max_blocks * kBlockTokens >= (int64_t(1) << 31) || c->max_context >= (int64_t(1) << 24)) {
+    set_last_error("max_blocks * block_tokens must be < 2^31 and max_context < 2^24");
     return DMS_ERR_INVALID_ARG;
   }
   const int64_t n_heads = int64_t(c->n_layers) * c->max_batch * c->n_kv_heads;
@@ -101,6 +101,8 @@ static dms_status plan_layout(const dms_pool_config* c, dms_pool_layout_t* lay) 
   lay->n_slots = off;     off = align256(off + uint64_t(n_heads) * 4);
   lay->n_retained = off;  off = align256(off + uint64_t(n_heads) * 4);
   lay->ring = off;        off = align256(off + uint64_t(n_heads) * c->window * 4);
+  lay->ring_row = off;    off = align256(off + uint64_t(n_heads) * c->window * 4);
+  lay->last_block = off;  off = align256(off + uint64_t(n_heads) * 4);
   lay->free_top = off;    off = align256(off + uint64_t(n_heads) * 4);
   lay->free_stack = off;  off = align256(off + uint64_t(n_heads) * kFreeStackCap * 4);
   lay->block_stack = off; off = align256(off + uint64_t(c->max_blocks) * 4);
@@ -147,6 +149,8 @@ static PoolView make_view(const dms_pool_config& c, const dms_pool_layout_t& lay
   v.n_slots = reinterpret_cast<int32_t*>(b + lay.n_slots);
   v.n_retained = reinterpret_cast<int32_t*>(b + lay.n_retained);
   v.ring = reinterpret_cast<uint32_t*>(b + lay.ring);
+  v.ring_row = reinterpret_cast<int32_t*>(b + lay.ring_row);
+  v.last_block = reinterpret_cast<int32_t*>(b + lay.last_block);
   v.free_top = reinterpret_cast<int32_t*>(b + lay.free_top);
   v.free_stack = reinterpret_cast<int32_t*>(b + lay.free_stack);
   v.block_stack = reinterpret_cast<int32_t*>(b + lay.block_stack);
@@ -228,7 +232,9 @@ __global__ void __launch_bounds__(1024) stats_kernel(PoolView v) {
     o->max_retained = mx;
     o->heads_nonempty = ne;
     o->pad0 = 0;
-    o->blocks_in_use = int64_t(v.hdr->next_block) - v.hdr->block_stack_top;
+    // an exhausted decode step may have bumped the counter past the pool
+    const int64_t handed = v.hdr->next_block < v.max_blocks ? v.hdr->next_block : v.max_blocks;
+    o->blocks_in_use = handed - v.hdr->block_stack_top;
     o->blocks_total = v.max_blocks;
     o->kv_bytes_in_use = o->blocks_in_use * v.block_bytes;
     o->kv_bytes_retained = ret * 2 * v.row_bytes;

@@ -187,6 +187,12 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(PoolView v, int laye
       v.n_slots[hd] = s_n[p];
       v.n_retained[hd] = s_n[p];
       v.free_top[hd] = 0;
+      if (nb > 0) {
+        const int a = s_base[p] + nb - 1;
+        v.last_block[hd] = a < stack ? v.block_stack[stack - 1 - a] : next + (a - stack);
+      } else {
+        v.last_block[hd] = -1;
+      }
     }
   }
   if (v.kv_dtype == DMS_FP8_E4M3) {
@@ -249,8 +255,10 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
     if (keep) {
       s_kept[rank] = threadIdx.x;
       if (j >= P - v.w) {
-        const uint32_t slot = uint32_t(base + rank);
-        v.ring[int64_t(hd) * v.w + (j % v.w)] = slot | (uint32_t(f != 0) << 31);
+        const int slot = base + rank;
+        const int64_t ri = int64_t(hd) * v.w + (j % v.w);
+        v.ring[ri] = uint32_t(slot) | (uint32_t(f != 0) << 31);
+        v.ring_row[ri] = v.bt[int64_t(hd) * v.mbh + slot / v.BT] * v.BT + slot % v.BT;
       }
     }
     __syncthreads();

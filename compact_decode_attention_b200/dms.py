@@ -52,8 +52,9 @@ class PoolConfig(ctypes.Structure):
 
 class PoolLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in
-                ("header", "blocks", "block_table", "n_slots", "n_retained", "ring", "free_top",
-                 "free_stack", "block_stack", "scales", "tickets", "scratch", "total")] + [
+                ("header", "blocks", "block_table", "n_slots", "n_retained", "ring", "ring_row",
+                 "last_block", "free_top", "free_stack", "block_stack", "scales", "tickets",
+                 "scratch", "total")] + [
         ("block_bytes", ctypes.c_int64), ("row_bytes", ctypes.c_int64),
         ("max_blocks_per_head", ctypes.c_int32), ("free_stack_cap", ctypes.c_int32),
         ("n_heads", ctypes.c_int32), ("fp8_layout", ctypes.c_int32)]

@@ -31,7 +31,8 @@
  *     table[s / BT], row s % BT), n_slots (slots ever handed out),
  *     n_retained (tokens held), a window ring of w entries
  *     (slot | flag << 31 for the last w positions; entry t mod w holds
- *     token t) and a LIFO free-slot stack;
+ *     token t) with a parallel ring of physical rows (block * BT + row),
+ *     the block of the head's last slot, and a LIFO free-slot stack;
  *   - a global free-block stack and bump counter, FP8 scales, an error word.
  * Slots of one head are dense: a retired slot is reused by the same step's
  * new token, so the held tokens are exactly slots [0, n_slots).
@@ -100,8 +101,8 @@ typedef struct dms_pool dms_pool;  /* opaque host handle */
 /* Byte offsets of each region inside the pool buffer, for inspection by
  * tests and tools (the pool is plain device memory). */
 typedef struct {
-  uint64_t header, blocks, block_table, n_slots, n_retained, ring, free_top,
-           free_stack, block_stack, scales, tickets, scratch, total;
+  uint64_t header, blocks, block_table, n_slots, n_retained, ring, ring_row, last_block,
+           free_top, free_stack, block_stack, scales, tickets, scratch, total;
   int64_t block_bytes;          /* bytes of one block (K tile + V tile)      */
   int64_t row_bytes;            /* bytes of one stored row (D * elem size)   */
   int32_t max_blocks_per_head;  /* block table width                         */

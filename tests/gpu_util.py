@@ -27,6 +27,8 @@ def read_state(pool) -> dict:
         "n_retained": reg("n_retained", torch.int32, nh),
         "free_top": reg("free_top", torch.int32, nh),
         "ring": reg("ring", torch.int32, nh * cfg.window).view(np.uint32).reshape(nh, cfg.window),
+        "ring_row": reg("ring_row", torch.int32, nh * cfg.window).reshape(nh, cfg.window),
+        "last_block": reg("last_block", torch.int32, nh),
         "bt": reg("block_table", torch.int32, nh * lay.max_blocks_per_head).reshape(nh, -1),
         "scales": reg("scales", torch.float32, cfg.n_layers * cfg.n_kv_heads * 2).reshape(
             cfg.n_layers, cfg.n_kv_heads, 2),
@@ -110,6 +112,10 @@ def check_head_store(pool, state, hd, store, rows_k_f32, rows_v_f32, kind, scale
     for idx, e in enumerate(store.ring):
         if e is not None:
             assert state["ring"][hd, idx] == (e[0] | (e[1] << 31)), (hd, idx)
+            slot = e[0]
+            assert state["ring_row"][hd, idx] == state["bt"][hd, slot // BT] * BT + slot % BT, (hd, idx)
+    if store.n_slots > 0 and store.n_slots % BT:
+        assert state["last_block"][hd] == state["bt"][hd, (store.n_slots - 1) // BT]
     n = store.n_slots
     got_k, got_v = stored_rows(pool, state, hd, n, kind)
     pos = [store.pos_of_slot[s] for s in range(n)]
