@@ -52,13 +52,16 @@ struct AttnTraits {
   static constexpr int QESZ = KV == KV_F32 ? 4 : 2;  // q / out element bytes
   static constexpr int ROWB = D * ESZ;
   static constexpr int TILEB = kBlockTokens * ROWB;
-  static constexpr int QB = 8 * D * QESZ;              // room for 8 query rows
+  // The fp32 path reads its query rows from the stage (QB bytes after the
+  // tiles); the tensor-core paths load query fragments from global memory.
+  static constexpr int QB = KV == KV_F32 ? 8 * D * QESZ : 0;
   static constexpr int STAGEB = 2 * TILEB + QB;
-  // 34 KB stages for bf16 D=128: 6 stages over 3 consumer warps (2 each);
-  // fp32 D=128 (68 KB stages): 3 stages, 3 warps; the others 8 (or 4) over 4.
-  static constexpr bool BIG = (KV == KV_BF16 && D == 128) || (KV == KV_F32 && D == 128);
-  static constexpr int NCW = BIG ? 3 : 4;              // consumer warps
+  // Tensor-core variants give every stage its own consumer warp (6 stages of
+  // 34 KB for bf16 D=128, 8 for the others): with two consumer warps per SM
+  // sub-partition one warp's MMA / ldmatrix latency hides behind the other's.
+  // fp32 (68 KB or 34 KB stages): 3 or 4 stages and warps.
   static constexpr int NS = KV == KV_F32 ? (D == 128 ? 3 : 4) : (KV == KV_BF16 && D == 128) ? 6 : 8;
+  static constexpr int NCW = NS;                        // consumer warps
   static constexpr int THREADS = 32 * (NCW + 1);       // + one producer warp
   static constexpr int COMBINE_FLOATS = NCW * 8 * D + 2 * NCW * 8;
   static constexpr int MISC_INTS = 16 + THREADS / 32;
@@ -132,14 +135,16 @@ struct MmaWarp {
     for (int i = 0; i < MTD; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   }
 
-  // Q^T B fragments from the stage's query rows (row n = lane / 4).
-  __device__ __forceinline__ void load_q(const uint8_t* qs, int lane) {
+  // Q^T B fragments of the group's query rows (row n = lane / 4 < g; the
+  // rows past g are the zero padding of the N = 8 side), from global memory.
+  __device__ __forceinline__ void load_q(const uint8_t* qg, int g, int lane) {
     const int n = lane >> 2, q2 = (lane & 3) * 2;
-    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(qs) + n * D;
+    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(qg) + n * D;
+    const bool real = n < g;
 #pragma unroll
     for (int kt = 0; kt < KSTEPS; ++kt) {
-      const uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + kt * 16 + q2);
-      const uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + kt * 16 + 8 + q2);
+      const uint32_t lo = real ? __ldg(reinterpret_cast<const unsigned int*>(qrow + kt * 16 + q2)) : 0u;
+      const uint32_t hi = real ? __ldg(reinterpret_cast<const unsigned int*>(qrow + kt * 16 + 8 + q2)) : 0u;
       if constexpr (KV == KV_FP8) {
         const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
         const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
@@ -163,22 +168,30 @@ struct MmaWarp {
     const uint8_t* Vs = stage + T::TILEB;
     const int q = lane & 3, r8 = lane >> 2;
     float s[4][4];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
     // ---- S^T = K Q^T over the 64 rows (4 m-tiles of 16 tokens) ----
+    // All four m-tiles are computed (rows past `rows` are masked to -inf
+    // below), k-step outer, so each k-step issues four independent MMAs.
+    if constexpr (KV == KV_BF16) {
+      const uint32_t kbase = smem_u32(Ks);
+#pragma unroll
+      for (int kt = 0; kt < KSTEPS; ++kt) {
+        const int ch = 2 * kt + (lane >> 4);
+        uint32_t a[4][4];
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          const int row = mt * 16 + (lane & 15);
+          ldmatrix_x4(a[mt], kbase + row * T::ROWB + (swz_chunk(ch, row) << 4));
+        }
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) mma(s[mt], a[mt], qf[kt][0], qf[kt][1]);
+      }
+    }
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
-      s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
-      if (mt * 16 < rows) {
-        if constexpr (KV == KV_BF16) {
-          const uint32_t kbase = smem_u32(Ks);
-          const int row = mt * 16 + (lane & 15);
-#pragma unroll
-          for (int kt = 0; kt < KSTEPS; ++kt) {
-            const int ch = 2 * kt + (lane >> 4);
-            uint32_t a[4];
-            ldmatrix_x4(a, kbase + row * T::ROWB + (swz_chunk(ch, row) << 4));
-            mma(s[mt], a, qf[kt][0], qf[kt][1]);
-          }
-        } else {  // FP8, D = 128: two 16-byte loads per row give all 8 k-steps
+      if constexpr (KV == KV_FP8) {
+        if (mt * 16 < rows) {  // FP8, D = 128: two 16-byte loads per row give all 8 k-steps
           const int r0 = mt * 16 + r8, r1 = r0 + 8;
           const uint4 a0lo = *reinterpret_cast<const uint4*>(Ks + r0 * 128 + (((2 * q) ^ (r0 & 7)) << 4));
           const uint4 a0hi = *reinterpret_cast<const uint4*>(Ks + r0 * 128 + (((2 * q + 1) ^ (r0 & 7)) << 4));
@@ -349,7 +362,7 @@ struct F32Warp {
       for (int e = 0; e < DPL; ++e) o[n][e] = 0.f;
     }
   }
-  __device__ __forceinline__ void load_q(const uint8_t*, int) {}
+  __device__ __forceinline__ void load_q(const uint8_t*, int, int) {}
 
   __device__ __forceinline__ float kval(const uint8_t* tile, int r, int d) const {
     return reinterpret_cast<const float*>(tile + r * T::ROWB + (swz_chunk(d >> 2, r) << 4))[d & 3];
@@ -463,12 +476,14 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     s_misc[0] = 0;
     fence_mbar_init();
   }
-  // query rows g..7 of every stage stay zero (padding of the N=8 side)
-  for (int s = 0; s < T::NS; ++s) {
-    uint4* qa = reinterpret_cast<uint4*>(stages + size_t(s) * T::STAGEB + 2 * T::TILEB);
-    for (int i = tid; i < T::QB / 16; i += kAttnThreads) qa[i] = make_uint4(0, 0, 0, 0);
+  if constexpr (T::QB > 0) {
+    // fp32 path: query rows g..7 of every stage stay zero (padding)
+    for (int s = 0; s < T::NS; ++s) {
+      uint4* qa = reinterpret_cast<uint4*>(stages + size_t(s) * T::STAGEB + 2 * T::TILEB);
+      for (int i = tid; i < T::QB / 16; i += kAttnThreads) qa[i] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();  // order these generic writes before later TMA writes
   }
-  fence_proxy_async_smem();  // order these generic writes before later TMA writes
 
   // everything above only touched shared memory; the pool state and the
   // queries may come from the kernel before this one (append/evict)
@@ -569,14 +584,14 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
             const uint32_t kbytes = uint32_t(jrows) * T::ROWB;
             const bool whole = jrows == kBlockTokens;
             const uint32_t vbytes = (whole || KV == KV_FP8) ? T::TILEB : kbytes;
-            mbar_arrive_expect_tx(&full[s], kbytes + vbytes + qrow_bytes);
+            mbar_arrive_expect_tx(&full[s], kbytes + vbytes + (T::QB > 0 ? qrow_bytes : 0));
             if (whole) {
               bulk_g2s(st, src, 2 * T::TILEB, &full[s], pol);
             } else {
               bulk_g2s(st, src, kbytes, &full[s], pol);
               bulk_g2s(st + T::TILEB, src + T::TILEB, vbytes, &full[s], pol);
             }
-            bulk_g2s(st + 2 * T::TILEB, qsrc, qrow_bytes, &full[s], qpol);
+            if constexpr (T::QB > 0) bulk_g2s(st + 2 * T::TILEB, qsrc, qrow_bytes, &full[s], qpol);
             issued = k + 1;
           }
         }
@@ -631,6 +646,13 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     if (k % kNCW == warp) {
       const int s = k % T::NS;
       const uint32_t ph = (k / T::NS) & 1;
+      if constexpr (KV != KV_F32) {
+        if (!have_q) {  // first block of this head for this warp: issue before the wait
+          st.load_q(p.q + int64_t(i / v.Hkv) * v.Hq * D * T::QESZ + int64_t(i % v.Hkv) * qrow_bytes,
+                    g, lane);
+          have_q = true;
+        }
+      }
       bool ok = false;
       if (!*s_abort) {
         ok = mbar_wait_bounded(&full[s], ph, s_abort);
@@ -642,15 +664,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         const uint8_t* stage = stages + size_t(s) * T::STAGEB;
-        if constexpr (KV == KV_F32) {
-          st.unit(stage, rows, lane);
-        } else {
-          if (!have_q) {
-            st.load_q(stage + 2 * T::TILEB, lane);
-            have_q = true;
-          }
-          st.unit(stage, rows, lane);
-        }
+        st.unit(stage, rows, lane);
       }
       // release the stage only after its copy was seen complete; after an
       // abort the producer issues nothing more and drains what it issued
@@ -940,3 +954,4 @@ extern "C" dms_status dms_decode_attn_layers_noalloc(dms_pool* pool, int layer0,
   if (v.kv_dtype == DMS_FP8_E4M3) return launch_attn<KV_FP8, 128>(prm, stream);
   return v.D == 128 ? launch_attn<KV_F32, 128>(prm, stream) : launch_attn<KV_F32, 64>(prm, stream);
 }
+

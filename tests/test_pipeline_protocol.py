@@ -19,7 +19,7 @@ import pytest
 
 # (stages, consumer warps) of each kernel variant: bf16 D=128, bf16 D=64,
 # FP8 D=128, fp32 D=64, fp32 D=128
-KERNEL_LAYOUTS = [(6, 3), (8, 4), (8, 4), (4, 4), (3, 3)]
+KERNEL_LAYOUTS = [(6, 6), (8, 8), (8, 8), (4, 4), (3, 3)]
 
 
 class MBarrier:
@@ -122,3 +122,4 @@ def test_shared_stages_break_the_protocol():
         except AssertionError:
             broken += 1
     assert broken > 0
+
