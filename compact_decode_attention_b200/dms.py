@@ -73,6 +73,12 @@ class PoolStats(ctypes.Structure):
         return {f: getattr(self, f) for f, _ in self._fields_ if f != "pad0"}
 
 
+class StepperLayout(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_size_t), ("v", ctypes.c_size_t), ("q", ctypes.c_size_t),
+                ("evict", ctypes.c_size_t), ("in_bytes", ctypes.c_size_t),
+                ("out_bytes", ctypes.c_size_t), ("device_bytes", ctypes.c_size_t)]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _I64 = ctypes.c_int64
@@ -92,6 +98,11 @@ _SIGS = {
     "dms_decode_attn": (_I, [_P, _I, _I, _P, _I, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
     "dms_decode_attn_layers_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, ctypes.c_float, _P]),
     "dms_pool_stats": (_I, [_P, ctypes.POINTER(PoolStats), _P]),
+    "dms_stepper_layout": (_I, [_P, _I, _I, ctypes.POINTER(StepperLayout)]),
+    "dms_stepper_create": (_I, [_P, _I, _I, _I, ctypes.c_float, _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
+    "dms_stepper_step": (_I, [_P, _I64, _P, _P]),
+    "dms_stepper_join": (_I, [_P, _P]),
+    "dms_stepper_destroy": (_I, [_P]),
     "dms_synth_normal": (_I, [ctypes.c_uint64, _I, _I, _I, _I, _I64, _I, _I, _I, _I, _P, _P]),
     "dms_synth_flags": (_I, [ctypes.c_uint64, _I, _I, _I, _I64, _I, _I, _P, _P, _P]),
 }
@@ -205,6 +216,32 @@ def dms_pool_stats(pool: int, stream: int, check: bool = True) -> PoolStats:
     return st
 
 
+def dms_stepper_layout(pool: int, n_layers: int, batch: int) -> StepperLayout:
+    lay = StepperLayout()
+    _check(lib().dms_stepper_layout(pool, n_layers, batch, ctypes.byref(lay)), "dms_stepper_layout")
+    return lay
+
+
+def dms_stepper_create(pool: int, layer0: int, n_layers: int, batch: int, sm_scale: float,
+                       device_buf: int, device_bytes: int, stream: int) -> int:
+    h = _P()
+    _check(lib().dms_stepper_create(pool, layer0, n_layers, batch, sm_scale, device_buf, device_bytes,
+                                    stream, ctypes.byref(h)), "dms_stepper_create")
+    return h.value
+
+
+def dms_stepper_step(st: int, pos: int, host_in: int, host_out: int):
+    _check(lib().dms_stepper_step(st, pos, host_in, host_out), "dms_stepper_step")
+
+
+def dms_stepper_join(st: int, stream: int):
+    _check(lib().dms_stepper_join(st, stream), "dms_stepper_join")
+
+
+def dms_stepper_destroy(st: int):
+    _check(lib().dms_stepper_destroy(st), "dms_stepper_destroy")
+
+
 def dms_synth_normal(seed: int, stream_id: int, layer0: int, n_layers: int, batch: int, pos0: int,
                      n_pos: int, n_heads: int, head_dim: int, dtype: int, out: int, stream: int):
     _check(lib().dms_synth_normal(seed, stream_id, layer0, n_layers, batch, pos0, n_pos, n_heads,
@@ -302,3 +339,52 @@ class Pool:
         off = getattr(self.layout, name)
         esz = torch.empty(0, dtype=dtype).element_size()
         return self.buffer[off: off + count * esz].view(dtype)
+
+
+class Stepper:
+    """Decode steps fed from pinned host memory (dms_stepper_*): one call per
+    step enqueues the input copy, append/evict, decode attention and the
+    output copy, pipelined against the neighbouring steps."""
+
+    def __init__(self, pool: Pool, layer0, n_layers, batch, sm_scale=0.0, stream=None):
+        import torch
+        self.pool = pool
+        self.layout = dms_stepper_layout(pool.handle, n_layers, batch)
+        self.buffer = torch.empty(self.layout.device_bytes, dtype=torch.uint8, device=pool.buffer.device)
+        self.stream = _stream(stream)
+        self.handle = dms_stepper_create(pool.handle, layer0, n_layers, batch, sm_scale,
+                                         _ptr(self.buffer), self.layout.device_bytes, self.stream)
+        self._step = lib().dms_stepper_step
+        self.n_layers, self.batch = n_layers, batch
+
+    def host_inputs(self, n_steps: int):
+        """Pinned uint8 host buffer for n_steps packed step inputs."""
+        import torch
+        return torch.empty(n_steps, self.layout.in_bytes, dtype=torch.uint8).pin_memory()
+
+    def pack(self, dst, k, v, q, evict):
+        """Write one step's inputs (torch tensors, any device) into the packed
+        host row dst (uint8, layout.in_bytes)."""
+        lay = self.layout
+        for off, t in ((lay.k, k), (lay.v, v), (lay.q, q), (lay.evict, evict)):
+            b = t.contiguous().view(-1).view(dtype=__import__("torch").uint8)
+            dst[off: off + b.numel()].copy_(b)
+
+    def step(self, pos, host_in, host_out):
+        rc = self._step(self.handle, pos, host_in.data_ptr(), host_out.data_ptr())
+        if rc != DMS_OK:
+            _check(rc, "dms_stepper_step")
+
+    def join(self, stream=None):
+        dms_stepper_join(self.handle, _stream(stream))
+
+    def close(self):
+        if self.handle:
+            dms_stepper_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

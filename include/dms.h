@@ -238,6 +238,65 @@ dms_status dms_decode_attn_layers_noalloc(dms_pool* pool, int layer0, int n_laye
                                           const void* q, dms_dtype q_dtype, void* out,
                                           float sm_scale, cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Decode steps fed from host memory
+ *
+ * A stepper runs whole decode steps (dms_append_evict_layers, then
+ * dms_decode_attn_layers over the same layers) on inputs that live in host
+ * memory, and copies each step's output back to host memory.  Every step
+ * is one packed host->device copy, the two kernels and one device->host
+ * copy; the copies run on two streams of the stepper's own, double-buffered
+ * against the caller's compute stream, so the copies of one step overlap
+ * the kernels of its neighbours.  The pages have no counterpart: this is the
+ * serving-side plumbing around the method's decode step.
+ * ------------------------------------------------------------------------ */
+typedef struct dms_stepper dms_stepper;  /* opaque host handle */
+
+/* Packed host input of one step: four segments, each starting at a
+ * multiple of 256 bytes,
+ *   k      [n_layers, batch, Hkv, D]  in dtype (DMS_F32 for an F32 pool,
+ *   v      [n_layers, batch, Hkv, D]   else DMS_BF16)
+ *   q      [n_layers, batch, Hq, D]   same dtype
+ *   evict  [n_layers, batch, Hkv]     uint8
+ * The host output of one step is out [n_layers, batch, Hq, D] (q's dtype). */
+typedef struct {
+  size_t k, v, q, evict;  /* byte offsets of the segments */
+  size_t in_bytes;        /* bytes of one packed host input */
+  size_t out_bytes;       /* bytes of one host output */
+  size_t device_bytes;    /* device buffer dms_stepper_create needs */
+} dms_stepper_layout_t;
+
+dms_status dms_stepper_layout(const dms_pool* pool, int n_layers, int batch,
+                              dms_stepper_layout_t* out);
+
+/* Create a stepper for layers [layer0, layer0 + n_layers) and sequences
+ * 0..batch-1 of the pool.  device_buf (>= layout.device_bytes, 256-byte
+ * aligned, owned by the caller, no initialisation) holds two input staging
+ * buffers, two output buffers and the attention workspace.  `stream` is
+ * the compute stream the kernels run on; the stepper creates two copy
+ * streams and its events (no device memory).  The pool's device must be
+ * current.  sm_scale as for dms_decode_attn_layers. */
+dms_status dms_stepper_create(dms_pool* pool, int layer0, int n_layers, int batch,
+                              float sm_scale, void* device_buf, size_t device_bytes,
+                              cudaStream_t stream, dms_stepper** out);
+
+/* Enqueue the decode step at position pos: host_in (layout.in_bytes, host)
+ * -> device, append/evict + decode attention, output -> host_out
+ * (layout.out_bytes, host).  Returns at once.  Both host buffers should be
+ * page-locked (pinned) for the copies to be asynchronous, must stay valid
+ * and unchanged (host_in) / unread (host_out) until the step has finished
+ * (dms_stepper_join, then synchronise).  Positions follow the rules of
+ * dms_append_evict_layers. */
+dms_status dms_stepper_step(dms_stepper* st, int64_t pos, const void* host_in, void* host_out);
+
+/* Make `stream` wait for every step enqueued so far, output copies
+ * included. */
+dms_status dms_stepper_join(dms_stepper* st, cudaStream_t stream);
+
+/* Wait for the stepper's work, then release its streams, events and the
+ * host handle (device_buf stays the caller's). */
+dms_status dms_stepper_destroy(dms_stepper* st);
+
 /* Reduce the pool's counters on the device and copy them to *out (host).
  * Synchronises `stream`.  Returns DMS_ERR_DEVICE when the error word is
  * non-zero (*out is filled either way).  Source: real allocator memory,

@@ -203,6 +203,37 @@ def test_split_heads_merge_across_many_ctas():
     assert np.abs(got - exp).max() < TOL["bf16"]
 
 
+def test_many_short_heads_in_one_call():
+    """2 layers x 360 sequences x 8 kv-heads = 5760 heads of ~1-2 blocks in
+    one call: every CTA's range crosses dozens of heads, and the per-thread
+    head scan covers ~26 heads per thread; sampled sequences of both layers
+    match the oracle."""
+    L, B, Hq, Hkv, D, P, w = 2, 360, 8, 8, 128, 90, 16
+    pool = dms.Pool(L, B, Hq, Hkv, D, w, dms.DMS_BF16, L * B * Hkv * 3, P + 2)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).cuda()  # noqa: E731
+    data = []
+    for layer in range(L):
+        K = synth.kv_tokens(31, 0, layer, B, 0, P + 1, Hkv, D, "bf16")
+        V = synth.kv_tokens(31, 1, layer, B, 0, P + 1, Hkv, D, "bf16")
+        fl = synth.flag_tokens(31, layer, B, 0, P + 1, Hkv, [synth.keep_threshold(0.4)] * Hkv)
+        pool.compact_prefill(layer, dev(K[:, :P]), dev(V[:, :P]), torch.from_numpy(fl[:, :P].copy()).cuda())
+        data.append((K, V, fl))
+    kn = np.stack([d[0][:, P] for d in data])
+    vn = np.stack([d[1][:, P] for d in data])
+    fn = np.stack([d[2][:, P] for d in data])
+    pool.append_evict_layers(0, P, dev(kn), dev(vn), torch.from_numpy(fn.copy()).cuda())
+    Q = np.stack([synth.q_tokens(31, layer, B, P, Hq, D, "bf16") for layer in range(L)])
+    out = torch.empty(L, B, Hq, D, dtype=torch.bfloat16, device="cuda")
+    pool.decode_attn_layers(0, dev(Q), out)
+    got = out.float().cpu().numpy()
+    for layer in range(L):
+        K, V, fl = data[layer]
+        for b in (0, 1, 179, 358, 359):
+            exp = oatt.decode_attention(Q[layer, b].astype(np.float64), K[b], V[b], fl[b], P, w)
+            assert np.abs(got[layer, b] - exp).max() < TOL["bf16"], (layer, b)
+    assert read_state(pool)["error"] == 0
+
+
 def test_fp8_store_small():
     """FP8-E4M3 store: scales bit-exact, stored codes bit-exact, outputs within 6e-2."""
     B, Hkv, P, S, w, D = 2, 2, 500, 40, 64, 128
