@@ -298,7 +298,9 @@ def main():
     R = min(K, 64)                 # instrumented steps for the attention-kernel timing
     assert W >= 3 and K >= 1
     dw = DeviceWorkload(wl, W + K + R + E, device=f"cuda:{local}")
-    dw.prefill()
+    compact_ms_layers = dw.prefill(timed=True)
+    # median layer: the first call of each kernel also pays its module load
+    compact_ms = float(np.median(compact_ms_layers)) * len(compact_ms_layers)
     torch.cuda.synchronize()
 
     L, B, Hkv, D, w, P = wl.n_layers, wl.batch, wl.n_kv_heads, wl.head_dim, wl.window, wl.prompt
@@ -312,6 +314,17 @@ def main():
     retired = fl.sum(dim=(0, 1, 3)).cpu().numpy().astype(np.int64) if fl is not None else \
         np.zeros(NT, np.int64)
     base = int(dw.pool.stats().retained_tokens)
+    # compaction (prefill) bytes: flags + kept rows read in input precision and
+    # written in the store's precision (+ every prompt row once more for the
+    # FP8 scale pass)
+    in_row = 2 * D * (4 if wl.in_dtype == "f32" else 2)
+    compact_bytes = L * B * P * Hkv + base * (in_row + row_bytes)
+    if wl.kv_dtype == "fp8":
+        compact_bytes += L * B * P * Hkv * in_row
+    compaction = {"value": compact_bytes / (compact_ms * 1e-3) / 1e9, "unit": "GB/s",
+                  "ms_per_layer": compact_ms / L, "algorithmic_bytes_per_layer": compact_bytes / L,
+                  "timing": "CUDA events around each layer's dms_compact_prefill call (count, plan "
+                            "and scatter kernels); median layer"}
     held = base + np.cumsum(H - retired)                  # after step s
     bytes_step = held.astype(np.float64) * row_bytes
 
@@ -320,36 +333,48 @@ def main():
         dw.step(s)
     torch.cuda.synchronize()
 
-    # ---- device-timed region: exactly K steps, nothing between the kernels ----
+    # ---- device-timed region: exactly K steps, captured once into a CUDA graph
+    # (so host issue time cannot leave the GPU idle between kernels) and
+    # replayed once; positions advance every step, so each graph runs once ----
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     si = dw.step_inputs
-    with ClockSampler(local) as clk:
-        barrier()
-        torch.cuda.synchronize()
-        t_start.record(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
         for j in range(K):
             s = W + j
             dw.pool.append_evict_layers(0, P + s, si["k"][s], si["v"][s], si["evict"][s])
             dw.pool.decode_attn_layers(0, si["q"][s], dw.out)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        graph.replay()
         t_end.record(stream)
         torch.cuda.synchronize()
         barrier()
     ms = t_start.elapsed_time(t_end)
+    del graph
 
-    # ---- the attention kernel alone: a second pass of R steps with CUDA events
-    # around each attention launch (events between the kernels stop the
-    # programmatic overlap of append and attention, so the headline pass above
-    # carries none) ----
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(R)]
+    # ---- the attention kernel alone: a second graph of R steps with event
+    # nodes around each attention launch (an event between the kernels stops
+    # the programmatic overlap of append and attention, so the headline graph
+    # above carries none) ----
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(R)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for j in range(R):
+            s = W + K + j
+            dw.pool.append_evict_layers(0, P + s, si["k"][s], si["v"][s], si["evict"][s])
+            ev[j][0].record()
+            dw.pool.decode_attn_layers(0, si["q"][s], dw.out)
+            ev[j][1].record()
     torch.cuda.synchronize()
-    for j in range(R):
-        s = W + K + j
-        dw.pool.append_evict_layers(0, P + s, si["k"][s], si["v"][s], si["evict"][s])
-        ev[j][0].record(stream)
-        dw.pool.decode_attn_layers(0, si["q"][s], dw.out)
-        ev[j][1].record(stream)
+    graph.replay()
     torch.cuda.synchronize()
     attn_ms = np.array([a.elapsed_time(b) for a, b in ev])
+    del graph
     st = dw.pool.stats()
     if st.error_flags:
         raise SystemExit(f"device error word 0x{st.error_flags:x}")
@@ -370,8 +395,8 @@ def main():
                 "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "algorithmic_bytes_per_launch": float(rbytes.mean()),
                 "attn_us_per_launch": float(attn_ms.mean() * 1e3),
-                "timed_launches": R, "timing": "CUDA events around each attention launch, "
-                                                "second pass of R steps on the launch stream"}
+                "timed_launches": R, "timing": "CUDA event nodes around each attention launch in "
+                                                "a captured graph of R steps, replayed once"}
 
     # ---- end to end through the C ABI from host memory: dms_stepper_step per
     # step (packed pinned input -> device, append/evict, attention, output ->
@@ -413,7 +438,8 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
-            "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": ms_max / K, "timing": "CUDA events around one replay of a captured graph "
+                                                 "of the K steps", "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.kv_dtype == "bf16" else wl.kv_dtype, "data": "synthetic",
             "config": {"workload": wl.name, "layers": L, "batch": B, "q_heads": wl.n_q_heads,
                        "kv_heads": Hkv, "head_dim": D, "prompt": P, "window": w, "kv_dtype": wl.kv_dtype,
@@ -421,7 +447,7 @@ def main():
                        "l2": (f"no flush: {bytes_step[W] / 1e6:.0f} MB of held K/V read per step "
                               f"> 126 MB L2")},
             "decode_steps_per_s": world * K / (ms_max * 1e-3),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "compaction": compaction,
             "gpu_launches": 2 * K, "clocks": clk.summary(),
             "kernels_per_step": ["append_evict_kernel (1 launch, all layers)",
                                  "decode_attn_kernel (1 launch, all layers)"],

@@ -17,9 +17,9 @@
 //   count    per (sequence, 256-token chunk, head): warp ballot + popcount
 //   plan     one CTA: per-head chunk prefix sums, block allocation in
 //            (sequence, head) order, block tables, counters, FP8 scales
-//   scatter  per (sequence, chunk): ranks by ballot/popcount + the chunk
-//            base give each kept row its slot; copy (or quantise) the row
-//            into its block, fill the window ring.
+//   scatter  per (sequence, kv-head, chunk): ranks by ballot/popcount +
+//            the chunk base give each kept row its slot; copy (or quantise)
+//            the row into its block, fill the window ring.
 #include "dms_internal.cuh"
 
 namespace dms {
@@ -227,91 +227,107 @@ __global__ void __launch_bounds__(256) prefill_fp8_clear_tail_kernel(PoolView v,
 }
 
 // ---------------------------------------------------------------------------
+// One CTA per (256-token chunk, kv-head, sequence).
 template <typename InT, bool FP8>
 __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int layer, int P,
-                                                              const InT* k, const InT* vv,
-                                                              const uint8_t* evict) {
+                                                              const InT* __restrict__ k,
+                                                              const InT* __restrict__ vv,
+                                                              const uint8_t* __restrict__ evict) {
+  constexpr int kBatchItems = 4;          // 16-byte copies in flight per thread
   __shared__ int s_kept[kPrefillChunk];   // chunk-local token index of each kept rank
   __shared__ int s_wcnt[8];
   if (!v.hdr->prefill_go) return;
-  const int b = blockIdx.y, chunk = blockIdx.x;
+  const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = chunk * kPrefillChunk + threadIdx.x;
   const int64_t in_row_elems = v.D;
-  for (int h = 0; h < v.Hkv; ++h) {
-    const int hd = v.head(layer, b, h);
-    const uint8_t f = j < P ? evict[(int64_t(b) * P + j) * v.Hkv + h] : 0;
-    const bool keep = keep_token(j, P, v.w, f);
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) s_wcnt[warp] = __popc(m);
-    __syncthreads();
-    int before = 0, nkept = 0;
-    for (int q = 0; q < 8; ++q) {
-      before += q < warp ? s_wcnt[q] : 0;
-      nkept += s_wcnt[q];
+  const int hd = v.head(layer, b, h);
+  const uint8_t f = j < P ? evict[(int64_t(b) * P + j) * v.Hkv + h] : 0;
+  const bool keep = keep_token(j, P, v.w, f);
+  const unsigned m = __ballot_sync(0xffffffffu, keep);
+  if (lane == 0) s_wcnt[warp] = __popc(m);
+  __syncthreads();
+  int before = 0, nkept = 0;
+  for (int q = 0; q < 8; ++q) {
+    before += q < warp ? s_wcnt[q] : 0;
+    nkept += s_wcnt[q];
+  }
+  const int rank = before + __popc(m & ((1u << lane) - 1u));
+  const int base = v.chunk_counts[(int64_t(b) * v.Hkv + h) * v.n_chunks_max + chunk];
+  const int32_t* table = v.bt + int64_t(hd) * v.mbh;
+  if (keep) {
+    s_kept[rank] = threadIdx.x;
+    if (j >= P - v.w) {
+      const int slot = base + rank;
+      const int64_t ri = int64_t(hd) * v.w + (j % v.w);
+      v.ring[ri] = uint32_t(slot) | (uint32_t(f != 0) << 31);
+      v.ring_row[ri] = table[slot / v.BT] * v.BT + slot % v.BT;
     }
-    const int rank = before + __popc(m & ((1u << lane) - 1u));
-    const int base = v.chunk_counts[(int64_t(b) * v.Hkv + h) * v.n_chunks_max + chunk];
-    if (keep) {
-      s_kept[rank] = threadIdx.x;
-      if (j >= P - v.w) {
-        const int slot = base + rank;
-        const int64_t ri = int64_t(hd) * v.w + (j % v.w);
-        v.ring[ri] = uint32_t(slot) | (uint32_t(f != 0) << 31);
-        v.ring_row[ri] = v.bt[int64_t(hd) * v.mbh + slot / v.BT] * v.BT + slot % v.BT;
-      }
-    }
-    __syncthreads();
-    const int32_t* table = v.bt + int64_t(hd) * v.mbh;
-    if constexpr (!FP8) {
-      // bitwise row copy, 16-byte chunks, swizzled by row
-      const int nch = int(v.row_bytes >> 4);
-      for (int i = threadIdx.x; i < nkept * nch; i += blockDim.x) {
-        const int kk = i / nch, c = i % nch;
-        const int jj = chunk * kPrefillChunk + s_kept[kk];
-        const int slot = base + kk;
-        const int row = slot % v.BT;
-        if (!DMS_CHECK(slot < v.mbh * v.BT && table[slot / v.BT] >= 0 &&
-                       table[slot / v.BT] < v.max_blocks, v.hdr, 201, hd, slot))
-          continue;
-        uint8_t* blk = v.blocks + int64_t(table[slot / v.BT]) * v.block_bytes;
-        const int64_t src_off = ((int64_t(b) * P + jj) * v.Hkv + h) * v.row_bytes + c * 16;
-        const int64_t dst_off = int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;
-        const uint4 xk = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(k) + src_off);
-        const uint4 xv = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vv) + src_off);
-        *reinterpret_cast<uint4*>(blk + dst_off) = xk;
-        *reinterpret_cast<uint4*>(blk + v.tile_bytes + dst_off) = xv;
-      }
-    } else {
-      // FP8 (D = 128): each thread quantises 16 elements of one kept row
-      const float sK = v.scales[(int64_t(layer) * v.Hkv + h) * 2 + 0];
-      const float sV = v.scales[(int64_t(layer) * v.Hkv + h) * 2 + 1];
-      for (int i = threadIdx.x; i < nkept * 8; i += blockDim.x) {
-        const int kk = i >> 3, lc = i & 7;
-        const int jj = chunk * kPrefillChunk + s_kept[kk];
-        const int slot = base + kk;
-        const int row = slot % v.BT;
-        uint8_t* blk = v.blocks + int64_t(table[slot / v.BT]) * v.block_bytes;
-        const InT* srck = k + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
-        const InT* srcv = vv + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
-        uint8_t codes[16];
+  }
+  __syncthreads();
+  if constexpr (!FP8) {
+    // bitwise row copy in 16-byte chunks, swizzled by row; each thread loads
+    // kBatchItems K and V chunks before storing any
+    const int nch = int(v.row_bytes >> 4);
+    const int total = nkept * nch;
+    for (int i0 = 0; i0 < total; i0 += kBatchItems * blockDim.x) {
+      uint4 xk[kBatchItems], xv[kBatchItems];
+      uint8_t* dst[kBatchItems];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int pos = lc * 16 + e;
-          const int d = ((pos >> 2) & 7) * 16 + ((pos >> 1) & 1) * 8 + (pos >> 5) * 2 + (pos & 1);
-          codes[e] = f32_to_e4m3(__fdiv_rn(to_f32(srck[d]), sK));
+      for (int u = 0; u < kBatchItems; ++u) {
+        const int i = i0 + u * blockDim.x + threadIdx.x;
+        dst[u] = nullptr;
+        if (i < total) {
+          const int kk = i / nch, c = i % nch;
+          const int jj = chunk * kPrefillChunk + s_kept[kk];
+          const int slot = base + kk;
+          const int row = slot % v.BT;
+          if (DMS_CHECK(slot < v.mbh * v.BT && table[slot / v.BT] >= 0 &&
+                            table[slot / v.BT] < v.max_blocks, v.hdr, 201, hd, slot)) {
+            dst[u] = v.blocks + int64_t(table[slot / v.BT]) * v.block_bytes +
+                     int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;
+            const int64_t src_off = ((int64_t(b) * P + jj) * v.Hkv + h) * v.row_bytes + c * 16;
+            xk[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(k) + src_off));
+            xv[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vv) + src_off));
+          }
         }
-        *reinterpret_cast<uint4*>(blk + row * 128 + ((lc ^ (row & 7)) << 4)) =
-            *reinterpret_cast<const uint4*>(codes);
-        // V: elements d = lc*16 .. lc*16+15 of this token, transposed tile
+      }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int d = lc * 16 + e;
-          blk[v.tile_bytes + fp8v_byte(row, d)] = f32_to_e4m3(__fdiv_rn(to_f32(srcv[d]), sV));
+      for (int u = 0; u < kBatchItems; ++u) {
+        if (dst[u]) {
+          *reinterpret_cast<uint4*>(dst[u]) = xk[u];
+          *reinterpret_cast<uint4*>(dst[u] + v.tile_bytes) = xv[u];
         }
       }
     }
-    __syncthreads();
+  } else {
+    // FP8 (D = 128): each thread quantises 16 elements of one kept row
+    const float sK = v.scales[(int64_t(layer) * v.Hkv + h) * 2 + 0];
+    const float sV = v.scales[(int64_t(layer) * v.Hkv + h) * 2 + 1];
+    for (int i = threadIdx.x; i < nkept * 8; i += blockDim.x) {
+      const int kk = i >> 3, lc = i & 7;
+      const int jj = chunk * kPrefillChunk + s_kept[kk];
+      const int slot = base + kk;
+      const int row = slot % v.BT;
+      uint8_t* blk = v.blocks + int64_t(table[slot / v.BT]) * v.block_bytes;
+      const InT* srck = k + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
+      const InT* srcv = vv + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
+      uint8_t codes[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int pos = lc * 16 + e;
+        const int d = ((pos >> 2) & 7) * 16 + ((pos >> 1) & 1) * 8 + (pos >> 5) * 2 + (pos & 1);
+        codes[e] = f32_to_e4m3(__fdiv_rn(to_f32(srck[d]), sK));
+      }
+      *reinterpret_cast<uint4*>(blk + row * 128 + ((lc ^ (row & 7)) << 4)) =
+          *reinterpret_cast<const uint4*>(codes);
+      // V: elements d = lc*16 .. lc*16+15 of this token, transposed tile
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int d = lc * 16 + e;
+        blk[v.tile_bytes + fp8v_byte(row, d)] = f32_to_e4m3(__fdiv_rn(to_f32(srcv[d]), sV));
+      }
+    }
   }
 }
 
@@ -346,6 +362,10 @@ extern "C" dms_status dms_compact_prefill(dms_pool* pool, int layer, int batch, 
     set_last_error("k and v must be 16-byte aligned");
     return DMS_ERR_INVALID_ARG;
   }
+  if (batch > 65535) {
+    set_last_error("batch %d exceeds the 65535 sequences of one prefill launch", batch);
+    return DMS_ERR_UNSUPPORTED;
+  }
   const int n_chunks = (prompt_len + kPrefillChunk - 1) / kPrefillChunk;
   const dim3 grid(n_chunks, batch);
   dms_status st;
@@ -378,20 +398,21 @@ extern "C" dms_status dms_compact_prefill(dms_pool* pool, int layer, int batch, 
     st = cuda_status(cudaGetLastError(), "prefill_fp8_clear_tail_kernel");
     if (st != DMS_OK) return st;
   }
+  const dim3 sgrid(n_chunks, pv.Hkv, batch);
   if (in_dtype == DMS_BF16) {
     auto kk = static_cast<const __nv_bfloat16*>(k);
     auto vv = static_cast<const __nv_bfloat16*>(v);
     if (fp8)
-      prefill_scatter_kernel<__nv_bfloat16, true><<<grid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<__nv_bfloat16, true><<<sgrid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
     else
-      prefill_scatter_kernel<__nv_bfloat16, false><<<grid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<__nv_bfloat16, false><<<sgrid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
   } else {
     auto kk = static_cast<const float*>(k);
     auto vv = static_cast<const float*>(v);
     if (fp8)
-      prefill_scatter_kernel<float, true><<<grid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<float, true><<<sgrid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
     else
-      prefill_scatter_kernel<float, false><<<grid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<float, false><<<sgrid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
   }
   return cuda_status(cudaGetLastError(), "prefill_scatter_kernel");
 }

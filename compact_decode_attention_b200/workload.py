@@ -99,19 +99,33 @@ class DeviceWorkload:
         return {"k": k, "v": v, "q": q, "evict": e, "pos0": pos0}
 
     # ---- the path ---------------------------------------------------------
-    def prefill(self, layers=None):
-        """Compact every layer's prompt (inputs drawn on the device, one layer at a time)."""
+    def prefill(self, layers=None, timed=False):
+        """Compact every layer's prompt (inputs drawn on the device, one layer at a
+        time).  With timed=True, returns the device milliseconds of each layer's
+        compaction call alone (CUDA events around each dms_compact_prefill)."""
         t = self.torch
         P = self.wl.prompt
         kbuf = t.empty(1, self.batch, P, self.Hkv, self.D, dtype=self.in_dtype, device=self.device)
         vbuf = t.empty_like(kbuf)
         fbuf = t.empty(1, self.batch, P, self.Hkv, dtype=t.uint8, device=self.device)
+        events = []
+        stream = t.cuda.current_stream(self.device)
         for layer in (range(self.L) if layers is None else layers):
             self.normal(STREAM_K, layer, 1, 0, P, self.Hkv, out=kbuf)
             self.normal(STREAM_V, layer, 1, 0, P, self.Hkv, out=vbuf)
             self.flags(layer, 1, 0, P, out=fbuf)
+            if timed:
+                e = (t.cuda.Event(enable_timing=True), t.cuda.Event(enable_timing=True))
+                e[0].record(stream)
             self.pool.compact_prefill(layer, kbuf[0], vbuf[0], fbuf[0])
+            if timed:
+                e[1].record(stream)
+                events.append(e)
+        t.cuda.synchronize(self.device)
         del kbuf, vbuf, fbuf
+        if timed:
+            return [float(a.elapsed_time(b)) for a, b in events]
+        return None
 
     def step(self, s: int, out=None):
         """Decode step s (position prompt + s): append/evict all layers, then attention."""
