@@ -65,8 +65,9 @@ struct AttnTraits {
   static constexpr int THREADS = 32 * (NCW + 1);       // + one producer warp
   static constexpr int COMBINE_FLOATS = NCW * 8 * D + 2 * NCW * 8;
   static constexpr int MISC_INTS = 16 + THREADS / 32;
+  static constexpr int HEAD_WIN = 256;                 // held counts of the CTA's first heads
   static constexpr size_t SMEM = size_t(NS) * STAGEB + COMBINE_FLOATS * 4 + 2 * NS * 8 +
-                                 MISC_INTS * 4;
+                                 MISC_INTS * 4 + HEAD_WIN * 4;
   static_assert(NS % NCW == 0, "each stage must always belong to the same consumer warp");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(STAGEB % 128 == 0, "stage alignment");
@@ -535,6 +536,12 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   }
   __syncthreads();
   const int i0 = s_misc[1], p0 = s_misc[2];
+  // held counts of heads i0 .. i0 + HEAD_WIN - 1 in shared memory, so that the
+  // walks below need no dependent global loads (the scan just loaded them)
+  int* s_nwin = s_misc + T::MISC_INTS;
+  for (int i = max(hb, i0); i < min(he, i0 + T::HEAD_WIN); ++i) s_nwin[i - i0] = n_of(p, i);
+  __syncthreads();
+  auto n_at = [&](int i) { return i - i0 < T::HEAD_WIN ? s_nwin[i - i0] : n_of(p, i); };
   const int qrow_bytes = g * D * T::QESZ;
 
   if (warp == kNCW) {
@@ -543,7 +550,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     const uint64_t qpol = policy_evict_last();   // query rows: re-read per block
     int k = 0, issued = 0;
     bool aborted = false;
-    int i = i0, pp = p0, n = n_of(p, i0), nu = units_of(n);
+    int i = i0, pp = p0, n = n_at(i0), nu = units_of(n);
     for (int ub = u_beg; ub < u_end; ub += 32) {
       const int u = ub + lane;
       int mi = i, mp = pp, mn = n, mnu = nu;
@@ -552,7 +559,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
         while (u >= mp + mnu) {
           mp += mnu;
           ++mi;
-          mn = n_of(p, mi);
+          mn = n_at(mi);
           mnu = units_of(mn);
         }
         const int bi = u - mp;
@@ -620,7 +627,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   float* my_ow = s_ow + warp * 8 * D;
   float* my_mw = s_mw + warp * 8;
   float* my_lw = s_lw + warp * 8;
-  int i = i0, pp = p0, n = n_of(p, i0), nu = units_of(n);
+  int i = i0, pp = p0, n = n_at(i0), nu = units_of(n);
   bool have_q = false;
   auto set_head_scales = [&](int head_i) {
     st.scale = p.scale_log2;
@@ -638,7 +645,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     while (u >= pp + nu) {
       pp += nu;
       ++i;
-      n = n_of(p, i);
+      n = n_at(i);
       nu = units_of(n);
       set_head_scales(i);
     }
