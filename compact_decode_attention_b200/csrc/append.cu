@@ -39,10 +39,26 @@ constexpr int kAppendThreads = 32 * kAppendHeadsPerCta;
 // One warp per (layer, sequence, kv-head).  Lane 0 does the bookkeeping; all
 // lanes load the new K/V row first (it does not depend on the bookkeeping)
 // and store it once the destination is known.
+// Pop a block from the global free-block stack (blocks released by finished
+// sequences); -1 when it is empty.  Only pops run during an append, so a
+// successful compare-and-swap owns the entry below the old top.
+__device__ __forceinline__ int pop_free_block(const PoolView& v) {
+  int top = *reinterpret_cast<volatile int*>(&v.hdr->block_stack_top);
+  while (top > 0) {
+    const int prev = atomicCAS(&v.hdr->block_stack_top, top, top - 1);
+    if (prev == top) return v.block_stack[top - 1];
+    top = prev;
+  }
+  return -1;
+}
+
+// seq_ids (nullable): pool sequence of batch row b, else b.  pos_arr
+// (nullable): position of batch row b, else `pos` for every row.
 template <typename InT, bool FP8>
 __global__ void __launch_bounds__(kAppendThreads)
     append_evict_kernel(PoolView v, int l0, int nl, int batch, int64_t pos, const InT* k,
-                        const InT* vv, const uint8_t* evict) {
+                        const InT* vv, const uint8_t* evict, const int32_t* seq_ids,
+                        const int64_t* pos_arr) {
   // the new rows and the pool state may have been written by the kernel
   // before this one; once they are visible, let the next kernel (decode
   // attention) be scheduled
@@ -52,9 +68,15 @@ __global__ void __launch_bounds__(kAppendThreads)
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * kAppendHeadsPerCta + (threadIdx.x >> 5);
   if (i >= H) return;
-  const int h = i % v.Hkv, b = (i / v.Hkv) % batch, l = l0 + i / (v.Hkv * batch);
+  const int h = i % v.Hkv, bi = (i / v.Hkv) % batch, l = l0 + i / (v.Hkv * batch);
+  const int b = seq_ids ? seq_ids[bi] : bi;
+  const int64_t tpos = pos_arr ? pos_arr[bi] : pos;
+  if (b < 0 || b >= v.Bmax || tpos < 0 || tpos >= (int64_t(1) << 31)) {
+    if (lane == 0) report_error(v.hdr, DMS_DEVERR_BAD_SEQUENCE, l, bi, h);
+    return;
+  }
   const int hd = v.head(l, b, h);
-  const int t = int(pos);
+  const int t = int(tpos);
   const int64_t ri = int64_t(hd) * v.w + t % v.w;
 
   // ---- new rows into registers (bf16/fp32: 16-byte chunks, K then V) ----
@@ -99,8 +121,9 @@ __global__ void __launch_bounds__(kAppendThreads)
     } else if (ns / v.BT < v.mbh) {
       slot = ns;
       ns += 1;
-      if (slot % v.BT == 0) {  // the slot opens a new block: bump the block counter
-        const int id = atomicAdd(&v.hdr->next_block, 1);
+      if (slot % v.BT == 0) {  // the slot opens a new block: a released one, else a fresh one
+        int id = pop_free_block(v);
+        if (id < 0) id = atomicAdd(&v.hdr->next_block, 1);
         if (id < v.max_blocks) {
           v.bt[int64_t(hd) * v.mbh + slot / v.BT] = id;
           v.last_block[hd] = id;
@@ -181,10 +204,12 @@ __global__ void __launch_bounds__(kAppendThreads)
 
 using namespace dms;
 
-extern "C" dms_status dms_append_evict_layers(dms_pool* pool, int layer0, int n_layers, int batch,
-                                              int64_t pos, const void* k, const void* v,
-                                              dms_dtype in_dtype, const uint8_t* evict,
-                                              cudaStream_t stream) {
+// Checks shared by the entry points, then one launch over n_layers x batch
+// heads.  seq_ids / pos_arr are device arrays or null.
+static dms_status launch_append(dms_pool* pool, int layer0, int n_layers, int batch, int64_t pos,
+                                const void* k, const void* v, dms_dtype in_dtype,
+                                const uint8_t* evict, const int32_t* seq_ids,
+                                const int64_t* pos_arr, cudaStream_t stream) {
   if (!pool) {
     set_last_error("null pool");
     return DMS_ERR_INVALID_ARG;
@@ -215,7 +240,7 @@ extern "C" dms_status dms_append_evict_layers(dms_pool* pool, int layer0, int n_
 #define DMS_LAUNCH_APPEND(T, F)                                                                   \
   st = cuda_status(launch_pdl(append_evict_kernel<T, F>, grid, dim3(kAppendThreads), 0, stream,  \
                               pv, layer0, n_layers, batch, pos, static_cast<const T*>(k),         \
-                              static_cast<const T*>(v), evict),                                   \
+                              static_cast<const T*>(v), evict, seq_ids, pos_arr),                 \
                    "append_evict_kernel")
   if (in_dtype == DMS_BF16) {
     if (fp8) DMS_LAUNCH_APPEND(__nv_bfloat16, true);
@@ -226,6 +251,27 @@ extern "C" dms_status dms_append_evict_layers(dms_pool* pool, int layer0, int n_
   }
 #undef DMS_LAUNCH_APPEND
   return st;
+}
+
+extern "C" dms_status dms_append_evict_layers(dms_pool* pool, int layer0, int n_layers, int batch,
+                                              int64_t pos, const void* k, const void* v,
+                                              dms_dtype in_dtype, const uint8_t* evict,
+                                              cudaStream_t stream) {
+  return launch_append(pool, layer0, n_layers, batch, pos, k, v, in_dtype, evict, nullptr, nullptr,
+                       stream);
+}
+
+extern "C" dms_status dms_append_evict_seqs(dms_pool* pool, int layer0, int n_layers, int n_seqs,
+                                            const int32_t* seq_ids, const int64_t* pos,
+                                            const void* k, const void* v, dms_dtype in_dtype,
+                                            const uint8_t* evict, cudaStream_t stream) {
+  if (!seq_ids || !pos || (reinterpret_cast<uintptr_t>(pos) & 7) ||
+      (reinterpret_cast<uintptr_t>(seq_ids) & 3)) {
+    set_last_error("seq_ids and pos must be non-null, 4- and 8-byte aligned device arrays");
+    return DMS_ERR_INVALID_ARG;
+  }
+  return launch_append(pool, layer0, n_layers, n_seqs, 0, k, v, in_dtype, evict, seq_ids, pos,
+                       stream);
 }
 
 extern "C" dms_status dms_append_evict(dms_pool* pool, int layer, int batch, int64_t pos,

@@ -81,6 +81,7 @@ struct AttnParams {
   float scale_log2;   // sm_scale * log2(e)
   float* ws_o;        // [(G + Htot) * g * D]
   float* ws_ml;       // [(G + Htot) * g * 2]
+  const int32_t* seq_ids;  // pool sequence of batch row b (device), or null: row b
   int G;
 };
 
@@ -92,14 +93,26 @@ __device__ __forceinline__ void consumer_bar() {
 
 __device__ __forceinline__ int units_of(int n) { return (n + kBlockTokens - 1) / kBlockTokens; }
 
-// head index i of the call -> pool head id
+// head index i of the call -> pool head id, or -1 for a sequence id out of range
 __device__ __forceinline__ int pool_head(const AttnParams& p, int i) {
   const int h = i % p.v.Hkv;
   const int lb = i / p.v.Hkv;  // li * batch + b
-  return p.v.head(p.l0 + lb / p.batch, lb % p.batch, h);
+  const int b = lb % p.batch;
+  const int seq = p.seq_ids ? p.seq_ids[b] : b;
+  if (seq < 0 || seq >= p.v.Bmax) return -1;
+  return p.v.head(p.l0 + lb / p.batch, seq, h);
 }
 
-__device__ __forceinline__ int n_of(const AttnParams& p, int i) { return p.v.n_slots[pool_head(p, i)]; }
+// held rows of call head i (a bad sequence id holds none and is reported)
+__device__ __forceinline__ int n_of(const AttnParams& p, int i) {
+  const int hd = pool_head(p, i);
+  if (hd < 0) {
+    report_error(p.v.hdr, DMS_DEVERR_BAD_SEQUENCE, p.l0 + (i / p.v.Hkv) / p.batch, (i / p.v.Hkv) % p.batch,
+                 i % p.v.Hkv);
+    return 0;
+  }
+  return p.v.n_slots[hd];
+}
 
 // CTA whose unit range holds unit u (U units cut into G ranges).
 __device__ __forceinline__ int cta_of(int64_t u, int64_t U, int G) {
@@ -687,7 +700,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
       const bool whole = cf == cl;
       const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
       const int pid = c + i;
-      DMS_CHECK(i < Htot && pid < G + Htot && cf >= 0 && cl < Geff, v.hdr, 303, i, pid);
+      (void)DMS_CHECK(i < Htot && pid < G + Htot && cf >= 0 && cl < Geff, v.hdr, 303, i, pid);
       for (int idx = tid; idx < g * D; idx += kCons) {
         const int nn = idx / D, d = idx % D;
         float M = -INFINITY;
@@ -773,6 +786,34 @@ static size_t attn_workspace_bytes(const dms_pool* pool, int n_layers, int batch
   return o_bytes + parts * g * 2 * 4;
 }
 
+// Fill the kernel parameters and launch (arguments already checked).
+static dms_status run_attn(dms_pool* pool, int layer0, int n_layers, int batch, const void* q,
+                           void* out, float sm_scale, void* ws, const int32_t* seq_ids,
+                           cudaStream_t stream) {
+  const PoolView& v = pool->view;
+  const int g = v.Hq / v.Hkv;
+  const size_t parts = size_t(pool->sm_count) + size_t(n_layers) * batch * v.Hkv;
+  AttnParams prm;
+  prm.v = v;
+  prm.l0 = layer0;
+  prm.nl = n_layers;
+  prm.batch = batch;
+  prm.q = static_cast<const uint8_t*>(q);
+  prm.out = static_cast<uint8_t*>(out);
+  const float sc = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf(float(v.D));
+  prm.scale_log2 = sc * 1.4426950408889634f;
+  prm.ws_o = static_cast<float*>(ws);
+  prm.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                       ((parts * g * v.D * 4 + 255) & ~size_t(255)));
+  prm.seq_ids = seq_ids;
+  prm.G = pool->sm_count;
+  if (v.kv_dtype == DMS_BF16) {
+    return v.D == 128 ? launch_attn<KV_BF16, 128>(prm, stream) : launch_attn<KV_BF16, 64>(prm, stream);
+  }
+  if (v.kv_dtype == DMS_FP8_E4M3) return launch_attn<KV_FP8, 128>(prm, stream);
+  return v.D == 128 ? launch_attn<KV_F32, 128>(prm, stream) : launch_attn<KV_F32, 64>(prm, stream);
+}
+
 extern "C" dms_status dms_decode_workspace_bytes(const dms_pool* pool, int n_layers, int batch,
                                                  size_t* bytes) {
   if (!pool || !bytes || n_layers < 1 || batch < 1) {
@@ -783,10 +824,10 @@ extern "C" dms_status dms_decode_workspace_bytes(const dms_pool* pool, int n_lay
   return DMS_OK;
 }
 
-extern "C" dms_status dms_decode_attn_layers(dms_pool* pool, int layer0, int n_layers, int batch,
-                                             const void* q, dms_dtype q_dtype, void* out,
-                                             float sm_scale, void* workspace,
-                                             size_t workspace_bytes, cudaStream_t stream) {
+static dms_status decode_attn_checked(dms_pool* pool, int layer0, int n_layers, int batch,
+                                      const void* q, dms_dtype q_dtype, void* out, float sm_scale,
+                                      void* workspace, size_t workspace_bytes,
+                                      const int32_t* seq_ids, cudaStream_t stream) {
   if (!pool) {
     set_last_error("null pool");
     return DMS_ERR_INVALID_ARG;
@@ -814,26 +855,27 @@ extern "C" dms_status dms_decode_attn_layers(dms_pool* pool, int layer0, int n_l
     set_last_error("workspace has %zu bytes, needs %zu", workspace_bytes, need);
     return DMS_ERR_CAPACITY;
   }
-  const int g = v.Hq / v.Hkv;
-  const size_t parts = size_t(pool->sm_count) + size_t(n_layers) * batch * v.Hkv;
-  AttnParams prm;
-  prm.v = v;
-  prm.l0 = layer0;
-  prm.nl = n_layers;
-  prm.batch = batch;
-  prm.q = static_cast<const uint8_t*>(q);
-  prm.out = static_cast<uint8_t*>(out);
-  const float sc = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf(float(v.D));
-  prm.scale_log2 = sc * 1.4426950408889634f;
-  prm.ws_o = static_cast<float*>(workspace);
-  prm.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                       ((parts * g * v.D * 4 + 255) & ~size_t(255)));
-  prm.G = pool->sm_count;
-  if (v.kv_dtype == DMS_BF16) {
-    return v.D == 128 ? launch_attn<KV_BF16, 128>(prm, stream) : launch_attn<KV_BF16, 64>(prm, stream);
+  return run_attn(pool, layer0, n_layers, batch, q, out, sm_scale, workspace, seq_ids, stream);
+}
+
+extern "C" dms_status dms_decode_attn_layers(dms_pool* pool, int layer0, int n_layers, int batch,
+                                             const void* q, dms_dtype q_dtype, void* out,
+                                             float sm_scale, void* workspace,
+                                             size_t workspace_bytes, cudaStream_t stream) {
+  return decode_attn_checked(pool, layer0, n_layers, batch, q, q_dtype, out, sm_scale, workspace,
+                             workspace_bytes, nullptr, stream);
+}
+
+extern "C" dms_status dms_decode_attn_seqs(dms_pool* pool, int layer0, int n_layers, int n_seqs,
+                                           const int32_t* seq_ids, const void* q, dms_dtype q_dtype,
+                                           void* out, float sm_scale, void* workspace,
+                                           size_t workspace_bytes, cudaStream_t stream) {
+  if (!seq_ids || (reinterpret_cast<uintptr_t>(seq_ids) & 3)) {
+    set_last_error("seq_ids must be a non-null, 4-byte aligned device array");
+    return DMS_ERR_INVALID_ARG;
   }
-  if (v.kv_dtype == DMS_FP8_E4M3) return launch_attn<KV_FP8, 128>(prm, stream);
-  return v.D == 128 ? launch_attn<KV_F32, 128>(prm, stream) : launch_attn<KV_F32, 64>(prm, stream);
+  return decode_attn_checked(pool, layer0, n_layers, n_seqs, q, q_dtype, out, sm_scale, workspace,
+                             workspace_bytes, seq_ids, stream);
 }
 
 extern "C" dms_status dms_decode_attn(dms_pool* pool, int layer, int batch, const void* q,
@@ -940,25 +982,6 @@ extern "C" dms_status dms_decode_attn_layers_noalloc(dms_pool* pool, int layer0,
   void* ws = nullptr;
   st = static_workspace_address(dev, &ws);
   if (st != DMS_OK) return st;
-  const int g = v.Hq / v.Hkv;
-  const size_t parts = size_t(pool->sm_count) + size_t(n_layers) * batch * v.Hkv;
-  AttnParams prm;
-  prm.v = v;
-  prm.l0 = layer0;
-  prm.nl = n_layers;
-  prm.batch = batch;
-  prm.q = static_cast<const uint8_t*>(q);
-  prm.out = static_cast<uint8_t*>(out);
-  const float sc = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf(float(v.D));
-  prm.scale_log2 = sc * 1.4426950408889634f;
-  prm.ws_o = static_cast<float*>(ws);
-  prm.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                       ((parts * g * v.D * 4 + 255) & ~size_t(255)));
-  prm.G = pool->sm_count;
-  if (v.kv_dtype == DMS_BF16) {
-    return v.D == 128 ? launch_attn<KV_BF16, 128>(prm, stream) : launch_attn<KV_BF16, 64>(prm, stream);
-  }
-  if (v.kv_dtype == DMS_FP8_E4M3) return launch_attn<KV_FP8, 128>(prm, stream);
-  return v.D == 128 ? launch_attn<KV_F32, 128>(prm, stream) : launch_attn<KV_F32, 64>(prm, stream);
+  return run_attn(pool, layer0, n_layers, batch, q, out, sm_scale, ws, nullptr, stream);
 }
 

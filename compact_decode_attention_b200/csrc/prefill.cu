@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(256) prefill_count_kernel(PoolView v, int P, c
 
 // ---------------------------------------------------------------------------
 // One CTA of 1024 threads.  s_n holds the kept count of each (b, h) pair.
-__global__ void __launch_bounds__(1024) prefill_plan_kernel(PoolView v, int layer, int batch, int P) {
+__global__ void __launch_bounds__(1024) prefill_plan_kernel(PoolView v, int layer, int seq0, int batch,
+                                                            int P) {
   extern __shared__ int s_n[];   // [batch * Hkv] kept counts, then block prefix
   __shared__ int s_fail;
   __shared__ int s_warp[32];
@@ -101,12 +102,12 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(PoolView v, int laye
     v.hdr->prefill_go = 0;
   }
   __syncthreads();
-  // the layer must be empty
+  // the target sequences of the layer must be empty
   for (int p = tid; p < pairs; p += blockDim.x) {
-    const int hd = v.head(layer, p / v.Hkv, p % v.Hkv);
+    const int hd = v.head(layer, seq0 + p / v.Hkv, p % v.Hkv);
     if (v.n_slots[hd] != 0 || v.n_retained[hd] != 0) {
       atomicExch(&s_fail, 1);
-      report_error(v.hdr, DMS_DEVERR_LAYER_NOT_EMPTY, layer, p / v.Hkv, p % v.Hkv);
+      report_error(v.hdr, DMS_DEVERR_LAYER_NOT_EMPTY, layer, seq0 + p / v.Hkv, p % v.Hkv);
     }
   }
   __syncthreads();
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(PoolView v, int laye
       const int nb = p < pairs ? (s_n[p] + v.BT - 1) / v.BT : 0;
       if (p < pairs && nb > v.mbh) {
         atomicExch(&s_fail, 1);
-        report_error(v.hdr, DMS_DEVERR_HEAD_TABLE_FULL, layer, p / v.Hkv, p % v.Hkv);
+        report_error(v.hdr, DMS_DEVERR_HEAD_TABLE_FULL, layer, seq0 + p / v.Hkv, p % v.Hkv);
       }
       int incl = nb;
       for (int o = 1; o < 32; o <<= 1) {
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(PoolView v, int laye
   const int next = v.hdr->next_block;
   // block tables: allocation index a -> free stack top first, then bump
   for (int p = warp; p < pairs; p += nwarps) {
-    const int hd = v.head(layer, p / v.Hkv, p % v.Hkv);
+    const int hd = v.head(layer, seq0 + p / v.Hkv, p % v.Hkv);
     const int nb = (s_n[p] + v.BT - 1) / v.BT;
     for (int k = lane; k < nb; k += 32) {
       const int a = s_base[p] + k;
@@ -196,11 +197,14 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(PoolView v, int laye
     }
   }
   if (v.kv_dtype == DMS_FP8_E4M3) {
+    // the first prefill into a layer sets its scales (0 = not set yet); later
+    // prefills of other sequences reuse them, saturating like decode tokens
     for (int i = tid; i < 2 * v.Hkv; i += blockDim.x) {
       const float a = __uint_as_float(v.amax[i]);
       const float s = a > 0.f ? __fdiv_rn(a, 448.0f) : 1.0f;
       const int which = i / v.Hkv, h = i % v.Hkv;
-      v.scales[(int64_t(layer) * v.Hkv + h) * 2 + which] = s;
+      float* dst = v.scales + (int64_t(layer) * v.Hkv + h) * 2 + which;
+      if (*dst == 0.f) *dst = s;
     }
   }
   __syncthreads();
@@ -215,10 +219,10 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(PoolView v, int laye
 // FP8 only: clear the transposed V tile of each head's last, partly filled
 // block, so that token columns past n_slots decode to 0 (the attention kernel
 // reads whole V tiles).  One CTA per (sequence, kv-head).
-__global__ void __launch_bounds__(256) prefill_fp8_clear_tail_kernel(PoolView v, int layer) {
+__global__ void __launch_bounds__(256) prefill_fp8_clear_tail_kernel(PoolView v, int layer, int seq0) {
   if (!v.hdr->prefill_go) return;
   const int b = blockIdx.x / v.Hkv, h = blockIdx.x % v.Hkv;
-  const int hd = v.head(layer, b, h);
+  const int hd = v.head(layer, seq0 + b, h);
   const int n = v.n_slots[hd];
   if (n % v.BT == 0) return;
   uint8_t* blk = v.blocks + int64_t(v.bt[int64_t(hd) * v.mbh + n / v.BT]) * v.block_bytes;
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(256) prefill_fp8_clear_tail_kernel(PoolView v,
 // ---------------------------------------------------------------------------
 // One CTA per (256-token chunk, kv-head, sequence).
 template <typename InT, bool FP8>
-__global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int layer, int P,
+__global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int layer, int seq0, int P,
                                                               const InT* __restrict__ k,
                                                               const InT* __restrict__ vv,
                                                               const uint8_t* __restrict__ evict) {
@@ -241,7 +245,7 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = chunk * kPrefillChunk + threadIdx.x;
   const int64_t in_row_elems = v.D;
-  const int hd = v.head(layer, b, h);
+  const int hd = v.head(layer, seq0 + b, h);
   const uint8_t f = j < P ? evict[(int64_t(b) * P + j) * v.Hkv + h] : 0;
   const bool keep = keep_token(j, P, v.w, f);
   const unsigned m = __ballot_sync(0xffffffffu, keep);
@@ -338,14 +342,21 @@ using namespace dms;
 extern "C" dms_status dms_compact_prefill(dms_pool* pool, int layer, int batch, int prompt_len,
                                           const void* k, const void* v, dms_dtype in_dtype,
                                           const uint8_t* evict, cudaStream_t stream) {
+  return dms_compact_prefill_seqs(pool, layer, 0, batch, prompt_len, k, v, in_dtype, evict, stream);
+}
+
+extern "C" dms_status dms_compact_prefill_seqs(dms_pool* pool, int layer, int seq0, int batch,
+                                               int prompt_len, const void* k, const void* v,
+                                               dms_dtype in_dtype, const uint8_t* evict,
+                                               cudaStream_t stream) {
   if (!pool) {
     set_last_error("null pool");
     return DMS_ERR_INVALID_ARG;
   }
   const PoolView& pv = pool->view;
-  if (layer < 0 || layer >= pv.L || batch < 1 || batch > pv.Bmax || prompt_len < 0 ||
-      prompt_len > pool->cfg.max_context) {
-    set_last_error("bad layer/batch/prompt_len (%d, %d, %d)", layer, batch, prompt_len);
+  if (layer < 0 || layer >= pv.L || seq0 < 0 || batch < 1 || seq0 + batch > pv.Bmax ||
+      prompt_len < 0 || prompt_len > pool->cfg.max_context) {
+    set_last_error("bad layer/sequences/prompt_len (%d, %d+%d, %d)", layer, seq0, batch, prompt_len);
     return DMS_ERR_INVALID_ARG;
   }
   if (prompt_len == 0) return DMS_OK;
@@ -390,11 +401,11 @@ extern "C" dms_status dms_compact_prefill(dms_pool* pool, int layer, int batch, 
     set_last_error("batch * n_kv_heads too large for the prefill planner");
     return DMS_ERR_UNSUPPORTED;
   }
-  prefill_plan_kernel<<<1, 1024, plan_smem, stream>>>(pv, layer, batch, prompt_len);
+  prefill_plan_kernel<<<1, 1024, plan_smem, stream>>>(pv, layer, seq0, batch, prompt_len);
   st = cuda_status(cudaGetLastError(), "prefill_plan_kernel");
   if (st != DMS_OK) return st;
   if (fp8) {
-    prefill_fp8_clear_tail_kernel<<<batch * pv.Hkv, 256, 0, stream>>>(pv, layer);
+    prefill_fp8_clear_tail_kernel<<<batch * pv.Hkv, 256, 0, stream>>>(pv, layer, seq0);
     st = cuda_status(cudaGetLastError(), "prefill_fp8_clear_tail_kernel");
     if (st != DMS_OK) return st;
   }
@@ -403,16 +414,16 @@ extern "C" dms_status dms_compact_prefill(dms_pool* pool, int layer, int batch, 
     auto kk = static_cast<const __nv_bfloat16*>(k);
     auto vv = static_cast<const __nv_bfloat16*>(v);
     if (fp8)
-      prefill_scatter_kernel<__nv_bfloat16, true><<<sgrid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<__nv_bfloat16, true><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
     else
-      prefill_scatter_kernel<__nv_bfloat16, false><<<sgrid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<__nv_bfloat16, false><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
   } else {
     auto kk = static_cast<const float*>(k);
     auto vv = static_cast<const float*>(v);
     if (fp8)
-      prefill_scatter_kernel<float, true><<<sgrid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<float, true><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
     else
-      prefill_scatter_kernel<float, false><<<sgrid, 256, 0, stream>>>(pv, layer, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<float, false><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
   }
   return cuda_status(cudaGetLastError(), "prefill_scatter_kernel");
 }

@@ -28,6 +28,7 @@ DEVERR_FREE_STACK_FULL = 0x4
 DEVERR_TIMEOUT = 0x8
 DEVERR_LAYER_NOT_EMPTY = 0x10
 DEVERR_BOUNDS = 0x20
+DEVERR_BAD_SEQUENCE = 0x40
 
 BLOCK_TOKENS = 64
 
@@ -98,6 +99,10 @@ _SIGS = {
     "dms_decode_attn": (_I, [_P, _I, _I, _P, _I, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
     "dms_decode_attn_layers_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, ctypes.c_float, _P]),
     "dms_pool_stats": (_I, [_P, ctypes.POINTER(PoolStats), _P]),
+    "dms_compact_prefill_seqs": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P]),
+    "dms_append_evict_seqs": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P]),
+    "dms_decode_attn_seqs": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
+    "dms_release_seqs": (_I, [_P, _I, _P, _P]),
     "dms_stepper_layout": (_I, [_P, _I, _I, ctypes.POINTER(StepperLayout)]),
     "dms_stepper_create": (_I, [_P, _I, _I, _I, ctypes.c_float, _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
     "dms_stepper_step": (_I, [_P, _I64, _P, _P]),
@@ -216,6 +221,29 @@ def dms_pool_stats(pool: int, stream: int, check: bool = True) -> PoolStats:
     return st
 
 
+def dms_compact_prefill_seqs(pool: int, layer: int, seq0: int, batch: int, prompt_len: int, k: int,
+                             v: int, in_dtype: int, evict: int, stream: int):
+    _check(lib().dms_compact_prefill_seqs(pool, layer, seq0, batch, prompt_len, k, v, in_dtype, evict,
+                                          stream), "dms_compact_prefill_seqs")
+
+
+def dms_append_evict_seqs(pool: int, layer0: int, n_layers: int, n_seqs: int, seq_ids: int, pos: int,
+                          k: int, v: int, in_dtype: int, evict: int, stream: int):
+    _check(lib().dms_append_evict_seqs(pool, layer0, n_layers, n_seqs, seq_ids, pos, k, v, in_dtype,
+                                       evict, stream), "dms_append_evict_seqs")
+
+
+def dms_decode_attn_seqs(pool: int, layer0: int, n_layers: int, n_seqs: int, seq_ids: int, q: int,
+                         q_dtype: int, out: int, sm_scale: float, workspace: int, workspace_bytes: int,
+                         stream: int):
+    _check(lib().dms_decode_attn_seqs(pool, layer0, n_layers, n_seqs, seq_ids, q, q_dtype, out, sm_scale,
+                                      workspace, workspace_bytes, stream), "dms_decode_attn_seqs")
+
+
+def dms_release_seqs(pool: int, n_seqs: int, seq_ids: int, stream: int):
+    _check(lib().dms_release_seqs(pool, n_seqs, seq_ids, stream), "dms_release_seqs")
+
+
 def dms_stepper_layout(pool: int, n_layers: int, batch: int) -> StepperLayout:
     lay = StepperLayout()
     _check(lib().dms_stepper_layout(pool, n_layers, batch, ctypes.byref(lay)), "dms_stepper_layout")
@@ -329,6 +357,27 @@ class Pool:
         ws = self.workspace(nl, B, q.device)
         dms_decode_attn_layers(self.handle, layer0, nl, B, _ptr(q), torch_dtype_code(q.dtype),
                                _ptr(out), sm_scale, _ptr(ws), ws.numel(), _stream(stream))
+
+    # ---- continuous batching: sequence slots with their own positions ----
+    def compact_prefill_seqs(self, layer, seq0, k, v, evict, stream=None):
+        B, P = k.shape[0], k.shape[1]
+        dms_compact_prefill_seqs(self.handle, layer, seq0, B, P, _ptr(k), _ptr(v),
+                                 torch_dtype_code(k.dtype), _ptr(evict), _stream(stream))
+
+    def append_evict_seqs(self, layer0, seq_ids, pos, k, v, evict, stream=None):
+        """seq_ids int32 [n], pos int64 [n] (device); k, v [nl, n, Hkv, D]."""
+        nl, n = k.shape[0], k.shape[1]
+        dms_append_evict_seqs(self.handle, layer0, nl, n, _ptr(seq_ids), _ptr(pos), _ptr(k), _ptr(v),
+                              torch_dtype_code(k.dtype), _ptr(evict), _stream(stream))
+
+    def decode_attn_seqs(self, layer0, seq_ids, q, out, sm_scale=0.0, stream=None):
+        nl, n = q.shape[0], q.shape[1]
+        ws = self.workspace(nl, n, q.device)
+        dms_decode_attn_seqs(self.handle, layer0, nl, n, _ptr(seq_ids), _ptr(q), torch_dtype_code(q.dtype),
+                             _ptr(out), sm_scale, _ptr(ws), ws.numel(), _stream(stream))
+
+    def release_seqs(self, seq_ids, stream=None):
+        dms_release_seqs(self.handle, int(seq_ids.numel()), _ptr(seq_ids), _stream(stream))
 
     def stats(self, stream=None, check=True) -> PoolStats:
         return dms_pool_stats(self.handle, _stream(stream), check)

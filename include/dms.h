@@ -82,6 +82,7 @@ typedef enum { DMS_F32 = 0, DMS_BF16 = 1, DMS_FP8_E4M3 = 2 } dms_dtype;
 #define DMS_DEVERR_TIMEOUT          0x8u  /* a bounded wait gave up; outputs invalid     */
 #define DMS_DEVERR_LAYER_NOT_EMPTY  0x10u /* prefill into a layer that already holds data */
 #define DMS_DEVERR_BOUNDS           0x20u /* DMS_DEBUG builds: an index failed its check  */
+#define DMS_DEVERR_BAD_SEQUENCE     0x40u /* a device sequence id or position out of range; that head skipped */
 
 typedef struct {
   int32_t n_layers;
@@ -167,12 +168,65 @@ dms_status dms_pool_layout(const dms_pool* pool, dms_pool_layout_t* out);
  *   evict  [batch, P, Hkv]     uint8, non-zero = flagged
  * The layer must be empty (fresh pool or after dms_pool_reset), else the
  * device sets DMS_DEVERR_LAYER_NOT_EMPTY and writes nothing.  in_dtype
- * must equal kv_dtype, or be F32/BF16 for an FP8 pool.
+ * must equal kv_dtype, or be F32/BF16 for an FP8 pool.  (FP8: the scales
+ * are only set when the layer has none yet; see dms_compact_prefill_seqs.)
  * Source: compaction = the compact store of the FastDMS page; eviction
  * before FP8 quantisation = the same page's FP8 paragraph. */
 dms_status dms_compact_prefill(dms_pool* pool, int layer, int batch, int prompt_len,
                                const void* k, const void* v, dms_dtype in_dtype,
                                const uint8_t* evict, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Continuous batching.  Sequences start, decode and finish independently:
+ * each occupies one of the pool's max_batch sequence slots, has its own
+ * position, and on release gives its whole blocks back to the global
+ * free-block stack (the pool of per-head variable token counts of the
+ * FastDMS page, table "What's the catch?", row "PagedAttention / KV memory
+ * pool"; its memory figures count real allocator memory, paragraph before
+ * the memory table).  The calls below take device arrays so that a step can
+ * be captured in a CUDA graph; a sequence id or position out of range sets
+ * DMS_DEVERR_BAD_SEQUENCE and that head is skipped.
+ * ------------------------------------------------------------------------ */
+
+/* dms_compact_prefill for sequence slots [seq0, seq0 + batch) of a layer
+ * (inputs indexed 0..batch-1).  Those slots must be empty in that layer
+ * (fresh, reset, or released).  FP8: the first prefill into a layer sets
+ * its scales from the amax of its own rows; later prefills of other
+ * sequences of that layer reuse them and saturate, like decode tokens. */
+dms_status dms_compact_prefill_seqs(dms_pool* pool, int layer, int seq0, int batch,
+                                    int prompt_len, const void* k, const void* v,
+                                    dms_dtype in_dtype, const uint8_t* evict,
+                                    cudaStream_t stream);
+
+/* dms_append_evict_layers with a list of sequences, each at its own
+ * position: batch row r of k, v [n_layers, n_seqs, Hkv, D] and evict
+ * [n_layers, n_seqs, Hkv] is the token at position pos[r] of sequence slot
+ * seq_ids[r].  seq_ids int32 [n_seqs] and pos int64 [n_seqs] are device
+ * arrays; the ids must be distinct.  Each sequence's positions must
+ * increase by one per step from its prompt length.  A new block comes from
+ * the global free-block stack first (blocks of released sequences), then
+ * from the never-used tail of the pool. */
+dms_status dms_append_evict_seqs(dms_pool* pool, int layer0, int n_layers, int n_seqs,
+                                 const int32_t* seq_ids, const int64_t* pos, const void* k,
+                                 const void* v, dms_dtype in_dtype, const uint8_t* evict,
+                                 cudaStream_t stream);
+
+/* dms_decode_attn_layers over a list of sequences: row r of q, out
+ * [n_layers, n_seqs, Hq, D] belongs to sequence slot seq_ids[r] (int32
+ * device array).  Workspace as for dms_decode_attn_layers with batch =
+ * n_seqs. */
+dms_status dms_decode_attn_seqs(dms_pool* pool, int layer0, int n_layers, int n_seqs,
+                                const int32_t* seq_ids, const void* q, dms_dtype q_dtype,
+                                void* out, float sm_scale, void* workspace,
+                                size_t workspace_bytes, cudaStream_t stream);
+
+/* End sequences: for every layer and kv-head of the n_seqs sequence slots in
+ * seq_ids (int32 device array, distinct ids), push every block they hold on
+ * the global free-block stack and return their counters to empty, so the
+ * slots can be prefilled again and the blocks reused by any sequence.
+ * Calls that touch these sequences must be ordered before it. */
+dms_status dms_release_seqs(dms_pool* pool, int n_seqs, const int32_t* seq_ids,
+                            cudaStream_t stream);
 
 /* One decode step at position `pos` (= t) for layers [layer0, layer0 +
  * n_layers): for every (layer, b, h): if t >= w and token t-w was flagged,
