@@ -49,3 +49,19 @@ def decode_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, evict: np.ndar
         rows = slice(hkv * g, (hkv + 1) * g)
         out[rows] = attend(q[rows], K[vis, hkv], V[vis, hkv], sm_scale)
     return out
+
+
+def prefill_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, evict: np.ndarray, w: int,
+                      sm_scale: float | None = None) -> np.ndarray:
+    """Outputs of every prompt query of one sequence of one layer.
+
+    The delayed-eviction mask applies to every query, not only to decode
+    steps: query i sees key j <= i unless j is flagged and i - j >= w (the
+    same rule as decode_attention with t = i).
+    Q [P, Hq, D], K / V [P, Hkv, D], evict [P, Hkv] -> [P, Hq, D] fp64.
+    """
+    P = Q.shape[0]
+    out = np.zeros(Q.shape, dtype=np.float64)
+    for i in range(P):
+        out[i] = decode_attention(Q[i], K[:i + 1], V[:i + 1], evict[:i + 1], i, w, sm_scale)
+    return out

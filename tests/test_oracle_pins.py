@@ -127,6 +127,53 @@ def test_general_flags_match_sdpa_with_operational_mask():
         np.testing.assert_allclose(got, sdpa(q, K[:t + 1], V[:t + 1], 0.37, m), rtol=0, atol=1e-12)
 
 
+def sdpa_prefill(Q, K, V, scale, mask_):
+    """torch fp64 SDPA over all prompt queries: Q [P, Hq, D], K/V [P, Hkv, D],
+    mask_ [Hkv, P, P] boolean (query, key)."""
+    g = Q.shape[1] // K.shape[1]
+    qt = torch.from_numpy(np.asarray(Q, np.float64)).permute(1, 0, 2)[None]
+    Kt = torch.from_numpy(np.asarray(K, np.float64)).permute(1, 0, 2)[None]
+    Vt = torch.from_numpy(np.asarray(V, np.float64)).permute(1, 0, 2)[None]
+    am = torch.from_numpy(np.repeat(mask_, g, axis=0))[None]
+    out = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=am, scale=scale,
+                                                           enable_gqa=True)
+    return out[0].permute(1, 0, 2).numpy()
+
+
+def test_prefill_attention_matches_sdpa_with_operational_mask():
+    """Every prompt query, random flags: the oracle equals torch SDPA whose
+    (query, key) mask comes from the operational model's cache contents."""
+    rng = np.random.default_rng(11)
+    P, w, Hq, Hkv, D = 40, 6, 6, 3, 8
+    Q = rng.standard_normal((P, Hq, D))
+    _, K, V = rand_case(rng, P, Hq=Hq, Hkv=Hkv, D=D)
+    evict = (rng.random((P, Hkv)) < 0.6).astype(np.uint8)
+    m = np.zeros((Hkv, P, P), dtype=bool)
+    for h in range(Hkv):
+        for i, vis in enumerate(operational_cache_sets(evict[:, h], w)):
+            m[h, i, vis] = True
+    got = attention.prefill_attention(Q, K, V, evict, w, 0.41)
+    np.testing.assert_allclose(got, sdpa_prefill(Q, K, V, 0.41, m), rtol=0, atol=1e-12)
+
+
+def test_prefill_attention_endpoints():
+    """w >= P: plain causal attention (torch's is_causal); all flags and w = 1:
+    each query sees only itself, so the output is its own value row."""
+    rng = np.random.default_rng(12)
+    P, Hq, Hkv, D = 33, 4, 2, 8
+    Q = rng.standard_normal((P, Hq, D))
+    _, K, V = rand_case(rng, P, Hq=Hq, Hkv=Hkv, D=D)
+    flags = np.ones((P, Hkv), np.uint8)
+    got = attention.prefill_attention(Q, K, V, flags, P, 0.3)
+    qt = torch.from_numpy(Q).permute(1, 0, 2)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qt, torch.from_numpy(K).permute(1, 0, 2)[None], torch.from_numpy(V).permute(1, 0, 2)[None],
+        is_causal=True, scale=0.3, enable_gqa=True)[0].permute(1, 0, 2).numpy()
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    only_self = attention.prefill_attention(Q, K, V, flags, 1, 0.3)
+    np.testing.assert_allclose(only_self, np.repeat(V, Hq // Hkv, axis=1), rtol=0, atol=1e-12)
+
+
 def test_zero_keys_give_uniform_mean_of_visible_values():
     # flags on even positions, w = 3, t = 10: the visible set is the odd
     # positions plus the last three (8, 9, 10)
