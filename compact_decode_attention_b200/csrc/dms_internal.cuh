@@ -291,6 +291,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 dms_status cuda_status(cudaError_t e, const char* what);
 int device_sm_count(int device);
+}  // namespace dms
+struct dms_pool;
+namespace dms {
+dms_status prefill_plan_launch(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
+                               const uint8_t* evict, cudaStream_t stream);
 
 }  // namespace dms
 

@@ -339,6 +339,26 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
 
 using namespace dms;
 
+namespace dms {
+// Count kept tokens per 256-token chunk, then plan (prefix counts, block
+// tables, counters, FP8 scales); shared with the fused prefill attention.
+dms_status prefill_plan_launch(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
+                               const uint8_t* evict, cudaStream_t stream) {
+  const PoolView& pv = pool->view;
+  const int n_chunks = (prompt_len + kPrefillChunk - 1) / kPrefillChunk;
+  prefill_count_kernel<<<dim3(n_chunks, batch), 256, 0, stream>>>(pv, prompt_len, evict);
+  dms_status st = cuda_status(cudaGetLastError(), "prefill_count_kernel");
+  if (st != DMS_OK) return st;
+  const size_t plan_smem = sizeof(int) * (2 * size_t(batch) * pv.Hkv + 1);
+  if (plan_smem > 48 * 1024) {
+    set_last_error("batch * n_kv_heads too large for the prefill planner");
+    return DMS_ERR_UNSUPPORTED;
+  }
+  prefill_plan_kernel<<<1, 1024, plan_smem, stream>>>(pv, layer, seq0, batch, prompt_len);
+  return cuda_status(cudaGetLastError(), "prefill_plan_kernel");
+}
+}  // namespace dms
+
 extern "C" dms_status dms_compact_prefill(dms_pool* pool, int layer, int batch, int prompt_len,
                                           const void* k, const void* v, dms_dtype in_dtype,
                                           const uint8_t* evict, cudaStream_t stream) {
@@ -393,16 +413,7 @@ extern "C" dms_status dms_compact_prefill_seqs(dms_pool* pool, int layer, int se
     st = cuda_status(cudaGetLastError(), "prefill_amax_kernel");
     if (st != DMS_OK) return st;
   }
-  prefill_count_kernel<<<grid, 256, 0, stream>>>(pv, prompt_len, evict);
-  st = cuda_status(cudaGetLastError(), "prefill_count_kernel");
-  if (st != DMS_OK) return st;
-  const size_t plan_smem = sizeof(int) * (2 * size_t(batch) * pv.Hkv + 1);
-  if (plan_smem > 48 * 1024) {
-    set_last_error("batch * n_kv_heads too large for the prefill planner");
-    return DMS_ERR_UNSUPPORTED;
-  }
-  prefill_plan_kernel<<<1, 1024, plan_smem, stream>>>(pv, layer, seq0, batch, prompt_len);
-  st = cuda_status(cudaGetLastError(), "prefill_plan_kernel");
+  st = prefill_plan_launch(pool, layer, seq0, batch, prompt_len, evict, stream);
   if (st != DMS_OK) return st;
   if (fp8) {
     prefill_fp8_clear_tail_kernel<<<batch * pv.Hkv, 256, 0, stream>>>(pv, layer, seq0);

@@ -1,0 +1,389 @@
+// dms_prefill_attn: prompt attention under the DMS delayed-eviction mask,
+// fused with the compaction of the prompt into the compact store.
+//
+// The delayed-eviction rule holds for every query, prompt queries included:
+// query i sees key j <= i unless j is flagged and i - j >= w ("NVIDIA
+// veröffentlicht Qwen3-8B-DMS-8x ..." (mindverse), section "Dynamic Memory
+// Sparsification (DMS): Eine innovative Lösung"; "Nvidia DMS ..."
+// (stiva.ai), section "Ключевое изобретение: delayed eviction").  The keys
+// the last prompt query can see are exactly the rows the compact store keeps
+// ("FastDMS: vLLM BF16/FP8보다 빠른 6.4x KV cache 압축" (molayo1419.me),
+// opening paragraphs), so the kernel that streams the prompt's K/V tiles for
+// attention also writes the kept rows into their slots.
+//
+// One CTA of 4 warps per (128-query tile, query head, sequence), heaviest
+// (latest) query tiles first.  Per 128-key tile, on the 5th-generation
+// tensor cores with accumulators in tensor memory:
+//   S = Q K^T           (M = 128 queries, N = 128 keys, K = D)
+//   thread r owns query row r: masked online softmax on S[r] (tcgen05.ld),
+//   P[r] as bf16 into shared memory, O[r] rescaled in tensor memory when the
+//   row maximum moved
+//   O += P V            (M = 128 queries, N = D, K = 128 keys; V is staged
+//                        transposed so both operands are K-major)
+// Operands live in shared memory in the K-major 128-byte-swizzled layout of
+// umma.cuh.  The CTA of the first query head of each kv-head group writes,
+// at its diagonal key tile, the tile's kept rows into the pool (slots from
+// the prefix counts of the count and plan kernels) and the window ring.
+#include <math.h>
+
+#include "dms_internal.cuh"
+#include "umma.cuh"
+
+namespace dms {
+
+constexpr int kPaTile = 128;      // queries per CTA and keys per tile
+constexpr int kPaThreads = 128;   // one thread per query row
+
+template <int D>
+struct PaSmem {
+  static constexpr int Q = 0;                          // [128 x D] K-major
+  static constexpr int K = Q + kPaTile * D * 2;        // [128 keys x D]
+  static constexpr int VT = K + kPaTile * D * 2;       // [D x 128 keys]
+  static constexpr int P = VT + D * kPaTile * 2;       // [128 x 128 keys]
+  static constexpr int FLAGS = P + kPaTile * kPaTile * 2;
+  static constexpr int BARS = FLAGS + kPaTile;         // 2 mbarriers
+  static constexpr int MISC = BARS + 16;               // tmem base, scan
+  static constexpr int BYTES = MISC + 64 + 1024;       // + alignment slack
+};
+
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Rows [row0, row0 + 128) of one head of a [B, P, H, D] bf16 tensor into a
+// K-major swizzled tile; rows past P are zero.
+template <int D>
+__device__ __forceinline__ void load_rows(uint8_t* tile, const __nv_bfloat16* src, int64_t row_stride,
+                                          int row0, int P, int tid) {
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  for (int idx = tid; idx < kPaTile * CH; idx += kPaThreads) {
+    const int r = idx / CH, c = idx % CH;
+    uint4 x = make_uint4(0, 0, 0, 0);
+    if (row0 + r < P) x = __ldg(reinterpret_cast<const uint4*>(src + (row0 + r) * row_stride) + c);
+    *reinterpret_cast<uint4*>(tile + umma::sw128_offset(kPaTile, r, c * 8)) = x;
+  }
+}
+
+// V rows [row0, row0 + 128) transposed into a [D x 128 keys] K-major tile:
+// each thread takes two neighbouring keys and stores (v[r][d], v[r+1][d])
+// pairs as 32-bit words.
+template <int D>
+__device__ __forceinline__ void load_v_transposed(uint8_t* tile, const __nv_bfloat16* src,
+                                                  int64_t row_stride, int row0, int P, int tid) {
+  constexpr int CH = D / 8;
+  for (int idx = tid; idx < (kPaTile / 2) * CH; idx += kPaThreads) {
+    const int r = 2 * (idx / CH), c = idx % CH;
+    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+    if (row0 + r < P) a = __ldg(reinterpret_cast<const uint4*>(src + (row0 + r) * row_stride) + c);
+    if (row0 + r + 1 < P) b = __ldg(reinterpret_cast<const uint4*>(src + (row0 + r + 1) * row_stride) + c);
+    const __nv_bfloat16* va = reinterpret_cast<const __nv_bfloat16*>(&a);
+    const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(&b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      __nv_bfloat162 pr;
+      pr.x = va[e];
+      pr.y = vb[e];
+      *reinterpret_cast<__nv_bfloat162*>(tile + umma::sw128_offset(D, c * 8 + e, r)) = pr;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPaThreads, 1)
+    prefill_attn_kernel(PoolView v, int layer, int seq0, int P, const __nv_bfloat16* q,
+                        const __nv_bfloat16* k, const __nv_bfloat16* vv, const uint8_t* evict,
+                        __nv_bfloat16* out, float scale_log2, int n_qtiles, int compact) {
+  using S = PaSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qt = n_qtiles - 1 - int(blockIdx.x);  // heaviest query tiles first
+  const int hq = blockIdx.y, b = blockIdx.z;
+  const int g = v.Hq / v.Hkv, hkv = hq / g;
+  const int i0 = qt * kPaTile;
+  const int64_t q_stride = int64_t(v.Hq) * D, kv_stride = int64_t(v.Hkv) * D;
+  const __nv_bfloat16* qsrc = q + int64_t(b) * P * q_stride + int64_t(hq) * D;
+  const __nv_bfloat16* ksrc = k + int64_t(b) * P * kv_stride + int64_t(hkv) * D;
+  const __nv_bfloat16* vsrc = vv + int64_t(b) * P * kv_stride + int64_t(hkv) * D;
+  uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + S::BARS);
+  uint64_t* bar_o = bar_s + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::MISC);
+  int* s_scan = reinterpret_cast<int*>(smem + S::MISC) + 4;
+  uint8_t* s_flag = smem + S::FLAGS;
+
+  if (tid == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();  // tcgen05.alloc is warp-collective: lane 0 rejoins first
+  if (warp == 0) {
+    umma::tmem_alloc(s_tmem, 256);
+    umma::tmem_relinquish();
+  }
+  load_rows<D>(smem + S::Q, qsrc, q_stride, i0, P, tid);
+  umma::fence_before_sync();
+  __syncthreads();
+  umma::fence_after_sync();
+  const uint32_t tbase = *s_tmem;
+  const uint32_t t_s = tbase, t_o = tbase + kPaTile;
+  const uint32_t aQ = smem_u32(smem + S::Q), aK = smem_u32(smem + S::K);
+  const uint32_t aVT = smem_u32(smem + S::VT), aP = smem_u32(smem + S::P);
+  constexpr uint32_t idS = umma::idesc_bf16_f32(kPaTile, kPaTile);
+  constexpr uint32_t idO = umma::idesc_bf16_f32(kPaTile, D);
+  const int i = i0 + tid;  // this thread's query row
+  float m = -INFINITY, l = 0.f;
+  volatile int never = 0;
+  bool ok = true;
+
+  for (int kt = 0; kt <= qt; ++kt) {
+    const int j0 = kt * kPaTile;
+    if (kt > 0) {  // the previous P V product has finished with K, V^T and P
+      ok &= mbar_wait_bounded(bar_o, (kt - 1) & 1, &never);
+      __syncwarp();
+      umma::fence_after_sync();
+    }
+    load_rows<D>(smem + S::K, ksrc, kv_stride, j0, P, tid);
+    load_v_transposed<D>(smem + S::VT, vsrc, kv_stride, j0, P, tid);
+    {
+      const int j = j0 + tid;
+      s_flag[tid] = j < P ? evict[(int64_t(b) * P + j) * v.Hkv + hkv] : 1;
+    }
+    fence_proxy_async_smem();  // generic-proxy tile writes before the tensor cores read them
+    __syncthreads();
+    if (tid == 0) {
+      umma::fence_after_sync();
+#pragma unroll
+      for (int k0 = 0; k0 < D; k0 += 16)
+        umma::mma_bf16(t_s, umma::desc_k16(aQ, kPaTile, k0), umma::desc_k16(aK, kPaTile, k0), idS,
+                       k0 > 0);
+      umma::commit(bar_s);
+    }
+    ok &= mbar_wait_bounded(bar_s, kt & 1, &never);
+    __syncwarp();  // lanes leave the wait loop independently; tcgen05.ld is warp-collective
+    umma::fence_after_sync();
+
+    // ---- masked online softmax on query row i (log2 domain) ----
+    float s[kPaTile];
+#pragma unroll
+    for (int cb = 0; cb < kPaTile / 32; ++cb) {
+      float x[32];
+      umma::ld32(umma::taddr_of(t_s, warp, cb * 32), x);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) s[cb * 32 + e] = x[e];
+    }
+    umma::wait_ld();
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kPaTile; ++c) {
+      const int j = j0 + c;
+      const bool vis = j < P && j <= i && (s_flag[c] == 0 || i - j < v.w);
+      s[c] = vis ? s[c] * scale_log2 : -INFINITY;
+      mx = fmaxf(mx, s[c]);
+    }
+    const float mn = fmaxf(m, mx);
+    const float alpha = mn == -INFINITY ? 1.f : fast_exp2(m - mn);
+    float sum = 0.f;
+#pragma unroll
+    for (int c = 0; c < kPaTile; ++c) {
+      const float p = mn == -INFINITY ? 0.f : fast_exp2(s[c] - mn);
+      sum += p;
+      s[c] = p;
+    }
+    l = l * alpha + sum;
+    m = mn;
+#pragma unroll
+    for (int ch = 0; ch < kPaTile / 8; ++ch) {
+      uint4 w4;
+      w4.x = pack2_bf16(s[ch * 8 + 0], s[ch * 8 + 1]);
+      w4.y = pack2_bf16(s[ch * 8 + 2], s[ch * 8 + 3]);
+      w4.z = pack2_bf16(s[ch * 8 + 4], s[ch * 8 + 5]);
+      w4.w = pack2_bf16(s[ch * 8 + 6], s[ch * 8 + 7]);
+      *reinterpret_cast<uint4*>(smem + S::P + umma::sw128_offset(kPaTile, tid, ch * 8)) = w4;
+    }
+    // O row *= alpha when this warp has a row whose maximum moved
+    if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
+        float o[32];
+        umma::ld32(umma::taddr_of(t_o, warp, cb * 32), o);
+        umma::wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] *= alpha;
+        umma::st32(umma::taddr_of(t_o, warp, cb * 32), o);
+      }
+      umma::wait_st();
+    }
+    fence_proxy_async_smem();  // P before the tensor cores read it
+    umma::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+      umma::fence_after_sync();
+#pragma unroll
+      for (int k0 = 0; k0 < kPaTile; k0 += 16)
+        umma::mma_bf16(t_o, umma::desc_k16(aP, kPaTile, k0), umma::desc_k16(aVT, D, k0), idO,
+                       kt > 0 || k0 > 0);
+      umma::commit(bar_o);
+    }
+  }
+  ok &= mbar_wait_bounded(bar_o, qt & 1, &never);
+  __syncwarp();
+  umma::fence_after_sync();
+
+  // ---- output row i ----
+  // tcgen05.ld is warp-collective (.sync.aligned): every lane of the warp
+  // executes it, also lanes whose query lies past the prompt; only the
+  // stores are guarded
+  {
+    const float inv = i < P ? 1.f / l : 0.f;
+    __nv_bfloat16* dst = out + (int64_t(b) * P + i) * q_stride + int64_t(hq) * D;
+#pragma unroll
+    for (int cb = 0; cb < D / 32; ++cb) {
+      float o[32];
+      umma::ld32(umma::taddr_of(t_o, warp, cb * 32), o);
+      umma::wait_ld();
+      if (i < P) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 w4;
+          w4.x = pack2_bf16(o[e + 0] * inv, o[e + 1] * inv);
+          w4.y = pack2_bf16(o[e + 2] * inv, o[e + 3] * inv);
+          w4.z = pack2_bf16(o[e + 4] * inv, o[e + 5] * inv);
+          w4.w = pack2_bf16(o[e + 6] * inv, o[e + 7] * inv);
+          *reinterpret_cast<uint4*>(dst + cb * 32 + e) = w4;
+        }
+      }
+    }
+  }
+  if (!ok && tid == 0) report_error(v.hdr, DMS_DEVERR_TIMEOUT, layer, seq0 + b, hq);
+
+  // ---- fused compaction: the diagonal key tile's kept rows into the pool ----
+  // (K rows come from the tile in shared memory, V rows from the input, which
+  // this CTA has just read)
+  if (compact && hq % g == 0 && v.hdr->prefill_go) {
+    int* s_kept = reinterpret_cast<int*>(smem + S::P);  // P is no longer read
+    const int hd = v.head(layer, seq0 + b, hkv);
+    auto keep_of = [&](int j, uint8_t* fl) {
+      const uint8_t f = j < P ? evict[(int64_t(b) * P + j) * v.Hkv + hkv] : 0;
+      *fl = f;
+      return j < P && (f == 0 || (P - 1 - j) < v.w);
+    };
+    uint8_t f = 0, f_unused = 0;
+    const int j = i0 + tid;
+    const bool keep = keep_of(j, &f);
+    const unsigned bm = __ballot_sync(0xffffffffu, keep);
+    // the prefix counts cover 256-token chunks; a second-half tile adds the
+    // kept count of the first half
+    const bool first_half_keep = (qt & 1) ? keep_of(j - kPaTile, &f_unused) : false;
+    const unsigned bm1 = __ballot_sync(0xffffffffu, first_half_keep);
+    if (lane == 0) {
+      s_scan[warp] = __popc(bm);
+      s_scan[4 + warp] = __popc(bm1);
+    }
+    __syncthreads();
+    int before = 0, nkept = 0, first_half = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      before += w < warp ? s_scan[w] : 0;
+      nkept += s_scan[w];
+      first_half += s_scan[4 + w];
+    }
+    const int rank = before + __popc(bm & ((1u << lane) - 1u));
+    const int base = v.chunk_counts[(int64_t(b) * v.Hkv + hkv) * v.n_chunks_max + (qt >> 1)] + first_half;
+    const int32_t* table = v.bt + int64_t(hd) * v.mbh;
+    if (keep) {
+      s_kept[rank] = tid;
+      if (j >= P - v.w) {
+        const int slot = base + rank;
+        const int64_t ri = int64_t(hd) * v.w + (j % v.w);
+        v.ring[ri] = uint32_t(slot) | (uint32_t(f != 0) << 31);
+        v.ring_row[ri] = table[slot / v.BT] * v.BT + slot % v.BT;
+      }
+    }
+    __syncthreads();
+    constexpr int CH = D / 8;
+    for (int idx = tid; idx < nkept * CH; idx += kPaThreads) {
+      const int kk = idx / CH, c = idx % CH;
+      const int r = s_kept[kk];
+      const int slot = base + kk, row = slot % v.BT;
+      const int blk = table[slot / v.BT];
+      if (!DMS_CHECK(blk >= 0 && blk < v.max_blocks && slot / v.BT < v.mbh, v.hdr, 501, hd, slot)) continue;
+      uint8_t* dst = v.blocks + int64_t(blk) * v.block_bytes + int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(smem + S::K + umma::sw128_offset(kPaTile, r, c * 8));
+      *reinterpret_cast<uint4*>(dst + v.tile_bytes) =
+          __ldg(reinterpret_cast<const uint4*>(vsrc + (i0 + r) * kv_stride) + c);
+    }
+  }
+
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) umma::tmem_dealloc(tbase, 256);
+}
+
+}  // namespace dms
+
+using namespace dms;
+
+extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
+                                       const void* q, const void* k, const void* v,
+                                       dms_dtype in_dtype, const uint8_t* evict, void* out,
+                                       float sm_scale, cudaStream_t stream) {
+  if (!pool) {
+    set_last_error("null pool");
+    return DMS_ERR_INVALID_ARG;
+  }
+  const PoolView& pv = pool->view;
+  if (pv.kv_dtype != DMS_BF16 || in_dtype != DMS_BF16 || (pv.D != 64 && pv.D != 128)) {
+    set_last_error("dms_prefill_attn needs a bf16 pool, bf16 inputs and head_dim 64 or 128");
+    return DMS_ERR_UNSUPPORTED;
+  }
+  if (layer < 0 || layer >= pv.L || seq0 < 0 || batch < 1 || seq0 + batch > pv.Bmax ||
+      batch > 65535 || prompt_len < 1 || prompt_len > pool->cfg.max_context) {
+    set_last_error("bad layer/sequences/prompt_len (%d, %d+%d, %d)", layer, seq0, batch, prompt_len);
+    return DMS_ERR_INVALID_ARG;
+  }
+  if (!q || !k || !v || !evict || !out) {
+    set_last_error("null pointer argument");
+    return DMS_ERR_INVALID_ARG;
+  }
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
+       reinterpret_cast<uintptr_t>(out)) & 15) {
+    set_last_error("q, k, v and out must be 16-byte aligned");
+    return DMS_ERR_INVALID_ARG;
+  }
+  // prefix counts and block tables of the layer's sequences (the same count
+  // and plan kernels as dms_compact_prefill_seqs)
+  dms_status st = prefill_plan_launch(pool, layer, seq0, batch, prompt_len, evict, stream);
+  if (st != DMS_OK) return st;
+  const int n_qtiles = (prompt_len + kPaTile - 1) / kPaTile;
+  const dim3 grid(n_qtiles, pv.Hq, batch);
+  const float sc = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf(float(pv.D));
+  const float scale_log2 = sc * 1.4426950408889634f;
+  auto kq = static_cast<const __nv_bfloat16*>(q);
+  auto kk = static_cast<const __nv_bfloat16*>(k);
+  auto kv = static_cast<const __nv_bfloat16*>(v);
+  auto ko = static_cast<__nv_bfloat16*>(out);
+  if (pv.D == 128) {
+    static bool attr = false;
+    if (!attr) {
+      st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            PaSmem<128>::BYTES), "prefill attn smem attribute");
+      if (st != DMS_OK) return st;
+      attr = true;
+    }
+    prefill_attn_kernel<128><<<grid, kPaThreads, PaSmem<128>::BYTES, stream>>>(
+        pv, layer, seq0, prompt_len, kq, kk, kv, evict, ko, scale_log2, n_qtiles, 1);
+  } else {
+    static bool attr = false;
+    if (!attr) {
+      st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            PaSmem<64>::BYTES), "prefill attn smem attribute");
+      if (st != DMS_OK) return st;
+      attr = true;
+    }
+    prefill_attn_kernel<64><<<grid, kPaThreads, PaSmem<64>::BYTES, stream>>>(
+        pv, layer, seq0, prompt_len, kq, kk, kv, evict, ko, scale_log2, n_qtiles, 1);
+  }
+  return cuda_status(cudaGetLastError(), "prefill_attn_kernel");
+}

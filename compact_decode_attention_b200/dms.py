@@ -103,6 +103,7 @@ _SIGS = {
     "dms_append_evict_seqs": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P]),
     "dms_decode_attn_seqs": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
     "dms_release_seqs": (_I, [_P, _I, _P, _P]),
+    "dms_prefill_attn": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, ctypes.c_float, _P]),
     "dms_stepper_layout": (_I, [_P, _I, _I, ctypes.POINTER(StepperLayout)]),
     "dms_stepper_create": (_I, [_P, _I, _I, _I, ctypes.c_float, _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
     "dms_stepper_step": (_I, [_P, _I64, _P, _P]),
@@ -240,6 +241,12 @@ def dms_decode_attn_seqs(pool: int, layer0: int, n_layers: int, n_seqs: int, seq
                                       workspace, workspace_bytes, stream), "dms_decode_attn_seqs")
 
 
+def dms_prefill_attn(pool: int, layer: int, seq0: int, batch: int, prompt_len: int, q: int, k: int, v: int,
+                     in_dtype: int, evict: int, out: int, sm_scale: float, stream: int):
+    _check(lib().dms_prefill_attn(pool, layer, seq0, batch, prompt_len, q, k, v, in_dtype, evict, out,
+                                  sm_scale, stream), "dms_prefill_attn")
+
+
 def dms_release_seqs(pool: int, n_seqs: int, seq_ids: int, stream: int):
     _check(lib().dms_release_seqs(pool, n_seqs, seq_ids, stream), "dms_release_seqs")
 
@@ -375,6 +382,12 @@ class Pool:
         ws = self.workspace(nl, n, q.device)
         dms_decode_attn_seqs(self.handle, layer0, nl, n, _ptr(seq_ids), _ptr(q), torch_dtype_code(q.dtype),
                              _ptr(out), sm_scale, _ptr(ws), ws.numel(), _stream(stream))
+
+    def prefill_attn(self, layer, seq0, q, k, v, evict, out, sm_scale=0.0, stream=None):
+        """Prompt attention [B, P, Hq, D] under the DMS mask + compaction of the layer."""
+        B, P = k.shape[0], k.shape[1]
+        dms_prefill_attn(self.handle, layer, seq0, B, P, _ptr(q), _ptr(k), _ptr(v), torch_dtype_code(k.dtype),
+                         _ptr(evict), _ptr(out), sm_scale, _stream(stream))
 
     def release_seqs(self, seq_ids, stream=None):
         dms_release_seqs(self.handle, int(seq_ids.numel()), _ptr(seq_ids), _stream(stream))

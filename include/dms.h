@@ -220,6 +220,25 @@ dms_status dms_decode_attn_seqs(dms_pool* pool, int layer0, int n_layers, int n_
                                 void* out, float sm_scale, void* workspace,
                                 size_t workspace_bytes, cudaStream_t stream);
 
+/* Prompt attention under the delayed-eviction mask, fused with compaction:
+ * for sequences [seq0, seq0 + batch) of a layer, out[b, i, hq] =
+ * softmax(sm_scale * q[b, i, hq] . K^T) V over the keys j <= i that query i
+ * can see (j unflagged, or i - j < w; kv-head hq / g), and the layer's kept
+ * prompt rows are written into the pool exactly as dms_compact_prefill_seqs
+ * writes them (the kernel that streams each K/V tile for attention also
+ * stores the tile's kept rows).
+ *   q, out  [batch, P, Hq, D]  bf16      k, v  [batch, P, Hkv, D]  bf16
+ *   evict   [batch, P, Hkv]    uint8     sm_scale <= 0 selects 1/sqrt(D)
+ * Needs a bf16 pool with head_dim 64 or 128 (else DMS_ERR_UNSUPPORTED).
+ * The sequences must be empty in that layer (else DMS_DEVERR_LAYER_NOT_EMPTY
+ * and nothing is stored; the outputs are still computed).  Runs on the
+ * tensor cores (tcgen05, accumulators in tensor memory).
+ * Source: the mask holds for every query (mindverse page, DMS section;
+ * stiva.ai page, "delayed eviction"); compaction as dms_compact_prefill. */
+dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
+                            const void* q, const void* k, const void* v, dms_dtype in_dtype,
+                            const uint8_t* evict, void* out, float sm_scale, cudaStream_t stream);
+
 /* End sequences: for every layer and kv-head of the n_seqs sequence slots in
  * seq_ids (int32 device array, distinct ids), push every block they hold on
  * the global free-block stack and return their counters to empty, so the

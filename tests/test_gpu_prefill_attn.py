@@ -1,0 +1,81 @@
+"""dms_prefill_attn: prompt attention under the delayed-eviction mask on the
+tensor cores, fused with compaction (through the C ABI).  Outputs are
+compared with the fp64 oracle (every query on small prompts, sampled queries
+on a long one, max-abs 2e-2 as for every bf16 path); the pool the fused
+kernel fills must hold exactly what the oracle's compaction keeps."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import attention as oatt
+from compact_decode_attention_b200 import dms
+
+from gpu_util import check_block_invariants, check_head_store, head_id, oracle_store, read_state
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+def _inputs(seed, B, P, Hq, Hkv, D, p_keep):
+    K = synth.kv_tokens(seed, 0, 0, B, 0, P, Hkv, D, "bf16")
+    V = synth.kv_tokens(seed, 1, 0, B, 0, P, Hkv, D, "bf16")
+    Q = np.stack([synth.q_tokens(seed, 0, B, i, Hq, D, "bf16") for i in range(P)], axis=1)  # [B, P, Hq, D]
+    F = synth.flag_tokens(seed, 0, B, 0, P, Hkv, [synth.keep_threshold(p_keep)] * Hkv)
+    return Q, K, V, F
+
+
+def _run(pool, seq0, Q, K, V, F, layer=0):
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).cuda()  # noqa: E731
+    out = torch.full(Q.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    pool.prefill_attn(layer, seq0, dev(Q), dev(K), dev(V), torch.from_numpy(np.ascontiguousarray(F)).cuda(), out)
+    return out.float().cpu().numpy()
+
+
+def _check_store(pool, seq0, K, V, F, P, w):
+    state = read_state(pool)
+    assert state["error"] == 0
+    B, _, Hkv, _ = K.shape
+    for b in range(B):
+        for h in range(Hkv):
+            store = oracle_store(F[b, :, h], np.zeros(0, np.uint8), w, P)
+            check_head_store(pool, state, head_id(pool.cfg, 0, seq0 + b, h), store,
+                             {j: K[b, j, h] for j in range(P)}, {j: V[b, j, h] for j in range(P)}, "bf16")
+    check_block_invariants(pool, state)
+
+
+@pytest.mark.parametrize("D,P,w,p_keep", [(128, 300, 64, 0.3), (64, 300, 64, 0.3), (128, 200, 512, 0.1),
+                                          (128, 129, 1, 0.0), (64, 77, 16, 0.5)])
+def test_every_query_matches_the_oracle_and_the_store_matches_compaction(D, P, w, p_keep):
+    B, Hq, Hkv = 2, 8, 2
+    Q, K, V, F = _inputs(7 + D + P, B, P, Hq, Hkv, D, p_keep)
+    pool = dms.Pool(1, B, Hq, Hkv, D, w, dms.DMS_BF16, B * Hkv * (P // 64 + 2), P + 1)
+    got = _run(pool, 0, Q, K, V, F)
+    assert np.isfinite(got).all()
+    for b in range(B):
+        exp = oatt.prefill_attention(Q[b].astype(np.float64), K[b], V[b], F[b], w)
+        err = np.abs(got[b] - exp).max()
+        assert err < TOL, (b, err)
+    _check_store(pool, 0, K, V, F, P, w)
+
+
+def test_long_prompt_sampled_queries_and_sequence_offset():
+    B, P, Hq, Hkv, D, w = 1, 2048, 32, 8, 128, 512
+    Q, K, V, F = _inputs(91, B, P, Hq, Hkv, D, 0.15)
+    pool = dms.Pool(1, 3, Hq, Hkv, D, w, dms.DMS_BF16, 3 * Hkv * (P // 64 + 2), P + 1)
+    got = _run(pool, 2, Q, K, V, F)             # into sequence slot 2
+    rng = np.random.default_rng(5)
+    for i in sorted(set(rng.integers(0, P, 40).tolist()) | {0, 127, 128, 1023, P - 1}):
+        exp = oatt.decode_attention(Q[0, i].astype(np.float64), K[0, :i + 1], V[0, :i + 1], F[0, :i + 1], i, w)
+        assert np.abs(got[0, i] - exp).max() < TOL, i
+    _check_store(pool, 2, K, V, F, P, w)
+
+
+def test_unsupported_pools_are_refused():
+    pool = dms.Pool(1, 1, 8, 2, 128, 16, dms.DMS_FP8_E4M3, 16, 256)
+    x = torch.zeros(1, 64, 8, 128, dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros(1, 64, 2, 128, dtype=torch.bfloat16, device="cuda")
+    f = torch.zeros(1, 64, 2, dtype=torch.uint8, device="cuda")
+    with pytest.raises(dms.DmsError) as e:
+        pool.prefill_attn(0, 0, x, kv, kv, f, x)
+    assert e.value.status == dms.DMS_ERR_UNSUPPORTED
