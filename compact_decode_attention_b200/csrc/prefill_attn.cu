@@ -18,10 +18,12 @@
 //   thread r owns query row r: masked online softmax on S[r] (tcgen05.ld),
 //   P[r] as bf16 into shared memory, O[r] rescaled in tensor memory when the
 //   row maximum moved
-//   O += P V            (M = 128 queries, N = D, K = 128 keys; V is staged
-//                        transposed so both operands are K-major)
-// Operands live in shared memory in the K-major 128-byte-swizzled layout of
-// umma.cuh.  The CTA of the first query head of each kv-head group writes,
+//   O += P V            (M = 128 queries, N = D, K = 128 keys; V is read in
+//                        its own [keys x D] layout as an MN-major operand)
+// Tiles live in shared memory in the 128-byte-swizzled image of umma.cuh,
+// filled by 16-byte asynchronous copies into two buffers, so the next key
+// tile streams in while the current one is computed.  The CTA of the first
+// query head of each kv-head group writes,
 // at its diagonal key tile, the tile's kept rows into the pool (slots from
 // the prefix counts of the count and plan kernels) and the window ring.
 #include <math.h>
@@ -36,12 +38,13 @@ constexpr int kPaThreads = 128;   // one thread per query row
 
 template <int D>
 struct PaSmem {
-  static constexpr int Q = 0;                          // [128 x D] K-major
-  static constexpr int K = Q + kPaTile * D * 2;        // [128 keys x D]
-  static constexpr int VT = K + kPaTile * D * 2;       // [D x 128 keys]
-  static constexpr int P = VT + D * kPaTile * 2;       // [128 x 128 keys]
-  static constexpr int FLAGS = P + kPaTile * kPaTile * 2;
-  static constexpr int BARS = FLAGS + kPaTile;         // 2 mbarriers
+  static constexpr int TILE = kPaTile * D * 2;         // one [128 x D] bf16 tile
+  static constexpr int Q = 0;                          // queries, K-major
+  static constexpr int K = Q + TILE;                   // 2 buffers of keys, K-major
+  static constexpr int V = K + 2 * TILE;               // 2 buffers of values [keys x D] (MN-major B)
+  static constexpr int P = V + 2 * TILE;               // [128 queries x 128 keys] bf16
+  static constexpr int FLAGS = P + kPaTile * kPaTile * 2;  // 2 x 4 words of evict-flag bits
+  static constexpr int BARS = FLAGS + 2 * kPaTile;     // 2 mbarriers
   static constexpr int MISC = BARS + 16;               // tmem base, scan
   static constexpr int BYTES = MISC + 64 + 1024;       // + alignment slack
 };
@@ -51,41 +54,18 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Rows [row0, row0 + 128) of one head of a [B, P, H, D] bf16 tensor into a
-// K-major swizzled tile; rows past P are zero.
+// Asynchronous copy of rows [row0, row0 + 128) of one head of a [B, P, H, D]
+// bf16 tensor into the swizzled image of a tile with 128 rows; rows past P
+// are zero-filled.
 template <int D>
-__device__ __forceinline__ void load_rows(uint8_t* tile, const __nv_bfloat16* src, int64_t row_stride,
-                                          int row0, int P, int tid) {
+__device__ __forceinline__ void copy_rows_async(uint8_t* tile, const __nv_bfloat16* src,
+                                                int64_t row_stride, int row0, int P, int tid) {
   constexpr int CH = D / 8;  // 16-byte chunks per row
   for (int idx = tid; idx < kPaTile * CH; idx += kPaThreads) {
     const int r = idx / CH, c = idx % CH;
-    uint4 x = make_uint4(0, 0, 0, 0);
-    if (row0 + r < P) x = __ldg(reinterpret_cast<const uint4*>(src + (row0 + r) * row_stride) + c);
-    *reinterpret_cast<uint4*>(tile + umma::sw128_offset(kPaTile, r, c * 8)) = x;
-  }
-}
-
-// V rows [row0, row0 + 128) transposed into a [D x 128 keys] K-major tile:
-// each thread takes two neighbouring keys and stores (v[r][d], v[r+1][d])
-// pairs as 32-bit words.
-template <int D>
-__device__ __forceinline__ void load_v_transposed(uint8_t* tile, const __nv_bfloat16* src,
-                                                  int64_t row_stride, int row0, int P, int tid) {
-  constexpr int CH = D / 8;
-  for (int idx = tid; idx < (kPaTile / 2) * CH; idx += kPaThreads) {
-    const int r = 2 * (idx / CH), c = idx % CH;
-    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-    if (row0 + r < P) a = __ldg(reinterpret_cast<const uint4*>(src + (row0 + r) * row_stride) + c);
-    if (row0 + r + 1 < P) b = __ldg(reinterpret_cast<const uint4*>(src + (row0 + r + 1) * row_stride) + c);
-    const __nv_bfloat16* va = reinterpret_cast<const __nv_bfloat16*>(&a);
-    const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(&b);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      __nv_bfloat162 pr;
-      pr.x = va[e];
-      pr.y = vb[e];
-      *reinterpret_cast<__nv_bfloat162*>(tile + umma::sw128_offset(D, c * 8 + e, r)) = pr;
-    }
+    const bool valid = row0 + r < P;
+    const __nv_bfloat16* g = src + int64_t(valid ? row0 + r : 0) * row_stride + c * 8;
+    umma::cp_async16(tile + umma::sw128_offset(kPaTile, r, c * 8), g, valid);
   }
 }
 
@@ -110,7 +90,19 @@ __global__ void __launch_bounds__(kPaThreads, 1)
   uint64_t* bar_o = bar_s + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::MISC);
   int* s_scan = reinterpret_cast<int*>(smem + S::MISC) + 4;
-  uint8_t* s_flag = smem + S::FLAGS;
+
+  // stage keys and values of tile kt into buffer kt & 1 (asynchronous copies)
+  auto stage_tile = [&](int kt) {
+    const int buf = kt & 1, j0 = kt * kPaTile;
+    copy_rows_async<D>(smem + S::K + buf * S::TILE, ksrc, kv_stride, j0, P, tid);
+    copy_rows_async<D>(smem + S::V + buf * S::TILE, vsrc, kv_stride, j0, P, tid);
+  };
+  // evict flag of key j0 + tid of tile kt (loaded a tile ahead, packed later)
+  auto flag_of = [&](int kt) -> uint8_t {
+    const int j = kt * kPaTile + tid;
+    return j < P ? evict[(int64_t(b) * P + j) * v.Hkv + hkv] : 0;
+  };
+  uint32_t* s_fbits = reinterpret_cast<uint32_t*>(smem + S::FLAGS);  // [2][4]
 
   if (tid == 0) {
     mbar_init(bar_s, 1);
@@ -122,36 +114,47 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     umma::tmem_alloc(s_tmem, 256);
     umma::tmem_relinquish();
   }
-  load_rows<D>(smem + S::Q, qsrc, q_stride, i0, P, tid);
+  copy_rows_async<D>(smem + S::Q, qsrc, q_stride, i0, P, tid);
+  stage_tile(0);
+  umma::cp_async_commit();
+  uint8_t f_cur = flag_of(0);
   umma::fence_before_sync();
   __syncthreads();
   umma::fence_after_sync();
   const uint32_t tbase = *s_tmem;
   const uint32_t t_s = tbase, t_o = tbase + kPaTile;
-  const uint32_t aQ = smem_u32(smem + S::Q), aK = smem_u32(smem + S::K);
-  const uint32_t aVT = smem_u32(smem + S::VT), aP = smem_u32(smem + S::P);
+  const uint32_t aQ = smem_u32(smem + S::Q), aP = smem_u32(smem + S::P);
   constexpr uint32_t idS = umma::idesc_bf16_f32(kPaTile, kPaTile);
-  constexpr uint32_t idO = umma::idesc_bf16_f32(kPaTile, D);
+  constexpr uint32_t idO = umma::idesc_bf16_f32_bmn(kPaTile, D);
   const int i = i0 + tid;  // this thread's query row
   float m = -INFINITY, l = 0.f;
   volatile int never = 0;
   bool ok = true;
 
   for (int kt = 0; kt <= qt; ++kt) {
-    const int j0 = kt * kPaTile;
-    if (kt > 0) {  // the previous P V product has finished with K, V^T and P
+    const int cur = kt & 1, j0 = kt * kPaTile;
+    if (kt > 0) {  // P V of tile kt-1 is done: P and the other buffer are free
       ok &= mbar_wait_bounded(bar_o, (kt - 1) & 1, &never);
       __syncwarp();
       umma::fence_after_sync();
     }
-    load_rows<D>(smem + S::K, ksrc, kv_stride, j0, P, tid);
-    load_v_transposed<D>(smem + S::VT, vsrc, kv_stride, j0, P, tid);
-    {
-      const int j = j0 + tid;
-      s_flag[tid] = j < P ? evict[(int64_t(b) * P + j) * v.Hkv + hkv] : 1;
+    {  // this tile's flags as 4 words of bits (bit c = key j0 + c flagged)
+      const unsigned fw = __ballot_sync(0xffffffffu, f_cur != 0);
+      if (lane == 0) s_fbits[cur * 4 + warp] = fw;
     }
-    fence_proxy_async_smem();  // generic-proxy tile writes before the tensor cores read them
+    uint8_t f_next = 0;
+    if (kt < qt) {  // the next tile streams in while this one is computed
+      stage_tile(kt + 1);
+      umma::cp_async_commit();
+      f_next = flag_of(kt + 1);
+      umma::cp_async_wait<1>();
+    } else {
+      umma::cp_async_wait<0>();
+    }
+    fence_proxy_async_smem();  // copies before the tensor cores read them
     __syncthreads();
+    const uint32_t aK = smem_u32(smem + S::K + cur * S::TILE);
+    const uint32_t aV = smem_u32(smem + S::V + cur * S::TILE);
     if (tid == 0) {
       umma::fence_after_sync();
 #pragma unroll
@@ -165,6 +168,21 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     umma::fence_after_sync();
 
     // ---- masked online softmax on query row i (log2 domain) ----
+    // visibility of key j0 + c as bits: flag clear or inside the window
+    // (c >= i - w + 1 - j0), causal (c <= i - j0), inside the prompt (c < P - j0)
+    uint32_t vis[4];
+    {
+      const int hi = i - j0, lo = i - v.w + 1 - j0, end = P - j0;
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        const int c0 = 32 * wd;
+        const int x_le = hi - c0, x_ge = lo - c0, x_lt = end - c0;
+        const uint32_t le = x_le < 0 ? 0u : x_le >= 31 ? ~0u : (2u << x_le) - 1u;
+        const uint32_t ge = x_ge <= 0 ? ~0u : x_ge >= 32 ? 0u : ~((1u << x_ge) - 1u);
+        const uint32_t lt = x_lt <= 0 ? 0u : x_lt >= 32 ? ~0u : (1u << x_lt) - 1u;
+        vis[wd] = (~s_fbits[cur * 4 + wd] | ge) & le & lt;
+      }
+    }
     float s[kPaTile];
 #pragma unroll
     for (int cb = 0; cb < kPaTile / 32; ++cb) {
@@ -174,25 +192,29 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       for (int e = 0; e < 32; ++e) s[cb * 32 + e] = x[e];
     }
     umma::wait_ld();
-    float mx = -INFINITY;
+    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
     for (int c = 0; c < kPaTile; ++c) {
-      const int j = j0 + c;
-      const bool vis = j < P && j <= i && (s_flag[c] == 0 || i - j < v.w);
-      s[c] = vis ? s[c] * scale_log2 : -INFINITY;
-      mx = fmaxf(mx, s[c]);
+      s[c] = ((vis[c >> 5] >> (c & 31)) & 1u) ? s[c] * scale_log2 : -INFINITY;
+      mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
     }
-    const float mn = fmaxf(m, mx);
-    const float alpha = mn == -INFINITY ? 1.f : fast_exp2(m - mn);
-    float sum = 0.f;
+    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+    // lazy rescaling: the running maximum only moves when the row maximum
+    // grew by more than 8 (log2 units), so P stays <= 256 and O rarely needs
+    // a round trip through tensor memory
+    float alpha = 1.f;
+    if (mx > m + 8.f) {
+      alpha = m == -INFINITY ? 0.f : fast_exp2(m - mx);
+      m = mx;
+    }
+    float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < kPaTile; ++c) {
-      const float p = mn == -INFINITY ? 0.f : fast_exp2(s[c] - mn);
-      sum += p;
+      const float p = m == -INFINITY ? 0.f : fast_exp2(s[c] - m);
+      sum4[c & 3] += p;
       s[c] = p;
     }
-    l = l * alpha + sum;
-    m = mn;
+    l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
 #pragma unroll
     for (int ch = 0; ch < kPaTile / 8; ++ch) {
       uint4 w4;
@@ -215,6 +237,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       }
       umma::wait_st();
     }
+    f_cur = f_next;
     fence_proxy_async_smem();  // P before the tensor cores read it
     umma::fence_before_sync();
     __syncthreads();
@@ -222,7 +245,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       umma::fence_after_sync();
 #pragma unroll
       for (int k0 = 0; k0 < kPaTile; k0 += 16)
-        umma::mma_bf16(t_o, umma::desc_k16(aP, kPaTile, k0), umma::desc_k16(aVT, D, k0), idO,
+        umma::mma_bf16(t_o, umma::desc_k16(aP, kPaTile, k0), umma::desc_mn_k16(aV, kPaTile, k0), idO,
                        kt > 0 || k0 > 0);
       umma::commit(bar_o);
     }
@@ -259,8 +282,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
   if (!ok && tid == 0) report_error(v.hdr, DMS_DEVERR_TIMEOUT, layer, seq0 + b, hq);
 
   // ---- fused compaction: the diagonal key tile's kept rows into the pool ----
-  // (K rows come from the tile in shared memory, V rows from the input, which
-  // this CTA has just read)
+  // (its K and V rows are still in shared memory)
   if (compact && hq % g == 0 && v.hdr->prefill_go) {
     int* s_kept = reinterpret_cast<int*>(smem + S::P);  // P is no longer read
     const int hd = v.head(layer, seq0 + b, hkv);
@@ -310,9 +332,9 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       const int blk = table[slot / v.BT];
       if (!DMS_CHECK(blk >= 0 && blk < v.max_blocks && slot / v.BT < v.mbh, v.hdr, 501, hd, slot)) continue;
       uint8_t* dst = v.blocks + int64_t(blk) * v.block_bytes + int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;
-      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(smem + S::K + umma::sw128_offset(kPaTile, r, c * 8));
-      *reinterpret_cast<uint4*>(dst + v.tile_bytes) =
-          __ldg(reinterpret_cast<const uint4*>(vsrc + (i0 + r) * kv_stride) + c);
+      const uint32_t so = (qt & 1) * S::TILE + umma::sw128_offset(kPaTile, r, c * 8);
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(smem + S::K + so);
+      *reinterpret_cast<uint4*>(dst + v.tile_bytes) = *reinterpret_cast<const uint4*>(smem + S::V + so);
     }
   }
 

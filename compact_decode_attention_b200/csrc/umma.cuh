@@ -43,11 +43,44 @@ __device__ __forceinline__ uint64_t desc_k16(uint32_t tile_addr, int R, int k0) 
   return desc_sw128(tile_addr + uint32_t((k0 >> 6) * R * 128 + (k0 & 63) * 2));
 }
 
+// MN-major operand (the MMA's M or N index contiguous): a tile stored with
+// the same image as a K-major tile whose rows are the K index (e.g. V as
+// [keys x D] for O += P V).  Leading byte offset = distance between 64-wide
+// blocks of the MN index (R * 128 bytes), stride byte offset = one 8-row group
+// of K (1024); the K = 16 slice at k0 starts k0 rows (k0 * 128 bytes) in.
+__device__ __forceinline__ uint64_t desc_mn_k16(uint32_t tile_addr, int R, int k0) {
+  const uint32_t addr = tile_addr + uint32_t(k0 * 128);
+  uint64_t d = 0;
+  d |= uint64_t((addr & 0x3FFFF) >> 4);
+  d |= uint64_t((uint32_t(R) * 128) >> 4) << 16;
+  d |= uint64_t(1024 >> 4) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
 // ---- instruction descriptor: kind::f16, bf16 x bf16 -> fp32, both K-major ----
 // bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format
 // (1 = bf16), 15 / 16 A / B major (0 = K), 17-22 N >> 3, 24-28 M >> 4.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// same with B MN-major (bit 16)
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
+  return idesc_bf16_f32(M, N) | (1u << 16);
+}
+
+// ---- 16-byte asynchronous global -> shared copy (zero-filled when !valid) ----
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ---- tensor memory ----
