@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(configs.BY_NAME))
     ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-attention measurement")
     ap.add_argument("--cpu-heads", type=int, default=72)
     ap.add_argument("--cpu-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -68,6 +69,57 @@ def measured_peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def measured_bf16_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p))["bf16_tflops"]), "measured burst cuBLAS bf16 (MEASURED_PEAKS.json bf16_tflops)"
+    return 1590.0, "fallback 1.59 PFLOP/s"
+
+
+def prefill_attention_line(wl, device, n_layers=3):
+    """dms_prefill_attn (prompt attention under the DMS mask on the tensor
+    cores, fused with compaction) at the workload's prompt shapes: one layer
+    per call, the median of n_layers calls, each into an empty layer of a
+    small pool.  FLOPs = the causal 128 x 128 tiles the kernel computes
+    (QK and PV, 2 flops per multiply-add)."""
+    import torch
+    from compact_decode_attention_b200 import dms
+    from compact_decode_attention_b200.workload import DeviceWorkload, STREAM_K, STREAM_Q, STREAM_V
+    if wl.kv_dtype != "bf16" or wl.head_dim not in (64, 128):
+        return None
+    P, B, Hq, Hkv, D = wl.prompt, wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    gen = DeviceWorkload(wl, 0, device=device, max_blocks=16)
+    k = gen.normal(STREAM_K, 0, 1, 0, P, Hkv)[0]
+    v = gen.normal(STREAM_V, 0, 1, 0, P, Hkv)[0]
+    q = gen.normal(STREAM_Q, 0, 1, 0, P, Hq)[0]
+    f = gen.flags(0, 1, 0, P)[0]
+    out = torch.empty_like(q)
+    pool = dms.Pool(n_layers + 1, B, Hq, Hkv, D, wl.window, dms.DMS_BF16,
+                    (n_layers + 1) * B * Hkv * (P // 64 + 2), P + 1, device=device)
+    pool.prefill_attn(0, 0, q, k, v, f, out)          # warm-up (module load, attributes)
+    torch.cuda.synchronize()
+    ts = []
+    for layer in range(1, n_layers + 1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pool.prefill_attn(layer, 0, q, k, v, f, out)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    if pool.stats(check=False).error_flags:
+        raise SystemExit("prefill attention set the device error word")
+    ms = float(np.median(ts))
+    n = (P + 127) // 128
+    flops = 4.0 * D * 128 * 128 * n * (n + 1) / 2 * Hq * B
+    peak, kind = measured_bf16_tflops()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"value": tf, "unit": "TFLOP/s", "ms_per_layer": ms, "prompt": P,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tf / peak, "peak_kind": kind},
+            "flops_basis": "causal 128x128 tiles computed (QK^T and PV), per layer",
+            "kernel": f"prefill_attn_kernel<{D}> (tcgen05, fused compaction)"}
 
 
 class ClockSampler:
@@ -430,6 +482,8 @@ def main():
                        "double-buffered against the neighbouring steps' kernels"}
         stp.close()
 
+    prefill = prefill_attention_line(wl, f"cuda:{local}") if not args.no_prefill else None
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, P + W, args.cpu_heads, args.cpu_steps, float(bytes_step[W]))
@@ -448,6 +502,7 @@ def main():
                               f"> 126 MB L2")},
             "decode_steps_per_s": world * K / (ms_max * 1e-3),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "compaction": compaction,
+            "prefill_attention": prefill,
             "gpu_launches": 2 * K, "clocks": clk.summary(),
             "kernels_per_step": ["append_evict_kernel (1 launch, all layers)",
                                  "decode_attn_kernel (1 launch, all layers)"],
