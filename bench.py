@@ -53,6 +53,10 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(configs.BY_NAME))
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-attention measurement")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the prefill-attention measurement and print it")
+    ap.add_argument("--prefill-prompt", type=int, default=0,
+                    help="prompt length for --prefill-only (default: the workload's)")
     ap.add_argument("--cpu-heads", type=int, default=72)
     ap.add_argument("--cpu-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -346,6 +350,14 @@ def main():
             dist.barrier()
 
     wl = configs.BY_NAME[args.workload]
+    if args.prefill_only:          # the prefill-attention measurement alone (one GPU)
+        import dataclasses
+        if args.prefill_prompt:
+            wl = dataclasses.replace(wl, prompt=args.prefill_prompt)
+        line = prefill_attention_line(wl, f"cuda:{local}")
+        if rank == 0:
+            print(json.dumps({"workload": wl.name, "prompt": wl.prompt, "prefill_attention": line}))
+        return 0
     W, K, E = args.warmup, args.steps, args.e2e_steps
     R = min(K, 64)                 # instrumented steps for the attention-kernel timing
     assert W >= 3 and K >= 1
