@@ -24,7 +24,7 @@ import torch
 
 import synth
 from synth import configs
-from oracle import attention, compaction, fp8, mask, reference, slots
+from oracle import attention, compaction, fp8, mask, projection, reference, slots
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 PAGE = json.load(open(os.path.join(GOLDEN, "page_figures.json")))
@@ -172,6 +172,41 @@ def test_prefill_attention_endpoints():
     np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
     only_self = attention.prefill_attention(Q, K, V, flags, 1, 0.3)
     np.testing.assert_allclose(only_self, np.repeat(V, Hq // Hkv, axis=1), rtol=0, atol=1e-12)
+
+
+def test_projection_one_hot_tokens_read_out_weight_rows():
+    """x = e_d: k and v are row d of the projection, the logit is the
+    predictor weight of row d plus the bias (pins the column split of k / v
+    per head and the predictor layout)."""
+    rng = np.random.default_rng(21)
+    dm, Hkv, D = 24, 3, 8
+    W = rng.standard_normal((dm, 2 * Hkv * D))
+    we, be = rng.standard_normal((dm, Hkv)), rng.standard_normal(Hkv)
+    for d in (0, 7, dm - 1):
+        x = np.zeros(dm)
+        x[d] = 1.0
+        k, v, logit = projection.project_token(x, W, we, be, Hkv, D)
+        for h in range(Hkv):
+            assert np.array_equal(k[h], W[d, h * D:(h + 1) * D])
+            assert np.array_equal(v[h], W[d, (Hkv + h) * D:(Hkv + h + 1) * D])
+        assert np.array_equal(logit, we[d] + be)
+    assert np.array_equal(projection.evict_flags(np.array([-1.0, 0.0, 1e-9]), 0.0), [0, 0, 1])
+
+
+def test_bf16_rounding_matches_torch_and_rounds_fp64_once():
+    """On fp32 inputs the oracle's bf16 rounding equals torch's; on fp64
+    values just above a tie it rounds up where fp64 -> fp32 -> bf16 would
+    round to even (a double-rounding trap)."""
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal(100000) * np.exp(rng.uniform(-20, 20, 100000))).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(projection.bf16_round(x.astype(np.float64)), ref)
+    one = 1.0
+    tie = one + 2.0 ** -8                      # halfway between bf16 1.0 and 1.0 + 2^-7
+    assert projection.bf16_round(np.array([tie]))[0] == 1.0          # tie to even
+    above = tie + 2.0 ** -40                   # rounds to 1.0 in fp32, but is above the tie
+    assert np.float32(above) == np.float32(tie)
+    assert projection.bf16_round(np.array([above]))[0] == 1.0 + 2.0 ** -7
 
 
 def test_zero_keys_give_uniform_mean_of_visible_values():
