@@ -82,6 +82,46 @@ def measured_bf16_tflops():
     return 1590.0, "fallback 1.59 PFLOP/s"
 
 
+def projection_line(wl, device, n_calls=8):
+    """dms_project_append (K/V projection + eviction decision + append, fused)
+    for one layer and the workload's batch, d_model = Hq * D (4096 for the
+    Qwen3-8B shapes), synthetic bf16 weights: the median of n_calls decode
+    steps.  Bytes = weights read (W_kv and the predictor) + x + rows written;
+    the kernel streams the weights once, so HBM bandwidth bounds it."""
+    import torch
+    from compact_decode_attention_b200 import dms
+    if wl.head_dim != 128 or wl.kv_dtype == "f32":
+        return None
+    B, Hq, Hkv, D = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    dm = Hq * D
+    g = torch.Generator(device=device).manual_seed(wl.seed)
+    w_kv = (torch.randn(dm, 2 * Hkv * D, device=device, generator=g) / dm ** 0.5).to(torch.bfloat16)
+    w_ev = (torch.randn(dm, Hkv, device=device, generator=g) / dm ** 0.5).to(torch.bfloat16)
+    x = torch.randn(n_calls + 1, B, dm, device=device, generator=g).to(torch.bfloat16)
+    code = {"bf16": dms.DMS_BF16, "fp8": dms.DMS_FP8_E4M3}[wl.kv_dtype]
+    pool = dms.Pool(1, B, Hq, Hkv, D, wl.window, code, B * Hkv * 4, n_calls + 2, device=device)
+    ts = []
+    for c in range(n_calls + 1):
+        pos = torch.full((B,), c, dtype=torch.int64, device=device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pool.project_append(0, None, pos, x[c], w_kv, w_ev)
+        e1.record()
+        torch.cuda.synchronize()
+        if c > 0:                                      # the first call loads the module
+            ts.append(e0.elapsed_time(e1))
+    if pool.stats(check=False).error_flags:
+        raise SystemExit("the projection set the device error word")
+    ms = float(np.median(ts))
+    nbytes = (w_kv.numel() + w_ev.numel() + B * dm) * 2 + B * Hkv * 2 * D * wl.kv_elem_bytes()
+    peak, kind = measured_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"value": gbs, "unit": "GB/s", "us_per_layer": ms * 1e3, "d_model": dm, "batch": B,
+            "algorithmic_bytes": nbytes,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak},
+            "kernel": "project_append_kernel<128> (split-K over d_model, epilogue appends)"}
+
+
 def prefill_attention_line(wl, device, n_layers=3):
     """dms_prefill_attn (prompt attention under the DMS mask on the tensor
     cores, fused with compaction) at the workload's prompt shapes: one layer
@@ -495,6 +535,7 @@ def main():
         stp.close()
 
     prefill = prefill_attention_line(wl, f"cuda:{local}") if not args.no_prefill else None
+    projection = projection_line(wl, f"cuda:{local}") if not args.no_prefill else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -514,7 +555,7 @@ def main():
                               f"> 126 MB L2")},
             "decode_steps_per_s": world * K / (ms_max * 1e-3),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "compaction": compaction,
-            "prefill_attention": prefill,
+            "prefill_attention": prefill, "kv_projection_append": projection,
             "gpu_launches": 2 * K, "clocks": clk.summary(),
             "kernels_per_step": ["append_evict_kernel (1 launch, all layers)",
                                  "decode_attn_kernel (1 launch, all layers)"],

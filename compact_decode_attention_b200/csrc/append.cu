@@ -20,7 +20,7 @@
 // state (slots, counts, rings, stored bytes) is a deterministic function of
 // the inputs; which physical block a head gets during decode is not (prefill
 // hands blocks out by a prefix sum and is deterministic).
-#include "dms_internal.cuh"
+#include "append_core.cuh"
 
 namespace dms {
 
@@ -39,19 +39,6 @@ constexpr int kAppendThreads = 32 * kAppendHeadsPerCta;
 // One warp per (layer, sequence, kv-head).  Lane 0 does the bookkeeping; all
 // lanes load the new K/V row first (it does not depend on the bookkeeping)
 // and store it once the destination is known.
-// Pop a block from the global free-block stack (blocks released by finished
-// sequences); -1 when it is empty.  Only pops run during an append, so a
-// successful compare-and-swap owns the entry below the old top.
-__device__ __forceinline__ int pop_free_block(const PoolView& v) {
-  int top = *reinterpret_cast<volatile int*>(&v.hdr->block_stack_top);
-  while (top > 0) {
-    const int prev = atomicCAS(&v.hdr->block_stack_top, top, top - 1);
-    if (prev == top) return v.block_stack[top - 1];
-    top = prev;
-  }
-  return -1;
-}
-
 // seq_ids (nullable): pool sequence of batch row b, else b.  pos_arr
 // (nullable): position of batch row b, else `pos` for every row.
 template <typename InT, bool FP8>
@@ -77,7 +64,6 @@ __global__ void __launch_bounds__(kAppendThreads)
   }
   const int hd = v.head(l, b, h);
   const int t = int(tpos);
-  const int64_t ri = int64_t(hd) * v.w + t % v.w;
 
   // ---- new rows into registers (bf16/fp32: 16-byte chunks, K then V) ----
   const int nch = int(v.row_bytes >> 4);       // chunks per row: 8, 16 or 32
@@ -98,56 +84,11 @@ __global__ void __launch_bounds__(kAppendThreads)
   // ---- bookkeeping (lane 0; all its loads are independent) ----
   int slot = -1, prow = -1, opened = 0;
   if (lane == 0) {
-    int ns = v.n_slots[hd], nr = v.n_retained[hd], ft = v.free_top[hd];
-    const int lb = v.last_block[hd];
-    const uint32_t e = v.ring[ri];
-    const int er = v.ring_row[ri];
     const uint32_t flag = evict[i] != 0;     // [nl, batch, Hkv] flattened like i
-    if (t >= v.w && (e >> 31)) {
-      // DMS delayed eviction retires token t - w; its slot is pushed on the
-      // head's LIFO free stack and popped right back by the new token, so
-      // the pair is done in registers and the row comes from the row ring
-      if (ft < v.free_cap) {
-        slot = int(e & 0x7fffffffu);
-        prow = er;
-        nr -= 1;
-      } else {
-        report_error(v.hdr, DMS_DEVERR_FREE_STACK_FULL, l, b, h);
-      }
-    } else if (ft > 0) {      // a slot freed earlier and not reused yet
-      ft -= 1;
-      slot = v.free_stack[int64_t(hd) * v.free_cap + ft];
-      prow = v.bt[int64_t(hd) * v.mbh + slot / v.BT] * v.BT + slot % v.BT;
-    } else if (ns / v.BT < v.mbh) {
-      slot = ns;
-      ns += 1;
-      if (slot % v.BT == 0) {  // the slot opens a new block: a released one, else a fresh one
-        int id = pop_free_block(v);
-        if (id < 0) id = atomicAdd(&v.hdr->next_block, 1);
-        if (id < v.max_blocks) {
-          v.bt[int64_t(hd) * v.mbh + slot / v.BT] = id;
-          v.last_block[hd] = id;
-          prow = id * v.BT;
-          opened = 1;
-        } else {
-          report_error(v.hdr, DMS_DEVERR_BLOCKS_EXHAUSTED, l, b, h);
-          slot = -1;
-        }
-      } else {
-        prow = lb * v.BT + slot % v.BT;
-      }
-    } else {
-      report_error(v.hdr, DMS_DEVERR_HEAD_TABLE_FULL, l, b, h);
-    }
-    if (slot >= 0 && !DMS_CHECK(prow >= 0 && prow < v.max_blocks * v.BT, v.hdr, 101, hd, prow))
-      slot = -1;
-    if (slot >= 0) {
-      v.n_slots[hd] = ns;
-      v.n_retained[hd] = nr + 1;
-      v.free_top[hd] = ft;
-      v.ring[ri] = uint32_t(slot) | (flag << 31);
-      v.ring_row[ri] = prow;
-    }
+    const AppendSlot r = append_bookkeeping(v, l, b, h, hd, t, flag);
+    slot = r.slot;
+    prow = r.prow;
+    opened = r.opened;
   }
   slot = __shfl_sync(0xffffffffu, slot, 0);
   prow = __shfl_sync(0xffffffffu, prow, 0);

@@ -1,0 +1,133 @@
+// One decode step of one head of the compact store, shared by the append
+// kernel and the fused projection epilogue.
+//
+// DMS delayed eviction: at step t the token leaving the window is t - w,
+// found at ring index t mod w; when it was flagged its slot is pushed on the
+// head's free stack and the new token takes the top of that stack, else the
+// token takes slot n_slots, opening a new block when that slot starts one
+// ("NVIDIA veröffentlicht Qwen3-8B-DMS-8x ..." (mindverse), section
+// "Dynamic Memory Sparsification (DMS): Eine innovative Lösung"; slot reuse:
+// "FastDMS: vLLM BF16/FP8보다 빠른 6.4x KV cache 압축" (molayo1419.me),
+// opening paragraphs).
+#pragma once
+
+#include "dms_internal.cuh"
+
+namespace dms {
+
+// Pop a block from the global free-block stack (blocks released by finished
+// sequences); -1 when it is empty.  Only pops run during an append, so a
+// successful compare-and-swap owns the entry below the old top.
+__device__ __forceinline__ int pop_free_block(const PoolView& v) {
+  int top = *reinterpret_cast<volatile int*>(&v.hdr->block_stack_top);
+  while (top > 0) {
+    const int prev = atomicCAS(&v.hdr->block_stack_top, top, top - 1);
+    if (prev == top) return v.block_stack[top - 1];
+    top = prev;
+  }
+  return -1;
+}
+
+struct AppendSlot {
+  int slot;    // logical slot of token t, -1 when nothing may be written
+  int prow;    // physical row (block * BT + row)
+  int opened;  // the slot opened a new block
+};
+
+// Bookkeeping of token t (flag `flag`) for head hd = (layer l, sequence b,
+// kv-head h); one thread.  All its loads are independent of each other.
+__device__ __forceinline__ AppendSlot append_bookkeeping(const PoolView& v, int l, int b, int h,
+                                                         int hd, int t, uint32_t flag) {
+  AppendSlot r{-1, -1, 0};
+  const int64_t ri = int64_t(hd) * v.w + t % v.w;
+  int ns = v.n_slots[hd], nr = v.n_retained[hd], ft = v.free_top[hd];
+  const int lb = v.last_block[hd];
+  const uint32_t e = v.ring[ri];
+  const int er = v.ring_row[ri];
+  if (t >= v.w && (e >> 31)) {
+    // token t - w retires; its slot is pushed on the LIFO free stack and
+    // popped right back by the new token, so the pair is done in registers
+    // and the row comes from the row ring
+    if (ft < v.free_cap) {
+      r.slot = int(e & 0x7fffffffu);
+      r.prow = er;
+      nr -= 1;
+    } else {
+      report_error(v.hdr, DMS_DEVERR_FREE_STACK_FULL, l, b, h);
+    }
+  } else if (ft > 0) {      // a slot freed earlier and not reused yet
+    ft -= 1;
+    r.slot = v.free_stack[int64_t(hd) * v.free_cap + ft];
+    r.prow = v.bt[int64_t(hd) * v.mbh + r.slot / v.BT] * v.BT + r.slot % v.BT;
+  } else if (ns / v.BT < v.mbh) {
+    r.slot = ns;
+    ns += 1;
+    if (r.slot % v.BT == 0) {  // a new block: a released one, else a fresh one
+      int id = pop_free_block(v);
+      if (id < 0) id = atomicAdd(&v.hdr->next_block, 1);
+      if (id < v.max_blocks) {
+        v.bt[int64_t(hd) * v.mbh + r.slot / v.BT] = id;
+        v.last_block[hd] = id;
+        r.prow = id * v.BT;
+        r.opened = 1;
+      } else {
+        report_error(v.hdr, DMS_DEVERR_BLOCKS_EXHAUSTED, l, b, h);
+        r.slot = -1;
+      }
+    } else {
+      r.prow = lb * v.BT + r.slot % v.BT;
+    }
+  } else {
+    report_error(v.hdr, DMS_DEVERR_HEAD_TABLE_FULL, l, b, h);
+  }
+  if (r.slot >= 0 && !DMS_CHECK(r.prow >= 0 && r.prow < v.max_blocks * v.BT, v.hdr, 101, hd, r.prow))
+    r.slot = -1;
+  if (r.slot >= 0) {
+    v.n_slots[hd] = ns;
+    v.n_retained[hd] = nr + 1;
+    v.free_top[hd] = ft;
+    v.ring[ri] = uint32_t(r.slot) | (flag << 31);
+    v.ring_row[ri] = r.prow;
+  }
+  return r;
+}
+
+// Store one token's K and V rows, given as float values already rounded to
+// the store's input precision, into physical row prow (one warp).  bf16 and
+// fp32 stores copy the values; an FP8 store quantises them with the layer's
+// scales (E4M3 of x / scale, nearest even, saturating) and, when the token
+// opened its block, clears the block's transposed V tile first.
+__device__ __forceinline__ void store_row_from_float(const PoolView& v, int l, int h, int prow,
+                                                     int opened, const float* krow,
+                                                     const float* vrow, int lane) {
+  const int row = prow % v.BT;
+  uint8_t* blk = v.blocks + int64_t(prow / v.BT) * v.block_bytes;
+  if (v.kv_dtype == DMS_FP8_E4M3) {
+    if (opened) {
+      uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);
+      for (int c = lane; c < int(v.tile_bytes / 16); c += 32) tile[c] = make_uint4(0, 0, 0, 0);
+      __syncwarp();
+    }
+    const float sK = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 0];
+    const float sV = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 1];
+    for (int d = lane; d < v.D; d += 32) {
+      blk[fp8k_byte(row, d)] = f32_to_e4m3(__fdiv_rn(krow[d], sK));
+      blk[v.tile_bytes + fp8v_byte(row, d)] = f32_to_e4m3(__fdiv_rn(vrow[d], sV));
+    }
+    return;
+  }
+  const int esz = v.kv_dtype == DMS_F32 ? 4 : 2;
+  for (int d = lane; d < v.D; d += 32) {
+    const int c = d * esz / 16, within = (d * esz) % 16;
+    const int64_t off = int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16 + within;
+    if (esz == 4) {
+      *reinterpret_cast<float*>(blk + off) = krow[d];
+      *reinterpret_cast<float*>(blk + v.tile_bytes + off) = vrow[d];
+    } else {
+      *reinterpret_cast<__nv_bfloat16*>(blk + off) = __float2bfloat16_rn(krow[d]);
+      *reinterpret_cast<__nv_bfloat16*>(blk + v.tile_bytes + off) = __float2bfloat16_rn(vrow[d]);
+    }
+  }
+}
+
+}  // namespace dms

@@ -104,6 +104,8 @@ _SIGS = {
     "dms_decode_attn_seqs": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
     "dms_release_seqs": (_I, [_P, _I, _P, _P]),
     "dms_prefill_attn": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, ctypes.c_float, _P]),
+    "dms_project_workspace_bytes": (_I, [_P, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "dms_project_append": (_I, [_P, _I, _I, _P, _P, _P, _I, _P, _P, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
     "dms_stepper_layout": (_I, [_P, _I, _I, ctypes.POINTER(StepperLayout)]),
     "dms_stepper_create": (_I, [_P, _I, _I, _I, ctypes.c_float, _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
     "dms_stepper_step": (_I, [_P, _I64, _P, _P]),
@@ -247,6 +249,20 @@ def dms_prefill_attn(pool: int, layer: int, seq0: int, batch: int, prompt_len: i
                                   sm_scale, stream), "dms_prefill_attn")
 
 
+def dms_project_workspace_bytes(pool: int, n_seqs: int, d_model: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().dms_project_workspace_bytes(pool, n_seqs, d_model, ctypes.byref(n)),
+           "dms_project_workspace_bytes")
+    return n.value
+
+
+def dms_project_append(pool: int, layer: int, n_seqs: int, seq_ids: int, pos: int, x: int, d_model: int,
+                       w_kv: int, w_evict: int, b_evict: int, threshold: float, workspace: int,
+                       workspace_bytes: int, stream: int):
+    _check(lib().dms_project_append(pool, layer, n_seqs, seq_ids, pos, x, d_model, w_kv, w_evict, b_evict,
+                                    threshold, workspace, workspace_bytes, stream), "dms_project_append")
+
+
 def dms_release_seqs(pool: int, n_seqs: int, seq_ids: int, stream: int):
     _check(lib().dms_release_seqs(pool, n_seqs, seq_ids, stream), "dms_release_seqs")
 
@@ -388,6 +404,19 @@ class Pool:
         B, P = k.shape[0], k.shape[1]
         dms_prefill_attn(self.handle, layer, seq0, B, P, _ptr(q), _ptr(k), _ptr(v), torch_dtype_code(k.dtype),
                          _ptr(evict), _ptr(out), sm_scale, _stream(stream))
+
+    def project_append(self, layer, seq_ids, pos, x, w_kv, w_evict, b_evict=None, threshold=0.0, stream=None):
+        """x [n, d_model] bf16; appends one projected token per sequence (seq_ids may be None)."""
+        import torch
+        n, dm = x.shape
+        key = ("proj", n, dm)
+        if key not in self._ws:
+            nb = dms_project_workspace_bytes(self.handle, n, dm)
+            self._ws[key] = torch.empty(max(nb, 16), dtype=torch.uint8, device=x.device)
+        ws = self._ws[key]
+        dms_project_append(self.handle, layer, n, 0 if seq_ids is None else _ptr(seq_ids), _ptr(pos), _ptr(x), dm,
+                           _ptr(w_kv), _ptr(w_evict), 0 if b_evict is None else _ptr(b_evict), threshold,
+                           _ptr(ws), ws.numel(), _stream(stream))
 
     def release_seqs(self, seq_ids, stream=None):
         dms_release_seqs(self.handle, int(seq_ids.numel()), _ptr(seq_ids), _stream(stream))

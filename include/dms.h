@@ -239,6 +239,31 @@ dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int batch, int 
                             const void* q, const void* k, const void* v, dms_dtype in_dtype,
                             const uint8_t* evict, void* out, float sm_scale, cudaStream_t stream);
 
+/* Workspace bytes dms_project_append needs (fp32 partial sums). */
+dms_status dms_project_workspace_bytes(const dms_pool* pool, int n_seqs, int d_model,
+                                       size_t* bytes);
+
+/* The model's K/V projection of one decode token per sequence with the
+ * eviction decision and the append fused into its epilogue.  For sequence
+ * row s (slot seq_ids[s], or s when seq_ids is null; position pos[s]) and
+ * kv-head h:
+ *   k = bf16(x[s] W_kv[:, h*D : (h+1)*D])
+ *   v = bf16(x[s] W_kv[:, (Hkv+h)*D : (Hkv+h+1)*D])
+ *   flag = x[s] . w_evict[:, h] + b_evict[h] > threshold
+ * then the token is appended exactly as dms_append_evict_seqs appends it.
+ *   x        [n_seqs, d_model]       bf16
+ *   w_kv     [d_model, 2 * Hkv * D]  bf16, row-major, 16-byte aligned
+ *   w_evict  [d_model, Hkv]          bf16 (the predictor's weights: an input)
+ *   b_evict  [Hkv] float, or null;   seq_ids int32 / pos int64 [n_seqs] device
+ * fp32 accumulation, k and v rounded to nearest-even bf16.  Needs head_dim 128
+ * and a bf16 or FP8 pool.  workspace >= dms_project_workspace_bytes.
+ * Source: a learned per-head predictor decides which tokens to evict
+ * (mindverse page, DMS section); decode runs the projection step by step. */
+dms_status dms_project_append(dms_pool* pool, int layer, int n_seqs, const int32_t* seq_ids,
+                              const int64_t* pos, const void* x, int d_model, const void* w_kv,
+                              const void* w_evict, const float* b_evict, float threshold,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* End sequences: for every layer and kv-head of the n_seqs sequence slots in
  * seq_ids (int32 device array, distinct ids), push every block they hold on
  * the global free-block stack and return their counters to empty, so the
