@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-attention measurement")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill-attention measurement and print it")
+    ap.add_argument("--projection-only", action="store_true",
+                    help="run only the fused K/V projection + append measurement and print it")
     ap.add_argument("--prefill-prompt", type=int, default=0,
                     help="prompt length for --prefill-only (default: the workload's)")
     ap.add_argument("--cpu-heads", type=int, default=72)
@@ -85,8 +87,8 @@ def measured_bf16_tflops():
 def projection_line(wl, device, n_calls=8):
     """dms_project_append (K/V projection + eviction decision + append, fused)
     for one layer and the workload's batch, d_model = Hq * D (4096 for the
-    Qwen3-8B shapes), synthetic bf16 weights: the median of n_calls decode
-    steps.  Bytes = weights read (W_kv and the predictor) + x + rows written;
+    Qwen3-8B shapes), synthetic bf16 weights: n_calls decode steps captured
+    in a CUDA graph, mean time per call.  Bytes = weights read (W_kv and the predictor) + x + rows written;
     the kernel streams the weights once, so HBM bandwidth bounds it."""
     import torch
     from compact_decode_attention_b200 import dms
@@ -100,19 +102,24 @@ def projection_line(wl, device, n_calls=8):
     x = torch.randn(n_calls + 1, B, dm, device=device, generator=g).to(torch.bfloat16)
     code = {"bf16": dms.DMS_BF16, "fp8": dms.DMS_FP8_E4M3}[wl.kv_dtype]
     pool = dms.Pool(1, B, Hq, Hkv, D, wl.window, code, B * Hkv * 4, n_calls + 2, device=device)
-    ts = []
-    for c in range(n_calls + 1):
-        pos = torch.full((B,), c, dtype=torch.int64, device=device)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        pool.project_append(0, None, pos, x[c], w_kv, w_ev)
-        e1.record()
-        torch.cuda.synchronize()
-        if c > 0:                                      # the first call loads the module
-            ts.append(e0.elapsed_time(e1))
+    pos = [torch.full((B,), c, dtype=torch.int64, device=device) for c in range(n_calls + 1)]
+    pool.project_append(0, None, pos[0], x[0], w_kv, w_ev)      # module load, workspace
+    torch.cuda.synchronize()
+    # the timed calls are captured once into a graph and replayed once, so the
+    # host's issue time cannot leave the GPU idle inside the timed region
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for c in range(1, n_calls + 1):
+            pool.project_append(0, None, pos[c], x[c], w_kv, w_ev)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
     if pool.stats(check=False).error_flags:
         raise SystemExit("the projection set the device error word")
-    ms = float(np.median(ts))
+    ms = e0.elapsed_time(e1) / n_calls
     nbytes = (w_kv.numel() + w_ev.numel() + B * dm) * 2 + B * Hkv * 2 * D * wl.kv_elem_bytes()
     peak, kind = measured_peaks()
     gbs = nbytes / (ms * 1e-3) / 1e9
@@ -390,6 +397,11 @@ def main():
             dist.barrier()
 
     wl = configs.BY_NAME[args.workload]
+    if args.projection_only:       # the fused projection measurement alone (one GPU)
+        line = projection_line(wl, f"cuda:{local}")
+        if rank == 0:
+            print(json.dumps({"workload": wl.name, "kv_projection_append": line}))
+        return 0
     if args.prefill_only:          # the prefill-attention measurement alone (one GPU)
         import dataclasses
         if args.prefill_prompt:

@@ -239,7 +239,8 @@ dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int batch, int 
                             const void* q, const void* k, const void* v, dms_dtype in_dtype,
                             const uint8_t* evict, void* out, float sm_scale, cudaStream_t stream);
 
-/* Workspace bytes dms_project_append needs (fp32 partial sums). */
+/* Workspace bytes dms_project_append needs: 0 (its partial sums are reduced
+ * in distributed shared memory); kept so callers can size generically. */
 dms_status dms_project_workspace_bytes(const dms_pool* pool, int n_seqs, int d_model,
                                        size_t* bytes);
 
@@ -256,7 +257,8 @@ dms_status dms_project_workspace_bytes(const dms_pool* pool, int n_seqs, int d_m
  *   w_evict  [d_model, Hkv]          bf16 (the predictor's weights: an input)
  *   b_evict  [Hkv] float, or null;   seq_ids int32 / pos int64 [n_seqs] device
  * fp32 accumulation, k and v rounded to nearest-even bf16.  Needs head_dim 128
- * and a bf16 or FP8 pool.  workspace >= dms_project_workspace_bytes.
+ * and a bf16 or FP8 pool.  workspace may be null (no scratch is needed).
+ * Runs as one thread-block cluster of 8 CTAs per kv-head.
  * Source: a learned per-head predictor decides which tokens to evict
  * (mindverse page, DMS section); decode runs the projection step by step. */
 dms_status dms_project_append(dms_pool* pool, int layer, int n_seqs, const int32_t* seq_ids,
