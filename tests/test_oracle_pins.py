@@ -24,7 +24,7 @@ import torch
 
 import synth
 from synth import configs
-from oracle import attention, compaction, fp8, mask, projection, reference, slots
+from oracle import attention, compaction, fp8, int4, mask, projection, reference, slots
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 PAGE = json.load(open(os.path.join(GOLDEN, "page_figures.json")))
@@ -207,6 +207,44 @@ def test_bf16_rounding_matches_torch_and_rounds_fp64_once():
     above = tie + 2.0 ** -40                   # rounds to 1.0 in fp32, but is above the tie
     assert np.float32(above) == np.float32(tie)
     assert projection.bf16_round(np.array([above]))[0] == 1.0 + 2.0 ** -7
+
+
+def test_int4_codes_are_the_nearest_multiples_of_the_group_scale():
+    """Brute force: each code is the q in [-7, 7] whose q * scale is nearest
+    to x (ties to the even q), the scale is the fp16 rounding of amax / 7 in
+    fp32, and the largest magnitude of a group maps to +-7."""
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal((50, 128)) * np.exp(rng.uniform(-6, 4, (50, 1)))).astype(np.float32)
+    x[3, 32:64] = 0.0                                   # a group of zeros
+    q, s = int4.quantize(x)
+    amax = np.abs(x.reshape(50, 4, 32)).max(-1)
+    assert np.array_equal(s, np.float16(amax.astype(np.float32) / np.float32(7)).astype(np.float32))
+    assert np.all(s[3, 1] == 0) and np.all(q[3, 32:64] == 0)
+    cand = np.arange(-7, 8, dtype=np.float64)
+    sx = np.repeat(s.astype(np.float64), 32, axis=-1)
+    for i in range(50):
+        for d in range(0, 128, 7):
+            if sx[i, d] == 0:
+                continue
+            err = np.abs(np.float64(np.float32(x[i, d]) / np.float32(sx[i, d])) - cand)
+            best = cand[err == err.min()]
+            want = best[0] if len(best) == 1 else best[(best % 2) == 0][0]
+            assert q[i, d] == want, (i, d)
+    big = np.abs(x.reshape(50, 4, 32)).argmax(-1)
+    for i in range(50):
+        for g in range(4):
+            if s[i, g] > 0:
+                assert abs(int(q[i, g * 32 + big[i, g]])) == 7
+
+
+def test_int4_error_is_within_half_a_scale_step():
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((200, 128)).astype(np.float32)
+    q, s = int4.quantize(x)
+    err = np.abs(int4.dequantize(q, s) - x.astype(np.float64))
+    # half a step, plus the fp16 rounding of the scale stretched over 7 steps
+    bound = np.repeat(s.astype(np.float64), 32, axis=-1) * (0.5 + 7 * 2.0 ** -11) + 1e-30
+    assert np.all(err <= bound)
 
 
 def test_zero_keys_give_uniform_mean_of_visible_values():
