@@ -41,7 +41,8 @@ constexpr int kAppendThreads = 32 * kAppendHeadsPerCta;
 // and store it once the destination is known.
 // seq_ids (nullable): pool sequence of batch row b, else b.  pos_arr
 // (nullable): position of batch row b, else `pos` for every row.
-template <typename InT, bool FP8>
+// STORE: 0 = copy (bf16 / fp32 store), 1 = FP8, 2 = 4-bit
+template <typename InT, int STORE>
 __global__ void __launch_bounds__(kAppendThreads)
     append_evict_kernel(PoolView v, int l0, int nl, int batch, int64_t pos, const InT* k,
                         const InT* vv, const uint8_t* evict, const int32_t* seq_ids,
@@ -69,7 +70,7 @@ __global__ void __launch_bounds__(kAppendThreads)
   const int nch = int(v.row_bytes >> 4);       // chunks per row: 8, 16 or 32
   constexpr int kMaxPerLane = 2;               // 2 * 32 chunks per lane pair covers fp32 D=128
   uint4 chunk[kMaxPerLane];
-  if constexpr (!FP8) {
+  if constexpr (STORE == 0) {
 #pragma unroll
     for (int r = 0; r < kMaxPerLane; ++r) {
       const int c = lane + 32 * r;
@@ -98,7 +99,20 @@ __global__ void __launch_bounds__(kAppendThreads)
   uint8_t* blk = v.blocks + int64_t(prow / v.BT) * v.block_bytes;
 
   // ---- store the row ----
-  if constexpr (!FP8) {
+  if constexpr (STORE == 2) {
+    if (opened) {   // tokens past the last one of a new block decode to 0
+      uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);
+      for (int c = lane; c < int(v.tile_bytes / 16); c += 32) tile[c] = make_uint4(0, 0, 0, 0);
+      __syncwarp();
+    }
+    float k4[4], v4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      k4[e] = in_to_f32(k[int64_t(i) * v.D + 4 * lane + e]);
+      v4[e] = in_to_f32(vv[int64_t(i) * v.D + 4 * lane + e]);
+    }
+    store_row_int4(v, prow, k4, v4, lane);
+  } else if constexpr (STORE == 0) {
 #pragma unroll
     for (int r = 0; r < kMaxPerLane; ++r) {
       const int c = lane + 32 * r;
@@ -166,8 +180,8 @@ static dms_status launch_append(dms_pool* pool, int layer0, int n_layers, int ba
     set_last_error("null input pointer");
     return DMS_ERR_INVALID_ARG;
   }
-  const bool fp8 = pv.kv_dtype == DMS_FP8_E4M3;
-  if (!(in_dtype == DMS_F32 || in_dtype == DMS_BF16) || (!fp8 && int(in_dtype) != pv.kv_dtype)) {
+  const bool fp8 = pv.kv_dtype == DMS_FP8_E4M3, int4 = pv.kv_dtype == DMS_INT4;
+  if (!(in_dtype == DMS_F32 || in_dtype == DMS_BF16) || (!fp8 && !int4 && int(in_dtype) != pv.kv_dtype)) {
     set_last_error("in_dtype %d does not match kv_dtype %d", int(in_dtype), pv.kv_dtype);
     return DMS_ERR_INVALID_ARG;
   }
@@ -183,12 +197,15 @@ static dms_status launch_append(dms_pool* pool, int layer0, int n_layers, int ba
                               pv, layer0, n_layers, batch, pos, static_cast<const T*>(k),         \
                               static_cast<const T*>(v), evict, seq_ids, pos_arr),                 \
                    "append_evict_kernel")
+  const int mode = fp8 ? 1 : int4 ? 2 : 0;
   if (in_dtype == DMS_BF16) {
-    if (fp8) DMS_LAUNCH_APPEND(__nv_bfloat16, true);
-    else DMS_LAUNCH_APPEND(__nv_bfloat16, false);
+    if (mode == 1) DMS_LAUNCH_APPEND(__nv_bfloat16, 1);
+    else if (mode == 2) DMS_LAUNCH_APPEND(__nv_bfloat16, 2);
+    else DMS_LAUNCH_APPEND(__nv_bfloat16, 0);
   } else {
-    if (fp8) DMS_LAUNCH_APPEND(float, true);
-    else DMS_LAUNCH_APPEND(float, false);
+    if (mode == 1) DMS_LAUNCH_APPEND(float, 1);
+    else if (mode == 2) DMS_LAUNCH_APPEND(float, 2);
+    else DMS_LAUNCH_APPEND(float, 0);
   }
 #undef DMS_LAUNCH_APPEND
   return st;

@@ -92,16 +92,95 @@ __device__ __forceinline__ AppendSlot append_bookkeeping(const PoolView& v, int 
   return r;
 }
 
+// ---- 4-bit rows (DMS_INT4, head_dim 128) ----
+// Scale of a group of 32: fp16(amax / 7) (fp32 quotient, nearest even,
+// 65504 at most); code = clamp(rint(x / scale), -7, 7), kept as the nibble
+// code + 8; scale 0 gives code 0.
+__device__ __forceinline__ float int4_group_scale(float amax) {
+  const float s = __half2float(__float2half_rn(__fdiv_rn(amax, 7.f)));
+  return s > 65504.f ? 65504.f : s;
+}
+__device__ __forceinline__ uint32_t int4_nibble(float x, float scale) {
+  if (!(scale > 0.f)) return 8u;
+  const float r = fminf(fmaxf(rintf(__fdiv_rn(x, scale)), -7.f), 7.f);
+  return uint32_t(int(r) + 8);
+}
+
+// One token's K and V rows into a 4-bit store (one warp): lane l holds
+// elements 4l .. 4l+3 of each row (values in input precision).  K words and
+// scales are written whole; V nibbles share 32-bit words with 7 other tokens
+// of the block, so they are cleared and set with atomics.
+__device__ __forceinline__ void store_row_int4(const PoolView& v, int prow, const float (&k4)[4],
+                                               const float (&v4)[4], int lane) {
+  const int row = prow % v.BT;
+  uint8_t* blk = v.blocks + int64_t(prow / v.BT) * v.block_bytes;
+  uint8_t* vt = blk + v.tile_bytes;
+  // group of lane l: elements 4l.. lie in group l / 8; amax over its 8 lanes
+  float ka = fmaxf(fmaxf(fabsf(k4[0]), fabsf(k4[1])), fmaxf(fabsf(k4[2]), fabsf(k4[3])));
+  float va = fmaxf(fmaxf(fabsf(v4[0]), fabsf(v4[1])), fmaxf(fabsf(v4[2]), fabsf(v4[3])));
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    ka = fmaxf(ka, __shfl_xor_sync(0xffffffffu, ka, o));
+    va = fmaxf(va, __shfl_xor_sync(0xffffffffu, va, o));
+  }
+  const float ks = int4_group_scale(ka), vs = int4_group_scale(va);
+  uint32_t c16 = 0;                  // the lane's four K nibbles, element 4l + i at bits 4i
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c16 |= int4_nibble(k4[i], ks) << (4 * i);
+  // K word (owner q, word kw) for lanes 0..15: element d = 32kw + 16j + 8hi + 2q + lo
+  // comes from lane 8kw + 4j + 2hi + q/2, nibble 2(q&1) + lo
+  uint32_t word = 0;
+  const int q = (lane >> 2) & 3, kw = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+#pragma unroll
+    for (int hi = 0; hi < 2; ++hi) {
+      const int src = lane < 16 ? 8 * kw + 4 * j + 2 * hi + (q >> 1) : lane;
+      const uint32_t pair = (__shfl_sync(0xffffffffu, c16, src) >> (8 * (q & 1))) & 0xFFu;
+      word |= (pair & 0xFu) << (8 * j + 4 * hi);
+      word |= (pair >> 4) << (8 * j + 4 * hi + 16);
+    }
+  }
+  if (lane < 16) *reinterpret_cast<uint32_t*>(blk + row * 64 + q * 16 + kw * 4) = word;
+  if ((lane & 7) == 0) {
+    *reinterpret_cast<__half*>(blk + int4k_scale(row, lane >> 3)) = __float2half_rn(ks);
+    *reinterpret_cast<__half*>(vt + int4v_scale(row, lane >> 3)) = __float2half_rn(vs);
+  }
+  const int sh = int4v_shift(row);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t* w = reinterpret_cast<uint32_t*>(vt + int4v_word(4 * lane + i, row));
+    atomicAnd(w, ~(0xFu << sh));
+    atomicOr(w, int4_nibble(v4[i], vs) << sh);
+  }
+}
+
 // Store one token's K and V rows, given as float values already rounded to
 // the store's input precision, into physical row prow (one warp).  bf16 and
 // fp32 stores copy the values; an FP8 store quantises them with the layer's
-// scales (E4M3 of x / scale, nearest even, saturating) and, when the token
-// opened its block, clears the block's transposed V tile first.
+// scales (E4M3 of x / scale, nearest even, saturating), a 4-bit store with
+// per-group scales; both clear the block's transposed V tile first when the
+// token opened its block.
 __device__ __forceinline__ void store_row_from_float(const PoolView& v, int l, int h, int prow,
                                                      int opened, const float* krow,
                                                      const float* vrow, int lane) {
   const int row = prow % v.BT;
   uint8_t* blk = v.blocks + int64_t(prow / v.BT) * v.block_bytes;
+  if (v.kv_dtype == DMS_INT4) {
+    if (opened) {   // tokens past the last one of a new block decode to 0
+      uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);
+      for (int c = lane; c < int(v.tile_bytes / 16); c += 32) tile[c] = make_uint4(0, 0, 0, 0);
+      __syncwarp();
+    }
+    float k4[4], v4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      k4[i] = krow[4 * lane + i];
+      v4[i] = vrow[4 * lane + i];
+    }
+    store_row_int4(v, prow, k4, v4, lane);
+    return;
+  }
   if (v.kv_dtype == DMS_FP8_E4M3) {
     if (opened) {
       uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);

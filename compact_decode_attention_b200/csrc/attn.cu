@@ -38,7 +38,18 @@
 
 namespace dms {
 
-enum { KV_F32 = 0, KV_BF16 = 1, KV_FP8 = 2 };
+enum { KV_F32 = 0, KV_BF16 = 1, KV_FP8 = 2, KV_INT4 = 3 };
+
+// 4-bit codes at bits 0 and 16 of x (stored as code + 8) -> f16x2 of the codes, exact
+__device__ __forceinline__ uint32_t int4x2_to_f16x2(uint32_t x) {
+  const uint32_t h = (x & 0x000F000Fu) | 0x64006400u;   // 1024 + nibble
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h), __half2half2(__ushort_as_half(0x6408)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
 
 // Stage ownership: unit k goes to stage k % NS and to consumer warp k % NCW.
 // NS must be a multiple of NCW so that every stage always belongs to the same
@@ -50,7 +61,8 @@ template <int KV, int D>
 struct AttnTraits {
   static constexpr int ESZ = KV == KV_F32 ? 4 : KV == KV_BF16 ? 2 : 1;
   static constexpr int QESZ = KV == KV_F32 ? 4 : 2;  // q / out element bytes
-  static constexpr int ROWB = D * ESZ;
+  // 4-bit rows: 64 bytes of nibbles + 4 fp16 group scales (see DMS_INT4)
+  static constexpr int ROWB = KV == KV_INT4 ? D / 2 + D / 16 : D * ESZ;
   static constexpr int TILEB = kBlockTokens * ROWB;
   // The fp32 path reads its query rows from the stage (QB bytes after the
   // tiles); the tensor-core paths load query fragments from global memory.
@@ -159,7 +171,7 @@ struct MmaWarp {
     for (int kt = 0; kt < KSTEPS; ++kt) {
       const uint32_t lo = real ? __ldg(reinterpret_cast<const unsigned int*>(qrow + kt * 16 + q2)) : 0u;
       const uint32_t hi = real ? __ldg(reinterpret_cast<const unsigned int*>(qrow + kt * 16 + 8 + q2)) : 0u;
-      if constexpr (KV == KV_FP8) {
+      if constexpr (KV == KV_FP8 || KV == KV_INT4) {
         const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
         const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
         qf[kt][0] = pack_f16x2(a.x, a.y);
@@ -173,7 +185,7 @@ struct MmaWarp {
 
   __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                       uint32_t b1) {
-    if constexpr (KV == KV_FP8) mma_f16_16816(d, a, b0, b1);
+    if constexpr (KV == KV_FP8 || KV == KV_INT4) mma_f16_16816(d, a, b0, b1);
     else mma_bf16_16816(d, a, b0, b1);
   }
 
@@ -225,6 +237,35 @@ struct MmaWarp {
         }
       }
     }
+    if constexpr (KV == KV_INT4) {
+      // each lane reads its 32 K nibbles of a row in one 16-byte load; k-step
+      // kt takes 4 of them from word kt/2 and scales them by group kt/2
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        if (mt * 16 < rows) {
+          const int r0 = mt * 16 + r8, r1 = r0 + 8;
+          const uint4 k0 = *reinterpret_cast<const uint4*>(Ks + r0 * 64 + q * 16);
+          const uint4 k1 = *reinterpret_cast<const uint4*>(Ks + r1 * 64 + q * 16);
+          const uint2 c0 = *reinterpret_cast<const uint2*>(Ks + kInt4Nibbles + r0 * 8);
+          const uint2 c1 = *reinterpret_cast<const uint2*>(Ks + kInt4Nibbles + r1 * 8);
+          const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+          const uint32_t s0[4] = {__byte_perm(c0.x, 0, 0x1010), __byte_perm(c0.x, 0, 0x3232),
+                                  __byte_perm(c0.y, 0, 0x1010), __byte_perm(c0.y, 0, 0x3232)};
+          const uint32_t s1[4] = {__byte_perm(c1.x, 0, 0x1010), __byte_perm(c1.x, 0, 0x3232),
+                                  __byte_perm(c1.y, 0, 0x1010), __byte_perm(c1.y, 0, 0x3232)};
+#pragma unroll
+          for (int kt = 0; kt < KSTEPS; ++kt) {
+            const int sh = 8 * (kt & 1);
+            uint32_t a[4];
+            a[0] = hmul2_u32(int4x2_to_f16x2(w0[kt >> 1] >> sh), s0[kt >> 1]);
+            a[1] = hmul2_u32(int4x2_to_f16x2(w1[kt >> 1] >> sh), s1[kt >> 1]);
+            a[2] = hmul2_u32(int4x2_to_f16x2(w0[kt >> 1] >> (sh + 4)), s0[kt >> 1]);
+            a[3] = hmul2_u32(int4x2_to_f16x2(w1[kt >> 1] >> (sh + 4)), s1[kt >> 1]);
+            mma(s[mt], a, qf[kt][0], qf[kt][1]);
+          }
+        }
+      }
+    }
     // ---- scale, mask rows past `rows`, online softmax ----
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -263,7 +304,7 @@ struct MmaWarp {
       const float p2 = fast_exp2(s[mt][2] - mn0), p3 = fast_exp2(s[mt][3] - mn1);
       l[0] += p0 + p2;
       l[1] += p1 + p3;
-      if constexpr (KV == KV_FP8) {
+      if constexpr (KV == KV_FP8 || KV == KV_INT4) {
         pb[mt][0] = movmatrix_trans(pack_f16x2(p0, p1));
         pb[mt][1] = movmatrix_trans(pack_f16x2(p2, p3));
       } else {
@@ -287,6 +328,29 @@ struct MmaWarp {
           const int ch = 2 * md + ((lane >> 3) & 1);
           uint32_t a[4];
           ldmatrix_x4_trans(a, vbase + row * T::ROWB + (swz_chunk(ch, row) << 4));
+          if (partial) {
+            a[0] &= m01;
+            a[1] &= m01;
+            a[2] &= m23;
+            a[3] &= m23;
+          }
+          mma(o[md], a, pb[mt][0], pb[mt][1]);
+        }
+      } else if constexpr (KV == KV_INT4) {  // V^T tile [D][64 tokens] of nibbles
+        const int t0 = mt * 16 + 2 * q, sh = 8 * (mt & 1);
+#pragma unroll
+        for (int md = 0; md < MTD; ++md) {
+          const int d0 = md * 16 + r8, gq = md >> 1;
+          const uint2 x0 = *reinterpret_cast<const uint2*>(Vs + d0 * 32 + q * 8);
+          const uint2 x1 = *reinterpret_cast<const uint2*>(Vs + (d0 + 8) * 32 + q * 8);
+          const uint32_t w0 = (mt >> 1) ? x0.y : x0.x, w1 = (mt >> 1) ? x1.y : x1.x;
+          const uint32_t sA = *reinterpret_cast<const uint32_t*>(Vs + kInt4Nibbles + gq * 128 + t0 * 2);
+          const uint32_t sB = *reinterpret_cast<const uint32_t*>(Vs + kInt4Nibbles + gq * 128 + (t0 + 8) * 2);
+          uint32_t a[4];
+          a[0] = hmul2_u32(int4x2_to_f16x2(w0 >> sh), sA);
+          a[1] = hmul2_u32(int4x2_to_f16x2(w1 >> sh), sA);
+          a[2] = hmul2_u32(int4x2_to_f16x2(w0 >> (sh + 4)), sB);
+          a[3] = hmul2_u32(int4x2_to_f16x2(w1 >> (sh + 4)), sB);
           if (partial) {
             a[0] &= m01;
             a[1] &= m01;
@@ -602,9 +666,11 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
             const uint8_t* qsrc = p.q + int64_t(ji / v.Hkv) * v.Hq * D * T::QESZ +
                                   int64_t(ji % v.Hkv) * qrow_bytes;
             const uint32_t kbytes = uint32_t(jrows) * T::ROWB;
-            const bool whole = jrows == kBlockTokens;
+            // 4-bit tiles keep their scales after the nibbles: always copied whole
+            const bool whole = jrows == kBlockTokens || KV == KV_INT4;
             const uint32_t vbytes = (whole || KV == KV_FP8) ? T::TILEB : kbytes;
-            mbar_arrive_expect_tx(&full[s], kbytes + vbytes + (T::QB > 0 ? qrow_bytes : 0));
+            mbar_arrive_expect_tx(&full[s], (whole ? T::TILEB : kbytes) + vbytes +
+                                                (T::QB > 0 ? qrow_bytes : 0));
             if (whole) {
               bulk_g2s(st, src, 2 * T::TILEB, &full[s], pol);
             } else {
@@ -811,6 +877,7 @@ static dms_status run_attn(dms_pool* pool, int layer0, int n_layers, int batch, 
     return v.D == 128 ? launch_attn<KV_BF16, 128>(prm, stream) : launch_attn<KV_BF16, 64>(prm, stream);
   }
   if (v.kv_dtype == DMS_FP8_E4M3) return launch_attn<KV_FP8, 128>(prm, stream);
+  if (v.kv_dtype == DMS_INT4) return launch_attn<KV_INT4, 128>(prm, stream);
   return v.D == 128 ? launch_attn<KV_F32, 128>(prm, stream) : launch_attn<KV_F32, 64>(prm, stream);
 }
 

@@ -110,6 +110,25 @@ __host__ __device__ __forceinline__ int fp8v_byte(int r, int d) {
   return d * 64 + ((((r & 7) >> 1) << 4) | ((r >> 4) << 2) | (((r >> 3) & 1) << 1) | (r & 1));
 }
 
+// 4-bit rows (head_dim 128): see DMS_INT4 in dms.h.  Byte offset of the
+// 32-bit word holding element d of K row r, and the bit of its nibble;
+// the same for token t of V element row d; scale offsets in a tile.
+constexpr int kInt4Nibbles = 4096;  // nibble bytes of a tile; scales follow
+__host__ __device__ __forceinline__ int int4k_word(int r, int d) {
+  return r * 64 + (((d & 7) >> 1) << 4) + ((d >> 5) << 2);
+}
+__host__ __device__ __forceinline__ int int4k_shift(int d) {
+  return 8 * ((d >> 4) & 1) + 4 * ((d >> 3) & 1) + 16 * (d & 1);
+}
+__host__ __device__ __forceinline__ int int4v_word(int d, int t) {
+  return d * 32 + (((t & 7) >> 1) << 3) + ((t >> 5) << 2);
+}
+__host__ __device__ __forceinline__ int int4v_shift(int t) {
+  return 8 * ((t >> 4) & 1) + 4 * ((t >> 3) & 1) + 16 * (t & 1);
+}
+__host__ __device__ __forceinline__ int int4k_scale(int r, int j) { return kInt4Nibbles + r * 8 + j * 2; }
+__host__ __device__ __forceinline__ int int4v_scale(int t, int j) { return kInt4Nibbles + j * 128 + t * 2; }
+
 // ------------------------------------------------------------------------
 // PTX wrappers
 // ------------------------------------------------------------------------

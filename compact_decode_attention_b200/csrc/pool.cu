@@ -65,7 +65,8 @@ static dms_status plan_layout(const dms_pool_config* c, dms_pool_layout_t* lay) 
     set_last_error("GQA group %d > 8 is not built", g);
     return DMS_ERR_UNSUPPORTED;
   }
-  if (c->kv_dtype != DMS_F32 && c->kv_dtype != DMS_BF16 && c->kv_dtype != DMS_FP8_E4M3) {
+  if (c->kv_dtype != DMS_F32 && c->kv_dtype != DMS_BF16 && c->kv_dtype != DMS_FP8_E4M3 &&
+      c->kv_dtype != DMS_INT4) {
     set_last_error("bad kv_dtype %d", c->kv_dtype);
     return DMS_ERR_INVALID_ARG;
   }
@@ -73,8 +74,8 @@ static dms_status plan_layout(const dms_pool_config* c, dms_pool_layout_t* lay) 
     set_last_error("head_dim %d not built (64, 128)", c->head_dim);
     return DMS_ERR_UNSUPPORTED;
   }
-  if (c->kv_dtype == DMS_FP8_E4M3 && c->head_dim != 128) {
-    set_last_error("FP8 pools are built for head_dim 128 only");
+  if ((c->kv_dtype == DMS_FP8_E4M3 || c->kv_dtype == DMS_INT4) && c->head_dim != 128) {
+    set_last_error("FP8 and 4-bit pools are built for head_dim 128 only");
     return DMS_ERR_UNSUPPORTED;
   }
   if (c->block_tokens != kBlockTokens) {
@@ -92,7 +93,9 @@ static dms_status plan_layout(const dms_pool_config* c, dms_pool_layout_t* lay) 
     return DMS_ERR_INVALID_ARG;
   }
   const int64_t n_chunks = (c->max_context + kPrefillChunk - 1) / kPrefillChunk;
-  const int64_t row_bytes = int64_t(c->head_dim) * elem_bytes(c->kv_dtype);
+  // 4-bit rows: D/2 bytes of nibbles + one fp16 scale per 32 elements
+  const int64_t row_bytes = c->kv_dtype == DMS_INT4 ? int64_t(c->head_dim) / 2 + c->head_dim / 16
+                                                    : int64_t(c->head_dim) * elem_bytes(c->kv_dtype);
 
   memset(lay, 0, sizeof(*lay));
   uint64_t off = 0;
@@ -120,7 +123,7 @@ static dms_status plan_layout(const dms_pool_config* c, dms_pool_layout_t* lay) 
   lay->max_blocks_per_head = int32_t(mbh);
   lay->free_stack_cap = kFreeStackCap;
   lay->n_heads = int32_t(n_heads);
-  lay->fp8_layout = c->kv_dtype == DMS_FP8_E4M3 ? 1 : 0;
+  lay->fp8_layout = c->kv_dtype == DMS_FP8_E4M3 ? 1 : c->kv_dtype == DMS_INT4 ? 2 : 0;
   return DMS_OK;
 }
 

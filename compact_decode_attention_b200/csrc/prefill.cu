@@ -20,7 +20,7 @@
 //   scatter  per (sequence, kv-head, chunk): ranks by ballot/popcount +
 //            the chunk base give each kept row its slot; copy (or quantise)
 //            the row into its block, fill the window ring.
-#include "dms_internal.cuh"
+#include "append_core.cuh"
 
 namespace dms {
 
@@ -231,8 +231,9 @@ __global__ void __launch_bounds__(256) prefill_fp8_clear_tail_kernel(PoolView v,
 }
 
 // ---------------------------------------------------------------------------
-// One CTA per (256-token chunk, kv-head, sequence).
-template <typename InT, bool FP8>
+// One CTA per (256-token chunk, kv-head, sequence).  STORE: 0 = copy
+// (bf16 / fp32 store), 1 = FP8, 2 = 4-bit.
+template <typename InT, int STORE>
 __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int layer, int seq0, int P,
                                                               const InT* __restrict__ k,
                                                               const InT* __restrict__ vv,
@@ -269,7 +270,24 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
     }
   }
   __syncthreads();
-  if constexpr (!FP8) {
+  if constexpr (STORE == 2) {
+    // 4-bit: one warp quantises one kept row (lane l: elements 4l .. 4l+3)
+    for (int kk = warp; kk < nkept; kk += blockDim.x / 32) {
+      const int jj = chunk * kPrefillChunk + s_kept[kk];
+      const int slot = base + kk;
+      const int blk = table[slot / v.BT];
+      if (!DMS_CHECK(blk >= 0 && blk < v.max_blocks, v.hdr, 202, hd, slot)) continue;
+      const InT* srck = k + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
+      const InT* srcv = vv + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
+      float k4[4], v4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        k4[e] = to_f32(srck[4 * lane + e]);
+        v4[e] = to_f32(srcv[4 * lane + e]);
+      }
+      store_row_int4(v, blk * v.BT + slot % v.BT, k4, v4, lane);
+    }
+  } else if constexpr (STORE == 0) {
     // bitwise row copy in 16-byte chunks, swizzled by row; each thread loads
     // kBatchItems K and V chunks before storing any
     const int nch = int(v.row_bytes >> 4);
@@ -384,8 +402,8 @@ extern "C" dms_status dms_compact_prefill_seqs(dms_pool* pool, int layer, int se
     set_last_error("null input pointer");
     return DMS_ERR_INVALID_ARG;
   }
-  const bool fp8 = pv.kv_dtype == DMS_FP8_E4M3;
-  if (!(in_dtype == DMS_F32 || in_dtype == DMS_BF16) || (!fp8 && int(in_dtype) != pv.kv_dtype)) {
+  const bool fp8 = pv.kv_dtype == DMS_FP8_E4M3, int4 = pv.kv_dtype == DMS_INT4;
+  if (!(in_dtype == DMS_F32 || in_dtype == DMS_BF16) || (!fp8 && !int4 && int(in_dtype) != pv.kv_dtype)) {
     set_last_error("in_dtype %d does not match kv_dtype %d", int(in_dtype), pv.kv_dtype);
     return DMS_ERR_INVALID_ARG;
   }
@@ -415,7 +433,7 @@ extern "C" dms_status dms_compact_prefill_seqs(dms_pool* pool, int layer, int se
   }
   st = prefill_plan_launch(pool, layer, seq0, batch, prompt_len, evict, stream);
   if (st != DMS_OK) return st;
-  if (fp8) {
+  if (fp8 || int4) {   // the V tile of each head's partly filled last block
     prefill_fp8_clear_tail_kernel<<<batch * pv.Hkv, 256, 0, stream>>>(pv, layer, seq0);
     st = cuda_status(cudaGetLastError(), "prefill_fp8_clear_tail_kernel");
     if (st != DMS_OK) return st;
@@ -425,16 +443,20 @@ extern "C" dms_status dms_compact_prefill_seqs(dms_pool* pool, int layer, int se
     auto kk = static_cast<const __nv_bfloat16*>(k);
     auto vv = static_cast<const __nv_bfloat16*>(v);
     if (fp8)
-      prefill_scatter_kernel<__nv_bfloat16, true><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<__nv_bfloat16, 1><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
+    else if (int4)
+      prefill_scatter_kernel<__nv_bfloat16, 2><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
     else
-      prefill_scatter_kernel<__nv_bfloat16, false><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<__nv_bfloat16, 0><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
   } else {
     auto kk = static_cast<const float*>(k);
     auto vv = static_cast<const float*>(v);
     if (fp8)
-      prefill_scatter_kernel<float, true><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<float, 1><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
+    else if (int4)
+      prefill_scatter_kernel<float, 2><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
     else
-      prefill_scatter_kernel<float, false><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
+      prefill_scatter_kernel<float, 0><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
   }
   return cuda_status(cudaGetLastError(), "prefill_scatter_kernel");
 }

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libdms_debug.so" if os.environ.get("DMS_LIBRARY"
                         else "libdms.so")
 
 DMS_OK, DMS_ERR_INVALID_ARG, DMS_ERR_CAPACITY, DMS_ERR_CUDA, DMS_ERR_UNSUPPORTED, DMS_ERR_DEVICE = range(6)
-DMS_F32, DMS_BF16, DMS_FP8_E4M3 = 0, 1, 2
+DMS_F32, DMS_BF16, DMS_FP8_E4M3, DMS_INT4 = 0, 1, 2, 3
 
 DEVERR_BLOCKS_EXHAUSTED = 0x1
 DEVERR_HEAD_TABLE_FULL = 0x2

@@ -73,7 +73,7 @@ typedef enum {
   DMS_ERR_DEVICE = 5         /* the pool's device error word is non-zero   */
 } dms_status;
 
-typedef enum { DMS_F32 = 0, DMS_BF16 = 1, DMS_FP8_E4M3 = 2 } dms_dtype;
+typedef enum { DMS_F32 = 0, DMS_BF16 = 1, DMS_FP8_E4M3 = 2, DMS_INT4 = 3 } dms_dtype;
 
 /* Bits of the device error word (dms_pool_stats_t.error_flags). */
 #define DMS_DEVERR_BLOCKS_EXHAUSTED 0x1u  /* global block pool ran out; write skipped   */
@@ -109,8 +109,30 @@ typedef struct {
   int32_t max_blocks_per_head;  /* block table width                         */
   int32_t free_stack_cap;       /* per-head free stack capacity              */
   int32_t n_heads;              /* n_layers * max_batch * n_kv_heads         */
-  int32_t fp8_layout;           /* 1: FP8 rows use the permuted layout below */
+  int32_t fp8_layout;           /* 1: FP8 rows use the permuted layout below; 2: 4-bit rows (below) */
 } dms_pool_layout_t;
+
+/* DMS_INT4 pools (head_dim 128 only): a stored row is 128 signed 4-bit codes
+ * q in [-7, 7], kept as the nibble q + 8, with one fp16 scale per group of 32
+ * elements (scale = fp16(amax / 7), q = rint(x / scale); the stored value is
+ * q * scale).  row_bytes = 72 (64 bytes of nibbles + 4 scales).  A block is
+ *   K tile: [64 rows x 64 B nibbles][64 rows x 4 fp16 scales]
+ *   V tile: [128 element rows x 32 B nibbles, token-major][4 groups x 64 tokens fp16 scales]
+ * Nibble placement (the attention kernel's MMA fragments come out of one
+ * 16-byte load per row): element d of K row r lies in the 32-bit word at
+ * byte r*64 + q*16 + (kt>>1)*4 with q = (d&7)>>1, kt = d>>4, at bit
+ * 8*(kt&1) + 4*((d>>3)&1) + 16*(d&1); token t of V element row d lies in
+ * the word at byte d*32 + q*8 + (m>>1)*4 with q = (t&7)>>1, m = t>>4, at bit
+ * 8*(m&1) + 4*((t>>3)&1) + 16*(t&1).  Scale of K row r, group j: byte
+ * 4096 + r*8 + j*2; of V token t, group j: byte 4096 + j*128 + t*2.
+ * Decode attention on a 4-bit pool multiplies each code by its scale in
+ * fp16 and runs the dot products on fp16 operands with fp32 accumulation
+ * (the query is rounded to fp16 too), so stored values and queries must
+ * stay within the fp16 range (|x| <= 65504).
+ * Source: the pages pair token eviction with lower-bit KV (FastDMS page,
+ * paragraph after the speed table, and its comparison with 4-bit KV) but
+ * give no 4-bit format; the symmetric per-group format above is the plain
+ * reading. */
 
 typedef struct {
   int64_t retained_tokens;      /* sum of n_retained over all heads           */
@@ -163,12 +185,13 @@ dms_status dms_pool_layout(const dms_pool* pool, dms_pool_layout_t* out);
  * count and fills the window ring with positions max(0,P-w)..P-1.
  * For an FP8 pool the per-(layer, kv-head) scales become amax/448 over all
  * P*batch rows of that head (before eviction), K and V separately, and rows
- * are stored as e4m3(x / scale) (round to nearest even, saturating).
+ * are stored as e4m3(x / scale) (round to nearest even, saturating).  A
+ * 4-bit pool quantises each kept row with its own group scales (DMS_INT4).
  *   k, v   [batch, P, Hkv, D]  in_dtype (DMS_F32 or DMS_BF16)
  *   evict  [batch, P, Hkv]     uint8, non-zero = flagged
  * The layer must be empty (fresh pool or after dms_pool_reset), else the
  * device sets DMS_DEVERR_LAYER_NOT_EMPTY and writes nothing.  in_dtype
- * must equal kv_dtype, or be F32/BF16 for an FP8 pool.  (FP8: the scales
+ * must equal kv_dtype, or be F32/BF16 for an FP8 or 4-bit pool.  (FP8: the scales
  * are only set when the layer has none yet; see dms_compact_prefill_seqs.)
  * Source: compaction = the compact store of the FastDMS page; eviction
  * before FP8 quantisation = the same page's FP8 paragraph. */
@@ -257,7 +280,7 @@ dms_status dms_project_workspace_bytes(const dms_pool* pool, int n_seqs, int d_m
  *   w_evict  [d_model, Hkv]          bf16 (the predictor's weights: an input)
  *   b_evict  [Hkv] float, or null;   seq_ids int32 / pos int64 [n_seqs] device
  * fp32 accumulation, k and v rounded to nearest-even bf16.  Needs head_dim 128
- * and a bf16 or FP8 pool.  workspace may be null (no scratch is needed).
+ * and a bf16, FP8 or 4-bit pool.  workspace may be null (no scratch is needed).
  * Runs as one thread-block cluster of 8 CTAs per kv-head.
  * Source: a learned per-head predictor decides which tokens to evict
  * (mindverse page, DMS section); decode runs the projection step by step. */

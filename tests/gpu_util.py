@@ -83,6 +83,43 @@ def stored_rows(pool, state, hd: int, n: int, kind: str):
     return (_unpermute_rows(k_raw, rows, kind, D, "K"), _unpermute_rows(v_raw, rows, kind, D, "V"))
 
 
+def int4_rows(pool, state, hd: int, n: int):
+    """Codes and scales held in slots 0..n-1 of head hd of a 4-bit store:
+    (codes_k, scales_k, codes_v, scales_v), codes int8 [n, D] (nibble - 8),
+    scales float32 [n, D / 32], undoing the DMS_INT4 layout of include/dms.h."""
+    lay = pool.layout
+    D = pool.cfg.head_dim
+    tile = BT * (D // 2 + D // 16)
+    nib = BT * D // 2
+    slots = np.arange(n)
+    blk = state["bt"][hd, slots // BT].astype(np.int64)
+    rows = slots % BT
+    raw = {}
+    for b in np.unique(blk):
+        o = int(lay.blocks + b * lay.block_bytes)
+        raw[int(b)] = pool.buffer[o:o + 2 * tile].cpu().numpy()
+    d = np.arange(D)
+    kword = ((d & 7) >> 1) * 16 + (d >> 5) * 4                 # + row * 64
+    kshift = 8 * ((d >> 4) & 1) + 4 * ((d >> 3) & 1) + 16 * (d & 1)
+    ck = np.zeros((n, D), np.int8)
+    cv = np.zeros((n, D), np.int8)
+    sk = np.zeros((n, D // 32), np.float32)
+    sv = np.zeros((n, D // 32), np.float32)
+    for i in range(n):
+        kt = raw[int(blk[i])][:tile]
+        vt = raw[int(blk[i])][tile:]
+        r = int(rows[i])
+        kw = kt[:nib].view(np.uint32)[(r * 64 + kword) // 4]
+        ck[i] = ((kw >> kshift.astype(np.uint32)) & 0xF).astype(np.int16) - 8
+        vword = d * 32 + ((r & 7) >> 1) * 8 + (r >> 5) * 4
+        vshift = 8 * ((r >> 4) & 1) + 4 * ((r >> 3) & 1) + 16 * (r & 1)
+        vw = vt[:nib].view(np.uint32)[vword // 4]
+        cv[i] = ((vw >> np.uint32(vshift)) & 0xF).astype(np.int16) - 8
+        sk[i] = kt[nib:].view(np.float16).reshape(BT, D // 32)[r].astype(np.float32)
+        sv[i] = vt[nib:].view(np.float16).reshape(D // 32, BT)[:, r].astype(np.float32)
+    return ck, sk, cv, sv
+
+
 def expected_row_bytes(values_f32: np.ndarray, kind: str, scale=None) -> np.ndarray:
     """Bytes the store should hold for rows given in input precision (float32 array)."""
     if kind == "f32":
