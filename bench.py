@@ -21,6 +21,7 @@ Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 from __future__ import annotations
 
 import argparse
+import glob
 import hashlib
 import json
 import os
@@ -41,7 +42,9 @@ from synth import configs  # noqa: E402
 METRIC = "compact-KV decode attn: retained-KV GB/s vs HBM peak; decode steps/s at ctx 8K"
 DEFAULT_WORKLOAD = configs.QWEN8B_CTX8K.name
 ATTN_KERNEL_SRC = os.path.join(ROOT, "compact_decode_attention_b200", "csrc", "attn.cu")
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_attn_qwen3-8b_ctx8k.md")
+PROFILES = os.path.join(ROOT, "profiles")
+L2_BYTES = 126 * 1024 * 1024
+L2_FLUSH_BYTES = 512 * 1024 * 1024   # written between timed steps when the held K/V fits in L2
 
 
 def parse_args():
@@ -51,6 +54,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(configs.BY_NAME))
+    ap.add_argument("--kv-dtype", default=None, choices=["f32", "bf16", "fp8", "int4"],
+                    help="store the workload's K/V in this dtype instead of its own")
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-attention measurement")
     ap.add_argument("--prefill-only", action="store_true",
@@ -68,6 +73,21 @@ def parse_args():
 # ---------------------------------------------------------------------------
 # measured peaks, clocks
 # ---------------------------------------------------------------------------
+
+KV_TAGS = {"f32": "fp32", "bf16": "bf16", "fp8": "fp8e4m3", "int4": "int4g32"}
+
+
+def with_kv_dtype(wl, kv_dtype):
+    """The workload with its K/V stored in another dtype (the name's dtype
+    tag follows)."""
+    if not kv_dtype or kv_dtype == wl.kv_dtype:
+        return wl
+    import dataclasses
+    old, new = "_" + KV_TAGS[wl.kv_dtype], "_" + KV_TAGS[kv_dtype]
+    i = wl.name.rfind(old)
+    name = wl.name[:i] + new + wl.name[i + len(old):] if i >= 0 else wl.name + new
+    return dataclasses.replace(wl, name=name, kv_dtype=kv_dtype)
+
 
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -100,7 +120,7 @@ def projection_line(wl, device, n_calls=8):
     w_kv = (torch.randn(dm, 2 * Hkv * D, device=device, generator=g) / dm ** 0.5).to(torch.bfloat16)
     w_ev = (torch.randn(dm, Hkv, device=device, generator=g) / dm ** 0.5).to(torch.bfloat16)
     x = torch.randn(n_calls + 1, B, dm, device=device, generator=g).to(torch.bfloat16)
-    code = {"bf16": dms.DMS_BF16, "fp8": dms.DMS_FP8_E4M3}[wl.kv_dtype]
+    code = {"bf16": dms.DMS_BF16, "fp8": dms.DMS_FP8_E4M3, "int4": dms.DMS_INT4}[wl.kv_dtype]
     pool = dms.Pool(1, B, Hq, Hkv, D, wl.window, code, B * Hkv * 4, n_calls + 2, device=device)
     pos = [torch.full((B,), c, dtype=torch.int64, device=device) for c in range(n_calls + 1)]
     pool.project_append(0, None, pos[0], x[0], w_kv, w_ev)      # module load, workspace
@@ -120,7 +140,7 @@ def projection_line(wl, device, n_calls=8):
     if pool.stats(check=False).error_flags:
         raise SystemExit("the projection set the device error word")
     ms = e0.elapsed_time(e1) / n_calls
-    nbytes = (w_kv.numel() + w_ev.numel() + B * dm) * 2 + B * Hkv * 2 * D * wl.kv_elem_bytes()
+    nbytes = (w_kv.numel() + w_ev.numel() + B * dm) * 2 + B * Hkv * 2 * wl.kv_row_bytes()
     peak, kind = measured_peaks()
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"value": gbs, "unit": "GB/s", "us_per_layer": ms * 1e3, "d_model": dm, "batch": B,
@@ -254,7 +274,8 @@ def cpu_baseline(wl, t0: int, n_heads: int, n_steps: int, bytes_per_step: float)
         flags = oref.head_flags(wl, layer, b, h, T)
         need = np.unique(np.concatenate([oracle_visible(t, flags, wl.window) for t in (t0, T - 1)]))
         need = np.unique(np.concatenate([need, np.arange(max(0, t0 - wl.window), T)]))
-        K, V = oref.stored_rows(wl, layer, b, h, need)
+        K, V = oref.stored_rows(wl, layer, b, h, need,
+                                oref.fp8_head_scales(wl, layer, h) if wl.kv_dtype == "fp8" else None)
         Kf = np.zeros((T, wl.head_dim))
         Vf = np.zeros((T, wl.head_dim))
         Kf[need], Vf[need] = K, V
@@ -292,7 +313,7 @@ def expected_bytes_per_step(wl):
     """Expected retained K/V bytes per step from the workload's keep probabilities."""
     p = wl.keep_probs()
     n = np.minimum(wl.prompt, wl.window) + p * max(0, wl.prompt - wl.window)
-    return float(n.sum() * wl.batch * 2 * wl.head_dim * wl.kv_elem_bytes())
+    return float(n.sum() * wl.batch * 2 * wl.kv_row_bytes())
 
 
 # ---------------------------------------------------------------------------
@@ -307,19 +328,20 @@ def attn_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic_ratio():
+def profiled_traffic_ratio(workload: str):
     """DRAM bytes (read + write) per algorithmic byte of the attention kernel
-    from the committed ncu summary, when it was taken on the current kernel
-    source; else None.  The captured launch held fewer tokens than the timed
-    ones, so traffic is scaled by held bytes (read traffic tracks them 1:1)."""
-    if not os.path.exists(PROFILE_SUMMARY):
-        return None, None
-    txt = open(PROFILE_SUMMARY).read()
-    m_src = re.search(r"kernel source hash:\s*([0-9a-f]+)", txt)
-    m_tr = re.search(r"dram bytes per algorithmic byte:\s*([0-9.eE+]+)", txt)
-    if not (m_src and m_tr) or m_src.group(1) != attn_source_hash():
-        return None, None
-    return float(m_tr.group(1)), m_src.group(1)
+    from the committed ncu summary of this workload, when it was taken on the
+    current kernel source; else None.  The captured launch held fewer tokens
+    than the timed ones, so traffic is scaled by held bytes (read traffic
+    tracks them 1:1)."""
+    for f in sorted(glob.glob(os.path.join(PROFILES, "decode_attn_*.md"))):
+        txt = open(f).read()
+        m_wl = re.search(r"^workload:\s*(\S+)", txt, re.M)
+        m_src = re.search(r"kernel source hash:\s*([0-9a-f]+)", txt)
+        m_tr = re.search(r"dram bytes per algorithmic byte:\s*([0-9.eE+]+)", txt)
+        if m_wl and m_src and m_tr and m_wl.group(1) == workload and m_src.group(1) == attn_source_hash():
+            return float(m_tr.group(1)), m_src.group(1)
+    return None, None
 
 
 # ---------------------------------------------------------------------------
@@ -349,7 +371,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = configs.BY_NAME[args.workload]
+    wl = with_kv_dtype(configs.BY_NAME[args.workload], args.kv_dtype)
     bps = expected_bytes_per_step(wl)
     t0 = time.perf_counter()
     steps = max(1, args.steps)
@@ -396,7 +418,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    wl = configs.BY_NAME[args.workload]
+    wl = with_kv_dtype(configs.BY_NAME[args.workload], args.kv_dtype)
     if args.projection_only:       # the fused projection measurement alone (one GPU)
         line = projection_line(wl, f"cuda:{local}")
         if rank == 0:
@@ -421,7 +443,7 @@ def main():
 
     L, B, Hkv, D, w, P = wl.n_layers, wl.batch, wl.n_kv_heads, wl.head_dim, wl.window, wl.prompt
     H = L * B * Hkv
-    row_bytes = 2 * D * wl.kv_elem_bytes()           # K row + V row of one token
+    row_bytes = 2 * wl.kv_row_bytes()                # K row + V row of one token
 
     # exact held tokens after each step: +1 per head, -1 per head whose token
     # t - w carried a flag (flags drawn by the same device generator)
@@ -454,12 +476,31 @@ def main():
     # replayed once; positions advance every step, so each graph runs once ----
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     si = dw.step_inputs
+    # a held K/V that fits in L2 would be read from L2 by the next step: then
+    # every timed step starts after an L2 flush (a write of L2_FLUSH_BYTES,
+    # then a read of it, so that no dirty line is left for the step to write
+    # back), outside the event pair that times it, and the step times are summed
+    flush = bool(bytes_step[W] <= L2_BYTES)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{local}") if flush else None
+    flush_sink = torch.empty((), dtype=torch.int32, device=f"cuda:{local}")
+
+    def l2_flush(j):
+        flush_buf.fill_(j & 0xff)
+        torch.amax(flush_buf.view(torch.int32), dim=0, out=flush_sink)
+
+    step_ev = [(torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(K if flush else 0)]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for j in range(K):
             s = W + j
+            if flush:
+                l2_flush(j)
+                step_ev[j][0].record()
             dw.pool.append_evict_layers(0, P + s, si["k"][s], si["v"][s], si["evict"][s])
             dw.pool.decode_attn_layers(0, si["q"][s], dw.out)
+            if flush:
+                step_ev[j][1].record()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         barrier()
@@ -469,7 +510,7 @@ def main():
         t_end.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms = t_start.elapsed_time(t_end)
+    ms = sum(a.elapsed_time(b) for a, b in step_ev) if flush else t_start.elapsed_time(t_end)
     del graph
 
     # ---- the attention kernel alone: a second graph of R steps with event
@@ -482,6 +523,8 @@ def main():
     with torch.cuda.graph(graph):
         for j in range(R):
             s = W + K + j
+            if flush:
+                l2_flush(j)
             dw.pool.append_evict_layers(0, P + s, si["k"][s], si["v"][s], si["evict"][s])
             ev[j][0].record()
             dw.pool.decode_attn_layers(0, si["q"][s], dw.out)
@@ -503,11 +546,11 @@ def main():
     peak, peak_kind = measured_peaks()
     rbytes = bytes_step[W + K:W + K + R]
     achieved = float(rbytes.sum() / (attn_ms.sum() * 1e-3) / 1e9)
-    ratio, _ = profiled_traffic_ratio()
+    ratio, _ = profiled_traffic_ratio(wl.name)
     traffic = None if ratio is None else ratio * float(rbytes.mean())
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": "decode_attn_kernel<bf16,128>" if wl.kv_dtype == "bf16" and D == 128 else "decode_attn_kernel",
+                "kernel": f"decode_attn_kernel<{wl.kv_dtype},{D}>",
                 "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "algorithmic_bytes_per_launch": float(rbytes.mean()),
                 "attn_us_per_launch": float(attn_ms.mean() * 1e3),
@@ -526,17 +569,28 @@ def main():
         for j in range(E):
             s = e0s + j
             stp.pack(hin[j], si["k"][s], si["v"][s], si["q"][s], si["evict"][s])
+        flush_ms = 0.0
+        if flush:      # the flushes alone, subtracted from the timed loop below
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for j in range(E):
+                l2_flush(j)
+            f1.record(stream)
+            torch.cuda.synchronize()
+            flush_ms = f0.elapsed_time(f1)
         barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for j in range(E):
+            if flush:
+                l2_flush(j)
             stp.step(P + e0s + j, hin[j], hout[j])
         stp.join(stream)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms, e_bytes = reduce_over_ranks(e0.elapsed_time(e1), float(bytes_step[e0s:e0s + E].sum()),
+        e_ms, e_bytes = reduce_over_ranks(e0.elapsed_time(e1) - flush_ms, float(bytes_step[e0s:e0s + E].sum()),
                                           device=f"cuda:{local}")
         e2e = {"value": e_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": int(stp.layout.in_bytes), "d2h_bytes_per_step": int(stp.layout.out_bytes),
@@ -544,6 +598,9 @@ def main():
                "path": "dms_stepper_step: one packed pinned-host input copy, append/evict, decode "
                        "attention, one pinned-host output copy per step; copies on their own streams, "
                        "double-buffered against the neighbouring steps' kernels"}
+        if flush:
+            e2e["l2"] = (f"an L2 flush ({L2_FLUSH_BYTES >> 20} MB written then read) on the compute stream before each "
+                         f"step; their time alone ({flush_ms / E * 1e3:.1f} us per flush) is subtracted")
         stp.close()
 
     prefill = prefill_attention_line(wl, f"cuda:{local}") if not args.no_prefill else None
@@ -557,13 +614,18 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
-            "ms_per_step": ms_max / K, "timing": "CUDA events around one replay of a captured graph "
-                                                 "of the K steps", "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": ms_max / K,
+            "timing": ("sum of CUDA event pairs around each step in one replay of a captured graph of "
+                       "the K steps (an L2 flush between steps, outside the pairs)" if flush else
+                       "CUDA events around one replay of a captured graph of the K steps"), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.kv_dtype == "bf16" else wl.kv_dtype, "data": "synthetic",
             "config": {"workload": wl.name, "layers": L, "batch": B, "q_heads": wl.n_q_heads,
                        "kv_heads": Hkv, "head_dim": D, "prompt": P, "window": w, "kv_dtype": wl.kv_dtype,
                        "seed": wl.seed, "parallelism": f"replicas x{world}",
-                       "l2": (f"no flush: {bytes_step[W] / 1e6:.0f} MB of held K/V read per step "
+                       "l2": (f"flush: {L2_FLUSH_BYTES >> 20} MB written then read before each timed step, outside "
+                              f"its events ({bytes_step[W] / 1e6:.0f} MB of held K/V per step fits in "
+                              f"the 126 MB L2)" if flush else
+                              f"no flush: {bytes_step[W] / 1e6:.0f} MB of held K/V read per step "
                               f"> 126 MB L2")},
             "decode_steps_per_s": world * K / (ms_max * 1e-3),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "compaction": compaction,

@@ -40,12 +40,12 @@ namespace dms {
 
 enum { KV_F32 = 0, KV_BF16 = 1, KV_FP8 = 2, KV_INT4 = 3 };
 
-// 4-bit codes at bits 0 and 16 of x (stored as code + 8) -> f16x2 of the codes, exact
-__device__ __forceinline__ uint32_t int4x2_to_f16x2(uint32_t x) {
-  const uint32_t h = (x & 0x000F000Fu) | 0x64006400u;   // 1024 + nibble
-  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h), __half2half2(__ushort_as_half(0x6408)));
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
+// 4-bit codes: a LOP3 of the packed word with 0x64006400 turns the nibble
+// at bits 0-3 (and 16-19) into the f16 value 1024 + n, and the nibble at
+// bits 4-7 (and 20-23) into 1024 + 16 n; both are exact.  The offsets and
+// the factor 16 are taken out in fp32 / on the other MMA operand.
+__device__ __forceinline__ uint32_t nib_lo_f16x2(uint32_t w) { return (w & 0x000F000Fu) | 0x64006400u; }
+__device__ __forceinline__ uint32_t nib_hi_f16x2(uint32_t w) { return (w & 0x00F000F0u) | 0x64006400u; }
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
   return *reinterpret_cast<const uint32_t*>(&r);
@@ -72,8 +72,11 @@ struct AttnTraits {
   // 34 KB for bf16 D=128, 8 for the others): with two consumer warps per SM
   // sub-partition one warp's MMA / ldmatrix latency hides behind the other's.
   // fp32 (68 KB or 34 KB stages): 3 or 4 stages and warps.
-  static constexpr int NS = KV == KV_F32 ? (D == 128 ? 3 : 4) : (KV == KV_BF16 && D == 128) ? 6 : 8;
-  static constexpr int NCW = NS;                        // consumer warps
+  // 4-bit stages are 9 KB: two per consumer warp keep 147 KB in flight.
+  static constexpr int NS = KV == KV_F32 ? (D == 128 ? 3 : 4)
+                          : KV == KV_INT4 ? 16
+                          : (KV == KV_BF16 && D == 128) ? 6 : 8;
+  static constexpr int NCW = KV == KV_INT4 ? 8 : NS;   // consumer warps
   static constexpr int THREADS = 32 * (NCW + 1);       // + one producer warp
   static constexpr int COMBINE_FLOATS = NCW * 8 * D + 2 * NCW * 8;
   static constexpr int MISC_INTS = 16 + THREADS / 32;
@@ -153,12 +156,21 @@ struct MmaWarp {
   uint32_t qf[KSTEPS][2];
   float scale;  // log2-domain score scale (includes the K scale for FP8)
   float vscale; // V scale (FP8), else 1
+  // 4-bit stores only: per 32-element group g, the offset that the 1024 + m n
+  // decoding adds to q . k for query columns 2(lane&3) and 2(lane&3)+1 ...
+  float cq[4][2];
+  // ... and the one it adds to each output row of group g (accumulated like o)
+  float eo[4][4];
 
   __device__ __forceinline__ void reset() {
     m[0] = m[1] = -INFINITY;
     l[0] = l[1] = 0.f;
 #pragma unroll
     for (int i = 0; i < MTD; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    if constexpr (KV == KV_INT4) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) eo[i][0] = eo[i][1] = eo[i][2] = eo[i][3] = 0.f;
+    }
   }
 
   // Q^T B fragments of the group's query rows (row n = lane / 4 < g; the
@@ -171,14 +183,41 @@ struct MmaWarp {
     for (int kt = 0; kt < KSTEPS; ++kt) {
       const uint32_t lo = real ? __ldg(reinterpret_cast<const unsigned int*>(qrow + kt * 16 + q2)) : 0u;
       const uint32_t hi = real ? __ldg(reinterpret_cast<const unsigned int*>(qrow + kt * 16 + 8 + q2)) : 0u;
-      if constexpr (KV == KV_FP8 || KV == KV_INT4) {
+      if constexpr (KV == KV_FP8) {
         const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
         const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
         qf[kt][0] = pack_f16x2(a.x, a.y);
         qf[kt][1] = pack_f16x2(b.x, b.y);
+      } else if constexpr (KV == KV_INT4) {
+        // k-columns 8..15 of a k-step meet K nibbles decoded as 1024 + 16 n:
+        // their query values enter divided by 16 (exact)
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+        qf[kt][0] = pack_f16x2(a.x, a.y);
+        qf[kt][1] = pack_f16x2(b.x * 0.0625f, b.y * 0.0625f);
       } else {
         qf[kt][0] = lo;
         qf[kt][1] = hi;
+      }
+    }
+    if constexpr (KV == KV_INT4) {
+      // Sum over group g of q'_d (1024 + 8 m_d), q' the f16 operand and m_d
+      // its nibble factor (1 or 16): what the decoding adds to the group's
+      // dot product.  This lane holds query row lane/4; columns 2(lane&3),
+      // 2(lane&3)+1 of the MMA accumulator need rows 2(lane&3) and +1.
+#pragma unroll
+      for (int gq = 0; gq < 4; ++gq) {
+        float c = 0.f;
+#pragma unroll
+        for (int kt = 2 * gq; kt < 2 * gq + 2; ++kt) {
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&qf[kt][0]));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&qf[kt][1]));
+          c += 1032.f * (a.x + a.y) + 1152.f * (b.x + b.y);
+        }
+        c += __shfl_xor_sync(0xffffffffu, c, 1);
+        c += __shfl_xor_sync(0xffffffffu, c, 2);
+        cq[gq][0] = __shfl_sync(0xffffffffu, c, 8 * (lane & 3));
+        cq[gq][1] = __shfl_sync(0xffffffffu, c, 8 * (lane & 3) + 4);
       }
     }
   }
@@ -238,8 +277,9 @@ struct MmaWarp {
       }
     }
     if constexpr (KV == KV_INT4) {
-      // each lane reads its 32 K nibbles of a row in one 16-byte load; k-step
-      // kt takes 4 of them from word kt/2 and scales them by group kt/2
+      // one 16-byte load gives a lane its 32 K nibbles of a row: word g holds
+      // group g (k-steps 2g and 2g+1).  Per group, two MMAs start from minus
+      // the decoding offset, and the group's K scale multiplies the result.
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
         if (mt * 16 < rows) {
@@ -249,19 +289,31 @@ struct MmaWarp {
           const uint2 c0 = *reinterpret_cast<const uint2*>(Ks + kInt4Nibbles + r0 * 8);
           const uint2 c1 = *reinterpret_cast<const uint2*>(Ks + kInt4Nibbles + r1 * 8);
           const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-          const uint32_t s0[4] = {__byte_perm(c0.x, 0, 0x1010), __byte_perm(c0.x, 0, 0x3232),
-                                  __byte_perm(c0.y, 0, 0x1010), __byte_perm(c0.y, 0, 0x3232)};
-          const uint32_t s1[4] = {__byte_perm(c1.x, 0, 0x1010), __byte_perm(c1.x, 0, 0x3232),
-                                  __byte_perm(c1.y, 0, 0x1010), __byte_perm(c1.y, 0, 0x3232)};
+          const float2 s0a = __half22float2(*reinterpret_cast<const __half2*>(&c0.x));
+          const float2 s0b = __half22float2(*reinterpret_cast<const __half2*>(&c0.y));
+          const float2 s1a = __half22float2(*reinterpret_cast<const __half2*>(&c1.x));
+          const float2 s1b = __half22float2(*reinterpret_cast<const __half2*>(&c1.y));
+          const float ks0[4] = {s0a.x, s0a.y, s0b.x, s0b.y}, ks1[4] = {s1a.x, s1a.y, s1b.x, s1b.y};
 #pragma unroll
-          for (int kt = 0; kt < KSTEPS; ++kt) {
-            const int sh = 8 * (kt & 1);
+          for (int gq = 0; gq < 4; ++gq) {
+            float t[4];
             uint32_t a[4];
-            a[0] = hmul2_u32(int4x2_to_f16x2(w0[kt >> 1] >> sh), s0[kt >> 1]);
-            a[1] = hmul2_u32(int4x2_to_f16x2(w1[kt >> 1] >> sh), s1[kt >> 1]);
-            a[2] = hmul2_u32(int4x2_to_f16x2(w0[kt >> 1] >> (sh + 4)), s0[kt >> 1]);
-            a[3] = hmul2_u32(int4x2_to_f16x2(w1[kt >> 1] >> (sh + 4)), s1[kt >> 1]);
-            mma(s[mt], a, qf[kt][0], qf[kt][1]);
+            a[0] = nib_lo_f16x2(w0[gq]);
+            a[1] = nib_lo_f16x2(w1[gq]);
+            a[2] = nib_hi_f16x2(w0[gq]);
+            a[3] = nib_hi_f16x2(w1[gq]);
+            mma_f16_16816_c(t, a, qf[2 * gq][0], qf[2 * gq][1], -cq[gq][0], -cq[gq][1], -cq[gq][0],
+                            -cq[gq][1]);
+            const uint32_t x0 = w0[gq] >> 8, x1 = w1[gq] >> 8;
+            a[0] = nib_lo_f16x2(x0);
+            a[1] = nib_lo_f16x2(x1);
+            a[2] = nib_hi_f16x2(x0);
+            a[3] = nib_hi_f16x2(x1);
+            mma_f16_16816(t, a, qf[2 * gq + 1][0], qf[2 * gq + 1][1]);
+            s[mt][0] = fmaf(ks0[gq], t[0], s[mt][0]);
+            s[mt][1] = fmaf(ks0[gq], t[1], s[mt][1]);
+            s[mt][2] = fmaf(ks1[gq], t[2], s[mt][2]);
+            s[mt][3] = fmaf(ks1[gq], t[3], s[mt][3]);
           }
         }
       }
@@ -296,6 +348,15 @@ struct MmaWarp {
       o[md][1] *= al1;
       o[md][2] *= al0;
       o[md][3] *= al1;
+    }
+    if constexpr (KV == KV_INT4) {
+#pragma unroll
+      for (int gq = 0; gq < 4; ++gq) {
+        eo[gq][0] *= al0;
+        eo[gq][1] *= al1;
+        eo[gq][2] *= al0;
+        eo[gq][3] *= al1;
+      }
     }
     uint32_t pb[4][2];
 #pragma unroll
@@ -337,27 +398,38 @@ struct MmaWarp {
           mma(o[md], a, pb[mt][0], pb[mt][1]);
         }
       } else if constexpr (KV == KV_INT4) {  // V^T tile [D][64 tokens] of nibbles
-        const int t0 = mt * 16 + 2 * q, sh = 8 * (mt & 1);
+        // The group's V scales of tokens t0, t0+1 (t0+8, t0+9) multiply the
+        // probabilities, and tokens 8..15 of the m-tile (nibbles decoded as
+        // 1024 + 16 n) take a further 1/16; a constant-A MMA accumulates what
+        // the decoding adds to every output row of the group (1032 or 1152
+        // times each weight), taken off when the state is written.
+        const uint32_t kSixteenth = 0x2C002C00u;       // f16x2 (1/16, 1/16)
+        const uint32_t ac[4] = {0x64086408u, 0x64086408u, 0x64806480u, 0x64806480u};  // 1032, 1152
+        const uint32_t pb1 = hmul2_u32(pb[mt][1], kSixteenth);
+        const int sh = 8 * (mt & 1);
 #pragma unroll
-        for (int md = 0; md < MTD; ++md) {
-          const int d0 = md * 16 + r8, gq = md >> 1;
-          const uint2 x0 = *reinterpret_cast<const uint2*>(Vs + d0 * 32 + q * 8);
-          const uint2 x1 = *reinterpret_cast<const uint2*>(Vs + (d0 + 8) * 32 + q * 8);
-          const uint32_t w0 = (mt >> 1) ? x0.y : x0.x, w1 = (mt >> 1) ? x1.y : x1.x;
+        for (int gq = 0; gq < 4; ++gq) {
           const uint32_t sA = *reinterpret_cast<const uint32_t*>(Vs + kInt4Nibbles + gq * 128 + t0 * 2);
           const uint32_t sB = *reinterpret_cast<const uint32_t*>(Vs + kInt4Nibbles + gq * 128 + (t0 + 8) * 2);
-          uint32_t a[4];
-          a[0] = hmul2_u32(int4x2_to_f16x2(w0 >> sh), sA);
-          a[1] = hmul2_u32(int4x2_to_f16x2(w1 >> sh), sA);
-          a[2] = hmul2_u32(int4x2_to_f16x2(w0 >> (sh + 4)), sB);
-          a[3] = hmul2_u32(int4x2_to_f16x2(w1 >> (sh + 4)), sB);
+          uint32_t b0 = hmul2_u32(pb[mt][0], sA), b1 = hmul2_u32(pb1, sB);
           if (partial) {
-            a[0] &= m01;
-            a[1] &= m01;
-            a[2] &= m23;
-            a[3] &= m23;
+            b0 &= m01;
+            b1 &= m23;
           }
-          mma(o[md], a, pb[mt][0], pb[mt][1]);
+          mma(eo[gq], ac, b0, b1);
+#pragma unroll
+          for (int md = 2 * gq; md < 2 * gq + 2; ++md) {
+            const int d0 = md * 16 + r8;
+            const uint2 x0 = *reinterpret_cast<const uint2*>(Vs + d0 * 32 + q * 8);
+            const uint2 x1 = *reinterpret_cast<const uint2*>(Vs + (d0 + 8) * 32 + q * 8);
+            const uint32_t w0 = ((mt >> 1) ? x0.y : x0.x) >> sh, w1 = ((mt >> 1) ? x1.y : x1.x) >> sh;
+            uint32_t a[4];
+            a[0] = nib_lo_f16x2(w0);
+            a[1] = nib_lo_f16x2(w1);
+            a[2] = nib_hi_f16x2(w0);
+            a[3] = nib_hi_f16x2(w1);
+            mma(o[md], a, b0, b1);
+          }
         }
       } else {  // FP8: V^T tile [D][64], 16 bytes per (d row, owner lane)
 #pragma unroll
@@ -386,6 +458,15 @@ struct MmaWarp {
 
   // Write this warp's state for query heads n < g into the combine area.
   __device__ __forceinline__ void write_state(float* ow, float* mw, float* lw, int g, int lane) {
+    if constexpr (KV == KV_INT4) {
+#pragma unroll
+      for (int md = 0; md < MTD; ++md) {
+        o[md][0] -= eo[md >> 1][0];
+        o[md][1] -= eo[md >> 1][1];
+        o[md][2] -= eo[md >> 1][2];
+        o[md][3] -= eo[md >> 1][3];
+      }
+    }
     float l0 = l[0], l1 = l[1];
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {

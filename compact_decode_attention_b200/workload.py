@@ -18,7 +18,7 @@ STREAM_K, STREAM_V, STREAM_Q = 0, 1, 2
 
 
 def _dtype_code(name: str) -> int:
-    return {"f32": dms.DMS_F32, "bf16": dms.DMS_BF16, "fp8": dms.DMS_FP8_E4M3}[name]
+    return {"f32": dms.DMS_F32, "bf16": dms.DMS_BF16, "fp8": dms.DMS_FP8_E4M3, "int4": dms.DMS_INT4}[name]
 
 
 def expected_blocks(wl, steps: int, sigmas: float = 8.0) -> int:

@@ -2,8 +2,9 @@
 
 Glue between ``synth`` (inputs) and the oracle's definitions: it regenerates
 the inputs of one (layer, sequence, kv-head) from the seed, forms the values
-the store holds (the model's K/V in their input precision, or for an FP8
-store their E4M3 codes times the per-head scale) and evaluates the oracle's
+the store holds (the model's K/V in their input precision, for an FP8 store
+their E4M3 codes times the per-head scale, for a 4-bit store their group
+codes times the group scales) and evaluates the oracle's
 mask, compaction, slot simulator and attention on them.  Everything is fp64
 except where the stored precision is the point (bf16 rounding, fp32 quotient
 before E4M3 rounding).
@@ -16,6 +17,7 @@ import synth
 
 from .attention import attend
 from .fp8 import dequantize, fp8_scale, quantize
+from .int4 import stored as int4_stored
 from .mask import visible_positions
 
 
@@ -54,6 +56,8 @@ def stored_rows(wl, layer: int, b: int, h: int, pos: np.ndarray, scales=None):
                          np.arange(wl.head_dim)[None, :], wl.in_dtype)
         if wl.kv_dtype == "fp8":
             out.append(dequantize(quantize(x, scales[i]), scales[i]))
+        elif wl.kv_dtype == "int4":
+            out.append(int4_stored(x))
         else:
             out.append(x.astype(np.float64))
     return out[0], out[1]

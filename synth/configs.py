@@ -30,7 +30,7 @@ class Workload:
     prompt: int
     decode: int
     window: int
-    kv_dtype: str          # storage dtype in the pool: "f32" | "bf16" | "fp8"
+    kv_dtype: str          # storage dtype in the pool: "f32" | "bf16" | "fp8" | "int4"
     in_dtype: str          # dtype of the K/V/Q the model hands over: "f32" | "bf16"
     seed: int
     keep: str              # "const" | "uniform" | "heavy_tail"
@@ -65,8 +65,12 @@ class Workload:
         """int64 [n_layers, n_kv_heads] 24-bit keep thresholds."""
         return keep_threshold(self.keep_probs())
 
-    def kv_elem_bytes(self) -> int:
-        return {"f32": 4, "bf16": 2, "fp8": 1}[self.kv_dtype]
+    def kv_row_bytes(self) -> int:
+        """Bytes of one stored K (or V) row: 4-bit rows carry 4 bits per
+        element plus one fp16 scale per group of 32."""
+        if self.kv_dtype == "int4":
+            return self.head_dim // 2 + self.head_dim // 16
+        return self.head_dim * {"f32": 4, "bf16": 2, "fp8": 1}[self.kv_dtype]
 
     def in_elem_bytes(self) -> int:
         return {"f32": 4, "bf16": 2}[self.in_dtype]
