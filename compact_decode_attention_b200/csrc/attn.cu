@@ -72,11 +72,13 @@ struct AttnTraits {
   // 34 KB for bf16 D=128, 8 for the others): with two consumer warps per SM
   // sub-partition one warp's MMA / ldmatrix latency hides behind the other's.
   // fp32 (68 KB or 34 KB stages): 3 or 4 stages and warps.
-  // 4-bit stages are 9 KB: two per consumer warp keep 147 KB in flight.
+  // 4-bit stages are 9 KB: two per consumer warp keep 129 KB in flight;
+  // 7 consumer warps + the producer leave two warps per SM sub-partition
+  // (up to 255 registers a thread).
   static constexpr int NS = KV == KV_F32 ? (D == 128 ? 3 : 4)
-                          : KV == KV_INT4 ? 16
+                          : KV == KV_INT4 ? 14
                           : (KV == KV_BF16 && D == 128) ? 6 : 8;
-  static constexpr int NCW = KV == KV_INT4 ? 8 : NS;   // consumer warps
+  static constexpr int NCW = KV == KV_INT4 ? 7 : NS;   // consumer warps
   static constexpr int THREADS = 32 * (NCW + 1);       // + one producer warp
   static constexpr int COMBINE_FLOATS = NCW * 8 * D + 2 * NCW * 8;
   static constexpr int MISC_INTS = 16 + THREADS / 32;
@@ -156,8 +158,8 @@ struct MmaWarp {
   uint32_t qf[KSTEPS][2];
   float scale;  // log2-domain score scale (includes the K scale for FP8)
   float vscale; // V scale (FP8), else 1
-  // 4-bit stores only: per 32-element group g, the offset that the 1024 + m n
-  // decoding adds to q . k for query columns 2(lane&3) and 2(lane&3)+1 ...
+  // 4-bit stores only: per 32-element group g, minus the offset that the
+  // 1024 + m n decoding adds to q . k for query columns 2(lane&3), +1 ...
   float cq[4][2];
   // ... and the one it adds to each output row of group g (accumulated like o)
   float eo[4][4];
@@ -216,8 +218,8 @@ struct MmaWarp {
         }
         c += __shfl_xor_sync(0xffffffffu, c, 1);
         c += __shfl_xor_sync(0xffffffffu, c, 2);
-        cq[gq][0] = __shfl_sync(0xffffffffu, c, 8 * (lane & 3));
-        cq[gq][1] = __shfl_sync(0xffffffffu, c, 8 * (lane & 3) + 4);
+        cq[gq][0] = -__shfl_sync(0xffffffffu, c, 8 * (lane & 3));
+        cq[gq][1] = -__shfl_sync(0xffffffffu, c, 8 * (lane & 3) + 4);
       }
     }
   }
@@ -282,7 +284,7 @@ struct MmaWarp {
       // the decoding offset, and the group's K scale multiplies the result.
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
-        if (mt * 16 < rows) {
+        {  // all four m-tiles: nibbles always decode to finite values
           const int r0 = mt * 16 + r8, r1 = r0 + 8;
           const uint4 k0 = *reinterpret_cast<const uint4*>(Ks + r0 * 64 + q * 16);
           const uint4 k1 = *reinterpret_cast<const uint4*>(Ks + r1 * 64 + q * 16);
@@ -302,8 +304,8 @@ struct MmaWarp {
             a[1] = nib_lo_f16x2(w1[gq]);
             a[2] = nib_hi_f16x2(w0[gq]);
             a[3] = nib_hi_f16x2(w1[gq]);
-            mma_f16_16816_c(t, a, qf[2 * gq][0], qf[2 * gq][1], -cq[gq][0], -cq[gq][1], -cq[gq][0],
-                            -cq[gq][1]);
+            mma_f16_16816_c(t, a, qf[2 * gq][0], qf[2 * gq][1], cq[gq][0], cq[gq][1], cq[gq][0],
+                            cq[gq][1]);
             const uint32_t x0 = w0[gq] >> 8, x1 = w1[gq] >> 8;
             a[0] = nib_lo_f16x2(x0);
             a[1] = nib_lo_f16x2(x1);
@@ -374,6 +376,53 @@ struct MmaWarp {
       }
     }
     // ---- O^T += V^T P^T ----
+    if constexpr (KV == KV_INT4) {
+      // V^T tile [D][64 tokens] of nibbles.  Per group g of 32 V elements:
+      // the group's V scales of the tokens multiply the probabilities, tokens
+      // 8..15 of each 16-token m-tile (nibbles decoded as 1024 + 16 n) take a
+      // further 1/16, and a constant-A MMA accumulates what the decoding adds
+      // to each output row of the group (1032 or 1152 times each weight),
+      // taken off when the state is written.  Token columns past `rows` hold
+      // scale 0 (a 4-bit block's V tile is cleared when it is opened) and
+      // probability 0, so every m-tile is computed.  One 8-byte load per
+      // output row gives a lane its nibbles of all 64 tokens.
+      const uint32_t kSixteenth = 0x2C002C00u;       // f16x2 (1/16, 1/16)
+      const uint32_t ac[4] = {0x64086408u, 0x64086408u, 0x64806480u, 0x64806480u};  // 1032, 1152
+#pragma unroll
+      for (int gq = 0; gq < 4; ++gq) {
+        uint32_t b[4][2];
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          const int t0 = mt * 16 + 2 * q;
+          const uint32_t sA = *reinterpret_cast<const uint32_t*>(Vs + kInt4Nibbles + gq * 128 + t0 * 2);
+          const uint32_t sB = *reinterpret_cast<const uint32_t*>(Vs + kInt4Nibbles + gq * 128 + (t0 + 8) * 2);
+          b[mt][0] = hmul2_u32(pb[mt][0], sA);
+          b[mt][1] = hmul2_u32(hmul2_u32(pb[mt][1], kSixteenth), sB);
+          mma(eo[gq], ac, b[mt][0], b[mt][1]);
+        }
+#pragma unroll
+        for (int md = 2 * gq; md < 2 * gq + 2; ++md) {
+          const int d0 = md * 16 + r8;
+          const uint2 x0 = *reinterpret_cast<const uint2*>(Vs + d0 * 32 + q * 8);
+          const uint2 x1 = *reinterpret_cast<const uint2*>(Vs + (d0 + 8) * 32 + q * 8);
+#pragma unroll
+          for (int mt = 0; mt < 4; ++mt) {
+            uint32_t w0 = (mt >> 1) ? x0.y : x0.x, w1 = (mt >> 1) ? x1.y : x1.x;
+            if (mt & 1) {
+              w0 >>= 8;
+              w1 >>= 8;
+            }
+            uint32_t a[4];
+            a[0] = nib_lo_f16x2(w0);
+            a[1] = nib_lo_f16x2(w1);
+            a[2] = nib_hi_f16x2(w0);
+            a[3] = nib_hi_f16x2(w1);
+            mma(o[md], a, b[mt][0], b[mt][1]);
+          }
+        }
+      }
+      return;
+    }
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
       if (mt * 16 >= rows) break;
@@ -396,40 +445,6 @@ struct MmaWarp {
             a[3] &= m23;
           }
           mma(o[md], a, pb[mt][0], pb[mt][1]);
-        }
-      } else if constexpr (KV == KV_INT4) {  // V^T tile [D][64 tokens] of nibbles
-        // The group's V scales of tokens t0, t0+1 (t0+8, t0+9) multiply the
-        // probabilities, and tokens 8..15 of the m-tile (nibbles decoded as
-        // 1024 + 16 n) take a further 1/16; a constant-A MMA accumulates what
-        // the decoding adds to every output row of the group (1032 or 1152
-        // times each weight), taken off when the state is written.
-        const uint32_t kSixteenth = 0x2C002C00u;       // f16x2 (1/16, 1/16)
-        const uint32_t ac[4] = {0x64086408u, 0x64086408u, 0x64806480u, 0x64806480u};  // 1032, 1152
-        const uint32_t pb1 = hmul2_u32(pb[mt][1], kSixteenth);
-        const int sh = 8 * (mt & 1);
-#pragma unroll
-        for (int gq = 0; gq < 4; ++gq) {
-          const uint32_t sA = *reinterpret_cast<const uint32_t*>(Vs + kInt4Nibbles + gq * 128 + t0 * 2);
-          const uint32_t sB = *reinterpret_cast<const uint32_t*>(Vs + kInt4Nibbles + gq * 128 + (t0 + 8) * 2);
-          uint32_t b0 = hmul2_u32(pb[mt][0], sA), b1 = hmul2_u32(pb1, sB);
-          if (partial) {
-            b0 &= m01;
-            b1 &= m23;
-          }
-          mma(eo[gq], ac, b0, b1);
-#pragma unroll
-          for (int md = 2 * gq; md < 2 * gq + 2; ++md) {
-            const int d0 = md * 16 + r8;
-            const uint2 x0 = *reinterpret_cast<const uint2*>(Vs + d0 * 32 + q * 8);
-            const uint2 x1 = *reinterpret_cast<const uint2*>(Vs + (d0 + 8) * 32 + q * 8);
-            const uint32_t w0 = ((mt >> 1) ? x0.y : x0.x) >> sh, w1 = ((mt >> 1) ? x1.y : x1.x) >> sh;
-            uint32_t a[4];
-            a[0] = nib_lo_f16x2(w0);
-            a[1] = nib_lo_f16x2(w1);
-            a[2] = nib_hi_f16x2(w0);
-            a[3] = nib_hi_f16x2(w1);
-            mma(o[md], a, b0, b1);
-          }
         }
       } else {  // FP8: V^T tile [D][64], 16 bytes per (d row, owner lane)
 #pragma unroll
@@ -800,17 +815,97 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     }
   };
   set_head_scales(i);
-  int k = 0;
-  for (int u = u_beg; u < u_end; ++u, ++k) {
-    while (u >= pp + nu) {
-      pp += nu;
-      ++i;
-      n = n_at(i);
-      nu = units_of(n);
+  // Each warp takes every kNCW-th unit of the CTA's range (unit k of the
+  // range lives in stage k % NS).  A head is finished (the warps' states
+  // combined) once no warp has a unit of it left: every warp passes every
+  // head end of the range, in order, so the consumer barriers match.
+  auto finish_head = [&]() {
+    st.write_state(my_ow, my_mw, my_lw, g, lane);
+    consumer_bar<kNCW>();
+    const int hd = pool_head(p, i);
+    const int cf = cta_of(pp, U, Geff), cl = cta_of(int64_t(pp) + nu - 1, U, Geff);
+    const bool whole = cf == cl;
+    const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
+    const int pid = c + i;
+    (void)DMS_CHECK(i < Htot && pid < G + Htot && cf >= 0 && cl < Geff, v.hdr, 303, i, pid);
+    for (int idx = tid; idx < g * D; idx += kCons) {
+      const int nn = idx / D, d = idx % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kNCW; ++w) M = fmaxf(M, s_mw[w * 8 + nn]);
+      float o = 0.f, L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kNCW; ++w) {
+        const float f = fast_exp2(s_mw[w * 8 + nn] - M);
+        o += f * s_ow[(w * 8 + nn) * D + d];
+        L += f * s_lw[w * 8 + nn];
+      }
+      if (whole) {
+        store_out<T::QESZ>(p.out, orow * D + idx, o / L);
+      } else {
+        p.ws_o[(int64_t(pid) * g + nn) * D + d] = o;
+        if (d == 0) {
+          p.ws_ml[(int64_t(pid) * g + nn) * 2 + 0] = M;
+          p.ws_ml[(int64_t(pid) * g + nn) * 2 + 1] = L;
+        }
+      }
+    }
+    if (!whole) {
+      consumer_bar<kNCW>();
+      if (tid == 0) {
+        __threadfence();
+        const int prev = atomicAdd(&v.tickets[hd], 1);
+        s_misc[3] = prev == cl - cf;
+      }
+      consumer_bar<kNCW>();
+      if (s_misc[3]) {
+        __threadfence();
+        for (int idx = tid; idx < g * D; idx += kCons) {
+          const int nn = idx / D, d = idx % D;
+          float M = -INFINITY;
+          for (int cc = cf; cc <= cl; ++cc)
+            M = fmaxf(M, __ldcg(&p.ws_ml[(int64_t(cc + i) * g + nn) * 2]));
+          float o = 0.f, L = 0.f;
+          for (int cc = cf; cc <= cl; ++cc) {
+            const int64_t id = int64_t(cc + i) * g + nn;
+            const float f = fast_exp2(__ldcg(&p.ws_ml[id * 2]) - M);
+            o += f * __ldcg(&p.ws_o[id * D + d]);
+            L += f * __ldcg(&p.ws_ml[id * 2 + 1]);
+          }
+          store_out<T::QESZ>(p.out, orow * D + idx, o / L);
+        }
+        if (tid == 0) v.tickets[hd] = 0;
+      }
+    }
+    consumer_bar<kNCW>();
+    st.reset();
+    have_q = false;
+  };
+  bool done = false;
+  for (int u = u_beg + warp; !done; u += kNCW) {
+    const int lim = u < u_end ? u : u_end;
+    while (pp + nu <= lim) {  // head i has no unit at or after u
+      finish_head();
+      if (pp + nu >= u_end) {
+        done = true;
+        break;
+      }
+      do {                    // next head with a unit (empty heads have none)
+        pp += nu;
+        ++i;
+        n = n_at(i);
+        nu = units_of(n);
+      } while (nu == 0 && i + 1 < Htot);
       set_head_scales(i);
     }
+    if (done) break;
+    if (u >= u_end) {         // the range ends inside head i
+      finish_head();
+      break;
+    }
+    const int k = u - u_beg;
     const int rows = min(kBlockTokens, n - (u - pp) * kBlockTokens);
-    if (k % kNCW == warp) {
+    {
       const int s = k % T::NS;
       const uint32_t ph = (k / T::NS) & 1;
       if constexpr (KV != KV_F32) {
@@ -837,69 +932,6 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
       // abort the producer issues nothing more and drains what it issued
       __syncwarp();
       if (ok && lane == 0) mbar_arrive(&empty[s]);
-    }
-    // ---- end of this CTA's piece of head i: combine the 4 warps ----
-    if (u + 1 == u_end || u + 1 >= pp + nu) {
-      st.write_state(my_ow, my_mw, my_lw, g, lane);
-      consumer_bar<kNCW>();
-      const int hd = pool_head(p, i);
-      const int cf = cta_of(pp, U, Geff), cl = cta_of(int64_t(pp) + nu - 1, U, Geff);
-      const bool whole = cf == cl;
-      const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
-      const int pid = c + i;
-      (void)DMS_CHECK(i < Htot && pid < G + Htot && cf >= 0 && cl < Geff, v.hdr, 303, i, pid);
-      for (int idx = tid; idx < g * D; idx += kCons) {
-        const int nn = idx / D, d = idx % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kNCW; ++w) M = fmaxf(M, s_mw[w * 8 + nn]);
-        float o = 0.f, L = 0.f;
-#pragma unroll
-        for (int w = 0; w < kNCW; ++w) {
-          const float f = fast_exp2(s_mw[w * 8 + nn] - M);
-          o += f * s_ow[(w * 8 + nn) * D + d];
-          L += f * s_lw[w * 8 + nn];
-        }
-        if (whole) {
-          store_out<T::QESZ>(p.out, orow * D + idx, o / L);
-        } else {
-          p.ws_o[(int64_t(pid) * g + nn) * D + d] = o;
-          if (d == 0) {
-            p.ws_ml[(int64_t(pid) * g + nn) * 2 + 0] = M;
-            p.ws_ml[(int64_t(pid) * g + nn) * 2 + 1] = L;
-          }
-        }
-      }
-      if (!whole) {
-        consumer_bar<kNCW>();
-        if (tid == 0) {
-          __threadfence();
-          const int prev = atomicAdd(&v.tickets[hd], 1);
-          s_misc[3] = prev == cl - cf;
-        }
-        consumer_bar<kNCW>();
-        if (s_misc[3]) {
-          __threadfence();
-          for (int idx = tid; idx < g * D; idx += kCons) {
-            const int nn = idx / D, d = idx % D;
-            float M = -INFINITY;
-            for (int cc = cf; cc <= cl; ++cc)
-              M = fmaxf(M, __ldcg(&p.ws_ml[(int64_t(cc + i) * g + nn) * 2]));
-            float o = 0.f, L = 0.f;
-            for (int cc = cf; cc <= cl; ++cc) {
-              const int64_t id = int64_t(cc + i) * g + nn;
-              const float f = fast_exp2(__ldcg(&p.ws_ml[id * 2]) - M);
-              o += f * __ldcg(&p.ws_o[id * D + d]);
-              L += f * __ldcg(&p.ws_ml[id * 2 + 1]);
-            }
-            store_out<T::QESZ>(p.out, orow * D + idx, o / L);
-          }
-          if (tid == 0) v.tickets[hd] = 0;
-        }
-      }
-      consumer_bar<kNCW>();
-      st.reset();
-      have_q = false;
     }
   }
 }
