@@ -230,7 +230,16 @@ struct MmaWarp {
     else mma_bf16_16816(d, a, b0, b1);
   }
 
+  // A whole block (64 rows) takes a copy of the unit code with every row
+  // check folded away; a head's last, partly filled block the general one.
   __device__ __forceinline__ void unit(const uint8_t* stage, int rows, int lane) {
+    if (rows == kBlockTokens) unit_rows<true>(stage, kBlockTokens, lane);
+    else unit_rows<false>(stage, rows, lane);
+  }
+
+  template <bool FULL>
+  __device__ __forceinline__ void unit_rows(const uint8_t* stage, int rows_in, int lane) {
+    const int rows = FULL ? kBlockTokens : rows_in;
     const uint8_t* Ks = stage;
     const uint8_t* Vs = stage + T::TILEB;
     const int q = lane & 3, r8 = lane >> 2;
