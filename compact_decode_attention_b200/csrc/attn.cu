@@ -75,10 +75,12 @@ struct AttnTraits {
   // 4-bit stages are 9 KB: two per consumer warp keep 129 KB in flight;
   // 7 consumer warps + the producer leave two warps per SM sub-partition
   // (up to 255 registers a thread).
+  // FP8 stages are 16 KB: two per consumer warp (6 warps, 192 KB in flight).
   static constexpr int NS = KV == KV_F32 ? (D == 128 ? 3 : 4)
                           : KV == KV_INT4 ? 14
+                          : KV == KV_FP8 ? 12
                           : (KV == KV_BF16 && D == 128) ? 6 : 8;
-  static constexpr int NCW = KV == KV_INT4 ? 7 : NS;   // consumer warps
+  static constexpr int NCW = KV == KV_INT4 ? 7 : KV == KV_FP8 ? 6 : NS;   // consumer warps
   static constexpr int THREADS = 32 * (NCW + 1);       // + one producer warp
   static constexpr int COMBINE_FLOATS = NCW * 8 * D + 2 * NCW * 8;
   static constexpr int MISC_INTS = 16 + THREADS / 32;
@@ -716,8 +718,31 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
       pre += nu;
     }
   }
+  // the head holding the range's last unit, and where it starts
+  if (u_beg < u_end && u_end - 1 >= excl && u_end - 1 < excl + su) {
+    int pre = excl;
+    for (int i = hb; i < he; ++i) {
+      const int n = n_of(p, i);
+      const int nu = units_of(n);
+      if (u_end - 1 < pre + nu) {
+        s_misc[4] = i;
+        s_misc[5] = pre;
+        s_misc[6] = n;
+        break;
+      }
+      pre += nu;
+    }
+  }
   __syncthreads();
   const int i0 = s_misc[1], p0 = s_misc[2];
+  // Processing order: first this CTA's piece of its last head (segment A,
+  // units [r, u_end)), then [u_beg, r) (segment B).  The range's two end
+  // heads are usually shared with the neighbouring CTAs and need the
+  // cross-CTA merge; this way both finish early and their merges overlap the
+  // copies already in flight, and the CTA ends on a head of its own.
+  const int iL = s_misc[4], pL = s_misc[5], nL = s_misc[6];
+  const int r = max(u_beg, pL);
+  const int nA = u_end - r;
   // held counts of heads i0 .. i0 + HEAD_WIN - 1 in shared memory, so that the
   // walks below need no dependent global loads (the scan just loaded them)
   int* s_nwin = s_misc + T::MISC_INTS;
@@ -732,12 +757,67 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     const uint64_t qpol = policy_evict_last();   // query rows: re-read per block
     int k = 0, issued = 0;
     bool aborted = false;
+    // lane 0 issues unit k (block jblk, jrows rows, of head ji) into stage k % NS
+    auto issue = [&](int jblk, int jrows, int ji) {
+      if (lane == 0 && !aborted) {
+        const int s = k % T::NS;
+        const uint32_t ph = (k / T::NS) & 1;
+        if (!DMS_CHECK(jblk >= 0 && jblk < v.max_blocks && jrows >= 1 && jrows <= kBlockTokens &&
+                           ji >= 0 && ji < Htot, v.hdr, 302, jblk, jrows)) {
+          aborted = true;
+          *s_abort = 1;
+        } else if (!mbar_wait_bounded(&empty[s], ph ^ 1, s_abort) || *s_abort) {
+          aborted = true;
+          if (!*s_abort) report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
+          *s_abort = 1;
+        } else {
+          uint8_t* st = stages + size_t(s) * T::STAGEB;
+          const uint8_t* src = v.blocks + int64_t(jblk) * v.block_bytes;
+          const uint8_t* qsrc = p.q + int64_t(ji / v.Hkv) * v.Hq * D * T::QESZ +
+                                int64_t(ji % v.Hkv) * qrow_bytes;
+          const uint32_t kbytes = uint32_t(jrows) * T::ROWB;
+          // 4-bit tiles keep their scales after the nibbles: always copied whole
+          const bool whole = jrows == kBlockTokens || KV == KV_INT4;
+          const uint32_t vbytes = (whole || KV == KV_FP8) ? T::TILEB : kbytes;
+          mbar_arrive_expect_tx(&full[s], (whole ? T::TILEB : kbytes) + vbytes +
+                                              (T::QB > 0 ? qrow_bytes : 0));
+          if (whole) {
+            bulk_g2s(st, src, 2 * T::TILEB, &full[s], pol);
+          } else {
+            bulk_g2s(st, src, kbytes, &full[s], pol);
+            bulk_g2s(st + T::TILEB, src + T::TILEB, vbytes, &full[s], pol);
+          }
+          if constexpr (T::QB > 0) bulk_g2s(st + 2 * T::TILEB, qsrc, qrow_bytes, &full[s], qpol);
+          issued = k + 1;
+        }
+      }
+      ++k;
+    };
+    // segment A: one head, units [r, u_end)
+    for (int ub = r; ub < u_end; ub += 32) {
+      const int u = ub + lane;
+      int blk = 0, rows = 0;
+      if (u < u_end) {
+        const int bi = u - pL;
+        if (DMS_CHECK(iL < Htot && bi >= 0 && bi < v.mbh, v.hdr, 304, iL, bi))
+          blk = v.bt[int64_t(pool_head(p, iL)) * v.mbh + bi];
+        rows = min(kBlockTokens, nL - bi * kBlockTokens);
+      }
+      const int cnt = min(32, u_end - ub);
+      for (int j = 0; j < cnt; ++j) {
+        const int jblk = __shfl_sync(0xffffffffu, blk, j);
+        const int jrows = __shfl_sync(0xffffffffu, rows, j);
+        issue(jblk, jrows, iL);
+      }
+      aborted = __shfl_sync(0xffffffffu, aborted, 0);
+    }
+    // segment B: units [u_beg, r), walking the heads from i0
     int i = i0, pp = p0, n = n_at(i0), nu = units_of(n);
-    for (int ub = u_beg; ub < u_end; ub += 32) {
+    for (int ub = u_beg; ub < r; ub += 32) {
       const int u = ub + lane;
       int mi = i, mp = pp, mn = n, mnu = nu;
       int blk = 0, rows = 0;
-      if (u < u_end) {
+      if (u < r) {
         while (u >= mp + mnu) {
           mp += mnu;
           ++mi;
@@ -749,44 +829,12 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
           blk = v.bt[int64_t(pool_head(p, mi)) * v.mbh + bi];
         rows = min(kBlockTokens, mn - bi * kBlockTokens);
       }
-      const int cnt = min(32, u_end - ub);
+      const int cnt = min(32, r - ub);
       for (int j = 0; j < cnt; ++j) {
         const int jblk = __shfl_sync(0xffffffffu, blk, j);
         const int jrows = __shfl_sync(0xffffffffu, rows, j);
         const int ji = __shfl_sync(0xffffffffu, mi, j);
-        if (lane == 0 && !aborted) {
-          const int s = k % T::NS;
-          const uint32_t ph = (k / T::NS) & 1;
-          if (!DMS_CHECK(jblk >= 0 && jblk < v.max_blocks && jrows >= 1 && jrows <= kBlockTokens &&
-                             ji >= 0 && ji < Htot, v.hdr, 302, jblk, jrows)) {
-            aborted = true;
-            *s_abort = 1;
-          } else if (!mbar_wait_bounded(&empty[s], ph ^ 1, s_abort) || *s_abort) {
-            aborted = true;
-            if (!*s_abort) report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
-            *s_abort = 1;
-          } else {
-            uint8_t* st = stages + size_t(s) * T::STAGEB;
-            const uint8_t* src = v.blocks + int64_t(jblk) * v.block_bytes;
-            const uint8_t* qsrc = p.q + int64_t(ji / v.Hkv) * v.Hq * D * T::QESZ +
-                                  int64_t(ji % v.Hkv) * qrow_bytes;
-            const uint32_t kbytes = uint32_t(jrows) * T::ROWB;
-            // 4-bit tiles keep their scales after the nibbles: always copied whole
-            const bool whole = jrows == kBlockTokens || KV == KV_INT4;
-            const uint32_t vbytes = (whole || KV == KV_FP8) ? T::TILEB : kbytes;
-            mbar_arrive_expect_tx(&full[s], (whole ? T::TILEB : kbytes) + vbytes +
-                                                (T::QB > 0 ? qrow_bytes : 0));
-            if (whole) {
-              bulk_g2s(st, src, 2 * T::TILEB, &full[s], pol);
-            } else {
-              bulk_g2s(st, src, kbytes, &full[s], pol);
-              bulk_g2s(st + T::TILEB, src + T::TILEB, vbytes, &full[s], pol);
-            }
-            if constexpr (T::QB > 0) bulk_g2s(st + 2 * T::TILEB, qsrc, qrow_bytes, &full[s], qpol);
-            issued = k + 1;
-          }
-        }
-        ++k;
+        issue(jblk, jrows, ji);
       }
       const int last = cnt - 1;
       i = __shfl_sync(0xffffffffu, mi, last);
@@ -890,57 +938,75 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     st.reset();
     have_q = false;
   };
-  bool done = false;
-  for (int u = u_beg + warp; !done; u += kNCW) {
-    const int lim = u < u_end ? u : u_end;
-    while (pp + nu <= lim) {  // head i has no unit at or after u
-      finish_head();
-      if (pp + nu >= u_end) {
-        done = true;
+  // unit k of the processing order (rows rows of head i) -> this warp
+  auto process_unit = [&](int k, int rows) {
+    const int s = k % T::NS;
+    const uint32_t ph = (k / T::NS) & 1;
+    if constexpr (KV != KV_F32) {
+      if (!have_q) {  // first block of this head for this warp: issue before the wait
+        st.load_q(p.q + int64_t(i / v.Hkv) * v.Hq * D * T::QESZ + int64_t(i % v.Hkv) * qrow_bytes,
+                  g, lane);
+        have_q = true;
+      }
+    }
+    bool ok = false;
+    if (!*s_abort) {
+      ok = mbar_wait_bounded(&full[s], ph, s_abort);
+      if (!ok && lane == 0) {
+        *s_abort = 1;
+        report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
+      }
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      const uint8_t* stage = stages + size_t(s) * T::STAGEB;
+      st.unit(stage, rows, lane);
+    }
+    // release the stage only after its copy was seen complete; after an
+    // abort the producer issues nothing more and drains what it issued
+    __syncwarp();
+    if (ok && lane == 0) mbar_arrive(&empty[s]);
+  };
+  int k = warp;
+  if (nA > 0) {               // segment A: the piece of head iL
+    i = iL;
+    pp = pL;
+    n = nL;
+    nu = units_of(nL);
+    set_head_scales(i);
+    for (; k < nA; k += kNCW) process_unit(k, min(kBlockTokens, n - (r + k - pp) * kBlockTokens));
+    finish_head();
+  }
+  if (r > u_beg) {            // segment B: [u_beg, r), ending on the head boundary r
+    i = i0;
+    pp = p0;
+    n = n_at(i0);
+    nu = units_of(n);
+    set_head_scales(i);
+    bool done = false;
+    for (; !done; k += kNCW) {
+      const int u = u_beg + (k - nA);
+      const int lim = u < r ? u : r;
+      while (pp + nu <= lim) {  // head i has no unit at or after u
+        finish_head();
+        if (pp + nu >= r) {
+          done = true;
+          break;
+        }
+        do {                    // next head with a unit (empty heads have none)
+          pp += nu;
+          ++i;
+          n = n_at(i);
+          nu = units_of(n);
+        } while (nu == 0 && i + 1 < Htot);
+        set_head_scales(i);
+      }
+      if (done) break;
+      if (u >= r) {
+        finish_head();
         break;
       }
-      do {                    // next head with a unit (empty heads have none)
-        pp += nu;
-        ++i;
-        n = n_at(i);
-        nu = units_of(n);
-      } while (nu == 0 && i + 1 < Htot);
-      set_head_scales(i);
-    }
-    if (done) break;
-    if (u >= u_end) {         // the range ends inside head i
-      finish_head();
-      break;
-    }
-    const int k = u - u_beg;
-    const int rows = min(kBlockTokens, n - (u - pp) * kBlockTokens);
-    {
-      const int s = k % T::NS;
-      const uint32_t ph = (k / T::NS) & 1;
-      if constexpr (KV != KV_F32) {
-        if (!have_q) {  // first block of this head for this warp: issue before the wait
-          st.load_q(p.q + int64_t(i / v.Hkv) * v.Hq * D * T::QESZ + int64_t(i % v.Hkv) * qrow_bytes,
-                    g, lane);
-          have_q = true;
-        }
-      }
-      bool ok = false;
-      if (!*s_abort) {
-        ok = mbar_wait_bounded(&full[s], ph, s_abort);
-        if (!ok && lane == 0) {
-          *s_abort = 1;
-          report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
-        }
-      }
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok) {
-        const uint8_t* stage = stages + size_t(s) * T::STAGEB;
-        st.unit(stage, rows, lane);
-      }
-      // release the stage only after its copy was seen complete; after an
-      // abort the producer issues nothing more and drains what it issued
-      __syncwarp();
-      if (ok && lane == 0) mbar_arrive(&empty[s]);
+      process_unit(k, min(kBlockTokens, n - (u - pp) * kBlockTokens));
     }
   }
 }
