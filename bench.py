@@ -582,10 +582,12 @@ def main():
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        h0 = time.perf_counter()
         for j in range(E):
             if flush:
                 l2_flush(j)
             stp.step(P + e0s + j, hin[j], hout[j])
+        host_issue_s = time.perf_counter() - h0
         stp.join(stream)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -595,9 +597,10 @@ def main():
         e2e = {"value": e_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": int(stp.layout.in_bytes), "d2h_bytes_per_step": int(stp.layout.out_bytes),
                "steps": E, "ms_per_step": e_ms / E,
+               "host_issue_us_per_step": host_issue_s / E * 1e6,
                "path": "dms_stepper_step: one packed pinned-host input copy, append/evict, decode "
                        "attention, one pinned-host output copy per step; copies on their own streams, "
-                       "double-buffered against the neighbouring steps' kernels"}
+                       "four buffers deep against the neighbouring steps' kernels"}
         if flush:
             e2e["l2"] = (f"an L2 flush ({L2_FLUSH_BYTES >> 20} MB written then read) on the compute stream before each "
                          f"step; their time alone ({flush_ms / E * 1e3:.1f} us per flush) is subtracted")

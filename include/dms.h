@@ -368,9 +368,9 @@ dms_status dms_decode_attn_layers_noalloc(dms_pool* pool, int layer0, int n_laye
  * dms_decode_attn_layers over the same layers) on inputs that live in host
  * memory, and copies each step's output back to host memory.  Every step
  * is one packed host->device copy, the two kernels and one device->host
- * copy; the copies run on two streams of the stepper's own, double-buffered
- * against the caller's compute stream, so the copies of one step overlap
- * the kernels of its neighbours.  The pages have no counterpart: this is the
+ * copy; the copies run on two streams of the stepper's own, with four
+ * staging and four output buffers in rotation against the caller's compute
+ * stream, so the copies of one step overlap the kernels of its neighbours.  The pages have no counterpart: this is the
  * serving-side plumbing around the method's decode step.
  * ------------------------------------------------------------------------ */
 typedef struct dms_stepper dms_stepper;  /* opaque host handle */
