@@ -65,7 +65,7 @@ def parse_args():
     ap.add_argument("--prefill-prompt", type=int, default=0,
                     help="prompt length for --prefill-only (default: the workload's)")
     ap.add_argument("--cpu-heads", type=int, default=72)
-    ap.add_argument("--cpu-steps", type=int, default=30)
+    ap.add_argument("--cpu-steps", type=int, default=90)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 

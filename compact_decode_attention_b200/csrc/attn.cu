@@ -679,24 +679,12 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   const int per = (Htot + kAttnThreads - 1) / kAttnThreads;
   const int hb = min(Htot, tid * per), he = min(Htot, hb + per);
   int su = 0;
-  for (int ib = hb; ib < he; ib += 4) {
-    // four heads' counts loaded together (one memory latency, not four)
-    int nn[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int hd = ib + j < he ? pool_head(p, ib + j) : -1;
-      nn[j] = hd >= 0 ? v.n_slots[hd] : 0;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int i = ib + j;
-      if (i >= he) break;
-      if (pool_head(p, i) < 0) (void)n_of(p, i);   // reports the bad sequence id
-      su += units_of(nn[j]);
-      if (nn[j] == 0 && i % G == c) {  // no key at all: define the output as 0
-        const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
-        for (int e = 0; e < g * D; ++e) store_out<T::QESZ>(p.out, orow * D + e, 0.f);
-      }
+  for (int i = hb; i < he; ++i) {
+    const int n = n_of(p, i);
+    su += units_of(n);
+    if (n == 0 && i % G == c) {  // no key at all: define the output as 0
+      const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
+      for (int e = 0; e < g * D; ++e) store_out<T::QESZ>(p.out, orow * D + e, 0.f);
     }
   }
   int incl = su;
