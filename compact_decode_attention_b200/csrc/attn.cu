@@ -44,8 +44,23 @@ enum { KV_F32 = 0, KV_BF16 = 1, KV_FP8 = 2, KV_INT4 = 3 };
 // at bits 0-3 (and 16-19) into the f16 value 1024 + n, and the nibble at
 // bits 4-7 (and 20-23) into 1024 + 16 n; both are exact.  The offsets and
 // the factor 16 are taken out in fp32 / on the other MMA operand.
-__device__ __forceinline__ uint32_t nib_lo_f16x2(uint32_t w) { return (w & 0x000F000Fu) | 0x64006400u; }
-__device__ __forceinline__ uint32_t nib_hi_f16x2(uint32_t w) { return (w & 0x00F000F0u) | 0x64006400u; }
+// (w & mask) | magic as one LOP3: mask and magic come in registers (a LOP3
+// takes a single immediate, and with two constants the compiler emits two).
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t w, uint32_t mask, uint32_t magic) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(mask), "r"(magic));
+  return r;
+}
+// The three decoding constants, held in registers for a warp's whole run
+// (a warp shuffle hides their values from constant folding).
+struct NibConsts {
+  uint32_t lo, hi, magic;
+  __device__ __forceinline__ void init() {
+    lo = __shfl_sync(0xffffffffu, 0x000F000Fu, 0);
+    hi = __shfl_sync(0xffffffffu, 0x00F000F0u, 0);
+    magic = __shfl_sync(0xffffffffu, 0x64006400u, 0);
+  }
+};
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
   return *reinterpret_cast<const uint32_t*>(&r);
@@ -165,6 +180,7 @@ struct MmaWarp {
   float cq[4][2];
   // ... and the one it adds to each output row of group g (accumulated like o)
   float eo[4][4];
+  NibConsts nc;  // 4-bit decoding constants
 
   __device__ __forceinline__ void reset() {
     m[0] = m[1] = -INFINITY;
@@ -174,6 +190,7 @@ struct MmaWarp {
     if constexpr (KV == KV_INT4) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) eo[i][0] = eo[i][1] = eo[i][2] = eo[i][3] = 0.f;
+      nc.init();
     }
   }
 
@@ -311,17 +328,17 @@ struct MmaWarp {
           for (int gq = 0; gq < 4; ++gq) {
             float t[4];
             uint32_t a[4];
-            a[0] = nib_lo_f16x2(w0[gq]);
-            a[1] = nib_lo_f16x2(w1[gq]);
-            a[2] = nib_hi_f16x2(w0[gq]);
-            a[3] = nib_hi_f16x2(w1[gq]);
+            a[0] = lop3_and_or(w0[gq], nc.lo, nc.magic);
+            a[1] = lop3_and_or(w1[gq], nc.lo, nc.magic);
+            a[2] = lop3_and_or(w0[gq], nc.hi, nc.magic);
+            a[3] = lop3_and_or(w1[gq], nc.hi, nc.magic);
             mma_f16_16816_c(t, a, qf[2 * gq][0], qf[2 * gq][1], cq[gq][0], cq[gq][1], cq[gq][0],
                             cq[gq][1]);
             const uint32_t x0 = w0[gq] >> 8, x1 = w1[gq] >> 8;
-            a[0] = nib_lo_f16x2(x0);
-            a[1] = nib_lo_f16x2(x1);
-            a[2] = nib_hi_f16x2(x0);
-            a[3] = nib_hi_f16x2(x1);
+            a[0] = lop3_and_or(x0, nc.lo, nc.magic);
+            a[1] = lop3_and_or(x1, nc.lo, nc.magic);
+            a[2] = lop3_and_or(x0, nc.hi, nc.magic);
+            a[3] = lop3_and_or(x1, nc.hi, nc.magic);
             mma_f16_16816(t, a, qf[2 * gq + 1][0], qf[2 * gq + 1][1]);
             s[mt][0] = fmaf(ks0[gq], t[0], s[mt][0]);
             s[mt][1] = fmaf(ks0[gq], t[1], s[mt][1]);
@@ -424,10 +441,10 @@ struct MmaWarp {
               w1 >>= 8;
             }
             uint32_t a[4];
-            a[0] = nib_lo_f16x2(w0);
-            a[1] = nib_lo_f16x2(w1);
-            a[2] = nib_hi_f16x2(w0);
-            a[3] = nib_hi_f16x2(w1);
+            a[0] = lop3_and_or(w0, nc.lo, nc.magic);
+            a[1] = lop3_and_or(w1, nc.lo, nc.magic);
+            a[2] = lop3_and_or(w0, nc.hi, nc.magic);
+            a[3] = lop3_and_or(w1, nc.hi, nc.magic);
             mma(o[md], a, b[mt][0], b[mt][1]);
           }
         }
