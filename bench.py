@@ -57,6 +57,8 @@ def parse_args():
     ap.add_argument("--kv-dtype", default=None, choices=["f32", "bf16", "fp8", "int4"],
                     help="store the workload's K/V in this dtype instead of its own")
     ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--no-numa-bind", action="store_true",
+                    help="do not pin the process to the CPUs local to its GPU")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-attention measurement")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill-attention measurement and print it")
@@ -87,6 +89,32 @@ def with_kv_dtype(wl, kv_dtype):
     i = wl.name.rfind(old)
     name = wl.name[:i] + new + wl.name[i + len(old):] if i >= 0 else wl.name + new
     return dataclasses.replace(wl, name=name, kv_dtype=kv_dtype)
+
+
+def bind_to_gpu_numa_node(device_index: int):
+    """Pin this process to the CPUs the GPU's PCI function reports as local
+    (sysfs local_cpulist), so that pinned host buffers are allocated on the
+    GPU's NUMA node.  Returns the CPU list, or None when it is unknown."""
+    import torch
+    prop = torch.cuda.get_device_properties(device_index)
+    path = "/sys/bus/pci/devices/%04x:%02x:%02x.0/local_cpulist" % (
+        prop.pci_domain_id, prop.pci_bus_id, prop.pci_device_id)
+    try:
+        text = open(path).read().strip()
+    except OSError:
+        return None
+    cpus = set()
+    for part in text.split(","):
+        if "-" in part:
+            a, b = part.split("-")
+            cpus.update(range(int(a), int(b) + 1))
+        elif part:
+            cpus.add(int(part))
+    cpus &= os.sched_getaffinity(0)
+    if not cpus:
+        return None
+    os.sched_setaffinity(0, cpus)
+    return text
 
 
 def measured_peaks():
@@ -410,6 +438,7 @@ def main():
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
+    numa = None if args.no_numa_bind else bind_to_gpu_numa_node(local)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
@@ -597,6 +626,7 @@ def main():
         e2e = {"value": e_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": int(stp.layout.in_bytes), "d2h_bytes_per_step": int(stp.layout.out_bytes),
                "steps": E, "ms_per_step": e_ms / E,
+               "host_cpus": numa or "not bound",
                "host_issue_us_per_step": host_issue_s / E * 1e6,
                "path": "dms_stepper_step: one packed pinned-host input copy, append/evict, decode "
                        "attention, one pinned-host output copy per step; copies on their own streams, "
