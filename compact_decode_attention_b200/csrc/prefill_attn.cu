@@ -11,13 +11,14 @@
 // opening paragraphs), so the kernel that streams the prompt's K/V tiles for
 // attention also writes the kept rows into their slots.
 //
-// One CTA of 4 warps per (128-query tile, query head, sequence), heaviest
+// One CTA of 8 warps per (128-query tile, query head, sequence), heaviest
 // (latest) query tiles first.  Per 128-key tile, on the 5th-generation
 // tensor cores with accumulators in tensor memory:
 //   S = Q K^T           (M = 128 queries, N = 128 keys, K = D)
-//   thread r owns query row r: masked online softmax on S[r] (tcgen05.ld),
-//   P[r] as bf16 into shared memory, O[r] rescaled in tensor memory when the
-//   row maximum moved
+//   threads r and r + 128 own query row r, 64 key columns each: masked
+//   online softmax on S[r] (tcgen05.ld; the row maximum is combined through
+//   shared memory), P[r] as bf16 into shared memory, O[r] rescaled in tensor
+//   memory when the row maximum moved
 //   O += P V            (M = 128 queries, N = D, K = 128 keys; V is read in
 //                        its own [keys x D] layout as an MN-major operand)
 // Tiles live in shared memory in the 128-byte-swizzled image of umma.cuh,
@@ -34,7 +35,14 @@
 namespace dms {
 
 constexpr int kPaTile = 128;      // queries per CTA and keys per tile
-constexpr int kPaThreads = 128;   // one thread per query row
+// threads per query row: each takes 128 / SPLIT key columns of S and D / SPLIT
+// columns of O (32 at least, the width of one tensor-memory load).  Two beat
+// one (the softmax issues from twice the warps) and four (more exchanges).
+template <int D>
+struct PaSplit {
+  static constexpr int SPLIT = 2;
+  static constexpr int THREADS = kPaTile * SPLIT;
+};
 
 template <int D>
 struct PaSmem {
@@ -46,7 +54,8 @@ struct PaSmem {
   static constexpr int FLAGS = P + kPaTile * kPaTile * 2;  // 2 x 4 words of evict-flag bits
   static constexpr int BARS = FLAGS + 2 * kPaTile;     // 2 mbarriers
   static constexpr int MISC = BARS + 16;               // tmem base, scan
-  static constexpr int BYTES = MISC + 64 + 1024;       // + alignment slack
+  static constexpr int RED = MISC + 64;                // [SPLIT parts][128 rows] floats
+  static constexpr int BYTES = RED + PaSplit<D>::SPLIT * kPaTile * 4 + 1024;  // + alignment slack
 };
 
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
@@ -61,7 +70,7 @@ template <int D>
 __device__ __forceinline__ void copy_rows_async(uint8_t* tile, const __nv_bfloat16* src,
                                                 int64_t row_stride, int row0, int P, int tid) {
   constexpr int CH = D / 8;  // 16-byte chunks per row
-  for (int idx = tid; idx < kPaTile * CH; idx += kPaThreads) {
+  for (int idx = tid; idx < kPaTile * CH; idx += PaSplit<D>::THREADS) {
     const int r = idx / CH, c = idx % CH;
     const bool valid = row0 + r < P;
     const __nv_bfloat16* g = src + int64_t(valid ? row0 + r : 0) * row_stride + c * 8;
@@ -70,7 +79,7 @@ __device__ __forceinline__ void copy_rows_async(uint8_t* tile, const __nv_bfloat
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPaThreads, 1)
+__global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
     prefill_attn_kernel(PoolView v, int layer, int seq0, int P, const __nv_bfloat16* q,
                         const __nv_bfloat16* k, const __nv_bfloat16* vv, const uint8_t* evict,
                         __nv_bfloat16* out, float scale_log2, int n_qtiles, int compact) {
@@ -78,6 +87,13 @@ __global__ void __launch_bounds__(kPaThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // query row r of the tile, key-column part h (columns HC h .. HC h + HC - 1
+  // of S, OC h .. of O); warps w, w + 4, ... share the tensor-memory lanes of
+  // rows 32 (w & 3) .. + 31
+  constexpr int SPLIT = PaSplit<D>::SPLIT, THREADS = PaSplit<D>::THREADS;
+  constexpr int HC = kPaTile / SPLIT, OC = D / SPLIT;  // S and O columns per thread
+  const int r = tid & (kPaTile - 1), h = tid >> 7;
+  float* s_red = reinterpret_cast<float*>(smem + S::RED);
   const int qt = n_qtiles - 1 - int(blockIdx.x);  // heaviest query tiles first
   const int hq = blockIdx.y, b = blockIdx.z;
   const int g = v.Hq / v.Hkv, hkv = hq / g;
@@ -97,10 +113,10 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     copy_rows_async<D>(smem + S::K + buf * S::TILE, ksrc, kv_stride, j0, P, tid);
     copy_rows_async<D>(smem + S::V + buf * S::TILE, vsrc, kv_stride, j0, P, tid);
   };
-  // evict flag of key j0 + tid of tile kt (loaded a tile ahead, packed later)
+  // evict flag of key j0 + r of tile kt (loaded a tile ahead, packed later)
   auto flag_of = [&](int kt) -> uint8_t {
-    const int j = kt * kPaTile + tid;
-    return j < P ? evict[(int64_t(b) * P + j) * v.Hkv + hkv] : 0;
+    const int j = kt * kPaTile + r;
+    return (h == 0 && j < P) ? evict[(int64_t(b) * P + j) * v.Hkv + hkv] : 0;
   };
   uint32_t* s_fbits = reinterpret_cast<uint32_t*>(smem + S::FLAGS);  // [2][4]
 
@@ -126,7 +142,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
   const uint32_t aQ = smem_u32(smem + S::Q), aP = smem_u32(smem + S::P);
   constexpr uint32_t idS = umma::idesc_bf16_f32(kPaTile, kPaTile);
   constexpr uint32_t idO = umma::idesc_bf16_f32_bmn(kPaTile, D);
-  const int i = i0 + tid;  // this thread's query row
+  const int i = i0 + r;  // this thread's query row
   float m = -INFINITY, l = 0.f;
   volatile int never = 0;
   bool ok = true;
@@ -140,7 +156,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     }
     {  // this tile's flags as 4 words of bits (bit c = key j0 + c flagged)
       const unsigned fw = __ballot_sync(0xffffffffu, f_cur != 0);
-      if (lane == 0) s_fbits[cur * 4 + warp] = fw;
+      if (lane == 0 && h == 0) s_fbits[cur * 4 + warp] = fw;
     }
     uint8_t f_next = 0;
     if (kt < qt) {  // the next tile streams in while this one is computed
@@ -170,35 +186,40 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     // ---- masked online softmax on query row i (log2 domain) ----
     // visibility of key j0 + c as bits: flag clear or inside the window
     // (c >= i - w + 1 - j0), causal (c <= i - j0), inside the prompt (c < P - j0)
-    uint32_t vis[4];
+    uint32_t vis[HC / 32];
     {
       const int hi = i - j0, lo = i - v.w + 1 - j0, end = P - j0;
 #pragma unroll
-      for (int wd = 0; wd < 4; ++wd) {
-        const int c0 = 32 * wd;
+      for (int x = 0; x < HC / 32; ++x) {
+        const int wd = (HC / 32) * h + x, c0 = 32 * wd;
         const int x_le = hi - c0, x_ge = lo - c0, x_lt = end - c0;
         const uint32_t le = x_le < 0 ? 0u : x_le >= 31 ? ~0u : (2u << x_le) - 1u;
         const uint32_t ge = x_ge <= 0 ? ~0u : x_ge >= 32 ? 0u : ~((1u << x_ge) - 1u);
         const uint32_t lt = x_lt <= 0 ? 0u : x_lt >= 32 ? ~0u : (1u << x_lt) - 1u;
-        vis[wd] = (~s_fbits[cur * 4 + wd] | ge) & le & lt;
+        vis[x] = (~s_fbits[cur * 4 + wd] | ge) & le & lt;
       }
     }
-    float s[kPaTile];
+    float s[HC];
 #pragma unroll
-    for (int cb = 0; cb < kPaTile / 32; ++cb) {
+    for (int cb = 0; cb < HC / 32; ++cb) {
       float x[32];
-      umma::ld32(umma::taddr_of(t_s, warp, cb * 32), x);
+      umma::ld32(umma::taddr_of(t_s, warp, h * HC + cb * 32), x);
 #pragma unroll
       for (int e = 0; e < 32; ++e) s[cb * 32 + e] = x[e];
     }
     umma::wait_ld();
     float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int c = 0; c < kPaTile; ++c) {
+    for (int c = 0; c < HC; ++c) {
       s[c] = ((vis[c >> 5] >> (c & 31)) & 1u) ? s[c] * scale_log2 : -INFINITY;
       mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
     }
-    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+    // the row maximum over the row's SPLIT threads (r, r + 128, ...)
+    s_red[h * kPaTile + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+    __syncthreads();
+    float mx = s_red[r];
+#pragma unroll
+    for (int x = 1; x < SPLIT; ++x) mx = fmaxf(mx, s_red[x * kPaTile + r]);
     // lazy rescaling: the running maximum only moves when the row maximum
     // grew by more than 8 (log2 units), so P stays <= 256 and O rarely needs
     // a round trip through tensor memory
@@ -209,31 +230,31 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     }
     float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < kPaTile; ++c) {
+    for (int c = 0; c < HC; ++c) {
       const float p = m == -INFINITY ? 0.f : fast_exp2(s[c] - m);
       sum4[c & 3] += p;
       s[c] = p;
     }
     l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
 #pragma unroll
-    for (int ch = 0; ch < kPaTile / 8; ++ch) {
+    for (int ch = 0; ch < HC / 8; ++ch) {
       uint4 w4;
       w4.x = pack2_bf16(s[ch * 8 + 0], s[ch * 8 + 1]);
       w4.y = pack2_bf16(s[ch * 8 + 2], s[ch * 8 + 3]);
       w4.z = pack2_bf16(s[ch * 8 + 4], s[ch * 8 + 5]);
       w4.w = pack2_bf16(s[ch * 8 + 6], s[ch * 8 + 7]);
-      *reinterpret_cast<uint4*>(smem + S::P + umma::sw128_offset(kPaTile, tid, ch * 8)) = w4;
+      *reinterpret_cast<uint4*>(smem + S::P + umma::sw128_offset(kPaTile, r, h * HC + ch * 8)) = w4;
     }
     // O row *= alpha when this warp has a row whose maximum moved
     if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-      for (int cb = 0; cb < D / 32; ++cb) {
+      for (int cb = 0; cb < OC / 32; ++cb) {
         float o[32];
-        umma::ld32(umma::taddr_of(t_o, warp, cb * 32), o);
+        umma::ld32(umma::taddr_of(t_o, warp, h * OC + cb * 32), o);
         umma::wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] *= alpha;
-        umma::st32(umma::taddr_of(t_o, warp, cb * 32), o);
+        umma::st32(umma::taddr_of(t_o, warp, h * OC + cb * 32), o);
       }
       umma::wait_st();
     }
@@ -259,12 +280,18 @@ __global__ void __launch_bounds__(kPaThreads, 1)
   // executes it, also lanes whose query lies past the prompt; only the
   // stores are guarded
   {
-    const float inv = i < P ? 1.f / l : 0.f;
-    __nv_bfloat16* dst = out + (int64_t(b) * P + i) * q_stride + int64_t(hq) * D;
+    // the row sum over the row's SPLIT threads
+    s_red[h * kPaTile + r] = l;
+    __syncthreads();
+    float lsum = s_red[r];
 #pragma unroll
-    for (int cb = 0; cb < D / 32; ++cb) {
+    for (int x = 1; x < SPLIT; ++x) lsum += s_red[x * kPaTile + r];
+    const float inv = i < P ? 1.f / lsum : 0.f;
+    __nv_bfloat16* dst = out + (int64_t(b) * P + i) * q_stride + int64_t(hq) * D + h * OC;
+#pragma unroll
+    for (int cb = 0; cb < OC / 32; ++cb) {
       float o[32];
-      umma::ld32(umma::taddr_of(t_o, warp, cb * 32), o);
+      umma::ld32(umma::taddr_of(t_o, warp, h * OC + cb * 32), o);
       umma::wait_ld();
       if (i < P) {
 #pragma unroll
@@ -292,14 +319,14 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       return j < P && (f == 0 || (P - 1 - j) < v.w);
     };
     uint8_t f = 0, f_unused = 0;
-    const int j = i0 + tid;
+    const int j = i0 + r;
     const bool keep = keep_of(j, &f);
     const unsigned bm = __ballot_sync(0xffffffffu, keep);
     // the prefix counts cover 256-token chunks; a second-half tile adds the
     // kept count of the first half
     const bool first_half_keep = (qt & 1) ? keep_of(j - kPaTile, &f_unused) : false;
     const unsigned bm1 = __ballot_sync(0xffffffffu, first_half_keep);
-    if (lane == 0) {
+    if (lane == 0 && h == 0) {
       s_scan[warp] = __popc(bm);
       s_scan[4 + warp] = __popc(bm1);
     }
@@ -314,8 +341,8 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     const int rank = before + __popc(bm & ((1u << lane) - 1u));
     const int base = v.chunk_counts[(int64_t(b) * v.Hkv + hkv) * v.n_chunks_max + (qt >> 1)] + first_half;
     const int32_t* table = v.bt + int64_t(hd) * v.mbh;
-    if (keep) {
-      s_kept[rank] = tid;
+    if (keep && h == 0) {
+      s_kept[rank] = r;
       if (j >= P - v.w) {
         const int slot = base + rank;
         const int64_t ri = int64_t(hd) * v.w + (j % v.w);
@@ -325,14 +352,14 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     }
     __syncthreads();
     constexpr int CH = D / 8;
-    for (int idx = tid; idx < nkept * CH; idx += kPaThreads) {
+    for (int idx = tid; idx < nkept * CH; idx += THREADS) {
       const int kk = idx / CH, c = idx % CH;
-      const int r = s_kept[kk];
+      const int kr = s_kept[kk];
       const int slot = base + kk, row = slot % v.BT;
       const int blk = table[slot / v.BT];
       if (!DMS_CHECK(blk >= 0 && blk < v.max_blocks && slot / v.BT < v.mbh, v.hdr, 501, hd, slot)) continue;
       uint8_t* dst = v.blocks + int64_t(blk) * v.block_bytes + int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;
-      const uint32_t so = (qt & 1) * S::TILE + umma::sw128_offset(kPaTile, r, c * 8);
+      const uint32_t so = (qt & 1) * S::TILE + umma::sw128_offset(kPaTile, kr, c * 8);
       *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(smem + S::K + so);
       *reinterpret_cast<uint4*>(dst + v.tile_bytes) = *reinterpret_cast<const uint4*>(smem + S::V + so);
     }
@@ -394,7 +421,7 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
       if (st != DMS_OK) return st;
       attr = true;
     }
-    prefill_attn_kernel<128><<<grid, kPaThreads, PaSmem<128>::BYTES, stream>>>(
+    prefill_attn_kernel<128><<<grid, PaSplit<128>::THREADS, PaSmem<128>::BYTES, stream>>>(
         pv, layer, seq0, prompt_len, kq, kk, kv, evict, ko, scale_log2, n_qtiles, 1);
   } else {
     static bool attr = false;
@@ -404,7 +431,7 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
       if (st != DMS_OK) return st;
       attr = true;
     }
-    prefill_attn_kernel<64><<<grid, kPaThreads, PaSmem<64>::BYTES, stream>>>(
+    prefill_attn_kernel<64><<<grid, PaSplit<64>::THREADS, PaSmem<64>::BYTES, stream>>>(
         pv, layer, seq0, prompt_len, kq, kk, kv, evict, ko, scale_log2, n_qtiles, 1);
   }
   return cuda_status(cudaGetLastError(), "prefill_attn_kernel");
