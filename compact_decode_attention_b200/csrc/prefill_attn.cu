@@ -27,6 +27,8 @@
 // query head of each kv-head group writes,
 // at its diagonal key tile, the tile's kept rows into the pool (slots from
 // the prefix counts of the count and plan kernels) and the window ring.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 
 #include "dms_internal.cuh"
@@ -52,8 +54,8 @@ struct PaSmem {
   static constexpr int V = K + 2 * TILE;               // 2 buffers of values [keys x D] (MN-major B)
   static constexpr int P = V + 2 * TILE;               // [128 queries x 128 keys] bf16
   static constexpr int FLAGS = P + kPaTile * kPaTile * 2;  // 2 x 4 words of evict-flag bits
-  static constexpr int BARS = FLAGS + 2 * kPaTile;     // 2 mbarriers
-  static constexpr int MISC = BARS + 16;               // tmem base, scan
+  static constexpr int BARS = FLAGS + 2 * kPaTile;     // mbarriers: S, O, Q, K/V x 2
+  static constexpr int MISC = BARS + 64;               // tmem base, scan
   static constexpr int RED = MISC + 64;                // [SPLIT parts][128 rows] floats
   static constexpr int BYTES = RED + PaSplit<D>::SPLIT * kPaTile * 4 + 1024;  // + alignment slack
 };
@@ -63,26 +65,12 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Asynchronous copy of rows [row0, row0 + 128) of one head of a [B, P, H, D]
-// bf16 tensor into the swizzled image of a tile with 128 rows; rows past P
-// are zero-filled.
-template <int D>
-__device__ __forceinline__ void copy_rows_async(uint8_t* tile, const __nv_bfloat16* src,
-                                                int64_t row_stride, int row0, int P, int tid) {
-  constexpr int CH = D / 8;  // 16-byte chunks per row
-  for (int idx = tid; idx < kPaTile * CH; idx += PaSplit<D>::THREADS) {
-    const int r = idx / CH, c = idx % CH;
-    const bool valid = row0 + r < P;
-    const __nv_bfloat16* g = src + int64_t(valid ? row0 + r : 0) * row_stride + c * 8;
-    umma::cp_async16(tile + umma::sw128_offset(kPaTile, r, c * 8), g, valid);
-  }
-}
-
 template <int D>
 __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
-    prefill_attn_kernel(PoolView v, int layer, int seq0, int P, const __nv_bfloat16* q,
-                        const __nv_bfloat16* k, const __nv_bfloat16* vv, const uint8_t* evict,
-                        __nv_bfloat16* out, float scale_log2, int n_qtiles, int compact) {
+    prefill_attn_kernel(PoolView v, int layer, int seq0, int P, const __grid_constant__ CUtensorMap tq,
+                        const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                        const uint8_t* evict, __nv_bfloat16* out, float scale_log2, int n_qtiles,
+                        int compact) {
   using S = PaSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -99,19 +87,26 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
   const int g = v.Hq / v.Hkv, hkv = hq / g;
   const int i0 = qt * kPaTile;
   const int64_t q_stride = int64_t(v.Hq) * D, kv_stride = int64_t(v.Hkv) * D;
-  const __nv_bfloat16* qsrc = q + int64_t(b) * P * q_stride + int64_t(hq) * D;
-  const __nv_bfloat16* ksrc = k + int64_t(b) * P * kv_stride + int64_t(hkv) * D;
-  const __nv_bfloat16* vsrc = vv + int64_t(b) * P * kv_stride + int64_t(hkv) * D;
+  (void)kv_stride;
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + S::BARS);
   uint64_t* bar_o = bar_s + 1;
+  uint64_t* bar_q = bar_s + 2;
+  uint64_t* bar_kv = bar_s + 3;  // [2]: K and V tiles of buffer 0 / 1
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::MISC);
   int* s_scan = reinterpret_cast<int*>(smem + S::MISC) + 4;
 
-  // stage keys and values of tile kt into buffer kt & 1 (asynchronous copies)
-  auto stage_tile = [&](int kt) {
-    const int buf = kt & 1, j0 = kt * kPaTile;
-    copy_rows_async<D>(smem + S::K + buf * S::TILE, ksrc, kv_stride, j0, P, tid);
-    copy_rows_async<D>(smem + S::V + buf * S::TILE, vsrc, kv_stride, j0, P, tid);
+  // keys and values of tile kt into buffer kt & 1: tensor-map loads of
+  // 64-column boxes (128 rows each, 128-byte swizzle: the operand image of
+  // umma.cuh); rows past the prompt arrive as zeros.  One thread.
+  auto load_tile = [&](int kt) {
+    const int buf = kt & 1;
+    mbar_arrive_expect_tx(&bar_kv[buf], 2 * S::TILE);
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb) {
+      const int off = buf * S::TILE + kb * kPaTile * 128;
+      umma::tma_load_3d(smem + S::K + off, &tk, hkv * D + kb * 64, kt * kPaTile, b, &bar_kv[buf]);
+      umma::tma_load_3d(smem + S::V + off, &tv, hkv * D + kb * 64, kt * kPaTile, b, &bar_kv[buf]);
+    }
   };
   // evict flag of key j0 + r of tile kt (loaded a tile ahead, packed later)
   auto flag_of = [&](int kt) -> uint8_t {
@@ -123,6 +118,9 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
   if (tid == 0) {
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
+    mbar_init(bar_q, 1);
+    mbar_init(&bar_kv[0], 1);
+    mbar_init(&bar_kv[1], 1);
     fence_mbar_init();
   }
   __syncwarp();  // tcgen05.alloc is warp-collective: lane 0 rejoins first
@@ -130,9 +128,14 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
     umma::tmem_alloc(s_tmem, 256);
     umma::tmem_relinquish();
   }
-  copy_rows_async<D>(smem + S::Q, qsrc, q_stride, i0, P, tid);
-  stage_tile(0);
-  umma::cp_async_commit();
+  __syncthreads();  // barriers initialised before any thread waits on them
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_q, S::TILE);
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb)
+      umma::tma_load_3d(smem + S::Q + kb * kPaTile * 128, &tq, hq * D + kb * 64, i0, b, bar_q);
+    load_tile(0);
+  }
   uint8_t f_cur = flag_of(0);
   umma::fence_before_sync();
   __syncthreads();
@@ -158,16 +161,13 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
       const unsigned fw = __ballot_sync(0xffffffffu, f_cur != 0);
       if (lane == 0 && h == 0) s_fbits[cur * 4 + warp] = fw;
     }
-    uint8_t f_next = 0;
-    if (kt < qt) {  // the next tile streams in while this one is computed
-      stage_tile(kt + 1);
-      umma::cp_async_commit();
-      f_next = flag_of(kt + 1);
-      umma::cp_async_wait<1>();
-    } else {
-      umma::cp_async_wait<0>();
-    }
-    fence_proxy_async_smem();  // copies before the tensor cores read them
+    const uint8_t f_next = kt < qt ? flag_of(kt + 1) : 0;
+    // the next tile streams in while this one is computed (its buffer was
+    // last read by P V of tile kt-1, complete above)
+    if (tid == 0 && kt < qt) load_tile(kt + 1);
+    if (kt == 0) ok &= mbar_wait_bounded(bar_q, 0, &never);
+    ok &= mbar_wait_bounded(&bar_kv[cur], (kt >> 1) & 1, &never);
+    __syncwarp();
     __syncthreads();
     const uint32_t aK = smem_u32(smem + S::K + cur * S::TILE);
     const uint32_t aV = smem_u32(smem + S::V + cur * S::TILE);
@@ -374,6 +374,42 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
 
 using namespace dms;
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library)
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Tensor map of a [batch, P, H * D] bf16 tensor: boxes of 64 elements x 128
+// rows x 1 sequence, 128-byte swizzle, zeros outside.
+static dms_status encode_bf16_map(CUtensorMap* m, const void* base, int batch, int P, int HD) {
+  auto enc = tensor_map_encoder();
+  if (!enc) {
+    set_last_error("cuTensorMapEncodeTiled is not available");
+    return DMS_ERR_CUDA;
+  }
+  const cuuint64_t dims[3] = {cuuint64_t(HD), cuuint64_t(P), cuuint64_t(batch)};
+  const cuuint64_t strides[2] = {cuuint64_t(HD) * 2, cuuint64_t(HD) * 2 * cuuint64_t(P)};
+  const cuuint32_t box[3] = {64, cuuint32_t(kPaTile), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_last_error("cuTensorMapEncodeTiled failed (%d)", int(r));
+    return DMS_ERR_CUDA;
+  }
+  return DMS_OK;
+}
+
 extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
                                        const void* q, const void* k, const void* v,
                                        dms_dtype in_dtype, const uint8_t* evict, void* out,
@@ -409,9 +445,11 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
   const dim3 grid(n_qtiles, pv.Hq, batch);
   const float sc = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf(float(pv.D));
   const float scale_log2 = sc * 1.4426950408889634f;
-  auto kq = static_cast<const __nv_bfloat16*>(q);
-  auto kk = static_cast<const __nv_bfloat16*>(k);
-  auto kv = static_cast<const __nv_bfloat16*>(v);
+  CUtensorMap tq, tk, tv;
+  st = encode_bf16_map(&tq, q, batch, prompt_len, pv.Hq * pv.D);
+  if (st == DMS_OK) st = encode_bf16_map(&tk, k, batch, prompt_len, pv.Hkv * pv.D);
+  if (st == DMS_OK) st = encode_bf16_map(&tv, v, batch, prompt_len, pv.Hkv * pv.D);
+  if (st != DMS_OK) return st;
   auto ko = static_cast<__nv_bfloat16*>(out);
   if (pv.D == 128) {
     static bool attr = false;
@@ -422,7 +460,7 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
       attr = true;
     }
     prefill_attn_kernel<128><<<grid, PaSplit<128>::THREADS, PaSmem<128>::BYTES, stream>>>(
-        pv, layer, seq0, prompt_len, kq, kk, kv, evict, ko, scale_log2, n_qtiles, 1);
+        pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, 1);
   } else {
     static bool attr = false;
     if (!attr) {
@@ -432,7 +470,7 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
       attr = true;
     }
     prefill_attn_kernel<64><<<grid, PaSplit<64>::THREADS, PaSmem<64>::BYTES, stream>>>(
-        pv, layer, seq0, prompt_len, kq, kk, kv, evict, ko, scale_log2, n_qtiles, 1);
+        pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, 1);
   }
   return cuda_status(cudaGetLastError(), "prefill_attn_kernel");
 }
