@@ -91,6 +91,18 @@ def with_kv_dtype(wl, kv_dtype):
     return dataclasses.replace(wl, name=name, kv_dtype=kv_dtype)
 
 
+def parse_cpulist(text: str) -> set:
+    """The CPUs of a sysfs cpu list such as "0-15,32-47"."""
+    cpus = set()
+    for part in text.strip().split(","):
+        if "-" in part:
+            a, b = part.split("-")
+            cpus.update(range(int(a), int(b) + 1))
+        elif part:
+            cpus.add(int(part))
+    return cpus
+
+
 def bind_to_gpu_numa_node(device_index: int):
     """Pin this process to the CPUs the GPU's PCI function reports as local
     (sysfs local_cpulist), so that pinned host buffers are allocated on the
@@ -103,14 +115,7 @@ def bind_to_gpu_numa_node(device_index: int):
         text = open(path).read().strip()
     except OSError:
         return None
-    cpus = set()
-    for part in text.split(","):
-        if "-" in part:
-            a, b = part.split("-")
-            cpus.update(range(int(a), int(b) + 1))
-        elif part:
-            cpus.add(int(part))
-    cpus &= os.sched_getaffinity(0)
+    cpus = parse_cpulist(text) & os.sched_getaffinity(0)
     if not cpus:
         return None
     os.sched_setaffinity(0, cpus)

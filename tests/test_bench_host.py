@@ -1,6 +1,7 @@
 """Host logic of bench.py on CPU: the cross-rank reduction with two gloo
-ranks (max of device times, sum of bytes), the expected-bytes formula and the
-reference arm's line."""
+ranks (max of device times, sum of bytes), the expected-bytes formula, the
+store-dtype override, the sysfs cpu-list parser, the lookup of a profiled
+traffic ratio and the reference arm's line."""
 import json
 import os
 import subprocess
@@ -54,6 +55,43 @@ def test_expected_bytes_of_the_default_workload():
     b = bench.expected_bytes_per_step(wl)
     # 288 heads, about 512 + 0.16 * 7680 kept tokens each, 512 bytes per token
     assert 200e6 < b < 300e6
+
+
+def test_kv_dtype_override_renames_and_resizes():
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import configs
+    wl = bench.with_kv_dtype(configs.QWEN8B_CTX8K, "int4")
+    assert wl.name == "qwen3-8b_l36_b1_ctx8192_s128_w512_int4g32" and wl.kv_dtype == "int4"
+    assert wl.kv_row_bytes() == 72 and configs.QWEN8B_CTX8K.kv_row_bytes() == 256
+    b8 = bench.with_kv_dtype(configs.QWEN8B_FP8_B8_CTX32K, "int4")
+    assert b8.name == "qwen3-8b_l36_b8_ctx32768_s256_w512_int4g32"
+    assert bench.with_kv_dtype(configs.QWEN8B_CTX8K, None) is configs.QWEN8B_CTX8K
+    assert bench.with_kv_dtype(configs.QWEN8B_CTX8K, "bf16") is configs.QWEN8B_CTX8K
+    # retained bytes scale with the row size: 2 x 72 instead of 2 x 256 bytes a token
+    r = bench.expected_bytes_per_step(wl) / bench.expected_bytes_per_step(configs.QWEN8B_CTX8K)
+    assert abs(r - 72 / 256) < 1e-12
+
+
+def test_parse_cpulist():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.parse_cpulist("0-3,8,10-11\n") == {0, 1, 2, 3, 8, 10, 11}
+    assert bench.parse_cpulist("5") == {5}
+
+
+def test_profiled_traffic_ratio_matches_workload_and_source(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    h = bench.attn_source_hash()
+    (tmp_path / "decode_attn_a.md").write_text(
+        f"workload: wl_a\nkernel source hash: {h}\n| dram bytes per algorithmic byte: 1.0200 | x |\n")
+    (tmp_path / "decode_attn_b.md").write_text(
+        "workload: wl_b\nkernel source hash: 0000000000000000\n| dram bytes per algorithmic byte: 1.5 |\n")
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    assert bench.profiled_traffic_ratio("wl_a") == (1.02, h)
+    assert bench.profiled_traffic_ratio("wl_b") == (None, None)   # taken on other sources
+    assert bench.profiled_traffic_ratio("wl_c") == (None, None)   # no summary
 
 
 @pytest.mark.slow
