@@ -11,7 +11,8 @@
 // opening paragraphs), so the kernel that streams the prompt's K/V tiles for
 // attention also writes the kept rows into their slots.
 //
-// One CTA of 8 warps per (128-query tile, query head, sequence), heaviest
+// One CTA of 8 warps per (128-query tile, query head, sequence), two CTAs
+// per SM (one CTA's softmax runs while the other's tensor cores work), heaviest
 // (latest) query tiles first.  Per 128-key tile, on the 5th-generation
 // tensor cores with accumulators in tensor memory:
 //   S = Q K^T           (M = 128 queries, N = 128 keys, K = D)
@@ -22,11 +23,12 @@
 //   O += P V            (M = 128 queries, N = D, K = 128 keys; V is read in
 //                        its own [keys x D] layout as an MN-major operand)
 // Tiles live in shared memory in the 128-byte-swizzled image of umma.cuh,
-// filled by 16-byte asynchronous copies into two buffers, so the next key
-// tile streams in while the current one is computed.  The CTA of the first
-// query head of each kv-head group writes,
-// at its diagonal key tile, the tile's kept rows into the pool (slots from
-// the prefix counts of the count and plan kernels) and the window ring.
+// filled by tensor-map (TMA) loads: the query tile once, then per key tile
+// its keys into the one tile buffer and, once S has read them, its values
+// into the same buffer while the softmax runs (about 100 KB a CTA, so that
+// two fit on an SM).  The CTA of the first query head of each kv-head group
+// writes, at its diagonal key tile, the tile's kept rows into the pool (slots
+// from the prefix counts of the count and plan kernels) and the window ring.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -50,11 +52,10 @@ template <int D>
 struct PaSmem {
   static constexpr int TILE = kPaTile * D * 2;         // one [128 x D] bf16 tile
   static constexpr int Q = 0;                          // queries, K-major
-  static constexpr int K = Q + TILE;                   // 2 buffers of keys, K-major
-  static constexpr int V = K + 2 * TILE;               // 2 buffers of values [keys x D] (MN-major B)
-  static constexpr int P = V + 2 * TILE;               // [128 queries x 128 keys] bf16
+  static constexpr int KV = Q + TILE;                  // keys (K-major), then values [keys x D] (MN-major B)
+  static constexpr int P = KV + TILE;                  // [128 queries x 128 keys] bf16
   static constexpr int FLAGS = P + kPaTile * kPaTile * 2;  // 2 x 4 words of evict-flag bits
-  static constexpr int BARS = FLAGS + 2 * kPaTile;     // mbarriers: S, O, Q, K/V x 2
+  static constexpr int BARS = FLAGS + 2 * kPaTile;     // mbarriers: S, O, Q, K, V
   static constexpr int MISC = BARS + 64;               // tmem base, scan
   static constexpr int RED = MISC + 64;                // [SPLIT parts][128 rows] floats
   static constexpr int BYTES = RED + PaSplit<D>::SPLIT * kPaTile * 4 + 1024;  // + alignment slack
@@ -66,7 +67,7 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
+__global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     prefill_attn_kernel(PoolView v, int layer, int seq0, int P, const __grid_constant__ CUtensorMap tq,
                         const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                         const uint8_t* evict, __nv_bfloat16* out, float scale_log2, int n_qtiles,
@@ -91,22 +92,19 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + S::BARS);
   uint64_t* bar_o = bar_s + 1;
   uint64_t* bar_q = bar_s + 2;
-  uint64_t* bar_kv = bar_s + 3;  // [2]: K and V tiles of buffer 0 / 1
+  uint64_t* bar_k = bar_s + 3;
+  uint64_t* bar_v = bar_s + 4;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::MISC);
   int* s_scan = reinterpret_cast<int*>(smem + S::MISC) + 4;
 
-  // keys and values of tile kt into buffer kt & 1: tensor-map loads of
-  // 64-column boxes (128 rows each, 128-byte swizzle: the operand image of
-  // umma.cuh); rows past the prompt arrive as zeros.  One thread.
-  auto load_tile = [&](int kt) {
-    const int buf = kt & 1;
-    mbar_arrive_expect_tx(&bar_kv[buf], 2 * S::TILE);
+  // tensor-map loads of one [128 x D] tile: boxes of 64 columns x 128 rows
+  // with 128-byte swizzle (the operand image of umma.cuh); rows past the
+  // prompt arrive as zeros.  One thread.
+  auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, int x0, int row0, uint64_t* bar) {
+    mbar_arrive_expect_tx(bar, S::TILE);
 #pragma unroll
-    for (int kb = 0; kb < D / 64; ++kb) {
-      const int off = buf * S::TILE + kb * kPaTile * 128;
-      umma::tma_load_3d(smem + S::K + off, &tk, hkv * D + kb * 64, kt * kPaTile, b, &bar_kv[buf]);
-      umma::tma_load_3d(smem + S::V + off, &tv, hkv * D + kb * 64, kt * kPaTile, b, &bar_kv[buf]);
-    }
+    for (int kb = 0; kb < D / 64; ++kb)
+      umma::tma_load_3d(dst + kb * kPaTile * 128, map, x0 + kb * 64, row0, b, bar);
   };
   // evict flag of key j0 + r of tile kt (loaded a tile ahead, packed later)
   auto flag_of = [&](int kt) -> uint8_t {
@@ -119,8 +117,8 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
     mbar_init(bar_q, 1);
-    mbar_init(&bar_kv[0], 1);
-    mbar_init(&bar_kv[1], 1);
+    mbar_init(bar_k, 1);
+    mbar_init(bar_v, 1);
     fence_mbar_init();
   }
   __syncwarp();  // tcgen05.alloc is warp-collective: lane 0 rejoins first
@@ -130,11 +128,8 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
   }
   __syncthreads();  // barriers initialised before any thread waits on them
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_q, S::TILE);
-#pragma unroll
-    for (int kb = 0; kb < D / 64; ++kb)
-      umma::tma_load_3d(smem + S::Q + kb * kPaTile * 128, &tq, hq * D + kb * 64, i0, b, bar_q);
-    load_tile(0);
+    load_tile(smem + S::Q, &tq, hq * D, i0, bar_q);
+    load_tile(smem + S::KV, &tk, hkv * D, 0, bar_k);
   }
   uint8_t f_cur = flag_of(0);
   umma::fence_before_sync();
@@ -152,25 +147,23 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
 
   for (int kt = 0; kt <= qt; ++kt) {
     const int cur = kt & 1, j0 = kt * kPaTile;
-    if (kt > 0) {  // P V of tile kt-1 is done: P and the other buffer are free
+    if (kt > 0) {  // P V of tile kt-1 is done: P and the tile buffer are free
       ok &= mbar_wait_bounded(bar_o, (kt - 1) & 1, &never);
       __syncwarp();
       umma::fence_after_sync();
+      if (tid == 0) load_tile(smem + S::KV, &tk, hkv * D, j0, bar_k);
+      __syncwarp();
     }
     {  // this tile's flags as 4 words of bits (bit c = key j0 + c flagged)
       const unsigned fw = __ballot_sync(0xffffffffu, f_cur != 0);
       if (lane == 0 && h == 0) s_fbits[cur * 4 + warp] = fw;
     }
     const uint8_t f_next = kt < qt ? flag_of(kt + 1) : 0;
-    // the next tile streams in while this one is computed (its buffer was
-    // last read by P V of tile kt-1, complete above)
-    if (tid == 0 && kt < qt) load_tile(kt + 1);
     if (kt == 0) ok &= mbar_wait_bounded(bar_q, 0, &never);
-    ok &= mbar_wait_bounded(&bar_kv[cur], (kt >> 1) & 1, &never);
+    ok &= mbar_wait_bounded(bar_k, kt & 1, &never);  // K_kt landed
     __syncwarp();
     __syncthreads();
-    const uint32_t aK = smem_u32(smem + S::K + cur * S::TILE);
-    const uint32_t aV = smem_u32(smem + S::V + cur * S::TILE);
+    const uint32_t aK = smem_u32(smem + S::KV), aV = aK;
     if (tid == 0) {
       umma::fence_after_sync();
 #pragma unroll
@@ -182,6 +175,10 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
     ok &= mbar_wait_bounded(bar_s, kt & 1, &never);
     __syncwarp();  // lanes leave the wait loop independently; tcgen05.ld is warp-collective
     umma::fence_after_sync();
+    // S read the keys: the values of the same tile stream into the buffer
+    // while the softmax runs
+    if (tid == 0) load_tile(smem + S::KV, &tv, hkv * D, j0, bar_v);
+    __syncwarp();
 
     // ---- masked online softmax on query row i (log2 domain) ----
     // visibility of key j0 + c as bits: flag clear or inside the window
@@ -264,12 +261,14 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
     __syncthreads();
     if (tid == 0) {
       umma::fence_after_sync();
+      ok &= mbar_wait_bounded(bar_v, kt & 1, &never);  // V_kt landed
 #pragma unroll
       for (int k0 = 0; k0 < kPaTile; k0 += 16)
         umma::mma_bf16(t_o, umma::desc_k16(aP, kPaTile, k0), umma::desc_mn_k16(aV, kPaTile, k0), idO,
                        kt > 0 || k0 > 0);
       umma::commit(bar_o);
     }
+    __syncwarp();
   }
   ok &= mbar_wait_bounded(bar_o, qt & 1, &never);
   __syncwarp();
@@ -306,11 +305,12 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
       }
     }
   }
-  if (!ok && tid == 0) report_error(v.hdr, DMS_DEVERR_TIMEOUT, layer, seq0 + b, hq);
-
   // ---- fused compaction: the diagonal key tile's kept rows into the pool ----
-  // (its K and V rows are still in shared memory)
+  // (its V rows are still in shared memory; its K rows come back into the
+  // query buffer, which no product reads any more)
   if (compact && hq % g == 0 && v.hdr->prefill_go) {
+    if (tid == 0) load_tile(smem + S::Q, &tk, hkv * D, qt * kPaTile, bar_q);
+    __syncwarp();
     int* s_kept = reinterpret_cast<int*>(smem + S::P);  // P is no longer read
     const int hd = v.head(layer, seq0 + b, hkv);
     auto keep_of = [&](int j, uint8_t* fl) {
@@ -350,6 +350,8 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
         v.ring_row[ri] = table[slot / v.BT] * v.BT + slot % v.BT;
       }
     }
+    ok &= mbar_wait_bounded(bar_q, 1, &never);  // K rows of the diagonal tile
+    __syncwarp();
     __syncthreads();
     constexpr int CH = D / 8;
     for (int idx = tid; idx < nkept * CH; idx += THREADS) {
@@ -359,12 +361,13 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 1)
       const int blk = table[slot / v.BT];
       if (!DMS_CHECK(blk >= 0 && blk < v.max_blocks && slot / v.BT < v.mbh, v.hdr, 501, hd, slot)) continue;
       uint8_t* dst = v.blocks + int64_t(blk) * v.block_bytes + int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;
-      const uint32_t so = (qt & 1) * S::TILE + umma::sw128_offset(kPaTile, kr, c * 8);
-      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(smem + S::K + so);
-      *reinterpret_cast<uint4*>(dst + v.tile_bytes) = *reinterpret_cast<const uint4*>(smem + S::V + so);
+      const uint32_t so = umma::sw128_offset(kPaTile, kr, c * 8);
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(smem + S::Q + so);
+      *reinterpret_cast<uint4*>(dst + v.tile_bytes) = *reinterpret_cast<const uint4*>(smem + S::KV + so);
     }
   }
 
+  if (!ok && tid == 0) report_error(v.hdr, DMS_DEVERR_TIMEOUT, layer, seq0 + b, hq);
   umma::fence_before_sync();
   __syncthreads();
   if (warp == 0) umma::tmem_dealloc(tbase, 256);
@@ -457,6 +460,10 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
       st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             PaSmem<128>::BYTES), "prefill attn smem attribute");
       if (st != DMS_OK) return st;
+      // two CTAs per SM: the whole shared-memory carveout
+      st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            int(cudaSharedmemCarveoutMaxShared)), "prefill attn carveout");
+      if (st != DMS_OK) return st;
       attr = true;
     }
     prefill_attn_kernel<128><<<grid, PaSplit<128>::THREADS, PaSmem<128>::BYTES, stream>>>(
@@ -466,6 +473,10 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
     if (!attr) {
       st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             PaSmem<64>::BYTES), "prefill attn smem attribute");
+      if (st != DMS_OK) return st;
+      // two CTAs per SM: the whole shared-memory carveout
+      st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            int(cudaSharedmemCarveoutMaxShared)), "prefill attn carveout");
       if (st != DMS_OK) return st;
       attr = true;
     }
