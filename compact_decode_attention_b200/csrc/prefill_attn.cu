@@ -141,7 +141,9 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
   constexpr uint32_t idS = umma::idesc_bf16_f32(kPaTile, kPaTile);
   constexpr uint32_t idO = umma::idesc_bf16_f32_bmn(kPaTile, D);
   const int i = i0 + r;  // this thread's query row
-  float m = -INFINITY, l = 0.f;
+  // running row maximum (log2 units); a large finite start instead of -inf
+  // keeps exp2(s - m) free of a check (masked entries are -inf and give 0)
+  float m = -1e30f, l = 0.f;
   volatile int never = 0;
   bool ok = true;
 
@@ -207,12 +209,12 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     umma::wait_ld();
     float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int c = 0; c < HC; ++c) {
-      s[c] = ((vis[c >> 5] >> (c & 31)) & 1u) ? s[c] * scale_log2 : -INFINITY;
+    for (int c = 0; c < HC; ++c) {  // unscaled scores; the scale enters the exponent below
+      s[c] = ((vis[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
       mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
     }
     // the row maximum over the row's SPLIT threads (r, r + 128, ...)
-    s_red[h * kPaTile + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+    s_red[h * kPaTile + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
     __syncthreads();
     float mx = s_red[r];
 #pragma unroll
@@ -222,13 +224,13 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     // a round trip through tensor memory
     float alpha = 1.f;
     if (mx > m + 8.f) {
-      alpha = m == -INFINITY ? 0.f : fast_exp2(m - mx);
+      alpha = fast_exp2(m - mx);
       m = mx;
     }
     float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < HC; ++c) {
-      const float p = m == -INFINITY ? 0.f : fast_exp2(s[c] - m);
+      const float p = fast_exp2(fmaf(s[c], scale_log2, -m));
       sum4[c & 3] += p;
       s[c] = p;
     }
