@@ -56,7 +56,7 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(configs.BY_NAME))
     ap.add_argument("--kv-dtype", default=None, choices=["f32", "bf16", "fp8", "int4"],
                     help="store the workload's K/V in this dtype instead of its own")
-    ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--e2e-steps", type=int, default=256)
     ap.add_argument("--no-numa-bind", action="store_true",
                     help="do not pin the process to the CPUs local to its GPU")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-attention measurement")

@@ -46,12 +46,17 @@ template <typename InT, int STORE>
 __global__ void __launch_bounds__(kAppendThreads)
     append_evict_kernel(PoolView v, int l0, int nl, int batch, int64_t pos, const InT* k,
                         const InT* vv, const uint8_t* evict, const int32_t* seq_ids,
-                        const int64_t* pos_arr) {
+                        const int64_t* pos_arr, const StepSync sync) {
   // the new rows and the pool state may have been written by the kernel
   // before this one; once they are visible, let the next kernel (decode
   // attention) be scheduled
   pdl_wait_prerequisites();
   pdl_launch_dependents();
+  if (sync.ready) {  // the step's inputs are copied in by another stream
+    if (threadIdx.x == 0 && !wait_counter_geq(sync.ready, sync.ready_value))
+      report_error(v.hdr, DMS_DEVERR_TIMEOUT, l0, -1, -1);
+    __syncthreads();
+  }
   const int H = nl * batch * v.Hkv;
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * kAppendHeadsPerCta + (threadIdx.x >> 5);
@@ -164,7 +169,8 @@ using namespace dms;
 static dms_status launch_append(dms_pool* pool, int layer0, int n_layers, int batch, int64_t pos,
                                 const void* k, const void* v, dms_dtype in_dtype,
                                 const uint8_t* evict, const int32_t* seq_ids,
-                                const int64_t* pos_arr, cudaStream_t stream) {
+                                const int64_t* pos_arr, cudaStream_t stream,
+                                const StepSync& sync = StepSync{}) {
   if (!pool) {
     set_last_error("null pool");
     return DMS_ERR_INVALID_ARG;
@@ -195,7 +201,7 @@ static dms_status launch_append(dms_pool* pool, int layer0, int n_layers, int ba
 #define DMS_LAUNCH_APPEND(T, F)                                                                   \
   st = cuda_status(launch_pdl(append_evict_kernel<T, F>, grid, dim3(kAppendThreads), 0, stream,  \
                               pv, layer0, n_layers, batch, pos, static_cast<const T*>(k),         \
-                              static_cast<const T*>(v), evict, seq_ids, pos_arr),                 \
+                              static_cast<const T*>(v), evict, seq_ids, pos_arr, sync),           \
                    "append_evict_kernel")
   const int mode = fp8 ? 1 : int4 ? 2 : 0;
   if (in_dtype == DMS_BF16) {
@@ -217,6 +223,15 @@ extern "C" dms_status dms_append_evict_layers(dms_pool* pool, int layer0, int n_
                                               cudaStream_t stream) {
   return launch_append(pool, layer0, n_layers, batch, pos, k, v, in_dtype, evict, nullptr, nullptr,
                        stream);
+}
+
+// The stepper's append launch: arguments as for dms_append_evict_layers,
+// plus the step counters.
+dms_status dms::append_layers_synced(dms_pool* pool, int layer0, int n_layers, int batch, int64_t pos,
+                                     const void* k, const void* v, dms_dtype in_dtype,
+                                     const uint8_t* evict, cudaStream_t stream, const StepSync& sync) {
+  return launch_append(pool, layer0, n_layers, batch, pos, k, v, in_dtype, evict, nullptr, nullptr,
+                       stream, sync);
 }
 
 extern "C" dms_status dms_append_evict_seqs(dms_pool* pool, int layer0, int n_layers, int n_seqs,

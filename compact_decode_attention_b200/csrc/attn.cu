@@ -117,6 +117,7 @@ struct AttnParams {
   float* ws_ml;       // [(G + Htot) * g * 2]
   const int32_t* seq_ids;  // pool sequence of batch row b (device), or null: row b
   int G;
+  StepSync sync;           // stepper counters (null pointers otherwise)
 };
 
 // Named barrier 1 among the consumer warps only (the producer never joins it).
@@ -691,6 +692,21 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   // queries may come from the kernel before this one (append/evict)
   pdl_launch_dependents();
   pdl_wait_prerequisites();
+  // stepper: the output buffer's previous copy-out must be done (thread 0;
+  // the scan's barrier below holds the other threads)
+  if (p.sync.drained && tid == 0 && !wait_counter_geq(p.sync.drained, p.sync.drained_value))
+    report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
+  // stepper: the last CTA to leave publishes the step as computed
+  auto sync_exit = [&]() {
+    if (p.sync.done && tid == 0) {
+      __threadfence();
+      if (atomicAdd(p.sync.exit_count, 1) == int(gridDim.x) - 1) {
+        *p.sync.exit_count = 0;
+        __threadfence();
+        st_release_gpu(p.sync.done, p.sync.done_value);
+      }
+    }
+  };
 
   // ---- find this CTA's unit range: per-thread head ranges + block scan ----
   const int per = (Htot + kAttnThreads - 1) / kAttnThreads;
@@ -721,7 +737,10 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   // with fewer blocks than CTAs only the first U CTAs take one block each,
   // so that every CTA in [0, Geff) has a non-empty range
   const int Geff = min(G, U);
-  if (c >= Geff) return;
+  if (c >= Geff) {
+    sync_exit();
+    return;
+  }
   const int u_beg = int((int64_t(c) * U) / Geff), u_end = int((int64_t(c + 1) * U) / Geff);
   if (u_beg < u_end && u_beg >= excl && u_beg < excl + su) {
     int pre = excl;
@@ -1026,6 +1045,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
       process_unit(k, min(kBlockTokens, n - (u - pp) * kBlockTokens));
     }
   }
+  sync_exit();  // after the last head's combine (its barriers ordered every consumer's writes)
 }
 
 template <int KV, int D>
@@ -1060,7 +1080,7 @@ static size_t attn_workspace_bytes(const dms_pool* pool, int n_layers, int batch
 // Fill the kernel parameters and launch (arguments already checked).
 static dms_status run_attn(dms_pool* pool, int layer0, int n_layers, int batch, const void* q,
                            void* out, float sm_scale, void* ws, const int32_t* seq_ids,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, const StepSync& sync = StepSync{}) {
   const PoolView& v = pool->view;
   const int g = v.Hq / v.Hkv;
   const size_t parts = size_t(pool->sm_count) + size_t(n_layers) * batch * v.Hkv;
@@ -1078,12 +1098,21 @@ static dms_status run_attn(dms_pool* pool, int layer0, int n_layers, int batch, 
                                        ((parts * g * v.D * 4 + 255) & ~size_t(255)));
   prm.seq_ids = seq_ids;
   prm.G = pool->sm_count;
+  prm.sync = sync;
   if (v.kv_dtype == DMS_BF16) {
     return v.D == 128 ? launch_attn<KV_BF16, 128>(prm, stream) : launch_attn<KV_BF16, 64>(prm, stream);
   }
   if (v.kv_dtype == DMS_FP8_E4M3) return launch_attn<KV_FP8, 128>(prm, stream);
   if (v.kv_dtype == DMS_INT4) return launch_attn<KV_INT4, 128>(prm, stream);
   return v.D == 128 ? launch_attn<KV_F32, 128>(prm, stream) : launch_attn<KV_F32, 64>(prm, stream);
+}
+
+// The stepper's attention launch: arguments as for dms_decode_attn_layers
+// (checked by the caller), plus the step counters.
+dms_status dms::decode_attn_layers_synced(dms_pool* pool, int layer0, int n_layers, int batch,
+                                          const void* q, void* out, float sm_scale, void* ws,
+                                          cudaStream_t stream, const StepSync& sync) {
+  return run_attn(pool, layer0, n_layers, batch, q, out, sm_scale, ws, nullptr, stream, sync);
 }
 
 extern "C" dms_status dms_decode_workspace_bytes(const dms_pool* pool, int n_layers, int batch,

@@ -185,6 +185,39 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Step counters shared with copy streams (the stepper): the copy streams
+// write and wait on them with stream memory operations, the kernels wait on
+// and publish them, so that the compute stream holds nothing but kernels.
+// A null pointer means no such condition.
+struct StepSync {
+  const int32_t* ready;    // append: inputs of this step landed once *ready >= ready_value
+  int32_t ready_value;
+  const int32_t* drained;  // attention: the output buffer's previous copy-out is done once
+  int32_t drained_value;   //            *drained >= drained_value
+  int32_t* done;           // attention: the last CTA to leave stores done_value
+  int32_t done_value;
+  int32_t* exit_count;     // attention: CTAs that left (the last one resets it)
+};
+
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Wait (one thread) until *p >= v; false after kWaitLimitNs.
+__device__ __forceinline__ bool wait_counter_geq(const int32_t* p, int32_t v) {
+  if (ld_acquire_gpu(p) >= v) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_gpu(p) < v) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(200);
+  }
+  return true;
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy (TMA) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -339,3 +372,13 @@ struct dms_pool {
   int device;
   int sm_count;
 };
+
+namespace dms {
+// stepper launches with step counters (csrc/append.cu, csrc/attn.cu)
+dms_status append_layers_synced(dms_pool* pool, int layer0, int n_layers, int batch, int64_t pos,
+                                const void* k, const void* v, dms_dtype in_dtype,
+                                const uint8_t* evict, cudaStream_t stream, const StepSync& sync);
+dms_status decode_attn_layers_synced(dms_pool* pool, int layer0, int n_layers, int batch,
+                                     const void* q, void* out, float sm_scale, void* ws,
+                                     cudaStream_t stream, const StepSync& sync);
+}  // namespace dms

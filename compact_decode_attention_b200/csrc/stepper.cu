@@ -3,16 +3,23 @@
 // Per step: one packed host->device copy of (k, v, q, evict) on the h2d
 // stream, append/evict and decode attention on the caller's compute stream,
 // one device->host copy of the output on the d2h stream.  kStepperDepth
-// staging buffers and as many output buffers rotate between steps; events
-// order the reuse (D = kStepperDepth):
-//   h2d(n)      waits  kernels(n-D) done    (staging[n % D] free again)
-//   kernels(n)  waits  h2d(n) done, d2h(n-D) done (output[n % D] free)
-//   d2h(n)      waits  kernels(n) done
-// With D = 4 the input copy of step n is issued three steps ahead of the
-// kernels that free its buffer, so it has landed before the compute stream
-// reaches step n and the waits there find their events complete (with two
-// buffers the copy waited for kernels(n-2) and the compute stream for the
-// copy, about 11 us a step on the Qwen3-8B ctx-8K workload).
+// staging buffers and as many output buffers rotate between steps (D =
+// kStepperDepth):
+//   h2d(n)      after  kernels(n-D)   (staging[n % D] free again)
+//   kernels(n)  after  h2d(n), d2h(n-D) (output[n % D] free)
+//   d2h(n)      after  kernels(n)
+// The compute stream holds only the kernels, so that the append of step
+// n+1 starts under the attention of step n (programmatic launch); the copy
+// streams wait on and set step counters in device memory (stream memory
+// operations), the append kernel waits for its inputs and the attention
+// kernel for its output buffer, and the attention's last CTA publishes the
+// step as computed.  Without the driver's stream memory operations the
+// same order is kept with events on all three streams.  With D = 4 the input
+// copy of step n is issued three steps ahead of the kernels that free its
+// buffer, so the waits find their conditions met (with two buffers the copy
+// waited for kernels(n-2) and the compute stream for the copy, about 11 us a
+// step on the Qwen3-8B ctx-8K workload).
+#include <cuda.h>
 #include <new>
 
 #include "dms_internal.cuh"
@@ -39,8 +46,21 @@ static dms_status stepper_layout(const dms_pool* pool, int n_layers, int batch,
   size_t ws = 0;
   dms_status st = dms_decode_workspace_bytes(pool, n_layers, batch, &ws);
   if (st != DMS_OK) return st;
-  o->device_bytes = kStepperDepth * (o->in_bytes + align256(qb)) + align256(ws);
+  // + 256 bytes of step counters (ready, done, drained, exit count)
+  o->device_bytes = kStepperDepth * (o->in_bytes + align256(qb)) + 256 + align256(ws);
   return DMS_OK;
+}
+
+// cuStreamWaitValue32 / cuStreamWriteValue32 through the runtime's driver
+// entry point (no link against the driver library); null when unavailable
+typedef CUresult (*StreamValueFn)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+static StreamValueFn stream_value_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<StreamValueFn>(p);
 }
 
 }  // namespace dms
@@ -60,6 +80,10 @@ struct dms_stepper {
   cudaStream_t compute, h2d, d2h;
   cudaEvent_t staged[kStepperDepth], computed[kStepperDepth], drained[kStepperDepth];
   int64_t steps;
+  // step counters in device memory: [0] steps staged, [1] steps computed,
+  // [2] steps copied out, [3] attention CTAs that left (self-resetting)
+  int32_t* counters;
+  StreamValueFn wait_value, write_value;  // both non-null: counter protocol
 };
 
 extern "C" dms_status dms_stepper_layout(const dms_pool* pool, int n_layers, int batch,
@@ -133,8 +157,13 @@ extern "C" dms_status dms_stepper_create(dms_pool* pool, int layer0, int n_layer
     s->out[j] = b;
     b += align256(lay.out_bytes);
   }
+  s->counters = reinterpret_cast<int32_t*>(b);
+  b += 256;
   s->ws = b;
   s->ws_bytes = device_bytes - size_t(b - static_cast<uint8_t*>(device_buf));
+  s->wait_value = stream_value_fn("cuStreamWaitValue32");
+  s->write_value = stream_value_fn("cuStreamWriteValue32");
+  if (!s->wait_value || !s->write_value) s->wait_value = s->write_value = nullptr;
   s->compute = stream;
   st = cuda_status(cudaStreamCreateWithFlags(&s->h2d, cudaStreamNonBlocking), "stepper h2d stream");
   if (st == DMS_OK)
@@ -146,6 +175,9 @@ extern "C" dms_status dms_stepper_create(dms_pool* pool, int layer0, int n_layer
     if (st == DMS_OK)
       st = cuda_status(cudaEventCreateWithFlags(&s->drained[j], cudaEventDisableTiming), "stepper event");
   }
+  if (st == DMS_OK)
+    st = cuda_status(cudaMemsetAsync(s->counters, 0, 256, stream), "stepper counters");
+  if (st == DMS_OK) st = cuda_status(cudaStreamSynchronize(stream), "stepper counters");
   if (st != DMS_OK) {
     stepper_release(s);
     return st;
@@ -165,6 +197,56 @@ extern "C" dms_status dms_stepper_step(dms_stepper* s, int64_t pos, const void* 
   const dms_stepper_layout_t& L = s->lay;
   uint8_t* stg = s->stage[j];
   dms_status st = DMS_OK;
+  if (s->wait_value) {
+    // Counter protocol: the compute stream holds only the two kernels, so
+    // the append of step n+1 and the attention of step n stay chained by
+    // programmatic launch; the copy streams wait on and set device counters.
+    const int32_t n = int32_t(s->steps);
+    auto dptr = [&](int i) { return CUdeviceptr(reinterpret_cast<uintptr_t>(s->counters + i)); };
+    auto drv = [&](CUresult r, const char* what) {
+      if (r == CUDA_SUCCESS) return DMS_OK;
+      set_last_error("%s failed (%d)", what, int(r));
+      return DMS_ERR_CUDA;
+    };
+    // host -> device once the kernels of step n-D are done with the buffer
+    if (reuse)
+      st = drv(s->wait_value(s->h2d, dptr(1), cuuint32_t(n - kStepperDepth + 1), CU_STREAM_WAIT_VALUE_GEQ),
+               "stepper wait (computed)");
+    if (st == DMS_OK)
+      st = cuda_status(cudaMemcpyAsync(stg, host_in, L.in_bytes, cudaMemcpyHostToDevice, s->h2d),
+                       "stepper input copy");
+    if (st == DMS_OK)
+      st = drv(s->write_value(s->h2d, dptr(0), cuuint32_t(n + 1), CU_STREAM_WRITE_VALUE_DEFAULT),
+               "stepper write (staged)");
+    StepSync in{};
+    in.ready = s->counters + 0;
+    in.ready_value = n + 1;
+    StepSync att{};
+    att.drained = reuse ? s->counters + 2 : nullptr;
+    att.drained_value = n - kStepperDepth + 1;
+    att.done = s->counters + 1;
+    att.done_value = n + 1;
+    att.exit_count = s->counters + 3;
+    if (st == DMS_OK)
+      st = append_layers_synced(s->pool, s->layer0, s->n_layers, s->batch, pos, stg + L.k, stg + L.v,
+                                s->dtype, stg + L.evict, s->compute, in);
+    if (st == DMS_OK)
+      st = decode_attn_layers_synced(s->pool, s->layer0, s->n_layers, s->batch, stg + L.q, s->out[j],
+                                     s->sm_scale, s->ws, s->compute, att);
+    // device -> host once the step is computed
+    if (st == DMS_OK)
+      st = drv(s->wait_value(s->d2h, dptr(1), cuuint32_t(n + 1), CU_STREAM_WAIT_VALUE_GEQ),
+               "stepper wait (computed)");
+    if (st == DMS_OK)
+      st = cuda_status(cudaMemcpyAsync(host_out, s->out[j], L.out_bytes, cudaMemcpyDeviceToHost, s->d2h),
+                       "stepper output copy");
+    if (st == DMS_OK)
+      st = drv(s->write_value(s->d2h, dptr(2), cuuint32_t(n + 1), CU_STREAM_WRITE_VALUE_DEFAULT),
+               "stepper write (drained)");
+    if (st == DMS_OK) st = cuda_status(cudaEventRecord(s->drained[j], s->d2h), "stepper record");
+    if (st == DMS_OK) ++s->steps;
+    return st;
+  }
   // host -> device: the staging buffer is free once the kernels of step n-D ran
   if (reuse) st = cuda_status(cudaStreamWaitEvent(s->h2d, s->computed[j], 0), "stepper wait");
   if (st == DMS_OK)
