@@ -468,8 +468,9 @@ def main():
         return 0
     W, K, E = args.warmup, args.steps, args.e2e_steps
     R = min(K, 64)                 # instrumented steps for the attention-kernel timing
+    RL = min(K, 16)                # steps issued as per-layer calls
     assert W >= 3 and K >= 1
-    dw = DeviceWorkload(wl, W + K + R + E, device=f"cuda:{local}")
+    dw = DeviceWorkload(wl, W + K + R + RL + E, device=f"cuda:{local}")
     compact_ms_layers = dw.prefill(timed=True)
     # median layer: the first call of each kernel also pays its module load
     compact_ms = float(np.median(compact_ms_layers)) * len(compact_ms_layers)
@@ -481,7 +482,7 @@ def main():
 
     # exact held tokens after each step: +1 per head, -1 per head whose token
     # t - w carried a flag (flags drawn by the same device generator)
-    NT = W + K + R + E
+    NT = W + K + R + RL + E
     fl = dw.flags(0, L, P - w, NT) if P - w >= 0 else None
     retired = fl.sum(dim=(0, 1, 3)).cpu().numpy().astype(np.int64) if fl is not None else \
         np.zeros(NT, np.int64)
@@ -568,6 +569,31 @@ def main():
     torch.cuda.synchronize()
     attn_ms = np.array([a.elapsed_time(b) for a, b in ev])
     del graph
+
+    # ---- the same decode step as 2 L launches (append, then attention, one
+    # layer per call), captured and replayed like the headline steps ----
+    dw.pool.workspace(1, B, dw.out.device)   # allocated before the capture
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for j in range(RL):
+            s = W + K + R + j
+            for layer in range(L):
+                dw.pool.append_evict_layers(layer, P + s, si["k"][s][layer:layer + 1],
+                                            si["v"][s][layer:layer + 1], si["evict"][s][layer:layer + 1])
+                dw.pool.decode_attn_layers(layer, si["q"][s][layer:layer + 1], dw.out[layer:layer + 1])
+    torch.cuda.synchronize()
+    pl0, pl1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pl0.record(stream)
+    graph.replay()
+    pl1.record(stream)
+    torch.cuda.synchronize()
+    pl_ms = pl0.elapsed_time(pl1) / RL
+    del graph
+    per_layer_calls = {"ms_per_step": pl_ms, "decode_steps_per_s": 1e3 / pl_ms,
+                       "value": float(bytes_step[W + K + R:W + K + R + RL].mean()) / (pl_ms * 1e-3) / 1e9,
+                       "unit": "GB/s", "launches_per_step": 2 * L, "steps": RL,
+                       "timing": "CUDA events around one replay of a captured graph of the steps, "
+                                 "each step one append and one attention call per layer"}
     st = dw.pool.stats()
     if st.error_flags:
         raise SystemExit(f"device error word 0x{st.error_flags:x}")
@@ -596,7 +622,7 @@ def main():
     # pinned host), copies inside the timed region ----
     e2e = None
     if E > 0:
-        e0s = W + K + R
+        e0s = W + K + R + RL
         stp = dms.Stepper(dw.pool, 0, L, B, stream=stream)
         hin = stp.host_inputs(E)
         hout = torch.empty(E, stp.layout.out_bytes, dtype=torch.uint8).pin_memory()
@@ -666,6 +692,7 @@ def main():
                               f"no flush: {bytes_step[W] / 1e6:.0f} MB of held K/V read per step "
                               f"> 126 MB L2")},
             "decode_steps_per_s": world * K / (ms_max * 1e-3),
+            "per_layer_calls": per_layer_calls,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "compaction": compaction,
             "prefill_attention": prefill, "kv_projection_append": projection,
             "gpu_launches": 2 * K, "clocks": clk.summary(),
