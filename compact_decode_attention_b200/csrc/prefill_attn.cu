@@ -424,8 +424,8 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
     return DMS_ERR_INVALID_ARG;
   }
   const PoolView& pv = pool->view;
-  if (pv.kv_dtype != DMS_BF16 || in_dtype != DMS_BF16 || (pv.D != 64 && pv.D != 128)) {
-    set_last_error("dms_prefill_attn needs a bf16 pool, bf16 inputs and head_dim 64 or 128");
+  if (pv.kv_dtype == DMS_F32 || in_dtype != DMS_BF16 || (pv.D != 64 && pv.D != 128)) {
+    set_last_error("dms_prefill_attn needs a bf16, FP8 or 4-bit pool, bf16 inputs and head_dim 64 or 128");
     return DMS_ERR_UNSUPPORTED;
   }
   if (layer < 0 || layer >= pv.L || seq0 < 0 || batch < 1 || seq0 + batch > pv.Bmax ||
@@ -442,9 +442,15 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
     set_last_error("q, k, v and out must be 16-byte aligned");
     return DMS_ERR_INVALID_ARG;
   }
-  // prefix counts and block tables of the layer's sequences (the same count
-  // and plan kernels as dms_compact_prefill_seqs)
-  dms_status st = prefill_plan_launch(pool, layer, seq0, batch, prompt_len, evict, stream);
+  // A bf16 store takes the kept rows from the attention kernel's tiles, after
+  // the prefix counts and block tables of the count and plan kernels.  FP8
+  // and 4-bit stores quantise them: the layer is compacted first, as by
+  // dms_compact_prefill_seqs (scales, plan, scatter), and the attention
+  // kernel stores nothing.
+  const int fused = pv.kv_dtype == DMS_BF16 ? 1 : 0;
+  dms_status st = fused ? prefill_plan_launch(pool, layer, seq0, batch, prompt_len, evict, stream)
+                        : dms_compact_prefill_seqs(pool, layer, seq0, batch, prompt_len, k, v, in_dtype,
+                                                   evict, stream);
   if (st != DMS_OK) return st;
   const int n_qtiles = (prompt_len + kPaTile - 1) / kPaTile;
   const dim3 grid(n_qtiles, pv.Hq, batch);
@@ -469,7 +475,7 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
       attr = true;
     }
     prefill_attn_kernel<128><<<grid, PaSplit<128>::THREADS, PaSmem<128>::BYTES, stream>>>(
-        pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, 1);
+        pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, fused);
   } else {
     static bool attr = false;
     if (!attr) {
@@ -483,7 +489,7 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
       attr = true;
     }
     prefill_attn_kernel<64><<<grid, PaSplit<64>::THREADS, PaSmem<64>::BYTES, stream>>>(
-        pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, 1);
+        pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, fused);
   }
   return cuda_status(cudaGetLastError(), "prefill_attn_kernel");
 }

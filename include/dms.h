@@ -252,7 +252,10 @@ dms_status dms_decode_attn_seqs(dms_pool* pool, int layer0, int n_layers, int n_
  * stores the tile's kept rows).
  *   q, out  [batch, P, Hq, D]  bf16      k, v  [batch, P, Hkv, D]  bf16
  *   evict   [batch, P, Hkv]    uint8     sm_scale <= 0 selects 1/sqrt(D)
- * Needs a bf16 pool with head_dim 64 or 128 (else DMS_ERR_UNSUPPORTED).
+ * Needs a bf16, FP8 or 4-bit pool with head_dim 64 or 128 (else
+ * DMS_ERR_UNSUPPORTED).  A bf16 pool is filled by the attention kernel
+ * itself; an FP8 or 4-bit pool is compacted first, as by
+ * dms_compact_prefill_seqs, and the attention reads the bf16 inputs.
  * The sequences must be empty in that layer (else DMS_DEVERR_LAYER_NOT_EMPTY
  * and nothing is stored; the outputs are still computed).  Runs on the
  * tensor cores (tcgen05, accumulators in tensor memory).

@@ -2,7 +2,8 @@
 tensor cores, fused with compaction (through the C ABI).  Outputs are
 compared with the fp64 oracle (every query on small prompts, sampled queries
 on a long one, max-abs 2e-2 as for every bf16 path); the pool the fused
-kernel fills must hold exactly what the oracle's compaction keeps."""
+kernel fills must hold exactly what the oracle's compaction keeps (FP8 and
+4-bit pools: compacted first, codes and scales bit-exact)."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +12,10 @@ import synth
 from oracle import attention as oatt
 from compact_decode_attention_b200 import dms
 
-from gpu_util import check_block_invariants, check_head_store, head_id, oracle_store, read_state
+from oracle import fp8 as ofp8
+from oracle import int4 as oint4
+
+from gpu_util import check_block_invariants, check_head_store, head_id, int4_rows, oracle_store, read_state
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2
@@ -71,8 +75,43 @@ def test_long_prompt_sampled_queries_and_sequence_offset():
     _check_store(pool, 2, K, V, F, P, w)
 
 
+@pytest.mark.parametrize("kind", ["fp8", "int4"])
+def test_quantised_pools_compact_first_then_attend(kind):
+    """FP8 and 4-bit stores: the layer is compacted as by
+    dms_compact_prefill_seqs (codes and scales bit-exact against the
+    oracle), and every query's output matches the oracle on the bf16 inputs."""
+    B, P, Hq, Hkv, D, w = 2, 333, 8, 2, 128, 64
+    Q, K, V, F = _inputs(41, B, P, Hq, Hkv, D, 0.3)
+    code = dms.DMS_FP8_E4M3 if kind == "fp8" else dms.DMS_INT4
+    pool = dms.Pool(1, B, Hq, Hkv, D, w, code, B * Hkv * (P // 64 + 2), P + 1)
+    got = _run(pool, 0, Q, K, V, F)
+    for b in range(B):
+        exp = oatt.prefill_attention(Q[b].astype(np.float64), K[b], V[b], F[b], w)
+        assert np.abs(got[b] - exp).max() < TOL, b
+    state = read_state(pool)
+    assert state["error"] == 0
+    for b in range(B):
+        for h in range(Hkv):
+            store = oracle_store(F[b, :, h], np.zeros(0, np.uint8), w, P)
+            hd = head_id(pool.cfg, 0, b, h)
+            assert state["n_slots"][hd] == store.n_slots
+            pos = np.array([store.pos_of_slot[x] for x in range(store.n_slots)])
+            if kind == "fp8":
+                scales = (ofp8.fp8_scale(np.abs(K[:, :, h]).max()), ofp8.fp8_scale(np.abs(V[:, :, h]).max()))
+                assert state["scales"][0, h, 0] == scales[0] and state["scales"][0, h, 1] == scales[1]
+                check_head_store(pool, state, hd, store, {j: K[b, j, h] for j in range(P)},
+                                 {j: V[b, j, h] for j in range(P)}, "fp8", scales)
+            else:
+                ck, sk, cv, sv = int4_rows(pool, state, hd, store.n_slots)
+                qk, ek = oint4.quantize(K[b, pos, h])
+                qv, ev = oint4.quantize(V[b, pos, h])
+                assert np.array_equal(ck, qk) and np.array_equal(sk, ek)
+                assert np.array_equal(cv, qv) and np.array_equal(sv, ev)
+    check_block_invariants(pool, state)
+
+
 def test_unsupported_pools_are_refused():
-    pool = dms.Pool(1, 1, 8, 2, 128, 16, dms.DMS_FP8_E4M3, 16, 256)
+    pool = dms.Pool(1, 1, 8, 2, 128, 16, dms.DMS_F32, 16, 256)
     x = torch.zeros(1, 64, 8, 128, dtype=torch.bfloat16, device="cuda")
     kv = torch.zeros(1, 64, 2, 128, dtype=torch.bfloat16, device="cuda")
     f = torch.zeros(1, 64, 2, dtype=torch.uint8, device="cuda")
