@@ -71,14 +71,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
   return idesc_bf16_f32(M, N) | (1u << 16);
 }
 
-// ---- 16-byte asynchronous global -> shared copy (zero-filled when !valid) ----
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
 // ---- tensor-map (TMA) tile load, 3-D, completion counted on an mbarrier ----
 // (x, y, z) is the box origin in elements; x * 2 bytes must be a multiple of
 // 16.  Elements outside the tensor arrive as zeros.  No multicast.
@@ -89,10 +81,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, in
       "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ---- tensor memory ----
