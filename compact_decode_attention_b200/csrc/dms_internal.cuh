@@ -55,7 +55,10 @@ struct PoolView {
   int32_t* tickets;         // [n_heads] split-K merge tickets (self-resetting)
   DevHeader* hdr;
   int32_t* chunk_counts;    // prefill scratch [Bmax][Hkv][n_chunks_max]
-  uint32_t* amax;           // prefill scratch [2][Hkv] (float bits, non-negative)
+  uint32_t* amax;           // prefill scratch [2][Hkv] (float bits, non-negative; left zeroed)
+  int32_t* prefill_tickets; // prefill scratch [Bmax + 1] arrival counters (self-resetting)
+  int32_t* pair_n;          // prefill scratch [Bmax][Hkv] kept tokens of each (sequence, head)
+  int32_t* pair_base;       // prefill scratch [Bmax * Hkv + 1] first allocation index of each pair
   void* stats;              // staging for dms_pool_stats
 
   __host__ __device__ __forceinline__ int head(int l, int b, int h) const {

@@ -114,6 +114,9 @@ static dms_status plan_layout(const dms_pool_config* c, dms_pool_layout_t* lay) 
   lay->scratch = off;
   off = align256(off + uint64_t(c->max_batch) * c->n_kv_heads * n_chunks * 4);  // chunk counts
   off = align256(off + uint64_t(2) * c->n_kv_heads * 4);                        // amax
+  off = align256(off + uint64_t(c->max_batch + 1) * 4);                         // prefill tickets
+  off = align256(off + uint64_t(c->max_batch) * c->n_kv_heads * 4);             // pair counts
+  off = align256(off + (uint64_t(c->max_batch) * c->n_kv_heads + 1) * 4);       // pair bases
   off = align256(off + sizeof(dms_pool_stats_t));                                // stats
   lay->blocks = off;
   lay->block_bytes = 2 * kBlockTokens * row_bytes;
@@ -165,6 +168,12 @@ static PoolView make_view(const dms_pool_config& c, const dms_pool_layout_t& lay
   s = align256(s + uint64_t(c.max_batch) * c.n_kv_heads * v.n_chunks_max * 4);
   v.amax = reinterpret_cast<uint32_t*>(b + s);
   s = align256(s + uint64_t(2) * c.n_kv_heads * 4);
+  v.prefill_tickets = reinterpret_cast<int32_t*>(b + s);
+  s = align256(s + uint64_t(c.max_batch + 1) * 4);
+  v.pair_n = reinterpret_cast<int32_t*>(b + s);
+  s = align256(s + uint64_t(c.max_batch) * c.n_kv_heads * 4);
+  v.pair_base = reinterpret_cast<int32_t*>(b + s);
+  s = align256(s + (uint64_t(c.max_batch) * c.n_kv_heads + 1) * 4);
   v.stats = b + s;
   return v;
 }

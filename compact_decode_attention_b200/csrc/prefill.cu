@@ -12,14 +12,21 @@
 // eviction and the kept rows are quantised (FastDMS page, FP8 paragraph:
 // eviction is decided before FP8 quantisation).
 //
-// Kernels, in stream order:
-//   amax     (FP8 only) per-(kv-head) |x| maximum over every prompt row
-//   count    per (sequence, 256-token chunk, head): warp ballot + popcount
-//   plan     one CTA: per-head chunk prefix sums, block allocation in
-//            (sequence, head) order, block tables, counters, FP8 scales
-//   scatter  per (sequence, kv-head, chunk): ranks by ballot/popcount +
-//            the chunk base give each kept row its slot; copy (or quantise)
-//            the row into its block, fill the window ring.
+// Two kernels, in stream order:
+//   plan     one CTA per (256-token chunk, sequence): per-head kept counts by
+//            warp ballot + popcount (and, for an FP8 store, the per-head |x|
+//            maximum of every prompt row).  The last CTA of a sequence to
+//            finish turns its heads' chunk counts into exclusive prefix sums;
+//            the last of those plans the layer: block allocation in
+//            (sequence, head) order, block tables, counters, FP8 scales.
+//            Arrival is counted with tickets, so no CTA ever waits.
+//   scatter  one CTA per (64- or 256-token piece, kv-head, sequence),
+//            launched as a programmatic dependent: it ranks its kept tokens
+//            from the flags while the planner runs, then waits for the plan
+//            and copies (or quantises) each kept row into its slot and fills
+//            the window ring.  For FP8 and 4-bit stores the CTA holding the
+//            last prompt token also clears the V rows past the head's last
+//            slot in its last block (the attention reads whole V tiles).
 #include "append_core.cuh"
 
 namespace dms {
@@ -33,241 +40,302 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
 
+// Two adjacent input elements (p 4- or 8-byte aligned) as floats.
+__device__ __forceinline__ void load_pair(const __nv_bfloat16* p, float& a, float& b) {
+  const __nv_bfloat162 x = __ldg(reinterpret_cast<const __nv_bfloat162*>(p));
+  a = __low2float(x);
+  b = __high2float(x);
+}
+__device__ __forceinline__ void load_pair(const float* p, float& a, float& b) {
+  const float2 x = __ldg(reinterpret_cast<const float2*>(p));
+  a = x.x;
+  b = x.y;
+}
+
 __device__ __forceinline__ bool keep_token(int j, int P, int w, uint8_t flag) {
   // visible to the last prompt query t = P - 1
   return j < P && (flag == 0 || (P - 1 - j) < w);
 }
 
 // ---------------------------------------------------------------------------
-template <typename InT>
-__global__ void __launch_bounds__(256) prefill_amax_kernel(PoolView v, int P, const InT* k,
-                                                           const InT* vv) {
-  extern __shared__ uint32_t s_amax[];  // [2][Hkv]
-  const int b = blockIdx.y;
-  const int j0 = blockIdx.x * kPrefillChunk;
-  const int nj = min(kPrefillChunk, P - j0);
-  for (int i = threadIdx.x; i < 2 * v.Hkv; i += blockDim.x) s_amax[i] = 0;
-  __syncthreads();
-  constexpr int VEC = 16 / sizeof(InT);
-  const int64_t row0 = (int64_t(b) * P + j0) * v.Hkv;  // first row of the chunk
-  const int64_t nvec = int64_t(nj) * v.Hkv * v.D / VEC;
-  for (int which = 0; which < 2; ++which) {
-    const uint4* src = reinterpret_cast<const uint4*>((which ? vv : k) + row0 * v.D);
-    for (int64_t i = threadIdx.x; i < nvec; i += blockDim.x) {
-      uint4 raw = src[i];
-      const InT* x = reinterpret_cast<const InT*>(&raw);
-      float m = 0.f;
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) m = fmaxf(m, fabsf(to_f32(x[e])));
-      const int h = int((i * VEC / v.D) % v.Hkv);
-      atomicMax(&s_amax[which * v.Hkv + h], __float_as_uint(m));
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 2 * v.Hkv; i += blockDim.x) atomicMax(&v.amax[i], s_amax[i]);
-}
-
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) prefill_count_kernel(PoolView v, int P, const uint8_t* evict) {
-  __shared__ int s_cnt[8];
-  const int b = blockIdx.y, chunk = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = chunk * kPrefillChunk + threadIdx.x;
-  for (int h = 0; h < v.Hkv; ++h) {
-    const uint8_t f = j < P ? evict[(int64_t(b) * P + j) * v.Hkv + h] : 0;
-    const unsigned m = __ballot_sync(0xffffffffu, keep_token(j, P, v.w, f));
-    if (lane == 0) s_cnt[warp] = __popc(m);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int c = 0;
-      for (int k = 0; k < 8; ++k) c += s_cnt[k];
-      v.chunk_counts[(int64_t(b) * v.Hkv + h) * v.n_chunks_max + chunk] = c;
-    }
-    __syncthreads();
-  }
-}
-
-// ---------------------------------------------------------------------------
-// One CTA of 1024 threads.  s_n holds the kept count of each (b, h) pair.
-__global__ void __launch_bounds__(1024) prefill_plan_kernel(PoolView v, int layer, int seq0, int batch,
-                                                            int P) {
-  extern __shared__ int s_n[];   // [batch * Hkv] kept counts, then block prefix
+// Layer plan, run by the last CTA of the plan kernel (256 threads) once every
+// sequence's chunk counts are scanned and pair_n holds each pair's kept count.
+__device__ void plan_layer(const PoolView& v, int layer, int seq0, int batch) {
   __shared__ int s_fail;
-  __shared__ int s_warp[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  __shared__ int s_warp[8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int pairs = batch * v.Hkv;
-  const int n_chunks = (P + kPrefillChunk - 1) / kPrefillChunk;
-  if (tid == 0) {
-    s_fail = 0;
-    v.hdr->prefill_go = 0;
-  }
+  const int stack = v.hdr->block_stack_top;
+  const int next = v.hdr->next_block;
+  if (tid == 0) s_fail = 0;
   __syncthreads();
-  // the target sequences of the layer must be empty
-  for (int p = tid; p < pairs; p += blockDim.x) {
-    const int hd = v.head(layer, seq0 + p / v.Hkv, p % v.Hkv);
-    if (v.n_slots[hd] != 0 || v.n_retained[hd] != 0) {
-      atomicExch(&s_fail, 1);
-      report_error(v.hdr, DMS_DEVERR_LAYER_NOT_EMPTY, layer, seq0 + p / v.Hkv, p % v.Hkv);
-    }
-  }
-  __syncthreads();
-  if (s_fail) return;
-  // per pair: exclusive scan of chunk counts (in place) and total
-  for (int p = warp; p < pairs; p += nwarps) {
-    int32_t* cc = v.chunk_counts + int64_t(p) * v.n_chunks_max;
-    int carry = 0;
-    for (int c0 = 0; c0 < n_chunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int x = c < n_chunks ? cc[c] : 0;
-      int incl = x;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+  // the target heads must be empty and each head's blocks must fit its
+  // table; blocks per pair -> exclusive prefix over pairs in (sequence, head)
+  // order
+  int running = 0;
+  for (int p0 = 0; p0 < pairs; p0 += blockDim.x) {
+    const int p = p0 + tid;
+    int nb = 0;
+    if (p < pairs) {
+      const int hd = v.head(layer, seq0 + p / v.Hkv, p % v.Hkv);
+      const int ns = v.n_slots[hd], nr = v.n_retained[hd], n = __ldcg(v.pair_n + p);
+      nb = (n + v.BT - 1) / v.BT;
+      if (ns != 0 || nr != 0) {
+        atomicExch(&s_fail, 1);
+        report_error(v.hdr, DMS_DEVERR_LAYER_NOT_EMPTY, layer, seq0 + p / v.Hkv, p % v.Hkv);
       }
-      if (c < n_chunks) cc[c] = carry + incl - x;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) s_n[p] = carry;
-  }
-  __syncthreads();
-  // blocks per pair, exclusive prefix over pairs in (b, h) order
-  int* s_base = s_n + pairs;
-  {
-    int running = 0;
-    for (int p0 = 0; p0 < pairs; p0 += blockDim.x) {
-      const int p = p0 + tid;
-      const int nb = p < pairs ? (s_n[p] + v.BT - 1) / v.BT : 0;
-      if (p < pairs && nb > v.mbh) {
+      if (nb > v.mbh) {
         atomicExch(&s_fail, 1);
         report_error(v.hdr, DMS_DEVERR_HEAD_TABLE_FULL, layer, seq0 + p / v.Hkv, p % v.Hkv);
       }
-      int incl = nb;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (lane == 31) s_warp[warp] = incl;
-      __syncthreads();
-      if (warp == 0) {
-        int t = lane < nwarps ? s_warp[lane] : 0;
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, t, o);
-          if (lane >= o) t += y;
-        }
-        s_warp[lane] = t;  // inclusive warp totals
-      }
-      __syncthreads();
-      const int before = (warp ? s_warp[warp - 1] : 0);
-      if (p < pairs) s_base[p] = running + before + incl - nb;
-      running += s_warp[nwarps - 1];
-      __syncthreads();
     }
-    if (tid == 0) s_base[pairs] = running;
+    int incl = nb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int before = 0, all = 0;
+    for (int q = 0; q < int(blockDim.x >> 5); ++q) {
+      before += q < warp ? s_warp[q] : 0;
+      all += s_warp[q];
+    }
+    if (p < pairs) v.pair_base[p] = running + before + incl - nb;
+    running += all;
+    __syncthreads();
   }
-  __syncthreads();
-  const int total = s_base[pairs];
-  const int stack = v.hdr->block_stack_top;
-  const int64_t avail = int64_t(stack) + (v.max_blocks - v.hdr->next_block);
-  if (tid == 0 && total > avail) {
+  const int total = running;
+  if (tid == 0 && int64_t(total) > int64_t(stack) + (v.max_blocks - next)) {
     s_fail = 1;
     report_error(v.hdr, DMS_DEVERR_BLOCKS_EXHAUSTED, layer, -1, -1);
   }
-  __syncthreads();
-  if (s_fail) return;
-  const int next = v.hdr->next_block;
-  // block tables: allocation index a -> free stack top first, then bump
-  for (int p = warp; p < pairs; p += nwarps) {
-    const int hd = v.head(layer, seq0 + p / v.Hkv, p % v.Hkv);
-    const int nb = (s_n[p] + v.BT - 1) / v.BT;
-    for (int k = lane; k < nb; k += 32) {
-      const int a = s_base[p] + k;
-      const int id = a < stack ? v.block_stack[stack - 1 - a] : next + (a - stack);
-      v.bt[int64_t(hd) * v.mbh + k] = id;
-    }
-    if (lane == 0) {
-      v.n_slots[hd] = s_n[p];
-      v.n_retained[hd] = s_n[p];
-      v.free_top[hd] = 0;
-      if (nb > 0) {
-        const int a = s_base[p] + nb - 1;
-        v.last_block[hd] = a < stack ? v.block_stack[stack - 1 - a] : next + (a - stack);
-      } else {
-        v.last_block[hd] = -1;
+  __syncthreads();   // pair_base visible to the whole CTA, s_fail final
+  const bool ok = s_fail == 0;
+  if (ok) {
+    // block tables: allocation index a -> free stack top first, then bump
+    for (int p = warp; p < pairs; p += blockDim.x >> 5) {
+      const int hd = v.head(layer, seq0 + p / v.Hkv, p % v.Hkv);
+      const int n = __ldcg(v.pair_n + p), base = __ldcg(v.pair_base + p);
+      const int nb = (n + v.BT - 1) / v.BT;
+      for (int k = lane; k < nb; k += 32) {
+        const int a = base + k;
+        v.bt[int64_t(hd) * v.mbh + k] = a < stack ? v.block_stack[stack - 1 - a] : next + (a - stack);
+      }
+      if (lane == 0) {
+        v.n_slots[hd] = n;
+        v.n_retained[hd] = n;
+        v.free_top[hd] = 0;
+        const int a = base + nb - 1;
+        v.last_block[hd] = nb == 0 ? -1 : a < stack ? v.block_stack[stack - 1 - a] : next + (a - stack);
       }
     }
   }
   if (v.kv_dtype == DMS_FP8_E4M3) {
     // the first prefill into a layer sets its scales (0 = not set yet); later
-    // prefills of other sequences reuse them, saturating like decode tokens
+    // prefills of other sequences reuse them, saturating like decode tokens.
+    // The maxima are cleared for the next call either way.
     for (int i = tid; i < 2 * v.Hkv; i += blockDim.x) {
-      const float a = __uint_as_float(v.amax[i]);
+      const float a = __uint_as_float(__ldcg(v.amax + i));
+      v.amax[i] = 0;
+      if (!ok) continue;
       const float s = a > 0.f ? __fdiv_rn(a, 448.0f) : 1.0f;
       const int which = i / v.Hkv, h = i % v.Hkv;
       float* dst = v.scales + (int64_t(layer) * v.Hkv + h) * 2 + which;
       if (*dst == 0.f) *dst = s;
     }
   }
-  __syncthreads();
   if (tid == 0) {
-    v.hdr->block_stack_top = stack > total ? stack - total : 0;
-    v.hdr->next_block = next + (total > stack ? total - stack : 0);
-    v.hdr->prefill_go = 1;
+    if (ok) {
+      v.hdr->block_stack_top = stack > total ? stack - total : 0;
+      v.hdr->next_block = next + (total > stack ? total - stack : 0);
+    }
+    v.hdr->prefill_go = ok ? 1 : 0;
   }
 }
 
 // ---------------------------------------------------------------------------
-// FP8 only: clear the transposed V tile of each head's last, partly filled
-// block, so that token columns past n_slots decode to 0 (the attention kernel
-// reads whole V tiles).  One CTA per (sequence, kv-head).
-__global__ void __launch_bounds__(256) prefill_fp8_clear_tail_kernel(PoolView v, int layer, int seq0) {
-  if (!v.hdr->prefill_go) return;
-  const int b = blockIdx.x / v.Hkv, h = blockIdx.x % v.Hkv;
-  const int hd = v.head(layer, seq0 + b, h);
-  const int n = v.n_slots[hd];
-  if (n % v.BT == 0) return;
-  uint8_t* blk = v.blocks + int64_t(v.bt[int64_t(hd) * v.mbh + n / v.BT]) * v.block_bytes;
-  uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);
-  for (int i = threadIdx.x; i < int(v.tile_bytes / 16); i += blockDim.x) tile[i] = make_uint4(0, 0, 0, 0);
+// One CTA of 256 threads per (256-token chunk, sequence).  AMAX: also fold
+// every prompt row of the chunk into the per-head |x| maxima (FP8 store).
+template <typename InT, bool AMAX>
+__global__ void __launch_bounds__(256) prefill_plan_kernel(PoolView v, int layer, int seq0, int batch,
+                                                           int P, const uint8_t* __restrict__ evict,
+                                                           const InT* __restrict__ k,
+                                                           const InT* __restrict__ vv) {
+  extern __shared__ uint32_t s_amax[];   // [2][Hkv], AMAX only
+  __shared__ int s_cnt[32][8];           // [head of a group of 32][warp]
+  __shared__ int s_last;
+  const int b = blockIdx.y, chunk = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = chunk * kPrefillChunk + tid;
+  const int n_chunks = gridDim.x;
+  for (int h0 = 0; h0 < v.Hkv; h0 += 32) {
+    const int nh = min(32, v.Hkv - h0);
+    const uint8_t* fl = evict + (int64_t(b) * P + j) * v.Hkv + h0;
+    uint8_t f[32];   // every flag load of the group in flight before the first ballot
+#pragma unroll
+    for (int hh = 0; hh < 32; ++hh) f[hh] = hh < nh && j < P ? __ldg(fl + hh) : 0;
+#pragma unroll
+    for (int hh = 0; hh < 32; ++hh) {
+      if (hh < nh) {
+        const unsigned m = __ballot_sync(0xffffffffu, keep_token(j, P, v.w, f[hh]));
+        if (lane == 0) s_cnt[hh][warp] = __popc(m);
+      }
+    }
+    __syncthreads();
+    if (tid < nh) {
+      int c = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) c += s_cnt[tid][q];
+      v.chunk_counts[(int64_t(b) * v.Hkv + h0 + tid) * v.n_chunks_max + chunk] = c;
+    }
+    __syncthreads();
+  }
+  if constexpr (AMAX) {
+    for (int i = tid; i < 2 * v.Hkv; i += blockDim.x) s_amax[i] = 0;
+    __syncthreads();
+    constexpr int VEC = 16 / sizeof(InT);
+    const int j0 = chunk * kPrefillChunk;
+    const int nj = min(kPrefillChunk, P - j0);
+    const int64_t row0 = (int64_t(b) * P + j0) * v.Hkv;  // first row of the chunk
+    const int64_t nvec = int64_t(nj) * v.Hkv * v.D / VEC;
+    const int vec_per_row = v.D / VEC;
+    for (int which = 0; which < 2; ++which) {
+      const uint4* src = reinterpret_cast<const uint4*>((which ? vv : k) + row0 * v.D);
+      // a thread's vectors mostly belong to one head (always when 256 vectors
+      // span a multiple of Hkv rows): keep its maximum in a register and fold
+      // it into shared memory when the head changes
+      float acc = 0.f;
+      int cur = -1;
+      for (int64_t i0 = tid; i0 < nvec; i0 += 4 * blockDim.x) {
+        uint4 raw[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t i = i0 + u * blockDim.x;
+          raw[u] = i < nvec ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t i = i0 + u * blockDim.x;
+          if (i >= nvec) break;
+          const InT* x = reinterpret_cast<const InT*>(&raw[u]);
+          float mx = 0.f;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) mx = fmaxf(mx, fabsf(to_f32(x[e])));
+          const int h = int((i / vec_per_row) % v.Hkv);
+          if (h != cur) {
+            if (cur >= 0) atomicMax(&s_amax[which * v.Hkv + cur], __float_as_uint(acc));
+            cur = h;
+            acc = 0.f;
+          }
+          acc = fmaxf(acc, mx);
+        }
+      }
+      if (cur >= 0) atomicMax(&s_amax[which * v.Hkv + cur], __float_as_uint(acc));
+    }
+    __syncthreads();
+    for (int i = tid; i < 2 * v.Hkv; i += blockDim.x) atomicMax(&v.amax[i], s_amax[i]);
+  }
+  // arrival: the last CTA of this sequence scans its heads' chunk counts
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&v.prefill_tickets[b], 1) == n_chunks - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int h = warp; h < v.Hkv; h += blockDim.x >> 5) {
+    int32_t* cc = v.chunk_counts + (int64_t(b) * v.Hkv + h) * v.n_chunks_max;
+    int carry = 0;
+    for (int c0 = 0; c0 < n_chunks; c0 += 32 * 8) {
+      int x[8], own = 0;   // lane owns chunks c0 + 8 * lane .. + 7
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + 8 * lane + u;
+        x[u] = c < n_chunks ? __ldcg(cc + c) : 0;
+        own += x[u];
+      }
+      int incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int run = carry + incl - own;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + 8 * lane + u;
+        if (c < n_chunks) cc[c] = run;
+        run += x[u];
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) v.pair_n[b * v.Hkv + h] = carry;
+  }
+  if (tid == 0) v.prefill_tickets[b] = 0;
+  // arrival: the last sequence to finish plans the layer
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&v.prefill_tickets[v.Bmax], 1) == batch - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  pdl_launch_dependents();   // the scatter grid may be scheduled while the plan is made
+  if (tid == 0) v.prefill_tickets[v.Bmax] = 0;
+  plan_layer(v, layer, seq0, batch);
 }
 
 // ---------------------------------------------------------------------------
-// One CTA per (256-token chunk, kv-head, sequence).  STORE: 0 = copy
-// (bf16 / fp32 store), 1 = FP8, 2 = 4-bit.
-template <typename InT, int STORE>
+// One CTA of 256 threads per (SUB-token piece, kv-head, sequence); the pieces
+// of one 256-token chunk share its planned base.  STORE: 0 = copy (bf16 /
+// fp32 store), 1 = FP8, 2 = 4-bit.
+template <typename InT, int STORE, int SUB>
 __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int layer, int seq0, int P,
                                                               const InT* __restrict__ k,
                                                               const InT* __restrict__ vv,
                                                               const uint8_t* __restrict__ evict) {
+  static_assert(kPrefillChunk % SUB == 0 && SUB % 32 == 0, "a piece is whole warps of a chunk");
+  constexpr int kPieces = kPrefillChunk / SUB, kPieceWarps = SUB / 32;
   constexpr int kBatchItems = 4;          // 16-byte copies in flight per thread
-  __shared__ int s_kept[kPrefillChunk];   // chunk-local token index of each kept rank
+  __shared__ int s_kept[SUB];             // chunk-local token index of each kept rank
   __shared__ int s_wcnt[8];
-  if (!v.hdr->prefill_go) return;
-  const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int chunk = blockIdx.x / kPieces, piece = blockIdx.x % kPieces;
+  const int h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = chunk * kPrefillChunk + threadIdx.x;
   const int64_t in_row_elems = v.D;
-  const int hd = v.head(layer, seq0 + b, h);
+  // ranks from the flags (inputs only: this overlaps the planner)
   const uint8_t f = j < P ? evict[(int64_t(b) * P + j) * v.Hkv + h] : 0;
   const bool keep = keep_token(j, P, v.w, f);
   const unsigned m = __ballot_sync(0xffffffffu, keep);
   if (lane == 0) s_wcnt[warp] = __popc(m);
   __syncthreads();
-  int before = 0, nkept = 0;
+  const int w0 = piece * kPieceWarps;     // the piece's first warp
+  const bool mine = warp >= w0 && warp < w0 + kPieceWarps;
+  int piece_base = 0, before = 0, nkept = 0;
+#pragma unroll
   for (int q = 0; q < 8; ++q) {
-    before += q < warp ? s_wcnt[q] : 0;
-    nkept += s_wcnt[q];
+    const int c = s_wcnt[q];
+    if (q < w0) {
+      piece_base += c;
+    } else if (q < w0 + kPieceWarps) {
+      nkept += c;
+      before += q < warp ? c : 0;
+    }
   }
   const int rank = before + __popc(m & ((1u << lane) - 1u));
-  const int base = v.chunk_counts[(int64_t(b) * v.Hkv + h) * v.n_chunks_max + chunk];
+  if (mine && keep) s_kept[rank] = threadIdx.x;
+  pdl_wait_prerequisites();               // the plan is complete and visible
+  const int go = v.hdr->prefill_go;
+  const int base = v.chunk_counts[(int64_t(b) * v.Hkv + h) * v.n_chunks_max + chunk] + piece_base;
+  if (!go) return;
+  const int hd = v.head(layer, seq0 + b, h);
   const int32_t* table = v.bt + int64_t(hd) * v.mbh;
-  if (keep) {
-    s_kept[rank] = threadIdx.x;
-    if (j >= P - v.w) {
-      const int slot = base + rank;
-      const int64_t ri = int64_t(hd) * v.w + (j % v.w);
-      v.ring[ri] = uint32_t(slot) | (uint32_t(f != 0) << 31);
-      v.ring_row[ri] = table[slot / v.BT] * v.BT + slot % v.BT;
-    }
+  if (mine && keep && j >= P - v.w) {
+    const int slot = base + rank;
+    const int64_t ri = int64_t(hd) * v.w + (j % v.w);
+    v.ring[ri] = uint32_t(slot) | (uint32_t(f != 0) << 31);
+    v.ring_row[ri] = table[slot / v.BT] * v.BT + slot % v.BT;
   }
   __syncthreads();
   if constexpr (STORE == 2) {
@@ -334,20 +402,63 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
       uint8_t* blk = v.blocks + int64_t(table[slot / v.BT]) * v.block_bytes;
       const InT* srck = k + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
       const InT* srcv = vv + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
+      // K: stored byte e of chunk lc is element d = 64 (lc & 1) + 2 (lc >> 1)
+      // + 16 (e >> 2) + 8 ((e >> 1) & 1) + (e & 1) (the fp8k_pos split): four
+      // pairs of adjacent elements per 16-element block, loaded as pairs
+      const int dk0 = (lc & 1) * 64 + (lc >> 1) * 2;
+      float kx[16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) load_pair(srck + dk0 + 16 * g + 8 * hi, kx[4 * g + 2 * hi], kx[4 * g + 2 * hi + 1]);
+      }
+      // V: elements d = 16 lc .. 16 lc + 15 of this token, one 16-byte load per 16 bytes
+      constexpr int kVecs = 16 * int(sizeof(InT)) / 16;
+      uint4 vraw[kVecs];
+#pragma unroll
+      for (int u = 0; u < kVecs; ++u) vraw[u] = __ldg(reinterpret_cast<const uint4*>(srcv + 16 * lc) + u);
+      const InT* vx = reinterpret_cast<const InT*>(vraw);
       uint8_t codes[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int pos = lc * 16 + e;
-        const int d = ((pos >> 2) & 7) * 16 + ((pos >> 1) & 1) * 8 + (pos >> 5) * 2 + (pos & 1);
-        codes[e] = f32_to_e4m3(__fdiv_rn(to_f32(srck[d]), sK));
-      }
+      for (int e = 0; e < 16; ++e) codes[e] = f32_to_e4m3(__fdiv_rn(kx[e], sK));
       *reinterpret_cast<uint4*>(blk + row * 128 + ((lc ^ (row & 7)) << 4)) =
           *reinterpret_cast<const uint4*>(codes);
-      // V: elements d = lc*16 .. lc*16+15 of this token, transposed tile
+      // V tile transposed: one byte per element
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int d = lc * 16 + e;
-        blk[v.tile_bytes + fp8v_byte(row, d)] = f32_to_e4m3(__fdiv_rn(to_f32(srcv[d]), sV));
+      for (int e = 0; e < 16; ++e)
+        blk[v.tile_bytes + fp8v_byte(row, 16 * lc + e)] = f32_to_e4m3(__fdiv_rn(to_f32(vx[e]), sV));
+    }
+  }
+  if constexpr (STORE != 0) {
+    // The piece holding the last prompt token holds the head's last slot n - 1
+    // (the window keeps that token): zero the V rows past it in its block, so
+    // those token columns decode to 0.  No other CTA writes those rows.
+    const int n = base + nkept;
+    const int r0 = n % v.BT;
+    if (int(blockIdx.x) == (P - 1) / SUB && r0 != 0) {
+      const int blk_id = table[(n - 1) / v.BT];
+      if (DMS_CHECK(blk_id >= 0 && blk_id < v.max_blocks, v.hdr, 203, hd, n)) {
+        uint8_t* vt = v.blocks + int64_t(blk_id) * v.block_bytes + v.tile_bytes;
+        if constexpr (STORE == 1) {
+          for (int i = threadIdx.x; i < (v.BT - r0) * v.D; i += blockDim.x)
+            vt[fp8v_byte(r0 + i / v.D, i % v.D)] = 0;
+        } else {
+          // word wi of element row d holds the nibbles of the 8 tokens
+          // t = 32 (wi & 1) + 16 e2 + 8 e1 + 2 (wi >> 1) + e0; other CTAs
+          // set the nibbles of rows < r0 with atomics, so clear with one too
+          for (int i = threadIdx.x; i < v.D * 8; i += blockDim.x) {
+            const int d = i >> 3, wi = i & 7;
+            uint32_t mask = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int t = (wi & 1) * 32 + ((e >> 2) & 1) * 16 + ((e >> 1) & 1) * 8 + (wi >> 1) * 2 + (e & 1);
+              if (t >= r0) mask |= 0xFu << int4v_shift(t);
+            }
+            if (mask) atomicAnd(reinterpret_cast<uint32_t*>(vt + int4v_word(d, (wi & 1) * 32 + (wi >> 1) * 2)), ~mask);
+          }
+          for (int i = threadIdx.x; i < (v.BT - r0) * (v.D / 32); i += blockDim.x)
+            *reinterpret_cast<__half*>(vt + int4v_scale(r0 + i / (v.D / 32), i % (v.D / 32))) = __float2half_rn(0.f);
+        }
       }
     }
   }
@@ -358,22 +469,45 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
 using namespace dms;
 
 namespace dms {
-// Count kept tokens per 256-token chunk, then plan (prefix counts, block
-// tables, counters, FP8 scales); shared with the fused prefill attention.
-dms_status prefill_plan_launch(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
-                               const uint8_t* evict, cudaStream_t stream) {
+// The plan kernel (counts, prefix sums, block tables, counters, FP8 scales);
+// shared with the fused prefill attention, which scatters the kept rows itself.
+template <typename InT, bool AMAX>
+static dms_status launch_plan(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
+                              const uint8_t* evict, const void* k, const void* v, cudaStream_t stream) {
   const PoolView& pv = pool->view;
   const int n_chunks = (prompt_len + kPrefillChunk - 1) / kPrefillChunk;
-  prefill_count_kernel<<<dim3(n_chunks, batch), 256, 0, stream>>>(pv, prompt_len, evict);
-  dms_status st = cuda_status(cudaGetLastError(), "prefill_count_kernel");
-  if (st != DMS_OK) return st;
-  const size_t plan_smem = sizeof(int) * (2 * size_t(batch) * pv.Hkv + 1);
-  if (plan_smem > 48 * 1024) {
-    set_last_error("batch * n_kv_heads too large for the prefill planner");
-    return DMS_ERR_UNSUPPORTED;
-  }
-  prefill_plan_kernel<<<1, 1024, plan_smem, stream>>>(pv, layer, seq0, batch, prompt_len);
+  const size_t smem = AMAX ? sizeof(uint32_t) * 2 * pv.Hkv : 0;
+  prefill_plan_kernel<InT, AMAX><<<dim3(n_chunks, batch), 256, smem, stream>>>(
+      pv, layer, seq0, batch, prompt_len, evict, static_cast<const InT*>(k), static_cast<const InT*>(v));
   return cuda_status(cudaGetLastError(), "prefill_plan_kernel");
+}
+
+dms_status prefill_plan_launch(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
+                               const uint8_t* evict, cudaStream_t stream) {
+  return launch_plan<__nv_bfloat16, false>(pool, layer, seq0, batch, prompt_len, evict, nullptr, nullptr,
+                                           stream);
+}
+
+template <typename InT, int STORE>
+static dms_status launch_scatter(const dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
+                                 const void* k, const void* v, const uint8_t* evict, cudaStream_t stream) {
+  const PoolView& pv = pool->view;
+  const int n_chunks = (prompt_len + kPrefillChunk - 1) / kPrefillChunk;
+  const int64_t ctas = int64_t(n_chunks) * pv.Hkv * batch;
+  // short prompts: 64-token pieces, so that the dense chunks (the window,
+  // keep-all heads) spread over four CTAs each; with two waves or more of
+  // 256-token CTAs (8 resident per SM) the dense ones balance out
+  const bool small = ctas < int64_t(2) * 8 * pool->sm_count;
+  const auto kk = static_cast<const InT*>(k);
+  const auto vv = static_cast<const InT*>(v);
+  cudaError_t e;
+  if (small)
+    e = launch_pdl(prefill_scatter_kernel<InT, STORE, 64>, dim3(n_chunks * 4, pv.Hkv, batch), dim3(256), 0,
+                   stream, pv, layer, seq0, prompt_len, kk, vv, evict);
+  else
+    e = launch_pdl(prefill_scatter_kernel<InT, STORE, 256>, dim3(n_chunks, pv.Hkv, batch), dim3(256), 0,
+                   stream, pv, layer, seq0, prompt_len, kk, vv, evict);
+  return cuda_status(e, "prefill_scatter_kernel");
 }
 }  // namespace dms
 
@@ -415,48 +549,19 @@ extern "C" dms_status dms_compact_prefill_seqs(dms_pool* pool, int layer, int se
     set_last_error("batch %d exceeds the 65535 sequences of one prefill launch", batch);
     return DMS_ERR_UNSUPPORTED;
   }
-  const int n_chunks = (prompt_len + kPrefillChunk - 1) / kPrefillChunk;
-  const dim3 grid(n_chunks, batch);
+  const bool bf16 = in_dtype == DMS_BF16;
   dms_status st;
-  if (fp8) {
-    st = cuda_status(cudaMemsetAsync(pv.amax, 0, sizeof(uint32_t) * 2 * pv.Hkv, stream), "amax clear");
-    if (st != DMS_OK) return st;
-    const size_t sm = sizeof(uint32_t) * 2 * pv.Hkv;
-    if (in_dtype == DMS_BF16)
-      prefill_amax_kernel<__nv_bfloat16><<<grid, 256, sm, stream>>>(
-          pv, prompt_len, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v));
-    else
-      prefill_amax_kernel<float><<<grid, 256, sm, stream>>>(
-          pv, prompt_len, static_cast<const float*>(k), static_cast<const float*>(v));
-    st = cuda_status(cudaGetLastError(), "prefill_amax_kernel");
-    if (st != DMS_OK) return st;
-  }
-  st = prefill_plan_launch(pool, layer, seq0, batch, prompt_len, evict, stream);
+  if (fp8)
+    st = bf16 ? launch_plan<__nv_bfloat16, true>(pool, layer, seq0, batch, prompt_len, evict, k, v, stream)
+              : launch_plan<float, true>(pool, layer, seq0, batch, prompt_len, evict, k, v, stream);
+  else
+    st = prefill_plan_launch(pool, layer, seq0, batch, prompt_len, evict, stream);
   if (st != DMS_OK) return st;
-  if (fp8 || int4) {   // the V tile of each head's partly filled last block
-    prefill_fp8_clear_tail_kernel<<<batch * pv.Hkv, 256, 0, stream>>>(pv, layer, seq0);
-    st = cuda_status(cudaGetLastError(), "prefill_fp8_clear_tail_kernel");
-    if (st != DMS_OK) return st;
-  }
-  const dim3 sgrid(n_chunks, pv.Hkv, batch);
-  if (in_dtype == DMS_BF16) {
-    auto kk = static_cast<const __nv_bfloat16*>(k);
-    auto vv = static_cast<const __nv_bfloat16*>(v);
-    if (fp8)
-      prefill_scatter_kernel<__nv_bfloat16, 1><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
-    else if (int4)
-      prefill_scatter_kernel<__nv_bfloat16, 2><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
-    else
-      prefill_scatter_kernel<__nv_bfloat16, 0><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
-  } else {
-    auto kk = static_cast<const float*>(k);
-    auto vv = static_cast<const float*>(v);
-    if (fp8)
-      prefill_scatter_kernel<float, 1><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
-    else if (int4)
-      prefill_scatter_kernel<float, 2><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
-    else
-      prefill_scatter_kernel<float, 0><<<sgrid, 256, 0, stream>>>(pv, layer, seq0, prompt_len, kk, vv, evict);
-  }
-  return cuda_status(cudaGetLastError(), "prefill_scatter_kernel");
+  if (bf16)
+    return fp8 ? launch_scatter<__nv_bfloat16, 1>(pool, layer, seq0, batch, prompt_len, k, v, evict, stream)
+         : int4 ? launch_scatter<__nv_bfloat16, 2>(pool, layer, seq0, batch, prompt_len, k, v, evict, stream)
+                : launch_scatter<__nv_bfloat16, 0>(pool, layer, seq0, batch, prompt_len, k, v, evict, stream);
+  return fp8 ? launch_scatter<float, 1>(pool, layer, seq0, batch, prompt_len, k, v, evict, stream)
+       : int4 ? launch_scatter<float, 2>(pool, layer, seq0, batch, prompt_len, k, v, evict, stream)
+              : launch_scatter<float, 0>(pool, layer, seq0, batch, prompt_len, k, v, evict, stream);
 }

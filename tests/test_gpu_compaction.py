@@ -1,0 +1,155 @@
+"""Prefill compaction at both piece sizes of the scatter kernel.
+
+The scatter kernel gives a CTA 64 prompt tokens when a layer has fewer than
+two waves of 256-token CTAs, else 256.  For each store (bf16, FP8, 4-bit) the
+same prompts are compacted once as a large batch (256-token pieces) and once
+as two sequences (64-token pieces), into pools whose blocks were filled with
+0xFF bytes first (NaN in bf16, FP8 and the f16 scales), with per-head keep
+probabilities from window-only to keep-all and a ragged last chunk.  Every
+checked head's counters, ring and stored rows must equal the oracle's bit for
+bit; in the quantised stores the V rows past a head's last slot must read zero
+(the attention reads whole V tiles); one decode step over every head must
+match the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import attention as oatt
+from oracle import fp8 as ofp8
+from oracle import int4 as oint4
+from compact_decode_attention_b200 import dms
+
+from gpu_util import (BT, check_block_invariants, check_head_store, head_id, int4_rows, oracle_store,
+                      read_state)
+
+pytestmark = pytest.mark.gpu
+
+CODE = {"bf16": dms.DMS_BF16, "fp8": dms.DMS_FP8_E4M3, "int4": dms.DMS_INT4}
+TOL = {"bf16": 2e-2, "fp8": 6e-2, "int4": 6e-2}
+KEEP = [0.3, 1.0, 0.0, 0.05, 0.5, 0.3, 0.9, 0.15]   # per kv-head
+
+
+def _dev(a, dt=torch.bfloat16):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dt).cuda()
+
+
+def _v_tail_bytes(pool, state, hd, n, kind):
+    """Bytes of the V rows r0..63 of the block holding slot n - 1 (r0 = n mod 64)."""
+    r0 = n % BT
+    blk = int(state["bt"][hd, (n - 1) // BT])
+    lay, D = pool.layout, pool.cfg.head_dim
+    o = int(lay.blocks + blk * lay.block_bytes)
+    rows = np.arange(r0, BT)
+    d = np.arange(D)
+    if kind == "fp8":
+        vt = pool.buffer[o + BT * D:o + 2 * BT * D].cpu().numpy()
+        f = (((rows & 7) >> 1) << 4) | ((rows >> 4) << 2) | (((rows >> 3) & 1) << 1) | (rows & 1)
+        return vt[d[:, None] * 64 + f[None, :]]
+    tile = BT * (D // 2 + D // 16)
+    vt = pool.buffer[o + tile:o + 2 * tile].cpu().numpy()
+    words = vt[:BT * D // 2].view(np.uint32)
+    wi = (d[:, None] * 32 + ((rows[None, :] & 7) >> 1) * 8 + (rows[None, :] >> 5) * 4) // 4
+    sh = 8 * ((rows >> 4) & 1) + 4 * ((rows >> 3) & 1) + 16 * (rows & 1)
+    nib = (words[wi] >> sh[None, :].astype(np.uint32)) & 0xF
+    scales = vt[BT * D // 2:].view(np.uint16).reshape(D // 32, BT)[:, rows]
+    return np.concatenate([nib.reshape(-1), scales.reshape(-1).astype(np.uint32)])
+
+
+def _device_inputs(seed, B, n_pos, Hkv, D, thr):
+    """K, V [B, n_pos, Hkv, D] bf16 and flags [B, n_pos, Hkv] drawn on the device
+    by the generator's device twin."""
+    st = torch.cuda.current_stream().cuda_stream
+    K = torch.empty(1, B, n_pos, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    F = torch.empty(1, B, n_pos, Hkv, dtype=torch.uint8, device="cuda")
+    dms.dms_synth_normal(seed, 0, 0, 1, B, 0, n_pos, Hkv, D, dms.DMS_BF16, K.data_ptr(), st)
+    dms.dms_synth_normal(seed, 1, 0, 1, B, 0, n_pos, Hkv, D, dms.DMS_BF16, V.data_ptr(), st)
+    t = torch.tensor([thr], dtype=torch.int32, device="cuda")
+    dms.dms_synth_flags(seed, 0, 1, B, 0, n_pos, Hkv, t.data_ptr(), F.data_ptr(), st)
+    return K[0], V[0], F[0]
+
+
+def _host_sequence(seed, b, n_pos, Hkv, D, thr):
+    """The same draws for one sequence, from the NumPy generator: [n_pos, Hkv, D] x 2, [n_pos, Hkv]."""
+    pos = np.arange(n_pos)
+    K = np.stack([synth.normal(seed, 0, 0, b, pos[:, None], h, np.arange(D)[None, :], "bf16")
+                  for h in range(Hkv)], axis=1)
+    V = np.stack([synth.normal(seed, 1, 0, b, pos[:, None], h, np.arange(D)[None, :], "bf16")
+                  for h in range(Hkv)], axis=1)
+    F = np.stack([synth.evict_flags(seed, 0, b, pos, h, thr[h]) for h in range(Hkv)], axis=1)
+    return K, V, F
+
+
+@pytest.mark.parametrize("kind", ["bf16", "fp8", "int4"])
+def test_both_piece_sizes_match_the_oracle(kind):
+    Hkv, Hq, D, P, w, seed = 8, 32, 128, 1000, 64, 91
+    sm = torch.cuda.get_device_properties(0).multi_processor_count
+    n_chunks = (P + 255) // 256
+    B_big = -(-2 * 8 * sm // (n_chunks * Hkv)) + 1
+    thr = [synth.keep_threshold(p) for p in KEEP]
+    Kd, Vd, Fd = _device_inputs(seed, B_big, P + 1, Hkv, D, thr)
+    rng = np.random.default_rng(seed)
+    host = {}
+    for B in (B_big, 2):
+        pool = dms.Pool(1, B, Hq, Hkv, D, w, CODE[kind], B * Hkv * (P // BT + 3), P + 2)
+        pool.buffer[pool.layout.blocks:].fill_(0xFF)       # stale bytes in every block
+        pool.compact_prefill(0, Kd[:B, :P].contiguous(), Vd[:B, :P].contiguous(), Fd[:B, :P].contiguous())
+        state = read_state(pool)
+        assert state["error"] == 0
+        check_block_invariants(pool, state)
+        scales = None
+        if kind == "fp8":   # amax over every prompt row of the batch (exact in any order)
+            scales = [(ofp8.fp8_scale(np.float32(Kd[:B, :P, h].float().abs().max().item())),
+                       ofp8.fp8_scale(np.float32(Vd[:B, :P, h].float().abs().max().item())))
+                      for h in range(Hkv)]
+            for h in range(Hkv):
+                assert state["scales"][0, h, 0] == scales[h][0] and state["scales"][0, h, 1] == scales[h][1]
+        seqs = sorted({0, 1, B - 1} | set(int(x) for x in rng.choice(B, size=min(B, 4), replace=False)))
+        for b in seqs:
+            if b not in host:
+                host[b] = _host_sequence(seed, b, P + 1, Hkv, D, thr)
+            K, V, F = host[b]
+            for h in range(Hkv):
+                hd = head_id(pool.cfg, 0, b, h)
+                store = oracle_store(F[:P, h], np.zeros(0, np.uint8), w, P)
+                n = store.n_slots
+                if kind == "int4":
+                    assert state["n_slots"][hd] == n and state["n_retained"][hd] == store.n_retained
+                    for idx, e in enumerate(store.ring):
+                        if e is not None:
+                            assert state["ring"][hd, idx] == (e[0] | (e[1] << 31)), (hd, idx)
+                    pos = np.array([store.pos_of_slot[s] for s in range(n)])
+                    ck, sk, cv, sv = int4_rows(pool, state, hd, n)
+                    qk, ek = oint4.quantize(K[pos, h])
+                    qv, ev = oint4.quantize(V[pos, h])
+                    assert np.array_equal(ck, qk) and np.array_equal(sk, ek), (B, b, h)
+                    assert np.array_equal(cv, qv) and np.array_equal(sv, ev), (B, b, h)
+                else:
+                    rk = {j: K[j, h] for j in range(P)}
+                    rv = {j: V[j, h] for j in range(P)}
+                    check_head_store(pool, state, hd, store, rk, rv, kind,
+                                     None if scales is None else scales[h])
+                if kind != "bf16" and n % BT:
+                    assert not _v_tail_bytes(pool, state, hd, n, kind).any(), (B, b, h)
+        # one decode step over every head; outputs of the sampled sequences
+        # against the oracle on the stored values
+        pool.append_evict_layers(0, P, Kd[None, :B, P].contiguous(), Vd[None, :B, P].contiguous(),
+                                 Fd[None, :B, P].contiguous())
+        Q = synth.q_tokens(seed, 0, B, P, Hq, D, "bf16")
+        out = torch.empty(1, B, Hq, D, dtype=torch.bfloat16, device="cuda")
+        pool.decode_attn_layers(0, _dev(Q[None]), out)
+        got = out[0].float().cpu().numpy()
+        assert np.isfinite(got).all()
+        for b in seqs:
+            K, V, F = host[b]
+            Ks, Vs = K.astype(np.float64), V.astype(np.float64)
+            if kind == "fp8":
+                for h in range(Hkv):
+                    Ks[:, h] = ofp8.dequantize(ofp8.quantize(K[:, h], scales[h][0]), scales[h][0])
+                    Vs[:, h] = ofp8.dequantize(ofp8.quantize(V[:, h], scales[h][1]), scales[h][1])
+            elif kind == "int4":
+                Ks, Vs = oint4.stored(K), oint4.stored(V)
+            exp = oatt.decode_attention(Q[b].astype(np.float64), Ks, Vs, F, P, w)
+            bound = TOL[kind] + (np.abs(exp) * 2.0 ** -8 + np.abs(Vs).max() * 2.0 ** -10 if kind == "int4" else 0)
+            assert (np.abs(got[b] - exp) < bound).all(), (kind, B, b)
