@@ -496,7 +496,10 @@ def main():
         compact_bytes += L * B * P * Hkv * in_row
     # the same rate counted as if every prompt row were read (the full-read variant)
     full_read_bytes = L * B * P * Hkv * (1 + in_row) + base * row_bytes
+    hbm_peak, hbm_kind = measured_peaks()
     compaction = {"value": compact_bytes / (compact_ms * 1e-3) / 1e9, "unit": "GB/s",
+                  "frac": compact_bytes / (compact_ms * 1e-3) / 1e9 / hbm_peak,
+                  "peak_kind": f"{hbm_kind} copy bandwidth",
                   "ms_per_layer": compact_ms / L, "algorithmic_bytes_per_layer": compact_bytes / L,
                   "full_read_value": full_read_bytes / (compact_ms * 1e-3) / 1e9,
                   "timing": "CUDA events around each layer's dms_compact_prefill call (plan and "

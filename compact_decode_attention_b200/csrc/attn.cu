@@ -17,12 +17,14 @@
 // CTA that finishes it last (an atomic ticket -- nobody waits).  Partial id
 // c + i is unique per (CTA c, head i) piece.
 //
-// Inside a CTA: warp 4 is the producer.  It issues one 1-D TMA bulk copy per
-// full block (K tile and V tile are adjacent in the pool, 32 KB for bf16
-// D=128) plus the g query rows of the head, into a ring of NS shared-memory
-// stages paced by mbarriers (expect-tx on "full", one arrive on "empty").
-// Warps 0-3 consume stages round-robin.  Each keeps its own online-softmax
-// state for the current head and computes on tensor cores with the GQA
+// Inside a CTA: the last warp is the producer.  It issues one 1-D TMA bulk
+// copy per full block (K tile and V tile are adjacent in the pool, 32 KB for
+// bf16 D=128) into a ring of NS shared-memory stages paced by mbarriers
+// (expect-tx on "full", one arrive on "empty").  The NCW consumer warps
+// before it take the stages round-robin (NS a multiple of NCW, see
+// AttnTraits).  Each keeps its own online-softmax state for the current head,
+// reads the head's query rows itself (the fp32 path: from the stage, where
+// the producer copies them with the block), and computes on tensor cores with the GQA
 // group as the N=8 side of mma.sync m16n8k16 (tokens as M): S^T = K Q^T,
 // then O^T += V^T P^T, P moved from accumulator to operand layout with
 // movmatrix.  The stored rows' 16-byte chunks are XOR-swizzled by row, so

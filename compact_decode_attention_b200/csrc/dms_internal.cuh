@@ -307,6 +307,11 @@ __device__ __forceinline__ void pdl_wait_prerequisites() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Bring the line holding p into L2 (no register written, nothing waits).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // 2^x with the hardware approximation (max rel. error ~2^-22).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

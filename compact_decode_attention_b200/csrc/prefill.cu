@@ -170,6 +170,14 @@ __global__ void __launch_bounds__(256) prefill_plan_kernel(PoolView v, int layer
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = chunk * kPrefillChunk + tid;
   const int n_chunks = gridDim.x;
+  if (chunk == 0 && b == 0) {   // warm L2 with what the planner reads cold
+    for (int p = tid; p < batch * v.Hkv; p += blockDim.x) {
+      const int hd = v.head(layer, seq0 + p / v.Hkv, p % v.Hkv);
+      prefetch_l2(v.n_slots + hd);
+      prefetch_l2(v.n_retained + hd);
+    }
+    if (tid == 0) prefetch_l2(v.hdr);
+  }
   for (int h0 = 0; h0 < v.Hkv; h0 += 32) {
     const int nh = min(32, v.Hkv - h0);
     const uint8_t* fl = evict + (int64_t(b) * P + j) * v.Hkv + h0;
@@ -196,43 +204,55 @@ __global__ void __launch_bounds__(256) prefill_plan_kernel(PoolView v, int layer
     for (int i = tid; i < 2 * v.Hkv; i += blockDim.x) s_amax[i] = 0;
     __syncthreads();
     constexpr int VEC = 16 / sizeof(InT);
+    constexpr int U = 4;                  // K and V vectors in flight per thread, each
     const int j0 = chunk * kPrefillChunk;
     const int nj = min(kPrefillChunk, P - j0);
     const int64_t row0 = (int64_t(b) * P + j0) * v.Hkv;  // first row of the chunk
-    const int64_t nvec = int64_t(nj) * v.Hkv * v.D / VEC;
     const int vec_per_row = v.D / VEC;
-    for (int which = 0; which < 2; ++which) {
-      const uint4* src = reinterpret_cast<const uint4*>((which ? vv : k) + row0 * v.D);
-      // a thread's vectors mostly belong to one head (always when 256 vectors
-      // span a multiple of Hkv rows): keep its maximum in a register and fold
-      // it into shared memory when the head changes
-      float acc = 0.f;
-      int cur = -1;
-      for (int64_t i0 = tid; i0 < nvec; i0 += 4 * blockDim.x) {
-        uint4 raw[4];
+    const int nvec = nj * v.Hkv * vec_per_row;
+    const uint4* srck = reinterpret_cast<const uint4*>(k + row0 * v.D);
+    const uint4* srcv = reinterpret_cast<const uint4*>(vv + row0 * v.D);
+    const int stride = blockDim.x;
+    // vector i belongs to head (i / vec_per_row) mod Hkv: every vector of a
+    // thread has the same head when the stride spans whole tokens
+    const bool fixed = stride % (vec_per_row * v.Hkv) == 0;
+    int cur = fixed ? (tid / vec_per_row) % v.Hkv : -1;
+    float ak = 0.f, av = 0.f;
+    const auto vmax = [](const uint4& raw) {
+      const InT* x = reinterpret_cast<const InT*>(&raw);
+      float m = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t i = i0 + u * blockDim.x;
-          raw[u] = i < nvec ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
-        }
+      for (int e = 0; e < VEC; ++e) m = fmaxf(m, fabsf(to_f32(x[e])));
+      return m;
+    };
+    for (int i0 = tid; i0 < nvec; i0 += U * stride) {
+      uint4 rk[U], rv[U];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t i = i0 + u * blockDim.x;
-          if (i >= nvec) break;
-          const InT* x = reinterpret_cast<const InT*>(&raw[u]);
-          float mx = 0.f;
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) mx = fmaxf(mx, fabsf(to_f32(x[e])));
-          const int h = int((i / vec_per_row) % v.Hkv);
-          if (h != cur) {
-            if (cur >= 0) atomicMax(&s_amax[which * v.Hkv + cur], __float_as_uint(acc));
-            cur = h;
-            acc = 0.f;
-          }
-          acc = fmaxf(acc, mx);
-        }
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * stride;
+        rk[u] = i < nvec ? __ldg(srck + i) : make_uint4(0, 0, 0, 0);   // zeros leave a maximum as it is
+        rv[u] = i < nvec ? __ldg(srcv + i) : make_uint4(0, 0, 0, 0);
       }
-      if (cur >= 0) atomicMax(&s_amax[which * v.Hkv + cur], __float_as_uint(acc));
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (!fixed) {
+          const int hh = ((i0 + u * stride) / vec_per_row) % v.Hkv;
+          if (hh != cur) {
+            if (cur >= 0) {
+              atomicMax(&s_amax[cur], __float_as_uint(ak));
+              atomicMax(&s_amax[v.Hkv + cur], __float_as_uint(av));
+            }
+            cur = hh;
+            ak = av = 0.f;
+          }
+        }
+        ak = fmaxf(ak, vmax(rk[u]));
+        av = fmaxf(av, vmax(rv[u]));
+      }
+    }
+    if (cur >= 0) {
+      atomicMax(&s_amax[cur], __float_as_uint(ak));
+      atomicMax(&s_amax[v.Hkv + cur], __float_as_uint(av));
     }
     __syncthreads();
     for (int i = tid; i < 2 * v.Hkv; i += blockDim.x) atomicMax(&v.amax[i], s_amax[i]);
@@ -273,31 +293,37 @@ __global__ void __launch_bounds__(256) prefill_plan_kernel(PoolView v, int layer
     if (lane == 0) v.pair_n[b * v.Hkv + h] = carry;
   }
   if (tid == 0) v.prefill_tickets[b] = 0;
-  // arrival: the last sequence to finish plans the layer
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&v.prefill_tickets[v.Bmax], 1) == batch - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  if (batch > 1) {
+    // arrival: the last sequence to finish plans the layer
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&v.prefill_tickets[v.Bmax], 1) == batch - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (tid == 0) v.prefill_tickets[v.Bmax] = 0;
+  } else {
+    __threadfence();   // pair_n of the one sequence, written above, is read through L2
+    __syncthreads();
+  }
   pdl_launch_dependents();   // the scatter grid may be scheduled while the plan is made
-  if (tid == 0) v.prefill_tickets[v.Bmax] = 0;
   plan_layer(v, layer, seq0, batch);
 }
 
 // ---------------------------------------------------------------------------
-// One CTA of 256 threads per (SUB-token piece, kv-head, sequence); the pieces
-// of one 256-token chunk share its planned base.  STORE: 0 = copy (bf16 /
-// fp32 store), 1 = FP8, 2 = 4-bit.
-template <typename InT, int STORE, int SUB>
+// One CTA of 256 threads per (SPAN-token span, kv-head, sequence): a 64-token
+// piece of a 256-token chunk (the pieces before it in the chunk give its
+// offset) or a whole chunk.  STORE: 0 = copy (bf16 / fp32 store), 1 = FP8,
+// 2 = 4-bit.
+template <typename InT, int STORE, int SPAN>
 __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int layer, int seq0, int P,
                                                               const InT* __restrict__ k,
                                                               const InT* __restrict__ vv,
                                                               const uint8_t* __restrict__ evict) {
-  static_assert(kPrefillChunk % SUB == 0 && SUB % 32 == 0, "a piece is whole warps of a chunk");
-  constexpr int kPieces = kPrefillChunk / SUB, kPieceWarps = SUB / 32;
+  static_assert(kPrefillChunk % SPAN == 0 && SPAN % 32 == 0, "a span is whole warps of one chunk");
+  constexpr int kPieces = kPrefillChunk / SPAN, kSpanWarps = SPAN / 32;
   constexpr int kBatchItems = 4;          // 16-byte copies in flight per thread
-  __shared__ int s_kept[SUB];             // chunk-local token index of each kept rank
+  __shared__ int s_kept[SPAN];            // chunk-local token index of each kept rank
   __shared__ int s_wcnt[8];
   const int chunk = blockIdx.x / kPieces, piece = blockIdx.x % kPieces;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -305,26 +331,85 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
   const int j = chunk * kPrefillChunk + threadIdx.x;
   const int64_t in_row_elems = v.D;
   // ranks from the flags (inputs only: this overlaps the planner)
-  const uint8_t f = j < P ? evict[(int64_t(b) * P + j) * v.Hkv + h] : 0;
+  const uint8_t f = j < P ? __ldg(evict + (int64_t(b) * P + j) * v.Hkv + h) : 0;
   const bool keep = keep_token(j, P, v.w, f);
   const unsigned m = __ballot_sync(0xffffffffu, keep);
   if (lane == 0) s_wcnt[warp] = __popc(m);
   __syncthreads();
-  const int w0 = piece * kPieceWarps;     // the piece's first warp
-  const bool mine = warp >= w0 && warp < w0 + kPieceWarps;
+  const int w0 = piece * kSpanWarps;      // the span's first warp
+  const bool mine = warp >= w0 && warp < w0 + kSpanWarps;
   int piece_base = 0, before = 0, nkept = 0;
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const int c = s_wcnt[q];
     if (q < w0) {
       piece_base += c;
-    } else if (q < w0 + kPieceWarps) {
+    } else if (q < w0 + kSpanWarps) {
       nkept += c;
       before += q < warp ? c : 0;
     }
   }
   const int rank = before + __popc(m & ((1u << lane) - 1u));
   if (mine && keep) s_kept[rank] = threadIdx.x;
+  __syncthreads();                        // s_kept complete
+  const auto src_row = [&](const InT* x, int kk) {
+    return x + ((int64_t(b) * P + chunk * kPrefillChunk + s_kept[kk]) * v.Hkv + h) * in_row_elems;
+  };
+  // The inputs are ready before the plan: each thread loads its first source
+  // data now, while the planner runs, and stores it once the slots are known.
+  // copy: 16-byte chunks, kBatchItems of K and of V per thread in flight
+  const int nch = int(v.row_bytes >> 4);
+  const int n_items = STORE == 0 ? nkept * nch : STORE == 1 ? nkept * 8 : nkept;
+  uint4 xk[kBatchItems], xv[kBatchItems];
+  const auto load_copy = [&](int i0) {
+#pragma unroll
+    for (int u = 0; u < kBatchItems; ++u) {
+      const int i = i0 + u * blockDim.x + threadIdx.x;
+      if (i < n_items) {
+        const int kk = i / nch, c = i % nch;
+        xk[u] = __ldg(reinterpret_cast<const uint4*>(src_row(k, kk)) + c);
+        xv[u] = __ldg(reinterpret_cast<const uint4*>(src_row(vv, kk)) + c);
+      }
+    }
+  };
+  // FP8 (D = 128): item i = 16 elements (chunk lc = i & 7) of kept row i >> 3.
+  // K: stored byte e of chunk lc is element d = 64 (lc & 1) + 2 (lc >> 1)
+  // + 16 (e >> 2) + 8 ((e >> 1) & 1) + (e & 1) (the fp8k_pos split): four
+  // pairs of adjacent elements per 16-element block, loaded as pairs.
+  // V: elements 16 lc .. 16 lc + 15, one 16-byte load per 16 bytes.
+  constexpr int kVecs = 16 * int(sizeof(InT)) / 16;
+  float kx[16];
+  uint4 vraw[kVecs];
+  const auto load_fp8 = [&](int i) {
+    const int kk = i >> 3, lc = i & 7;
+    const InT* srck = src_row(k, kk);
+    const int dk0 = (lc & 1) * 64 + (lc >> 1) * 2;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+#pragma unroll
+      for (int hi = 0; hi < 2; ++hi) load_pair(srck + dk0 + 16 * g + 8 * hi, kx[4 * g + 2 * hi], kx[4 * g + 2 * hi + 1]);
+    }
+#pragma unroll
+    for (int u = 0; u < kVecs; ++u) vraw[u] = __ldg(reinterpret_cast<const uint4*>(src_row(vv, kk) + 16 * lc) + u);
+  };
+  // 4-bit: one warp per kept row, lane l holds elements 4l .. 4l+3
+  float k4[4], v4[4];
+  const auto load_int4 = [&](int kk) {
+    const InT* srck = src_row(k, kk);
+    const InT* srcv = src_row(vv, kk);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      k4[e] = to_f32(srck[4 * lane + e]);
+      v4[e] = to_f32(srcv[4 * lane + e]);
+    }
+  };
+  if constexpr (STORE == 0) load_copy(0);
+  if constexpr (STORE == 1) {
+    if (int(threadIdx.x) < n_items) load_fp8(threadIdx.x);
+  }
+  if constexpr (STORE == 2) {
+    if (warp < n_items) load_int4(warp);
+  }
   pdl_wait_prerequisites();               // the plan is complete and visible
   const int go = v.hdr->prefill_go;
   const int base = v.chunk_counts[(int64_t(b) * v.Hkv + h) * v.n_chunks_max + chunk] + piece_base;
@@ -337,86 +422,42 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
     v.ring[ri] = uint32_t(slot) | (uint32_t(f != 0) << 31);
     v.ring_row[ri] = table[slot / v.BT] * v.BT + slot % v.BT;
   }
-  __syncthreads();
   if constexpr (STORE == 2) {
-    // 4-bit: one warp quantises one kept row (lane l: elements 4l .. 4l+3)
     for (int kk = warp; kk < nkept; kk += blockDim.x / 32) {
-      const int jj = chunk * kPrefillChunk + s_kept[kk];
+      if (kk != warp) load_int4(kk);
       const int slot = base + kk;
       const int blk = table[slot / v.BT];
       if (!DMS_CHECK(blk >= 0 && blk < v.max_blocks, v.hdr, 202, hd, slot)) continue;
-      const InT* srck = k + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
-      const InT* srcv = vv + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
-      float k4[4], v4[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        k4[e] = to_f32(srck[4 * lane + e]);
-        v4[e] = to_f32(srcv[4 * lane + e]);
-      }
       store_row_int4(v, blk * v.BT + slot % v.BT, k4, v4, lane);
     }
   } else if constexpr (STORE == 0) {
-    // bitwise row copy in 16-byte chunks, swizzled by row; each thread loads
-    // kBatchItems K and V chunks before storing any
-    const int nch = int(v.row_bytes >> 4);
-    const int total = nkept * nch;
-    for (int i0 = 0; i0 < total; i0 += kBatchItems * blockDim.x) {
-      uint4 xk[kBatchItems], xv[kBatchItems];
-      uint8_t* dst[kBatchItems];
+    // bitwise row copy, 16-byte chunks swizzled by row
+    for (int i0 = 0; i0 < n_items; i0 += kBatchItems * blockDim.x) {
+      if (i0) load_copy(i0);
 #pragma unroll
       for (int u = 0; u < kBatchItems; ++u) {
         const int i = i0 + u * blockDim.x + threadIdx.x;
-        dst[u] = nullptr;
-        if (i < total) {
-          const int kk = i / nch, c = i % nch;
-          const int jj = chunk * kPrefillChunk + s_kept[kk];
-          const int slot = base + kk;
-          const int row = slot % v.BT;
-          if (DMS_CHECK(slot < v.mbh * v.BT && table[slot / v.BT] >= 0 &&
-                            table[slot / v.BT] < v.max_blocks, v.hdr, 201, hd, slot)) {
-            dst[u] = v.blocks + int64_t(table[slot / v.BT]) * v.block_bytes +
-                     int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;
-            const int64_t src_off = ((int64_t(b) * P + jj) * v.Hkv + h) * v.row_bytes + c * 16;
-            xk[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(k) + src_off));
-            xv[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vv) + src_off));
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kBatchItems; ++u) {
-        if (dst[u]) {
-          *reinterpret_cast<uint4*>(dst[u]) = xk[u];
-          *reinterpret_cast<uint4*>(dst[u] + v.tile_bytes) = xv[u];
+        if (i >= n_items) break;
+        const int kk = i / nch, c = i % nch;
+        const int slot = base + kk;
+        const int row = slot % v.BT;
+        const int blk = table[slot / v.BT];
+        if (DMS_CHECK(slot < v.mbh * v.BT && blk >= 0 && blk < v.max_blocks, v.hdr, 201, hd, slot)) {
+          uint8_t* dst = v.blocks + int64_t(blk) * v.block_bytes + int64_t(row) * v.row_bytes + swz_chunk(c, row) * 16;
+          *reinterpret_cast<uint4*>(dst) = xk[u];
+          *reinterpret_cast<uint4*>(dst + v.tile_bytes) = xv[u];
         }
       }
     }
   } else {
-    // FP8 (D = 128): each thread quantises 16 elements of one kept row
     const float sK = v.scales[(int64_t(layer) * v.Hkv + h) * 2 + 0];
     const float sV = v.scales[(int64_t(layer) * v.Hkv + h) * 2 + 1];
-    for (int i = threadIdx.x; i < nkept * 8; i += blockDim.x) {
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+      if (i != int(threadIdx.x)) load_fp8(i);
       const int kk = i >> 3, lc = i & 7;
-      const int jj = chunk * kPrefillChunk + s_kept[kk];
       const int slot = base + kk;
       const int row = slot % v.BT;
       uint8_t* blk = v.blocks + int64_t(table[slot / v.BT]) * v.block_bytes;
-      const InT* srck = k + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
-      const InT* srcv = vv + ((int64_t(b) * P + jj) * v.Hkv + h) * in_row_elems;
-      // K: stored byte e of chunk lc is element d = 64 (lc & 1) + 2 (lc >> 1)
-      // + 16 (e >> 2) + 8 ((e >> 1) & 1) + (e & 1) (the fp8k_pos split): four
-      // pairs of adjacent elements per 16-element block, loaded as pairs
-      const int dk0 = (lc & 1) * 64 + (lc >> 1) * 2;
-      float kx[16];
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) load_pair(srck + dk0 + 16 * g + 8 * hi, kx[4 * g + 2 * hi], kx[4 * g + 2 * hi + 1]);
-      }
-      // V: elements d = 16 lc .. 16 lc + 15 of this token, one 16-byte load per 16 bytes
-      constexpr int kVecs = 16 * int(sizeof(InT)) / 16;
-      uint4 vraw[kVecs];
-#pragma unroll
-      for (int u = 0; u < kVecs; ++u) vraw[u] = __ldg(reinterpret_cast<const uint4*>(srcv + 16 * lc) + u);
       const InT* vx = reinterpret_cast<const InT*>(vraw);
       uint8_t codes[16];
 #pragma unroll
@@ -435,7 +476,7 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
     // those token columns decode to 0.  No other CTA writes those rows.
     const int n = base + nkept;
     const int r0 = n % v.BT;
-    if (int(blockIdx.x) == (P - 1) / SUB && r0 != 0) {
+    if (int(blockIdx.x) == (P - 1) / SPAN && r0 != 0) {
       const int blk_id = table[(n - 1) / v.BT];
       if (DMS_CHECK(blk_id >= 0 && blk_id < v.max_blocks, v.hdr, 203, hd, n)) {
         uint8_t* vt = v.blocks + int64_t(blk_id) * v.block_bytes + v.tile_bytes;
@@ -493,11 +534,12 @@ static dms_status launch_scatter(const dms_pool* pool, int layer, int seq0, int 
                                  const void* k, const void* v, const uint8_t* evict, cudaStream_t stream) {
   const PoolView& pv = pool->view;
   const int n_chunks = (prompt_len + kPrefillChunk - 1) / kPrefillChunk;
-  const int64_t ctas = int64_t(n_chunks) * pv.Hkv * batch;
-  // short prompts: 64-token pieces, so that the dense chunks (the window,
-  // keep-all heads) spread over four CTAs each; with two waves or more of
-  // 256-token CTAs (8 resident per SM) the dense ones balance out
-  const bool small = ctas < int64_t(2) * 8 * pool->sm_count;
+  const int64_t ctas = int64_t(n_chunks) * pv.Hkv * batch;   // with 256-token spans
+  // Short prompts: 64-token spans, so that the dense chunks (the window,
+  // keep-all heads) spread over four CTAs each; from 16 x SMs CTAs on (four
+  // rounds at four resident per SM) the dense ones balance out.  Spans of
+  // several chunks measured slower: a CTA's copy rounds are serial.
+  const bool small = ctas < int64_t(16) * pool->sm_count;
   const auto kk = static_cast<const InT*>(k);
   const auto vv = static_cast<const InT*>(v);
   cudaError_t e;
