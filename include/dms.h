@@ -47,8 +47,10 @@
  *   (pool exhausted, table overflow, a wait that timed out) set bits of the
  *   pool's error word, read back by dms_pool_stats.  No kernel traps or
  *   waits without a time limit.
- * - Calls that touch the same layer must be ordered (same stream or
- *   events).  Pointers are device pointers unless marked host.
+ * - Calls on one pool must be ordered (one stream, or events between
+ *   streams): compaction, append, release and the fused projection share
+ *   the pool's block counters and the planner's scratch, whatever layer
+ *   they touch.  Pointers are device pointers unless marked host.
  * - Layouts are row-major, C order.  B = batch (sequences 0..B-1 of the
  *   pool, B <= max_batch), P = prompt length, Hq / Hkv query / kv heads,
  *   g = Hq / Hkv (query head hq reads kv head hq / g), D = head_dim.
