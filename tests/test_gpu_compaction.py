@@ -156,3 +156,36 @@ def test_both_piece_sizes_match_the_oracle(kind):
             exp = oatt.decode_attention(Q[b].astype(np.float64), Ks, Vs, F, P, w)
             bound = TOL[kind] + (np.abs(exp) * 2.0 ** -8 + np.abs(Vs).max() * 2.0 ** -10 if kind == "int4" else 0)
             assert (np.abs(got[b] - exp) < bound).all(), (kind, B, b)
+
+
+def test_refused_call_leaves_the_planner_clean():
+    """A compaction the planner refuses (its layer is not empty) still resets
+    the arrival tickets and the FP8 maxima: the next call, into another layer,
+    takes its scales from its own rows only (the refused call's rows are 100x
+    larger) and stores every head bit-exactly."""
+    L, B, Hq, Hkv, D, P, w, seed = 2, 3, 4, 2, 128, 300, 32, 92
+    thr = [synth.keep_threshold(0.3)] * Hkv
+    pool = dms.Pool(L, B, Hq, Hkv, D, w, dms.DMS_FP8_E4M3, L * B * Hkv * (P // BT + 2), P + 1)
+    K = synth.kv_tokens(seed, 0, 0, B, 0, P, Hkv, D, "bf16")
+    V = synth.kv_tokens(seed, 1, 0, B, 0, P, Hkv, D, "bf16")
+    F = synth.flag_tokens(seed, 0, B, 0, P, Hkv, thr)
+    Fd = torch.from_numpy(np.ascontiguousarray(F)).cuda()
+    pool.compact_prefill(0, _dev(K), _dev(V), Fd)
+    pool.compact_prefill(0, _dev(K * 100), _dev(V * 100), Fd)          # refused: layer 0 is full
+    assert pool.stats(check=False).error_flags & dms.DEVERR_LAYER_NOT_EMPTY
+    K1 = synth.kv_tokens(seed, 0, 1, B, 0, P, Hkv, D, "bf16")
+    V1 = synth.kv_tokens(seed, 1, 1, B, 0, P, Hkv, D, "bf16")
+    F1 = synth.flag_tokens(seed, 1, B, 0, P, Hkv, thr)
+    pool.compact_prefill(1, _dev(K1), _dev(V1), torch.from_numpy(np.ascontiguousarray(F1)).cuda())
+    state = read_state(pool)
+    for layer, (Kx, Vx, Fx) in enumerate(((K, V, F), (K1, V1, F1))):
+        scales = [(ofp8.fp8_scale(np.abs(Kx[:, :, h]).max()), ofp8.fp8_scale(np.abs(Vx[:, :, h]).max()))
+                  for h in range(Hkv)]
+        for h in range(Hkv):
+            assert state["scales"][layer, h, 0] == scales[h][0] and state["scales"][layer, h, 1] == scales[h][1]
+            for b in range(B):
+                store = oracle_store(Fx[b, :, h], np.zeros(0, np.uint8), w, P)
+                check_head_store(pool, state, head_id(pool.cfg, layer, b, h), store,
+                                 {j: Kx[b, j, h] for j in range(P)}, {j: Vx[b, j, h] for j in range(P)},
+                                 "fp8", scales[h])
+    check_block_invariants(pool, state)
