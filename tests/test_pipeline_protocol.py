@@ -18,8 +18,8 @@ import random
 import pytest
 
 # (stages, consumer warps) of each kernel variant: bf16 D=128, bf16 D=64,
-# FP8 D=128, fp32 D=64, fp32 D=128
-KERNEL_LAYOUTS = [(6, 6), (8, 8), (8, 8), (4, 4), (3, 3)]
+# FP8 D=128, 4-bit D=128, fp32 D=64, fp32 D=128
+KERNEL_LAYOUTS = [(6, 6), (8, 8), (12, 6), (14, 7), (4, 4), (3, 3)]
 
 
 class MBarrier:
