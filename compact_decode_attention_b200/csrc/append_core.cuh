@@ -109,9 +109,12 @@ __device__ __forceinline__ uint32_t int4_nibble(float x, float scale) {
 // One token's K and V rows into a 4-bit store (one warp): lane l holds
 // elements 4l .. 4l+3 of each row (values in input precision).  K words and
 // scales are written whole; V nibbles share 32-bit words with 7 other tokens
-// of the block, so they are cleared and set with atomics.
+// of the block, so they are cleared and set with atomics -- or, with
+// s_vwords (a zeroed shared-memory image of the block's 1024 V nibble words),
+// OR-ed into that image for the caller to write out.
 __device__ __forceinline__ void store_row_int4(const PoolView& v, int prow, const float (&k4)[4],
-                                               const float (&v4)[4], int lane) {
+                                               const float (&v4)[4], int lane,
+                                               uint32_t* s_vwords = nullptr) {
   const int row = prow % v.BT;
   uint8_t* blk = v.blocks + int64_t(prow / v.BT) * v.block_bytes;
   uint8_t* vt = blk + v.tile_bytes;
@@ -149,9 +152,13 @@ __device__ __forceinline__ void store_row_int4(const PoolView& v, int prow, cons
   const int sh = int4v_shift(row);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    uint32_t* w = reinterpret_cast<uint32_t*>(vt + int4v_word(4 * lane + i, row));
-    atomicAnd(w, ~(0xFu << sh));
-    atomicOr(w, int4_nibble(v4[i], vs) << sh);
+    if (s_vwords) {
+      atomicOr(s_vwords + (int4v_word(4 * lane + i, row) >> 2), int4_nibble(v4[i], vs) << sh);
+    } else {
+      uint32_t* w = reinterpret_cast<uint32_t*>(vt + int4v_word(4 * lane + i, row));
+      atomicAnd(w, ~(0xFu << sh));
+      atomicOr(w, int4_nibble(v4[i], vs) << sh);
+    }
   }
 }
 

@@ -325,6 +325,8 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
   constexpr int kBatchItems = 4;          // 16-byte copies in flight per thread
   __shared__ int s_kept[SPAN];            // chunk-local token index of each kept rank
   __shared__ int s_wcnt[8];
+  // 4-bit store: V nibble words of the blocks the span's slots touch
+  __shared__ uint32_t s_vw[STORE == 2 ? SPAN / 64 + 1 : 1][STORE == 2 ? kInt4Nibbles / 4 : 1];
   const int chunk = blockIdx.x / kPieces, piece = blockIdx.x % kPieces;
   const int h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -423,12 +425,48 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
     v.ring_row[ri] = table[slot / v.BT] * v.BT + slot % v.BT;
   }
   if constexpr (STORE == 2) {
+    // V nibbles: the span's slots [base, base + nkept) touch at most
+    // SPAN / 64 + 1 blocks; their nibble words are built in shared memory
+    // and written once each -- whole when every token of the word is this
+    // CTA's, else with an AND / OR of this CTA's nibbles (neighbouring spans
+    // own the other tokens).  In the head's last block the rows past the last
+    // slot count as this CTA's (zero nibbles) when it holds the last token.
+    constexpr int kWords = kInt4Nibbles / 4;           // V nibble words of a block (D = 128)
+    const int kb0 = base / v.BT;
+    const int nbt = nkept > 0 ? (base + nkept - 1) / v.BT - kb0 + 1 : 0;
+    for (int i = threadIdx.x; i < nbt * kWords; i += blockDim.x) s_vw[i / kWords][i % kWords] = 0;
+    __syncthreads();
     for (int kk = warp; kk < nkept; kk += blockDim.x / 32) {
       if (kk != warp) load_int4(kk);
       const int slot = base + kk;
       const int blk = table[slot / v.BT];
       if (!DMS_CHECK(blk >= 0 && blk < v.max_blocks, v.hdr, 202, hd, slot)) continue;
-      store_row_int4(v, blk * v.BT + slot % v.BT, k4, v4, lane);
+      store_row_int4(v, blk * v.BT + slot % v.BT, k4, v4, lane, s_vw[slot / v.BT - kb0]);
+    }
+    __syncthreads();
+    const bool holds_last = int(blockIdx.x) == (P - 1) / SPAN;
+    for (int i = threadIdx.x; i < nbt * kWords; i += blockDim.x) {
+      const int kb = kb0 + i / kWords, d = (i % kWords) >> 3, wi = i & 7;
+      const int lo = max(base, kb * v.BT) - kb * v.BT;
+      const int hi = holds_last && kb == (base + nkept - 1) / v.BT ? v.BT - 1
+                                                                  : min(base + nkept, (kb + 1) * v.BT) - 1 - kb * v.BT;
+      uint32_t mask = 0;   // word wi of element row d: tokens 32 (wi & 1) + 16 e2 + 8 e1 + 2 (wi >> 1) + e0
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int t = (wi & 1) * 32 + ((e >> 2) & 1) * 16 + ((e >> 1) & 1) * 8 + (wi >> 1) * 2 + (e & 1);
+        if (t >= lo && t <= hi) mask |= 0xFu << int4v_shift(t);
+      }
+      const int blk = table[kb];
+      if (mask == 0 || !DMS_CHECK(blk >= 0 && blk < v.max_blocks, v.hdr, 204, hd, kb)) continue;
+      uint32_t* w = reinterpret_cast<uint32_t*>(v.blocks + int64_t(blk) * v.block_bytes + v.tile_bytes +
+                                                int4v_word(d, (wi & 1) * 32 + (wi >> 1) * 2));
+      const uint32_t x = s_vw[i / kWords][i % kWords];
+      if (mask == 0xFFFFFFFFu) {
+        *w = x;
+      } else {
+        atomicAnd(w, ~mask);
+        if (x) atomicOr(w, x);
+      }
     }
   } else if constexpr (STORE == 0) {
     // bitwise row copy, 16-byte chunks swizzled by row
@@ -483,20 +521,7 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
         if constexpr (STORE == 1) {
           for (int i = threadIdx.x; i < (v.BT - r0) * v.D; i += blockDim.x)
             vt[fp8v_byte(r0 + i / v.D, i % v.D)] = 0;
-        } else {
-          // word wi of element row d holds the nibbles of the 8 tokens
-          // t = 32 (wi & 1) + 16 e2 + 8 e1 + 2 (wi >> 1) + e0; other CTAs
-          // set the nibbles of rows < r0 with atomics, so clear with one too
-          for (int i = threadIdx.x; i < v.D * 8; i += blockDim.x) {
-            const int d = i >> 3, wi = i & 7;
-            uint32_t mask = 0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int t = (wi & 1) * 32 + ((e >> 2) & 1) * 16 + ((e >> 1) & 1) * 8 + (wi >> 1) * 2 + (e & 1);
-              if (t >= r0) mask |= 0xFu << int4v_shift(t);
-            }
-            if (mask) atomicAnd(reinterpret_cast<uint32_t*>(vt + int4v_word(d, (wi & 1) * 32 + (wi >> 1) * 2)), ~mask);
-          }
+        } else {   // 4-bit: the nibbles of those rows were written as zeros above
           for (int i = threadIdx.x; i < (v.BT - r0) * (v.D / 32); i += blockDim.x)
             *reinterpret_cast<__half*>(vt + int4v_scale(r0 + i / (v.D / 32), i % (v.D / 32))) = __float2half_rn(0.f);
         }
