@@ -334,7 +334,43 @@ def cpu_baseline(wl, t0: int, n_heads: int, n_steps: int, bytes_per_step: float)
                    f"t={t0}: slot bookkeeping + fp64 masked attention per head, {elapsed:.1f} s; "
                    f"per-step time = mean head-step time x {H} heads"),
         "seconds": elapsed, "step_seconds_extrapolated": step_time,
+        "compaction": oracle_compaction(wl, picks[:4 if wl.prompt <= 32768 else 1]),
     }
+
+
+def oracle_compaction(wl, picks):
+    """Time the oracle's prefill compaction (one thread) of the given heads:
+    kept positions, slots and window ring, the kept K/V rows gathered (FP8:
+    the head's maximum over its prompt rows and the kept rows quantised);
+    scaled to a layer by its head count."""
+    from oracle import compaction as ocomp
+    from oracle import fp8 as ofp8
+    from oracle import reference as oref
+    prep = []
+    for (layer, b, h) in picks:          # untimed: the head's inputs
+        prep.append((oref.head_flags(wl, layer, b, h, wl.prompt),
+                     oref.head_input(wl, 0, layer, b, h, 0, wl.prompt),
+                     oref.head_input(wl, 1, layer, b, h, 0, wl.prompt)))
+    in_row = 2 * wl.head_dim * (4 if wl.in_dtype == "f32" else 2)
+    nbytes = 0
+    start = time.perf_counter()
+    for flags, K, V in prep:
+        kept = ocomp.prefill_kept_positions(flags, wl.window)
+        ocomp.prefill_slots(flags, wl.window)
+        ocomp.prefill_ring(flags, wl.window)
+        Kc, Vc = K[kept], V[kept]
+        if wl.kv_dtype == "fp8":
+            ofp8.quantize(Kc, ofp8.fp8_scale(np.abs(K).max()))
+            ofp8.quantize(Vc, ofp8.fp8_scale(np.abs(V).max()))
+            nbytes += wl.prompt * in_row
+        nbytes += wl.prompt + len(kept) * (in_row + 2 * wl.kv_row_bytes())
+    elapsed = time.perf_counter() - start
+    heads_per_layer = wl.batch * wl.n_kv_heads
+    per_head = elapsed / max(1, len(prep))
+    return {"ms_per_layer": per_head * heads_per_layer * 1e3,
+            "value": nbytes / elapsed / 1e9 if elapsed > 0 else None, "unit": "GB/s", "cores": 1,
+            "sample": (f"{len(prep)} (sequence, kv-head) prompts of {wl.prompt} tokens, {elapsed:.2f} s; "
+                       f"per-layer time = mean head time x {heads_per_layer} heads")}
 
 
 def oracle_visible(t, flags, w):
@@ -417,7 +453,7 @@ def run_reference(args):
         "ms_per_step": cb["step_seconds_extrapolated"] * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "bytes_per_step": bps},
-        "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "compaction")},
         "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "note": ("the reference arm is the CPU oracle (the pages ship no code); each step is a bounded "
                  "sample of the workload's decode step, extrapolated by head count"),
@@ -680,7 +716,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, P + W, args.cpu_heads, args.cpu_steps, float(bytes_step[W]))
-        cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample", "compaction")}
 
     if rank == 0:
         line = {

@@ -103,3 +103,4 @@ def test_reference_arm_prints_one_line():
     assert r.returncode == 0, r.stderr
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["compaction"]["ms_per_layer"] > 0
