@@ -300,6 +300,10 @@ def cpu_baseline(wl, t0: int, n_heads: int, n_steps: int, bytes_per_step: float)
         b = int((i // wl.n_kv_heads) % wl.batch)
         layer = int(i // (wl.n_kv_heads * wl.batch))
         picks.append((layer, b, h))
+    if wl.keep == "heavy_tail":
+        # the sample always holds two keep-all heads (they dominate the bytes)
+        full = [(int(l), 0, int(h)) for l, h in np.argwhere(wl.keep_probs() >= 1.0)[:2]]
+        picks = full + [p for p in picks if p not in full][:max(0, len(picks) - len(full))]
     # untimed: inputs of each sampled head (flags, the rows it may see, queries)
     prep = []
     for (layer, b, h) in picks:
