@@ -35,5 +35,9 @@ Modules:
 
 Every function here is pinned by a ``-m "not gpu"`` test against something
 other than itself (closed forms, library routines, brute force, page
-figures); none is "parity unpinned".
+figures): the per-head glue of ``reference`` (flags, inputs, query rows,
+FP8 scales, stored rows, expected outputs) against whole tensors drawn from
+the generator, torch's fp64 scaled_dot_product_attention under the
+operational eviction mask and torch's float8 cast, for every (layer,
+sequence, kv-head) of a small workload; none is "parity unpinned".
 """

@@ -479,3 +479,125 @@ def test_oracle_and_product_do_not_import_each_other():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
+
+
+# ---------------------------------------------------------------------------
+# per-head glue of oracle/reference.py, against whole tensors drawn from the
+# generator and library routines (torch SDPA, torch's float8 cast)
+# ---------------------------------------------------------------------------
+
+def _glue_workload(kv_dtype="bf16", in_dtype="bf16", head_dim=16):
+    """Three layers, batch 3, GQA 4 and a keep probability drawn per
+    (layer, kv-head), so a slip in the layer / sequence / head indexing of
+    the glue picks other draws."""
+    return configs.Workload("glue_pin", 3, 3, 12, 3, head_dim, 90, 8, 20, kv_dtype, in_dtype, 17,
+                            "uniform", extra={"lo": 0.05, "hi": 0.9})
+
+
+def _torch_fp8_store(x, scale):
+    """Stored values of an FP8 store via torch: e4m3fn(x / scale) * scale, the
+    quotient in fp32, saturated to +-448 before the cast (torch's cast gives
+    NaN above 464; decode tokens may exceed the prompt's amax)."""
+    y = torch.from_numpy(np.asarray(x, np.float32)) / torch.tensor(scale, dtype=torch.float32)
+    y = torch.clamp(y, -448.0, 448.0)
+    return y.to(torch.float8_e4m3fn).to(torch.float64).numpy() * np.float64(scale)
+
+
+def test_glue_inputs_are_the_workload_tensors():
+    """head_flags / head_input / head_query return slices of the whole-tensor
+    draws of the same workload: (layer, sequence, kv-head) in the right
+    places, the query rows of kv-head h being query heads h*g .. h*g+g-1."""
+    wl = _glue_workload()
+    thr = wl.thresholds()
+    assert len(np.unique(thr)) == thr.size          # every (layer, head) draws its own rate
+    n = 50
+    for layer in range(wl.n_layers):
+        K = synth.kv_tokens(wl.seed, 0, layer, wl.batch, 0, n, wl.n_kv_heads, wl.head_dim, "bf16")
+        V = synth.kv_tokens(wl.seed, 1, layer, wl.batch, 0, n, wl.n_kv_heads, wl.head_dim, "bf16")
+        F = synth.flag_tokens(wl.seed, layer, wl.batch, 0, n, wl.n_kv_heads, thr[layer])
+        Q = synth.q_tokens(wl.seed, layer, wl.batch, 37, wl.n_q_heads, wl.head_dim, "bf16")
+        for b in range(wl.batch):
+            for h in range(wl.n_kv_heads):
+                assert np.array_equal(reference.head_flags(wl, layer, b, h, n), F[b, :, h])
+                assert np.array_equal(reference.head_input(wl, 0, layer, b, h, 5, 20), K[b, 5:25, h])
+                assert np.array_equal(reference.head_input(wl, 1, layer, b, h, 0, n), V[b, :, h])
+                g = wl.group
+                assert np.array_equal(reference.head_query(wl, layer, b, h, 37), Q[b, h * g:(h + 1) * g])
+
+
+def test_glue_fp8_scales_are_amax_over_every_sequence_and_prompt_row():
+    """fp8_head_scales = amax / 448 over all batch rows and all prompt
+    positions of the (layer, kv-head), before eviction; the decode tokens
+    after the prompt do not count.  A small chunk size makes the amax loop
+    cross chunk and sequence boundaries."""
+    wl = _glue_workload("fp8")
+    for layer in range(wl.n_layers):
+        K = synth.kv_tokens(wl.seed, 0, layer, wl.batch, 0, wl.prompt, wl.n_kv_heads, wl.head_dim, "bf16")
+        V = synth.kv_tokens(wl.seed, 1, layer, wl.batch, 0, wl.prompt, wl.n_kv_heads, wl.head_dim, "bf16")
+        for h in range(wl.n_kv_heads):
+            sk, sv = reference.fp8_head_scales(wl, layer, h, chunk=7)
+            want_k = (torch.from_numpy(K[:, :, h]).abs().max() / 448.0).item()
+            want_v = (torch.from_numpy(V[:, :, h]).abs().max() / 448.0).item()
+            assert sk == np.float32(want_k) and sv == np.float32(want_v), (layer, h)
+            # one sequence, or the rows after the prompt, give another amax
+            one = np.float32(np.abs(K[0, :, h]).max() / np.float32(448))
+            assert any(np.float32(np.abs(K[b, :, h]).max() / np.float32(448)) != sk
+                       for b in range(wl.batch)) or one == sk
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8", "f32"])
+def test_glue_expected_output_matches_sdpa_on_workload_tensors(kv_dtype):
+    """expected_output for every (layer, sequence, kv-head) at a few decode
+    positions equals torch's fp64 SDPA over the whole tensors of the
+    workload, masked by the operational model of delayed eviction, with the
+    store's values formed by torch (bf16 / fp32 inputs as drawn; FP8 through
+    torch's e4m3fn cast with scales from torch's amax)."""
+    in_dtype = "f32" if kv_dtype == "f32" else "bf16"
+    wl = _glue_workload(kv_dtype, in_dtype)
+    g, D, w = wl.group, wl.head_dim, wl.window
+    thr = wl.thresholds()
+    for layer in range(wl.n_layers):
+        T = wl.prompt + wl.decode
+        K = synth.kv_tokens(wl.seed, 0, layer, wl.batch, 0, T, wl.n_kv_heads, D, in_dtype)
+        V = synth.kv_tokens(wl.seed, 1, layer, wl.batch, 0, T, wl.n_kv_heads, D, in_dtype)
+        F = synth.flag_tokens(wl.seed, layer, wl.batch, 0, T, wl.n_kv_heads, thr[layer])
+        scales = {}
+        Ks, Vs = K.astype(np.float64), V.astype(np.float64)
+        if kv_dtype == "fp8":
+            for h in range(wl.n_kv_heads):
+                sk = np.float32((torch.from_numpy(K[:, :wl.prompt, h]).abs().max() / 448.0).item())
+                sv = np.float32((torch.from_numpy(V[:, :wl.prompt, h]).abs().max() / 448.0).item())
+                scales[h] = (sk, sv)
+                Ks[:, :, h] = _torch_fp8_store(K[:, :, h], sk)
+                Vs[:, :, h] = _torch_fp8_store(V[:, :, h], sv)
+        for t in (wl.prompt, wl.prompt + 3, T - 1):
+            Q = synth.q_tokens(wl.seed, layer, wl.batch, t, wl.n_q_heads, D, in_dtype)
+            for b in range(wl.batch):
+                m = np.zeros((wl.n_kv_heads, t + 1), dtype=bool)
+                for h in range(wl.n_kv_heads):
+                    m[h, operational_cache_sets(F[b, :t + 1, h], w)[t]] = True
+                ref = sdpa(Q[b], Ks[b, :t + 1], Vs[b, :t + 1], 1.0 / np.sqrt(D), m)
+                for h in range(wl.n_kv_heads):
+                    got = reference.expected_output(wl, layer, b, h, t, scales=scales.get(h))
+                    np.testing.assert_allclose(got, ref[h * g:(h + 1) * g], rtol=0, atol=1e-12,
+                                               err_msg=f"{kv_dtype} layer {layer} seq {b} head {h} t {t}")
+
+
+def test_glue_stored_rows_of_a_4bit_store_are_the_group_quantised_rows():
+    """stored_rows of a 4-bit workload: each row is its own group-scaled
+    4-bit rounding (brute force per element: the nearest multiple of the
+    group's fp16 scale among -7..7)."""
+    wl = _glue_workload("int4", head_dim=64)
+    pos = np.array([0, 3, 40, 89])
+    Kr, Vr = reference.stored_rows(wl, 1, 2, 1, pos)
+    for stream, got in ((0, Kr), (1, Vr)):
+        x = reference.head_input(wl, stream, 1, 2, 1, 0, wl.prompt)[pos]
+        for i in range(len(pos)):
+            for gq in range(wl.head_dim // 32):
+                grp = x[i, 32 * gq:32 * gq + 32]
+                s = np.float64(np.float16(np.float32(np.abs(grp).max()) / np.float32(7)))
+                cand = np.arange(-7, 8) * s
+                for d in range(32):
+                    err = np.abs(cand - grp[d])
+                    assert np.isclose(got[i, 32 * gq + d], cand[err.argmin()], rtol=0, atol=1e-12) or \
+                        np.sum(err == err.min()) > 1
