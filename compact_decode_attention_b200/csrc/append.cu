@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kAppendThreads)
   pdl_wait_prerequisites();
   pdl_launch_dependents();
   if (sync.ready) {  // the step's inputs are copied in by another stream
-    if (threadIdx.x == 0 && !wait_counter_geq(sync.ready, sync.ready_value))
+    if (threadIdx.x == 0 && !wait_counter_geq(sync.ready, sync.ready_value, v.wait_ns))
       report_error(v.hdr, DMS_DEVERR_TIMEOUT, l0, -1, -1);
     __syncthreads();
   }

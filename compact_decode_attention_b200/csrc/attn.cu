@@ -32,7 +32,8 @@
 // f16 in registers (exact) from a layout that gives each lane its fragment
 // bytes in two 16-byte loads; fp32 rows use CUDA-core FMA.
 //
-// Every wait is bounded (1 s); a timeout sets DMS_DEVERR_TIMEOUT and the CTA
+// Every wait is bounded (the pool's wait limit, 1 s unless set); a timeout
+// sets DMS_DEVERR_TIMEOUT and the CTA
 // drains its in-flight copies and returns.
 #include <math.h>
 
@@ -701,7 +702,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   pdl_wait_prerequisites();
   // stepper: the output buffer's previous copy-out must be done (thread 0;
   // the scan's barrier below holds the other threads)
-  if (p.sync.drained && tid == 0 && !wait_counter_geq(p.sync.drained, p.sync.drained_value))
+  if (p.sync.drained && tid == 0 && !wait_counter_geq(p.sync.drained, p.sync.drained_value, v.wait_ns))
     report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
   // stepper: the last CTA to leave publishes the step as computed
   auto sync_exit = [&]() {
@@ -810,7 +811,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
                            ji >= 0 && ji < Htot, v.hdr, 302, jblk, jrows)) {
           aborted = true;
           *s_abort = 1;
-        } else if (!mbar_wait_bounded(&empty[s], ph ^ 1, s_abort) || *s_abort) {
+        } else if (!mbar_wait_bounded(&empty[s], ph ^ 1, s_abort, v.wait_ns) || *s_abort) {
           aborted = true;
           if (!*s_abort) report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
           *s_abort = 1;
@@ -891,7 +892,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     if (lane == 0) {
       volatile int never = 0;
       for (int kk = max(0, issued - T::NS); kk < issued; ++kk)
-        mbar_wait_bounded(&full[kk % T::NS], (kk / T::NS) & 1, &never);
+        mbar_wait_bounded(&full[kk % T::NS], (kk / T::NS) & 1, &never, v.wait_ns);
     }
     return;
   }
@@ -995,7 +996,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     }
     bool ok = false;
     if (!*s_abort) {
-      ok = mbar_wait_bounded(&full[s], ph, s_abort);
+      ok = mbar_wait_bounded(&full[s], ph, s_abort, v.wait_ns);
       if (!ok && lane == 0) {
         *s_abort = 1;
         report_error(v.hdr, DMS_DEVERR_TIMEOUT, p.l0, -1, c);
@@ -1059,15 +1060,11 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
 template <int KV, int D>
 static dms_status launch_attn(const AttnParams& prm, cudaStream_t stream) {
   using T = AttnTraits<KV, D>;
-  static bool attr_set = false;  // per instantiation; set once per process
-  if (!attr_set) {
-    dms_status st = cuda_status(cudaFuncSetAttribute(decode_attn_kernel<KV, D>,
-                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                      int(T::SMEM)),
-                                "attn smem attribute");
-    if (st != DMS_OK) return st;
-    attr_set = true;
-  }
+  static FuncAttrCache smem_attr;  // per instantiation, per device
+  dms_status st = ensure_func_attr(reinterpret_cast<const void*>(decode_attn_kernel<KV, D>),
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, int(T::SMEM),
+                                   smem_attr, "attn smem attribute");
+  if (st != DMS_OK) return st;
   return cuda_status(launch_pdl(decode_attn_kernel<KV, D>, dim3(prm.G), dim3(T::THREADS), T::SMEM,
                                 stream, prm),
                      "decode_attn_kernel");
@@ -1210,12 +1207,14 @@ extern "C" dms_status dms_decode_attn(dms_pool* pool, int layer, int batch, cons
 // hand the array's name to a kernel (in host code it names a host-side
 // stand-in, not device memory), so the first call on each device looks up
 // its device address with cudaGetSymbolAddress while that device is current
-// and caches it; make that first call before any stream capture.  Every call
+// and caches it with the context it belongs to; make that first call (and
+// the first after a device reset) before any stream capture.  Every call
 // on a device shares the one array, which keeps the previous call's partial
 // results: nothing in it has to start at zero (each launch writes every
 // partial it later reads, and the merge tickets live in the pool), but calls
 // whose kernels overlap on the GPU race on it and must be ordered.
 // ---------------------------------------------------------------------------
+#include <cuda.h>
 #include <mutex>
 
 namespace dms {
@@ -1225,24 +1224,55 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
+// The address is looked up once per device and context: a device reset
+// (cudaDeviceReset, or a caller that makes another driver context current)
+// gives the array a new address in the new context, so the cache remembers
+// which context its address belongs to and looks it up again when the
+// current context differs.
+struct StaticWsEntry {
+  CUcontext ctx;
+  void* addr;
+};
 static std::mutex g_static_ws_mutex;
-static void* g_static_ws_addr[kMaxDevices] = {};
+static StaticWsEntry g_static_ws[kMaxDevices] = {};
 
-// Device address of g_static_workspace on the current device (looked up once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+static CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
+
+// Device address of g_static_workspace on the current device (set-up on
+// the first call in a device's context; cudaGetSymbolAddress runs there).
 static dms_status static_workspace_address(int device, void** addr) {
   if (device < 0 || device >= kMaxDevices) {
     set_last_error("device %d out of range for the fixed workspace table", device);
     return DMS_ERR_UNSUPPORTED;
   }
+  CUcontext ctx = nullptr;
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  if (!get || get(&ctx) != CUDA_SUCCESS) {
+    set_last_error("cuCtxGetCurrent is not available");
+    return DMS_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-  if (!g_static_ws_addr[device]) {
+  StaticWsEntry& e = g_static_ws[device];
+  if (!e.addr || e.ctx != ctx) {
     void* p = nullptr;
     dms_status st = cuda_status(cudaGetSymbolAddress(&p, g_static_workspace),
                                 "cudaGetSymbolAddress(g_static_workspace)");
     if (st != DMS_OK) return st;
-    g_static_ws_addr[device] = p;
+    e.ctx = ctx;
+    e.addr = p;
   }
-  *addr = g_static_ws_addr[device];
+  *addr = e.addr;
   return DMS_OK;
 }
 

@@ -7,6 +7,7 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 #include "dms.h"
@@ -16,7 +17,7 @@ namespace dms {
 constexpr int kBlockTokens = 64;     // BT: rows per physical block
 constexpr int kFreeStackCap = 4;     // per-head free slots awaiting reuse
 constexpr int kPrefillChunk = 256;   // prompt tokens per compaction CTA
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // every device wait gives up after 1 s
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // default limit of every device wait: 1 s
 
 // Device-side header at the start of the pool buffer.
 struct DevHeader {
@@ -38,6 +39,7 @@ struct PoolView {
   int32_t n_heads;
   int32_t n_chunks_max;     // prefill scratch: chunks per (b, h)
   int64_t max_blocks;
+  uint64_t wait_ns;         // limit of every bounded device wait (dms_pool_set_wait_limit)
   int64_t row_bytes;        // D * elem size
   int64_t tile_bytes;       // BT * row_bytes
   int64_t block_bytes;      // 2 * tile_bytes
@@ -175,16 +177,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase of `parity` to complete; gives up after kWaitLimitNs or
+// Wait for the phase of `parity` to complete; gives up after limit_ns or
 // when *abort becomes non-zero.  Returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort) {
+                                                  volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -210,12 +212,12 @@ __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
 __device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
   asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-// Wait (one thread) until *p >= v; false after kWaitLimitNs.
-__device__ __forceinline__ bool wait_counter_geq(const int32_t* p, int32_t v) {
+// Wait (one thread) until *p >= v; false after limit_ns.
+__device__ __forceinline__ bool wait_counter_geq(const int32_t* p, int32_t v, uint64_t limit_ns) {
   if (ld_acquire_gpu(p) >= v) return true;
   const uint64_t t0 = globaltimer_ns();
   while (ld_acquire_gpu(p) < v) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
     __nanosleep(200);
   }
   return true;
@@ -362,6 +364,17 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 dms_status cuda_status(cudaError_t e, const char* what);
 int device_sm_count(int device);
+// A kernel attribute (cudaFuncSetAttribute) takes effect on the current
+// device only, so it is set once per device: the cache remembers, per
+// device ordinal, the largest value set so far (a static object, zeroed at
+// load).  Two threads making their first call at once both set it, which is
+// harmless.  Devices past the table are set on every call.
+constexpr int kAttrDevices = 64;
+struct FuncAttrCache {
+  std::atomic<int> value[kAttrDevices];
+};
+dms_status ensure_func_attr(const void* func, cudaFuncAttribute attr, int value,
+                            FuncAttrCache& cache, const char* what);
 }  // namespace dms
 struct dms_pool;
 namespace dms {

@@ -33,6 +33,21 @@ dms_status cuda_status(cudaError_t e, const char* what) {
   return DMS_ERR_CUDA;
 }
 
+dms_status ensure_func_attr(const void* func, cudaFuncAttribute attr, int value,
+                            FuncAttrCache& cache, const char* what) {
+  int dev = -1;
+  dms_status st = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != DMS_OK) return st;
+  const bool cached = dev >= 0 && dev < kAttrDevices;
+  if (cached && cache.value[dev].load(std::memory_order_acquire) >= value) return DMS_OK;
+  st = cuda_status(cudaFuncSetAttribute(func, attr, value), what);
+  if (st != DMS_OK || !cached) return st;
+  int old = cache.value[dev].load(std::memory_order_relaxed);
+  while (old < value && !cache.value[dev].compare_exchange_weak(old, value, std::memory_order_release))
+    ;
+  return DMS_OK;
+}
+
 int device_sm_count(int device) {
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return 0;
@@ -147,6 +162,7 @@ static PoolView make_view(const dms_pool_config& c, const dms_pool_layout_t& lay
   v.n_heads = lay.n_heads;
   v.n_chunks_max = int32_t((c.max_context + kPrefillChunk - 1) / kPrefillChunk);
   v.max_blocks = c.max_blocks;
+  v.wait_ns = kWaitLimitNs;
   v.row_bytes = lay.row_bytes;
   v.tile_bytes = kBlockTokens * lay.row_bytes;
   v.block_bytes = lay.block_bytes;
@@ -350,6 +366,16 @@ dms_status dms_pool_reset(dms_pool* pool, cudaStream_t stream) {
     return DMS_ERR_INVALID_ARG;
   }
   return clear_pool(pool, stream);
+}
+
+dms_status dms_pool_set_wait_limit(dms_pool* pool, uint64_t limit_ns) {
+  if (!pool || limit_ns < 1000 || limit_ns > 60000000000ull) {
+    set_last_error("wait limit must be between 1 us and 60 s (got %llu ns)",
+                   (unsigned long long)limit_ns);
+    return DMS_ERR_INVALID_ARG;
+  }
+  pool->view.wait_ns = limit_ns;
+  return DMS_OK;
 }
 
 dms_status dms_pool_layout(const dms_pool* pool, dms_pool_layout_t* out) {

@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
   for (int kt = 0; kt <= qt; ++kt) {
     const int cur = kt & 1, j0 = kt * kPaTile;
     if (kt > 0) {  // P V of tile kt-1 is done: P and the tile buffer are free
-      ok &= mbar_wait_bounded(bar_o, (kt - 1) & 1, &never);
+      ok &= mbar_wait_bounded(bar_o, (kt - 1) & 1, &never, v.wait_ns);
       __syncwarp();
       umma::fence_after_sync();
       if (tid == 0) load_tile(smem + S::KV, &tk, hkv * D, j0, bar_k);
@@ -161,8 +161,8 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
       if (lane == 0 && h == 0) s_fbits[cur * 4 + warp] = fw;
     }
     const uint8_t f_next = kt < qt ? flag_of(kt + 1) : 0;
-    if (kt == 0) ok &= mbar_wait_bounded(bar_q, 0, &never);
-    ok &= mbar_wait_bounded(bar_k, kt & 1, &never);  // K_kt landed
+    if (kt == 0) ok &= mbar_wait_bounded(bar_q, 0, &never, v.wait_ns);
+    ok &= mbar_wait_bounded(bar_k, kt & 1, &never, v.wait_ns);  // K_kt landed
     __syncwarp();
     __syncthreads();
     const uint32_t aK = smem_u32(smem + S::KV), aV = aK;
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
                        k0 > 0);
       umma::commit(bar_s);
     }
-    ok &= mbar_wait_bounded(bar_s, kt & 1, &never);
+    ok &= mbar_wait_bounded(bar_s, kt & 1, &never, v.wait_ns);
     __syncwarp();  // lanes leave the wait loop independently; tcgen05.ld is warp-collective
     umma::fence_after_sync();
     // S read the keys: the values of the same tile stream into the buffer
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     __syncthreads();
     if (tid == 0) {
       umma::fence_after_sync();
-      ok &= mbar_wait_bounded(bar_v, kt & 1, &never);  // V_kt landed
+      ok &= mbar_wait_bounded(bar_v, kt & 1, &never, v.wait_ns);  // V_kt landed
 #pragma unroll
       for (int k0 = 0; k0 < kPaTile; k0 += 16)
         umma::mma_bf16(t_o, umma::desc_k16(aP, kPaTile, k0), umma::desc_mn_k16(aV, kPaTile, k0), idO,
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     }
     __syncwarp();
   }
-  ok &= mbar_wait_bounded(bar_o, qt & 1, &never);
+  ok &= mbar_wait_bounded(bar_o, qt & 1, &never, v.wait_ns);
   __syncwarp();
   umma::fence_after_sync();
 
@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
         v.ring_row[ri] = table[slot / v.BT] * v.BT + slot % v.BT;
       }
     }
-    ok &= mbar_wait_bounded(bar_q, 1, &never);  // K rows of the diagonal tile
+    ok &= mbar_wait_bounded(bar_q, 1, &never, v.wait_ns);  // K rows of the diagonal tile
     __syncwarp();
     __syncthreads();
     constexpr int CH = D / 8;
@@ -463,31 +463,29 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
   if (st != DMS_OK) return st;
   auto ko = static_cast<__nv_bfloat16*>(out);
   if (pv.D == 128) {
-    static bool attr = false;
-    if (!attr) {
-      st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            PaSmem<128>::BYTES), "prefill attn smem attribute");
-      if (st != DMS_OK) return st;
-      // two CTAs per SM: the whole shared-memory carveout
-      st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                            int(cudaSharedmemCarveoutMaxShared)), "prefill attn carveout");
-      if (st != DMS_OK) return st;
-      attr = true;
-    }
+    static FuncAttrCache smem_attr, carveout_attr;  // per device
+    st = ensure_func_attr(reinterpret_cast<const void*>(prefill_attn_kernel<128>),
+                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(PaSmem<128>::BYTES), smem_attr,
+                          "prefill attn smem attribute");
+    if (st != DMS_OK) return st;
+    // two CTAs per SM: the whole shared-memory carveout
+    st = ensure_func_attr(reinterpret_cast<const void*>(prefill_attn_kernel<128>),
+                          cudaFuncAttributePreferredSharedMemoryCarveout, int(cudaSharedmemCarveoutMaxShared),
+                          carveout_attr, "prefill attn carveout");
+    if (st != DMS_OK) return st;
     prefill_attn_kernel<128><<<grid, PaSplit<128>::THREADS, PaSmem<128>::BYTES, stream>>>(
         pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, fused);
   } else {
-    static bool attr = false;
-    if (!attr) {
-      st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            PaSmem<64>::BYTES), "prefill attn smem attribute");
-      if (st != DMS_OK) return st;
-      // two CTAs per SM: the whole shared-memory carveout
-      st = cuda_status(cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                            int(cudaSharedmemCarveoutMaxShared)), "prefill attn carveout");
-      if (st != DMS_OK) return st;
-      attr = true;
-    }
+    static FuncAttrCache smem_attr, carveout_attr;  // per device
+    st = ensure_func_attr(reinterpret_cast<const void*>(prefill_attn_kernel<64>),
+                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(PaSmem<64>::BYTES), smem_attr,
+                          "prefill attn smem attribute");
+    if (st != DMS_OK) return st;
+    // two CTAs per SM: the whole shared-memory carveout
+    st = ensure_func_attr(reinterpret_cast<const void*>(prefill_attn_kernel<64>),
+                          cudaFuncAttributePreferredSharedMemoryCarveout, int(cudaSharedmemCarveoutMaxShared),
+                          carveout_attr, "prefill attn carveout");
+    if (st != DMS_OK) return st;
     prefill_attn_kernel<64><<<grid, PaSplit<64>::THREADS, PaSmem<64>::BYTES, stream>>>(
         pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, fused);
   }

@@ -188,14 +188,11 @@ static dms_status launch_projection(const PoolView& v, int layer, const int32_t*
     set_last_error("d_model %d too large for the projection's shared memory", dm);
     return DMS_ERR_UNSUPPORTED;
   }
-  static size_t attr = 0;   // per instantiation: the largest size set so far
-  if (smem > attr) {
-    dms_status st = cuda_status(cudaFuncSetAttribute(project_append_kernel<128, S>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)),
-                                "projection smem attribute");
-    if (st != DMS_OK) return st;
-    attr = smem;
-  }
+  static FuncAttrCache smem_attr;   // per instantiation and device: the largest size set so far
+  dms_status ast = ensure_func_attr(reinterpret_cast<const void*>(project_append_kernel<128, S>),
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem), smem_attr,
+                                    "projection smem attribute");
+  if (ast != DMS_OK) return ast;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kProjCluster * v.Hkv);
   cfg.blockDim = dim3(kProjThreads);

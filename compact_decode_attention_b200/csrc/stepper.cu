@@ -84,6 +84,7 @@ struct dms_stepper {
   // [2] steps copied out, [3] attention CTAs that left (self-resetting)
   int32_t* counters;
   StreamValueFn wait_value, write_value;  // both non-null: counter protocol
+  bool drop_input_signal;                 // injected fault: skip the next "staged" write
 };
 
 extern "C" dms_status dms_stepper_layout(const dms_pool* pool, int n_layers, int batch,
@@ -215,9 +216,10 @@ extern "C" dms_status dms_stepper_step(dms_stepper* s, int64_t pos, const void* 
     if (st == DMS_OK)
       st = cuda_status(cudaMemcpyAsync(stg, host_in, L.in_bytes, cudaMemcpyHostToDevice, s->h2d),
                        "stepper input copy");
-    if (st == DMS_OK)
+    if (st == DMS_OK && !s->drop_input_signal)
       st = drv(s->write_value(s->h2d, dptr(0), cuuint32_t(n + 1), CU_STREAM_WRITE_VALUE_DEFAULT),
                "stepper write (staged)");
+    s->drop_input_signal = false;
     StepSync in{};
     in.ready = s->counters + 0;
     in.ready_value = n + 1;
@@ -272,6 +274,19 @@ extern "C" dms_status dms_stepper_step(dms_stepper* s, int64_t pos, const void* 
   if (st == DMS_OK) st = cuda_status(cudaEventRecord(s->drained[j], s->d2h), "stepper record");
   if (st == DMS_OK) ++s->steps;
   return st;
+}
+
+extern "C" dms_status dms_stepper_inject_fault(dms_stepper* s, int fault) {
+  if (!s || fault != DMS_FAULT_DROP_INPUT_SIGNAL) {
+    set_last_error("null stepper or unknown fault %d", fault);
+    return DMS_ERR_INVALID_ARG;
+  }
+  if (!s->wait_value) {
+    set_last_error("the stepper runs on events (no stream memory operations): no signal to drop");
+    return DMS_ERR_UNSUPPORTED;
+  }
+  s->drop_input_signal = true;
+  return DMS_OK;
 }
 
 extern "C" dms_status dms_stepper_join(dms_stepper* s, cudaStream_t stream) {

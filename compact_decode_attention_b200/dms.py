@@ -30,6 +30,8 @@ DEVERR_LAYER_NOT_EMPTY = 0x10
 DEVERR_BOUNDS = 0x20
 DEVERR_BAD_SEQUENCE = 0x40
 
+FAULT_DROP_INPUT_SIGNAL = 1
+
 BLOCK_TOKENS = 64
 
 
@@ -91,6 +93,8 @@ _SIGS = {
     "dms_pool_destroy": (_I, [_P]),
     "dms_pool_reset": (_I, [_P, _P]),
     "dms_pool_layout": (_I, [_P, ctypes.POINTER(PoolLayout)]),
+    "dms_pool_set_wait_limit": (_I, [_P, ctypes.c_uint64]),
+    "dms_stepper_inject_fault": (_I, [_P, _I]),
     "dms_compact_prefill": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P]),
     "dms_append_evict_layers": (_I, [_P, _I, _I, _I, _I64, _P, _P, _I, _P, _P]),
     "dms_append_evict": (_I, [_P, _I, _I, _I64, _P, _P, _I, _P, _P]),
@@ -164,6 +168,14 @@ def dms_pool_destroy(pool: int):
 
 def dms_pool_reset(pool: int, stream: int):
     _check(lib().dms_pool_reset(pool, stream), "dms_pool_reset")
+
+
+def dms_pool_set_wait_limit(pool: int, limit_ns: int):
+    _check(lib().dms_pool_set_wait_limit(pool, limit_ns), "dms_pool_set_wait_limit")
+
+
+def dms_stepper_inject_fault(st: int, fault: int):
+    _check(lib().dms_stepper_inject_fault(st, fault), "dms_stepper_inject_fault")
 
 
 def dms_pool_layout(pool: int) -> PoolLayout:
@@ -357,6 +369,9 @@ class Pool:
     def reset(self, stream=None):
         dms_pool_reset(self.handle, _stream(stream))
 
+    def set_wait_limit(self, limit_ns: int):
+        dms_pool_set_wait_limit(self.handle, int(limit_ns))
+
     def compact_prefill(self, layer, k, v, evict, stream=None):
         B, P = k.shape[0], k.shape[1]
         dms_compact_prefill(self.handle, layer, B, P, _ptr(k), _ptr(v), torch_dtype_code(k.dtype),
@@ -468,6 +483,9 @@ class Stepper:
 
     def join(self, stream=None):
         dms_stepper_join(self.handle, _stream(stream))
+
+    def inject_fault(self, fault: int):
+        dms_stepper_inject_fault(self.handle, fault)
 
     def close(self):
         if self.handle:

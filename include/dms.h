@@ -177,6 +177,15 @@ dms_status dms_pool_destroy(dms_pool* pool);
 /* Clear every head, the block stack and the error word (async on stream). */
 dms_status dms_pool_reset(dms_pool* pool, cudaStream_t stream);
 
+/* Limit of every bounded wait in the kernels launched on this pool from now
+ * on (default 1 s; 1 us .. 60 s, else DMS_ERR_INVALID_ARG).  A wait that
+ * runs out sets DMS_DEVERR_TIMEOUT in the error word and its kernel returns
+ * (no kernel waits without a limit).  The waits are the stepper's step
+ * counters and the attention kernels' copy barriers; a shorter limit makes a
+ * stalled producer (a copy that never lands, a signal that never comes)
+ * surface sooner.  Host-side setting of the handle: not stream-ordered. */
+dms_status dms_pool_set_wait_limit(dms_pool* pool, uint64_t limit_ns);
+
 /* Region offsets of the pool buffer. */
 dms_status dms_pool_layout(const dms_pool* pool, dms_pool_layout_t* out);
 
@@ -359,9 +368,12 @@ dms_status dms_decode_attn(dms_pool* pool, int layer, int batch, const void* q,
  * globals (present on every GPU that loads the library until exit) instead
  * of a caller workspace; calls needing more return DMS_ERR_CAPACITY.  The
  * first call on a device looks up the array's device address (make it
- * before any stream capture).  All calls on a device share the array:
+ * before any stream capture); after a device reset, or in another driver
+ * context, the next call looks it up again in the context then current (make
+ * that call before any capture too).  All calls on a device share the array:
  * nothing in it must start at zero, but calls whose kernels overlap on the
- * GPU race and must be ordered.  The current device must be the pool's. */
+ * GPU race and must be ordered -- also calls on different pools or streams,
+ * since the array is per device.  The current device must be the pool's. */
 dms_status dms_decode_attn_layers_noalloc(dms_pool* pool, int layer0, int n_layers, int batch,
                                           const void* q, dms_dtype q_dtype, void* out,
                                           float sm_scale, cudaStream_t stream);
@@ -399,8 +411,9 @@ dms_status dms_stepper_layout(const dms_pool* pool, int n_layers, int batch,
 
 /* Create a stepper for layers [layer0, layer0 + n_layers) and sequences
  * 0..batch-1 of the pool.  device_buf (>= layout.device_bytes, 256-byte
- * aligned, owned by the caller, no initialisation) holds two input staging
- * buffers, two output buffers and the attention workspace.  `stream` is
+ * aligned, owned by the caller, no initialisation) holds four input staging
+ * buffers, four output buffers, 256 bytes of step counters and the attention
+ * workspace.  `stream` is
  * the compute stream the kernels run on; the stepper creates two copy
  * streams and its events (no device memory).  The pool's device must be
  * current.  sm_scale as for dms_decode_attn_layers. */
@@ -416,6 +429,18 @@ dms_status dms_stepper_create(dms_pool* pool, int layer0, int n_layers, int batc
  * (dms_stepper_join, then synchronise).  Positions follow the rules of
  * dms_append_evict_layers. */
 dms_status dms_stepper_step(dms_stepper* st, int64_t pos, const void* host_in, void* host_out);
+
+/* Host-side fault injection for failure-detection tests (the pages have no
+ * counterpart).  DMS_FAULT_DROP_INPUT_SIGNAL: the next dms_stepper_step
+ * copies its inputs but does not signal "inputs staged" to the device, as if
+ * the copy engine's completion message were lost; that step's append kernel
+ * waits for the signal until the pool's wait limit (dms_pool_set_wait_limit),
+ * then sets DMS_DEVERR_TIMEOUT, and the step runs on (its outputs are
+ * invalid).  Nothing faults, traps or hangs: later steps signal as usual.
+ * Returns DMS_ERR_UNSUPPORTED when the stepper uses events (no driver stream
+ * memory operations), where there is no signal to drop. */
+#define DMS_FAULT_DROP_INPUT_SIGNAL 1
+dms_status dms_stepper_inject_fault(dms_stepper* st, int fault);
 
 /* Make `stream` wait for every step enqueued so far, output copies
  * included. */

@@ -78,3 +78,56 @@ def test_stepper_rejects_bad_arguments():
     with pytest.raises(dms.DmsError) as e:          # layer range past the pool
         dms.dms_stepper_create(pool.handle, 1, 2, 2, 0.0, buf.data_ptr(), lay.device_bytes, s)
     assert e.value.status == dms.DMS_ERR_INVALID_ARG
+
+
+def test_dropped_input_signal_times_out_and_the_device_keeps_answering():
+    """Failure detection without a GPU fault: the stepper is told to drop one
+    step's "inputs staged" signal (a lost completion message, injected on the
+    host).  That step's append kernel waits for it only until the pool's wait
+    limit (20 ms here instead of the default second), reports
+    DMS_DEVERR_TIMEOUT and returns; dms_pool_stats then answers
+    DMS_ERR_DEVICE, and later steps run on the same context as before."""
+    B, Hq, Hkv, D, P, S, w = 2, 8, 2, 64, 300, 5, 32
+    (pa, pb), K, V, fl, Q, dev, dt = _pools_and_inputs("bf16", B, Hq, Hkv, D, P, S, w, seed=43)
+    stream = torch.cuda.current_stream()
+    pb.set_wait_limit(20_000_000)
+    with pytest.raises(dms.DmsError) as e:
+        pb.set_wait_limit(0)
+    assert e.value.status == dms.DMS_ERR_INVALID_ARG
+    stp = dms.Stepper(pb, 0, 1, B, stream=stream)
+    hin = stp.host_inputs(S)
+    hout = torch.zeros(S, stp.layout.out_bytes, dtype=torch.uint8).pin_memory()
+    for s in range(S):
+        stp.pack(hin[s], dev(K[None, :, P + s]), dev(V[None, :, P + s]), dev(Q[None, s]),
+                 torch.from_numpy(np.ascontiguousarray(fl[None, :, P + s])).cuda())
+    for s in range(2):
+        stp.step(P + s, hin[s], hout[s])
+    stp.join(stream)
+    torch.cuda.synchronize()
+    assert pb.stats().error_flags == 0
+    try:
+        stp.inject_fault(dms.FAULT_DROP_INPUT_SIGNAL)
+    except dms.DmsError as err:        # event protocol: nothing to drop
+        assert err.status == dms.DMS_ERR_UNSUPPORTED
+        stp.close()
+        pytest.skip("stepper runs on events here")
+    import time
+    t0 = time.perf_counter()
+    stp.step(P + 2, hin[2], hout[2])
+    stp.join(stream)
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    st = pb.stats(check=False)
+    assert st.error_flags & dms.DEVERR_TIMEOUT, st.as_dict()
+    with pytest.raises(dms.DmsError) as e:
+        pb.stats()
+    assert e.value.status == dms.DMS_ERR_DEVICE
+    assert 0.015 < waited < 0.9, waited           # the 20 ms limit, not the default second
+    for s in range(3, S):                         # the context still answers
+        stp.step(P + s, hin[s], hout[s])
+    stp.join(stream)
+    torch.cuda.synchronize()
+    out = hout[S - 1].view(dt).view(1, B, Hq, D).float()
+    assert torch.isfinite(out).all()
+    stp.close()
+    assert float(torch.ones(4, device="cuda").sum().item()) == 4.0
