@@ -1,7 +1,8 @@
 """Per-head expected values for a seeded synthetic workload (oracle).
 
-Glue between ``synth`` (inputs) and the oracle's definitions: it regenerates
-the inputs of one (layer, sequence, kv-head) from the seed, forms the values
+Glue between ``synth`` (inputs, drawn by its C twin ``synth.fast`` for speed)
+and the oracle's definitions: it regenerates the inputs of one (layer,
+sequence, kv-head) from the seed, forms the values
 the store holds (the model's K/V in their input precision, for an FP8 store
 their E4M3 codes times the per-head scale, for a 4-bit store their group
 codes times the group scales) and evaluates the oracle's
@@ -14,6 +15,7 @@ from __future__ import annotations
 import numpy as np
 
 import synth
+from synth import fast as synth_fast
 
 from .attention import attend
 from .fp8 import dequantize, fp8_scale, quantize
@@ -29,12 +31,21 @@ def head_flags(wl, layer: int, b: int, h: int, n_pos: int) -> np.ndarray:
 
 def head_input(wl, stream: int, layer: int, b: int, h: int, pos0: int, n_pos: int) -> np.ndarray:
     """float32 [n_pos, D]: the model's K (stream 0) or V (stream 1) rows in input precision."""
-    return synth.normal(wl.seed, stream, layer, b, (pos0 + np.arange(n_pos))[:, None], h,
-                        np.arange(wl.head_dim)[None, :], wl.in_dtype)
+    return synth_fast.normal(wl.seed, stream, layer, b, pos0 + np.arange(n_pos), h, wl.head_dim,
+                             wl.in_dtype)
+
+
+def fp8_layer_scales(wl, layer: int) -> list:
+    """[(scale_K, scale_V)] of every kv-head of a layer: amax/448 over the
+    whole prompt of every sequence, before eviction."""
+    amax = [synth_fast.amax(wl.seed, stream, layer, wl.batch, 0, wl.prompt, wl.n_kv_heads,
+                            wl.head_dim, wl.in_dtype) for stream in (synth.STREAM_K, synth.STREAM_V)]
+    return [(fp8_scale(amax[0][h]), fp8_scale(amax[1][h])) for h in range(wl.n_kv_heads)]
 
 
 def fp8_head_scales(wl, layer: int, h: int, chunk: int = 4096) -> tuple:
-    """(scale_K, scale_V) of one (layer, kv-head): amax/448 over the whole prompt and batch."""
+    """(scale_K, scale_V) of one (layer, kv-head): amax/448 over the whole
+    prompt and batch, taken chunk by chunk of positions."""
     scales = []
     for stream in (synth.STREAM_K, synth.STREAM_V):
         amax = np.float32(0.0)
@@ -52,8 +63,7 @@ def stored_rows(wl, layer: int, b: int, h: int, pos: np.ndarray, scales=None):
     pos = np.asarray(pos, dtype=np.int64)
     out = []
     for i, stream in enumerate((synth.STREAM_K, synth.STREAM_V)):
-        x = synth.normal(wl.seed, stream, layer, b, pos[:, None], h,
-                         np.arange(wl.head_dim)[None, :], wl.in_dtype)
+        x = synth_fast.normal(wl.seed, stream, layer, b, pos, h, wl.head_dim, wl.in_dtype)
         if wl.kv_dtype == "fp8":
             out.append(dequantize(quantize(x, scales[i]), scales[i]))
         elif wl.kv_dtype == "int4":

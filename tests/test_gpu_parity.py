@@ -4,7 +4,8 @@ Bookkeeping (counts, slots, ring, stored bytes) must be bit-exact; attention
 outputs must be within max-abs 1e-5 (fp32 store), 2e-2 (bf16), 6e-2 (FP8).
 Small cases compare every head at every step; the workloads at full size run
 in the launch configuration the benchmark times (all layers per call, one
-CTA per SM) and compare sampled heads and steps.
+CTA per SM) and compare every head at one decode step (the 128K stress
+workload: sampled heads) and sampled heads at others.
 """
 import numpy as np
 import pytest
@@ -334,20 +335,29 @@ def _sample_heads(wl, n_extra=2):
     return sorted(heads)
 
 
-def _full_size(wl, check_steps, heads=None, step_scales=True):
+def _full_size(wl, check_steps, heads=None, all_heads_step=None):
+    """Prefill and decode a workload at full size in the launch configuration
+    the benchmark times.  Sampled heads are compared with the oracle at
+    check_steps; at all_heads_step every (layer, sequence, kv-head) is, so
+    that every CTA boundary, rotated range and cross-CTA merge of the real
+    partition is checked.  FP8: every (layer, kv-head) scale bit-exact."""
+    import oracle_jobs
     P, S, g = wl.prompt, wl.decode, wl.group
     dw = DeviceWorkload(wl, S, pregenerate_steps=wl.batch * wl.n_layers <= 288)
     dw.prefill()
     heads = heads or _sample_heads(wl)
-    scales = {}
-    if wl.kv_dtype == "fp8":
-        for (l, b, h) in heads:
-            if (l, h) not in scales:
-                scales[(l, h)] = oref.fp8_head_scales(wl, l, h)
+    scales = None
     state = read_state(dw.pool)
     assert state["error"] == 0
-    for (l, h), (sk, sv) in scales.items():
-        assert state["scales"][l, h, 0] == sk and state["scales"][l, h, 1] == sv
+    if wl.kv_dtype == "fp8":
+        scales = [oref.fp8_layer_scales(wl, l) for l in range(wl.n_layers)]
+        for l in range(wl.n_layers):
+            for h in range(wl.n_kv_heads):
+                assert state["scales"][l, h, 0] == scales[l][h][0], (l, h)
+                assert state["scales"][l, h, 1] == scales[l][h][1], (l, h)
+        l0, h0 = heads[0][0], heads[0][2]          # the chunked per-head definition agrees
+        assert oref.fp8_head_scales(wl, l0, h0) == scales[l0][h0]
+    every = [(l, b, h) for l in range(wl.n_layers) for b in range(wl.batch) for h in range(wl.n_kv_heads)]
     worst = 0.0
     for s in range(S):
         if dw.step_inputs is None:
@@ -356,11 +366,11 @@ def _full_size(wl, check_steps, heads=None, step_scales=True):
             dw.pool.decode_attn_layers(0, si["q"][0], dw.out)
         else:
             dw.step(s)
-        if s in check_steps:
+        if s in check_steps or s == all_heads_step:
             out = dw.out.float().cpu().numpy()
-            for (l, b, h) in heads:
-                sc = scales.get((l, h))
-                exp = oref.expected_output(wl, l, b, h, P + s, scales=sc)
+            which = every if s == all_heads_step else heads
+            exps = oracle_jobs.expected_outputs(wl, which, P + s, scales)
+            for (l, b, h), exp in zip(which, exps):
                 err = np.abs(out[l, b, h * g:(h + 1) * g] - exp).max()
                 worst = max(worst, err)
                 assert err < TOL[wl.kv_dtype], (l, b, h, s, err)
@@ -374,7 +384,7 @@ def _full_size(wl, check_steps, heads=None, step_scales=True):
         rk = dict(zip(pos, oref.head_input(wl, 0, l, b, h, 0, P + S)[pos]))
         rv = dict(zip(pos, oref.head_input(wl, 1, l, b, h, 0, P + S)[pos]))
         check_head_store(dw.pool, state, head_id(dw.pool.cfg, l, b, h), store, rk, rv,
-                         wl.kv_dtype, scales.get((l, h)))
+                         wl.kv_dtype, None if scales is None else scales[l][h])
     check_block_invariants(dw.pool, state)
     st = dw.pool.stats()
     assert st.error_flags == 0
@@ -382,19 +392,22 @@ def _full_size(wl, check_steps, heads=None, step_scales=True):
 
 
 def test_llama_1b_ctx8k_full_size():
+    """All 128 heads at decode step 64; sampled heads at four steps."""
     wl = configs.LLAMA1B_CTX8K
-    _full_size(wl, {0, 1, 64, wl.decode - 1})
+    _full_size(wl, {0, 1, wl.decode - 1}, all_heads_step=64)
 
 
 def test_qwen3_8b_ctx8k_full_size():
+    """All 288 heads at decode step 64; sampled heads at four steps."""
     wl = configs.QWEN8B_CTX8K
-    _full_size(wl, {0, 1, 64, wl.decode - 1})
+    _full_size(wl, {0, 1, wl.decode - 1}, all_heads_step=64)
 
 
 def test_qwen3_8b_fp8_b8_ctx32k_full_size():
+    """All 2304 heads at the last decode step; every FP8 scale."""
     wl = configs.QWEN8B_FP8_B8_CTX32K
     heads = [(0, 0, 0), (35, 7, 7), (17, 3, 4)]
-    _full_size(wl, {0, wl.decode - 1}, heads=heads)
+    _full_size(wl, {0}, heads=heads, all_heads_step=wl.decode - 1)
 
 
 @pytest.mark.slow

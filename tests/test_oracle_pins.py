@@ -601,3 +601,12 @@ def test_glue_stored_rows_of_a_4bit_store_are_the_group_quantised_rows():
                     err = np.abs(cand - grp[d])
                     assert np.isclose(got[i, 32 * gq + d], cand[err.argmin()], rtol=0, atol=1e-12) or \
                         np.sum(err == err.min()) > 1
+
+
+def test_glue_layer_scales_equal_the_per_head_scales():
+    """fp8_layer_scales (one threaded pass over a layer) gives each head the
+    scales fp8_head_scales takes chunk by chunk."""
+    wl = _glue_workload("fp8")
+    for layer in range(wl.n_layers):
+        assert reference.fp8_layer_scales(wl, layer) == [
+            reference.fp8_head_scales(wl, layer, h, chunk=11) for h in range(wl.n_kv_heads)]
