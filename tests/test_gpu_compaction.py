@@ -1,8 +1,8 @@
 """Prefill compaction at both piece sizes of the scatter kernel.
 
 The scatter kernel gives a CTA 64 prompt tokens when a layer would have fewer
-than 16 x SMs CTAs of 256 tokens, else 256.  For each store (bf16, FP8, 4-bit)
-the same prompts are compacted at a batch size that selects each span, into
+than 16 x SMs CTAs of 256 tokens, else 256.  For each store (bf16, FP8, 4-bit;
+the quantised stores from bf16 and from fp32 inputs) the same prompts are compacted at a batch size that selects each span, into
 pools whose blocks were filled with
 0xFF bytes first (NaN in bf16, FP8 and the f16 scales), with per-head keep
 probabilities from window-only to keep-all and a ragged last chunk.  Every
@@ -56,33 +56,35 @@ def _v_tail_bytes(pool, state, hd, n, kind):
     return np.concatenate([nib.reshape(-1), scales.reshape(-1).astype(np.uint32)])
 
 
-def _device_inputs(seed, B, n_pos, Hkv, D, thr):
-    """K, V [B, n_pos, Hkv, D] bf16 and flags [B, n_pos, Hkv] drawn on the device
-    by the generator's device twin."""
+def _device_inputs(seed, B, n_pos, Hkv, D, thr, in_kind="bf16"):
+    """K, V [B, n_pos, Hkv, D] (bf16 or fp32) and flags [B, n_pos, Hkv] drawn on
+    the device by the generator's device twin."""
     st = torch.cuda.current_stream().cuda_stream
-    K = torch.empty(1, B, n_pos, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    dt, code = (torch.float32, dms.DMS_F32) if in_kind == "f32" else (torch.bfloat16, dms.DMS_BF16)
+    K = torch.empty(1, B, n_pos, Hkv, D, dtype=dt, device="cuda")
     V = torch.empty_like(K)
     F = torch.empty(1, B, n_pos, Hkv, dtype=torch.uint8, device="cuda")
-    dms.dms_synth_normal(seed, 0, 0, 1, B, 0, n_pos, Hkv, D, dms.DMS_BF16, K.data_ptr(), st)
-    dms.dms_synth_normal(seed, 1, 0, 1, B, 0, n_pos, Hkv, D, dms.DMS_BF16, V.data_ptr(), st)
+    dms.dms_synth_normal(seed, 0, 0, 1, B, 0, n_pos, Hkv, D, code, K.data_ptr(), st)
+    dms.dms_synth_normal(seed, 1, 0, 1, B, 0, n_pos, Hkv, D, code, V.data_ptr(), st)
     t = torch.tensor([thr], dtype=torch.int32, device="cuda")
     dms.dms_synth_flags(seed, 0, 1, B, 0, n_pos, Hkv, t.data_ptr(), F.data_ptr(), st)
     return K[0], V[0], F[0]
 
 
-def _host_sequence(seed, b, n_pos, Hkv, D, thr):
+def _host_sequence(seed, b, n_pos, Hkv, D, thr, in_kind="bf16"):
     """The same draws for one sequence, from the NumPy generator: [n_pos, Hkv, D] x 2, [n_pos, Hkv]."""
     pos = np.arange(n_pos)
-    K = np.stack([synth.normal(seed, 0, 0, b, pos[:, None], h, np.arange(D)[None, :], "bf16")
+    K = np.stack([synth.normal(seed, 0, 0, b, pos[:, None], h, np.arange(D)[None, :], in_kind)
                   for h in range(Hkv)], axis=1)
-    V = np.stack([synth.normal(seed, 1, 0, b, pos[:, None], h, np.arange(D)[None, :], "bf16")
+    V = np.stack([synth.normal(seed, 1, 0, b, pos[:, None], h, np.arange(D)[None, :], in_kind)
                   for h in range(Hkv)], axis=1)
     F = np.stack([synth.evict_flags(seed, 0, b, pos, h, thr[h]) for h in range(Hkv)], axis=1)
     return K, V, F
 
 
-@pytest.mark.parametrize("kind", ["bf16", "fp8", "int4"])
-def test_both_piece_sizes_match_the_oracle(kind):
+@pytest.mark.parametrize("kind,in_kind", [("bf16", "bf16"), ("fp8", "bf16"), ("int4", "bf16"),
+                                          ("fp8", "f32"), ("int4", "f32")])
+def test_both_piece_sizes_match_the_oracle(kind, in_kind):
     Hkv, Hq, D, P, w, seed = 16, 32, 128, 1000, 64, 91
     sm = torch.cuda.get_device_properties(0).multi_processor_count
     n_chunks = (P + 255) // 256
@@ -90,7 +92,7 @@ def test_both_piece_sizes_match_the_oracle(kind):
     # and a batch of 2 (64-token spans)
     batches = [-(-16 * sm // (n_chunks * Hkv)) + 1, 2]
     thr = [synth.keep_threshold(p) for p in KEEP]
-    Kd, Vd, Fd = _device_inputs(seed, batches[0], P + 1, Hkv, D, thr)
+    Kd, Vd, Fd = _device_inputs(seed, batches[0], P + 1, Hkv, D, thr, in_kind)
     rng = np.random.default_rng(seed)
     host = {}
     for B in batches:
@@ -110,7 +112,7 @@ def test_both_piece_sizes_match_the_oracle(kind):
         seqs = sorted({0, B - 1, int(rng.integers(0, B))})
         for b in seqs:
             if b not in host:
-                host[b] = _host_sequence(seed, b, P + 1, Hkv, D, thr)
+                host[b] = _host_sequence(seed, b, P + 1, Hkv, D, thr, in_kind)
             K, V, F = host[b]
             for h in range(Hkv):
                 hd = head_id(pool.cfg, 0, b, h)
