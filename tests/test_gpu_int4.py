@@ -4,10 +4,12 @@ against the oracle, through the C ABI.
 Stored codes and group scales must equal the oracle's quantisation of the
 rows the slot simulator says are held (bit-exact, like all bookkeeping);
 attention over the stored values must be within the FP8 tolerance, 6e-2
-max-abs, of the fp64 oracle run on the dequantised rows, widened where values
-are far from unit scale by the two roundings that grow with them: the bf16
-output (half an ulp, 2^-9 of |out|) and the f16 probabilities of the P.V
-product (2^-11 of each weight, so at most 2^-11 of max |v|)."""
+max-abs, of the fp64 oracle run on the dequantised rows.  Only the test whose
+groups are scaled far from unit size (values up to a few thousand) widens it,
+by the two roundings that grow with the values: the bf16 output (half an
+ulp, 2^-9 of |out|, taken as 2^-8) and the f16 probabilities times f16 group
+scales of the P.V product (2^-11 of each weight twice, so at most 2^-10 of
+max |v|)."""
 import numpy as np
 import pytest
 import torch
@@ -60,7 +62,7 @@ def _check_store(pool, K, V, flags, P, w):
     check_block_invariants(pool, state)
 
 
-def _run(seed, B, P, S, Hq, Hkv, w, in_kind, p_keep=0.3, edit=None):
+def _run(seed, B, P, S, Hq, Hkv, w, in_kind, p_keep=0.3, edit=None, widen=False):
     D = 128
     K = synth.kv_tokens(seed, 0, 0, B, 0, P + S, Hkv, D, in_kind)
     V = synth.kv_tokens(seed, 1, 0, B, 0, P + S, Hkv, D, in_kind)
@@ -86,7 +88,9 @@ def _run(seed, B, P, S, Hq, Hkv, w, in_kind, p_keep=0.3, edit=None):
         for b in range(B):
             exp = oatt.decode_attention(Q[s, b].astype(np.float64), Ks[b, :t + 1], Vs[b, :t + 1],
                                         flags[b, :t + 1], t, w)
-            bound = TOL + np.abs(exp) * 2.0 ** -8 + np.abs(Vs[b, :t + 1]).max() * 2.0 ** -10
+            bound = TOL
+            if widen:     # values far from unit scale: the roundings that grow with them
+                bound = TOL + np.abs(exp) * 2.0 ** -8 + np.abs(Vs[b, :t + 1]).max() * 2.0 ** -10
             worst = max(worst, float((np.abs(got[b] - exp) / bound).max()))
     assert worst < 1.0, worst
     _check_store(pool, K, V, flags, P, w)
@@ -116,7 +120,7 @@ def test_int4_zero_and_large_groups():
         V[0, ::5, 1, 64:96] *= 1024.0
         K[:] = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(K))
         V[:] = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(V))
-    _run(83, 2, 150, 40, 8, 2, 24, "bf16", p_keep=0.4, edit=edit)
+    _run(83, 2, 150, 40, 8, 2, 24, "bf16", p_keep=0.4, edit=edit, widen=True)
 
 
 def test_int4_all_layers_fused_call_and_release():
