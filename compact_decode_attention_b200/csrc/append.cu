@@ -12,10 +12,11 @@
 // opening paragraphs).  Otherwise the token takes slot n_slots, opening a
 // new block when that slot starts one.
 //
-// One warp per head: the per-head state it needs (counters, last block, the
-// ring entry and the physical row of the token leaving the window) is read
-// with independent loads, so the kernel waits on memory about once before
-// its stores, and the rows are written by as many SMs as there are heads / 8.
+// One warp per head (append_head_warp in append_core.cuh): the per-head
+// state it needs (counters, last block, the ring entry and the physical row
+// of the token leaving the window) is read with independent loads, so the
+// kernel waits on memory about once before its stores, and the rows are
+// written by as many SMs as there are heads / 8.
 // A new block comes from an atomic bump of the block counter: the logical
 // state (slots, counts, rings, stored bytes) is a deterministic function of
 // the inputs; which physical block a head gets during decode is not (prefill
@@ -24,21 +25,10 @@
 
 namespace dms {
 
-template <typename T>
-__device__ __forceinline__ float in_to_f32(T x);
-template <>
-__device__ __forceinline__ float in_to_f32<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ float in_to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
-  return __bfloat162float(x);
-}
-
 constexpr int kAppendHeadsPerCta = 8;            // one warp per head
 constexpr int kAppendThreads = 32 * kAppendHeadsPerCta;
 
-// One warp per (layer, sequence, kv-head).  Lane 0 does the bookkeeping; all
-// lanes load the new K/V row first (it does not depend on the bookkeeping)
-// and store it once the destination is known.
+// One warp per (layer, sequence, kv-head) runs append_head_warp.
 // seq_ids (nullable): pool sequence of batch row b, else b.  pos_arr
 // (nullable): position of batch row b, else `pos` for every row.
 // STORE: 0 = copy (bf16 / fp32 store), 1 = FP8, 2 = 4-bit
@@ -68,96 +58,9 @@ __global__ void __launch_bounds__(kAppendThreads)
     if (lane == 0) report_error(v.hdr, DMS_DEVERR_BAD_SEQUENCE, l, bi, h);
     return;
   }
-  const int hd = v.head(l, b, h);
-  const int t = int(tpos);
-
-  // ---- new rows into registers (bf16/fp32: 16-byte chunks, K then V) ----
-  const int nch = int(v.row_bytes >> 4);       // chunks per row: 8, 16 or 32
-  constexpr int kMaxPerLane = 2;               // 2 * 32 chunks per lane pair covers fp32 D=128
-  uint4 chunk[kMaxPerLane];
-  if constexpr (STORE == 0) {
-#pragma unroll
-    for (int r = 0; r < kMaxPerLane; ++r) {
-      const int c = lane + 32 * r;
-      if (c < 2 * nch) {
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(c < nch ? k : vv) +
-                             int64_t(i) * v.row_bytes + (c % nch) * 16;
-        chunk[r] = *reinterpret_cast<const uint4*>(src);
-      }
-    }
-  }
-
-  // ---- bookkeeping (lane 0; all its loads are independent) ----
-  int slot = -1, prow = -1, opened = 0;
-  if (lane == 0) {
-    const uint32_t flag = evict[i] != 0;     // [nl, batch, Hkv] flattened like i
-    const AppendSlot r = append_bookkeeping(v, l, b, h, hd, t, flag);
-    slot = r.slot;
-    prow = r.prow;
-    opened = r.opened;
-  }
-  slot = __shfl_sync(0xffffffffu, slot, 0);
-  prow = __shfl_sync(0xffffffffu, prow, 0);
-  opened = __shfl_sync(0xffffffffu, opened, 0);
-  if (slot < 0) return;
-  const int row = prow % v.BT;
-  uint8_t* blk = v.blocks + int64_t(prow / v.BT) * v.block_bytes;
-
-  // ---- store the row ----
-  if constexpr (STORE == 2) {
-    if (opened) {   // tokens past the last one of a new block decode to 0
-      uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);
-      for (int c = lane; c < int(v.tile_bytes / 16); c += 32) tile[c] = make_uint4(0, 0, 0, 0);
-      __syncwarp();
-    }
-    float k4[4], v4[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      k4[e] = in_to_f32(k[int64_t(i) * v.D + 4 * lane + e]);
-      v4[e] = in_to_f32(vv[int64_t(i) * v.D + 4 * lane + e]);
-    }
-    store_row_int4(v, prow, k4, v4, lane);
-  } else if constexpr (STORE == 0) {
-#pragma unroll
-    for (int r = 0; r < kMaxPerLane; ++r) {
-      const int c = lane + 32 * r;
-      if (c < 2 * nch) {
-        uint8_t* dst = blk + (c < nch ? 0 : v.tile_bytes) + int64_t(row) * v.row_bytes +
-                       swz_chunk(c % nch, row) * 16;
-        *reinterpret_cast<uint4*>(dst) = chunk[r];
-      }
-    }
-  } else {
-    // a block opened by this step gets its transposed V tile cleared first,
-    // so token columns not yet written decode to 0 (the attention kernel
-    // reads whole V tiles)
-    if (opened) {
-      uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);
-      for (int c = lane; c < int(v.tile_bytes / 16); c += 32) tile[c] = make_uint4(0, 0, 0, 0);
-      __syncwarp();
-    }
-    const float sK = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 0];
-    const float sV = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 1];
-    const InT* srck = k + int64_t(i) * v.D;
-    const InT* srcv = vv + int64_t(i) * v.D;
-    if (lane < 8) {            // K: lane lc fills 16-byte chunk lc of the permuted row
-      const int lc = lane;
-      uint8_t codes[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int p = lc * 16 + e;
-        const int d = ((p >> 2) & 7) * 16 + ((p >> 1) & 1) * 8 + (p >> 5) * 2 + (p & 1);
-        codes[e] = f32_to_e4m3(__fdiv_rn(in_to_f32(srck[d]), sK));
-      }
-      *reinterpret_cast<uint4*>(blk + row * 128 + ((lc ^ (row & 7)) << 4)) =
-          *reinterpret_cast<const uint4*>(codes);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {  // V: 4 elements per lane into the transposed tile
-      const int d = lane * 4 + e;
-      blk[v.tile_bytes + fp8v_byte(row, d)] = f32_to_e4m3(__fdiv_rn(in_to_f32(srcv[d]), sV));
-    }
-  }
+  const uint32_t flag = lane == 0 ? uint32_t(evict[i] != 0) : 0u;  // [nl, batch, Hkv] flattened like i
+  append_head_warp<InT, STORE>(v, l, b, h, v.head(l, b, h), int(tpos), k + int64_t(i) * v.D,
+                               vv + int64_t(i) * v.D, flag, lane);
 }
 
 }  // namespace dms

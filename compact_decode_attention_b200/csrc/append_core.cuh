@@ -112,12 +112,12 @@ __device__ __forceinline__ uint32_t int4_nibble(float x, float scale) {
 // of the block, so they are cleared and set with atomics -- or, with
 // s_vwords (a zeroed shared-memory image of the block's 1024 V nibble words),
 // OR-ed into that image for the caller to write out.
-__device__ __forceinline__ void store_row_int4(const PoolView& v, int prow, const float (&k4)[4],
-                                               const float (&v4)[4], int lane,
-                                               uint32_t* s_vwords = nullptr) {
-  const int row = prow % v.BT;
-  uint8_t* blk = v.blocks + int64_t(prow / v.BT) * v.block_bytes;
-  uint8_t* vt = blk + v.tile_bytes;
+// store_row_int4_at writes row `row` of the block image at blk (global
+// memory, or a shared-memory stage: the atomics work on either).
+__device__ __forceinline__ void store_row_int4_at(uint8_t* blk, int row, int64_t tile_bytes,
+                                                  const float (&k4)[4], const float (&v4)[4],
+                                                  int lane, uint32_t* s_vwords = nullptr) {
+  uint8_t* vt = blk + tile_bytes;
   // group of lane l: elements 4l.. lie in group l / 8; amax over its 8 lanes
   float ka = fmaxf(fmaxf(fabsf(k4[0]), fabsf(k4[1])), fmaxf(fabsf(k4[2]), fabsf(k4[3])));
   float va = fmaxf(fmaxf(fabsf(v4[0]), fabsf(v4[1])), fmaxf(fabsf(v4[2]), fabsf(v4[3])));
@@ -160,6 +160,13 @@ __device__ __forceinline__ void store_row_int4(const PoolView& v, int prow, cons
       atomicOr(w, int4_nibble(v4[i], vs) << sh);
     }
   }
+}
+
+__device__ __forceinline__ void store_row_int4(const PoolView& v, int prow, const float (&k4)[4],
+                                               const float (&v4)[4], int lane,
+                                               uint32_t* s_vwords = nullptr) {
+  store_row_int4_at(v.blocks + int64_t(prow / v.BT) * v.block_bytes, prow % v.BT, v.tile_bytes, k4,
+                    v4, lane, s_vwords);
 }
 
 // Store one token's K and V rows, given as float values already rounded to
@@ -212,6 +219,111 @@ __device__ __forceinline__ void store_row_from_float(const PoolView& v, int l, i
     } else {
       *reinterpret_cast<__nv_bfloat16*>(blk + off) = __float2bfloat16_rn(krow[d]);
       *reinterpret_cast<__nv_bfloat16*>(blk + v.tile_bytes + off) = __float2bfloat16_rn(vrow[d]);
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float in_to_f32(T x);
+template <>
+__device__ __forceinline__ float in_to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float in_to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+// One decode step of one head, one warp: token t (flag `flag`, valid in
+// lane 0) of head hd = (layer l, sequence b, kv-head h) with input rows
+// krow, vrow (D elements each, 16-byte aligned).  Lane 0 does the
+// bookkeeping; all lanes load the new rows first (they do not depend on the
+// bookkeeping) and store them once the destination is known.
+// STORE: 0 = copy (bf16 / fp32 store, input in the store's dtype), 1 = FP8,
+// 2 = 4-bit.
+template <typename InT, int STORE>
+__device__ __forceinline__ void append_head_warp(const PoolView& v, int l, int b, int h, int hd, int t,
+                                                 const InT* krow, const InT* vrow, uint32_t flag,
+                                                 int lane) {
+  // ---- new rows into registers (bf16/fp32: 16-byte chunks, K then V) ----
+  const int nch = int(v.row_bytes >> 4);       // chunks per row: 8, 16 or 32
+  constexpr int kMaxPerLane = 2;               // 2 * 32 chunks per lane pair covers fp32 D=128
+  uint4 chunk[kMaxPerLane];
+  if constexpr (STORE == 0) {
+#pragma unroll
+    for (int r = 0; r < kMaxPerLane; ++r) {
+      const int c = lane + 32 * r;
+      if (c < 2 * nch) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(c < nch ? krow : vrow) + (c % nch) * 16;
+        chunk[r] = *reinterpret_cast<const uint4*>(src);
+      }
+    }
+  }
+
+  // ---- bookkeeping (lane 0; all its loads are independent) ----
+  int slot = -1, prow = -1, opened = 0;
+  if (lane == 0) {
+    const AppendSlot r = append_bookkeeping(v, l, b, h, hd, t, flag);
+    slot = r.slot;
+    prow = r.prow;
+    opened = r.opened;
+  }
+  slot = __shfl_sync(0xffffffffu, slot, 0);
+  prow = __shfl_sync(0xffffffffu, prow, 0);
+  opened = __shfl_sync(0xffffffffu, opened, 0);
+  if (slot < 0) return;
+  const int row = prow % v.BT;
+  uint8_t* blk = v.blocks + int64_t(prow / v.BT) * v.block_bytes;
+
+  // ---- store the row ----
+  if constexpr (STORE == 2) {
+    if (opened) {   // tokens past the last one of a new block decode to 0
+      uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);
+      for (int c = lane; c < int(v.tile_bytes / 16); c += 32) tile[c] = make_uint4(0, 0, 0, 0);
+      __syncwarp();
+    }
+    float k4[4], v4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      k4[e] = in_to_f32(krow[4 * lane + e]);
+      v4[e] = in_to_f32(vrow[4 * lane + e]);
+    }
+    store_row_int4(v, prow, k4, v4, lane);
+  } else if constexpr (STORE == 0) {
+#pragma unroll
+    for (int r = 0; r < kMaxPerLane; ++r) {
+      const int c = lane + 32 * r;
+      if (c < 2 * nch) {
+        uint8_t* dst = blk + (c < nch ? 0 : v.tile_bytes) + int64_t(row) * v.row_bytes +
+                       swz_chunk(c % nch, row) * 16;
+        *reinterpret_cast<uint4*>(dst) = chunk[r];
+      }
+    }
+  } else {
+    // a block opened by this step gets its transposed V tile cleared first,
+    // so token columns not yet written decode to 0 (the attention kernel
+    // reads whole V tiles)
+    if (opened) {
+      uint4* tile = reinterpret_cast<uint4*>(blk + v.tile_bytes);
+      for (int c = lane; c < int(v.tile_bytes / 16); c += 32) tile[c] = make_uint4(0, 0, 0, 0);
+      __syncwarp();
+    }
+    const float sK = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 0];
+    const float sV = v.scales[(int64_t(l) * v.Hkv + h) * 2 + 1];
+    if (lane < 8) {            // K: lane lc fills 16-byte chunk lc of the permuted row
+      const int lc = lane;
+      uint8_t codes[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int p = lc * 16 + e;
+        const int d = ((p >> 2) & 7) * 16 + ((p >> 1) & 1) * 8 + (p >> 5) * 2 + (p & 1);
+        codes[e] = f32_to_e4m3(__fdiv_rn(in_to_f32(krow[d]), sK));
+      }
+      *reinterpret_cast<uint4*>(blk + row * 128 + ((lc ^ (row & 7)) << 4)) =
+          *reinterpret_cast<const uint4*>(codes);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {  // V: 4 elements per lane into the transposed tile
+      const int d = lane * 4 + e;
+      blk[v.tile_bytes + fp8v_byte(row, d)] = f32_to_e4m3(__fdiv_rn(in_to_f32(vrow[d]), sV));
     }
   }
 }

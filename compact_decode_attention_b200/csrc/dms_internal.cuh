@@ -309,6 +309,12 @@ __device__ __forceinline__ void pdl_wait_prerequisites() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Bring `bytes` (a multiple of 16) from p into L2, asynchronously (TMA bulk
+// prefetch: no register written, nothing waits).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Bring the line holding p into L2 (no register written, nothing waits).
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
@@ -392,6 +398,7 @@ struct dms_pool {
   size_t bytes;
   int device;
   int sm_count;
+  int attn_kernel;  // DMS_ATTN_* (dms_pool_set_attn_kernel)
 };
 
 namespace dms {
@@ -402,4 +409,12 @@ dms_status append_layers_synced(dms_pool* pool, int layer0, int n_layers, int ba
 dms_status decode_attn_layers_synced(dms_pool* pool, int layer0, int n_layers, int batch,
                                      const void* q, void* out, float sm_scale, void* ws,
                                      cudaStream_t stream, const StepSync& sync);
+// one cluster per head for calls with few heads (csrc/step.cu): attention
+// only when knew is null, else the fused decode step; *done = false when
+// the call has too many heads for every cluster of two or more CTAs to be
+// resident at once (force: launch with clusters of one CTA then)
+dms_status cluster_attn(dms_pool* pool, int layer0, int n_layers, int batch, const void* q, void* out,
+                        float sm_scale, const void* knew, const void* vnew, dms_dtype in_dtype,
+                        const uint8_t* evict, int64_t pos, bool force, cudaStream_t stream,
+                        bool* done);
 }  // namespace dms

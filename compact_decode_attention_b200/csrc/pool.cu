@@ -345,6 +345,7 @@ dms_status dms_pool_create(const dms_pool_config* cfg, void* dev_buf, size_t byt
   p->bytes = bytes;
   p->device = dev;
   p->sm_count = device_sm_count(dev);
+  p->attn_kernel = DMS_ATTN_AUTO;
   p->view = make_view(*cfg, lay, dev_buf);
   st = clear_pool(p, stream);
   if (st != DMS_OK) {
@@ -375,6 +376,15 @@ dms_status dms_pool_set_wait_limit(dms_pool* pool, uint64_t limit_ns) {
     return DMS_ERR_INVALID_ARG;
   }
   pool->view.wait_ns = limit_ns;
+  return DMS_OK;
+}
+
+dms_status dms_pool_set_attn_kernel(dms_pool* pool, int kind) {
+  if (!pool || kind < DMS_ATTN_AUTO || kind > DMS_ATTN_CLUSTER) {
+    set_last_error("null pool or unknown attention kernel %d", kind);
+    return DMS_ERR_INVALID_ARG;
+  }
+  pool->attn_kernel = kind;
   return DMS_OK;
 }
 

@@ -31,6 +31,7 @@ DEVERR_BOUNDS = 0x20
 DEVERR_BAD_SEQUENCE = 0x40
 
 FAULT_DROP_INPUT_SIGNAL = 1
+ATTN_AUTO, ATTN_STREAM_K, ATTN_CLUSTER = 0, 1, 2
 
 BLOCK_TOKENS = 64
 
@@ -94,6 +95,9 @@ _SIGS = {
     "dms_pool_reset": (_I, [_P, _P]),
     "dms_pool_layout": (_I, [_P, ctypes.POINTER(PoolLayout)]),
     "dms_pool_set_wait_limit": (_I, [_P, ctypes.c_uint64]),
+    "dms_pool_set_attn_kernel": (_I, [_P, _I]),
+    "dms_decode_step_layers": (_I, [_P, _I, _I, _I, _I64, _P, _P, _I, _P, _P, _I, _P, ctypes.c_float, _P,
+                                    ctypes.c_size_t, _P]),
     "dms_stepper_inject_fault": (_I, [_P, _I]),
     "dms_compact_prefill": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P]),
     "dms_append_evict_layers": (_I, [_P, _I, _I, _I, _I64, _P, _P, _I, _P, _P]),
@@ -172,6 +176,18 @@ def dms_pool_reset(pool: int, stream: int):
 
 def dms_pool_set_wait_limit(pool: int, limit_ns: int):
     _check(lib().dms_pool_set_wait_limit(pool, limit_ns), "dms_pool_set_wait_limit")
+
+
+def dms_pool_set_attn_kernel(pool: int, kind: int):
+    _check(lib().dms_pool_set_attn_kernel(pool, kind), "dms_pool_set_attn_kernel")
+
+
+def dms_decode_step_layers(pool: int, layer0: int, n_layers: int, batch: int, pos: int, k: int, v: int,
+                           in_dtype: int, evict: int, q: int, q_dtype: int, out: int, sm_scale: float,
+                           workspace: int, workspace_bytes: int, stream: int):
+    _check(lib().dms_decode_step_layers(pool, layer0, n_layers, batch, pos, k, v, in_dtype, evict, q,
+                                        q_dtype, out, sm_scale, workspace, workspace_bytes, stream),
+           "dms_decode_step_layers")
 
 
 def dms_stepper_inject_fault(st: int, fault: int):
@@ -372,6 +388,9 @@ class Pool:
     def set_wait_limit(self, limit_ns: int):
         dms_pool_set_wait_limit(self.handle, int(limit_ns))
 
+    def set_attn_kernel(self, kind: int):
+        dms_pool_set_attn_kernel(self.handle, int(kind))
+
     def compact_prefill(self, layer, k, v, evict, stream=None):
         B, P = k.shape[0], k.shape[1]
         dms_compact_prefill(self.handle, layer, B, P, _ptr(k), _ptr(v), torch_dtype_code(k.dtype),
@@ -395,6 +414,14 @@ class Pool:
         ws = self.workspace(nl, B, q.device)
         dms_decode_attn_layers(self.handle, layer0, nl, B, _ptr(q), torch_dtype_code(q.dtype),
                                _ptr(out), sm_scale, _ptr(ws), ws.numel(), _stream(stream))
+
+    def decode_step_layers(self, layer0, pos, k, v, evict, q, out, sm_scale=0.0, stream=None):
+        """Append (k, v, evict [nl, B, Hkv(, D)]) then attend (q, out [nl, B, Hq, D]) in one call."""
+        nl, B = q.shape[0], q.shape[1]
+        ws = self.workspace(nl, B, q.device)
+        dms_decode_step_layers(self.handle, layer0, nl, B, pos, _ptr(k), _ptr(v), torch_dtype_code(k.dtype),
+                               _ptr(evict), _ptr(q), torch_dtype_code(q.dtype), _ptr(out), sm_scale, _ptr(ws),
+                               ws.numel(), _stream(stream))
 
     # ---- continuous batching: sequence slots with their own positions ----
     def compact_prefill_seqs(self, layer, seq0, k, v, evict, stream=None):

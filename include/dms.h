@@ -186,6 +186,25 @@ dms_status dms_pool_reset(dms_pool* pool, cudaStream_t stream);
  * surface sooner.  Host-side setting of the handle: not stream-ordered. */
 dms_status dms_pool_set_wait_limit(dms_pool* pool, uint64_t limit_ns);
 
+/* Which kernel decode attention uses (host setting of the handle, applied to
+ * calls made after it):
+ *   DMS_ATTN_AUTO      one thread-block cluster per head (up to 16 CTAs per
+ *                      head, partials merged in distributed shared memory)
+ *                      when every cluster of at least 2 CTAs of the call can
+ *                      be resident at once -- calls with few heads, e.g. one
+ *                      layer at a small batch; else the stream-K kernel
+ *                      (the held blocks of all heads cut evenly over one CTA
+ *                      per SM, merged through the workspace).  The default.
+ *   DMS_ATTN_STREAM_K  always the stream-K kernel.
+ *   DMS_ATTN_CLUSTER   always the cluster kernel (clusters of one CTA, in
+ *                      waves, when the call has more heads than fit).
+ * Both compute the same attention (rounding order aside).  The calls with
+ * device sequence lists (_seqs) and the stepper always use stream-K. */
+#define DMS_ATTN_AUTO 0
+#define DMS_ATTN_STREAM_K 1
+#define DMS_ATTN_CLUSTER 2
+dms_status dms_pool_set_attn_kernel(dms_pool* pool, int kind);
+
 /* Region offsets of the pool buffer. */
 dms_status dms_pool_layout(const dms_pool* pool, dms_pool_layout_t* out);
 
@@ -353,6 +372,28 @@ dms_status dms_decode_workspace_bytes(const dms_pool* pool, int n_layers, int ba
 dms_status dms_decode_attn_layers(dms_pool* pool, int layer0, int n_layers, int batch,
                                   const void* q, dms_dtype q_dtype, void* out, float sm_scale,
                                   void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream);
+
+/* One whole decode step at position `pos` for layers [layer0, layer0 +
+ * n_layers): the result of dms_append_evict_layers(k, v, evict) followed by
+ * dms_decode_attn_layers(q) -- the new token is stored exactly as the
+ * append stores it and the attention covers the same rows -- in one launch
+ * when the call has few heads (the cluster kernel: every CTA of a head reads
+ * the head's state from before the append, a cluster barrier orders that
+ * before the append, the slot the append reuses is masked and the new token
+ * enters the attention from the inputs); otherwise the two kernels run in
+ * turn.  The form a model issues layer by layer (layer l+1's query needs
+ * layer l's output).  Arguments as for the two calls:
+ *   k, v   [n_layers, batch, Hkv, D]  in_dtype;   evict [n_layers, batch, Hkv]
+ *   q, out [n_layers, batch, Hq, D]   q_dtype;    workspace as for
+ *   dms_decode_attn_layers (used only when the two kernels run).
+ * Source: delayed eviction and the attention over each head's retained
+ * tokens (mindverse page, DMS section); slot reclaim (FastDMS page, opening
+ * paragraphs). */
+dms_status dms_decode_step_layers(dms_pool* pool, int layer0, int n_layers, int batch, int64_t pos,
+                                  const void* k, const void* v, dms_dtype in_dtype,
+                                  const uint8_t* evict, const void* q, dms_dtype q_dtype, void* out,
+                                  float sm_scale, void* workspace, size_t workspace_bytes,
                                   cudaStream_t stream);
 
 /* Single-layer form of dms_decode_attn_layers (q, out [batch, Hq, D]). */

@@ -36,6 +36,7 @@ def _pools_and_inputs(kind, B, Hq, Hkv, D, P, S, w, seed):
 def test_stepper_matches_direct_calls_bit_exactly(kind, B, Hq, Hkv, D):
     P, S, w = 700, 7, 64
     (pa, pb), K, V, fl, Q, dev, dt = _pools_and_inputs(kind, B, Hq, Hkv, D, P, S, w, seed=41)
+    pa.set_attn_kernel(dms.ATTN_STREAM_K)   # the stepper's kernel, so the outputs can match bit for bit
     stream = torch.cuda.current_stream()
     stp = dms.Stepper(pb, 0, 1, B, stream=stream)
     hin = stp.host_inputs(S)
