@@ -396,7 +396,7 @@ def expected_bytes_per_step(wl):
 def attn_source_hash() -> str:
     h = hashlib.sha256()
     for f in sorted(os.listdir(os.path.dirname(ATTN_KERNEL_SRC))):
-        if f in ("attn.cu", "dms_internal.cuh"):
+        if f in ("attn.cu", "attn_warp.cuh", "step.cu", "dms_internal.cuh"):
             h.update(open(os.path.join(os.path.dirname(ATTN_KERNEL_SRC), f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -508,9 +508,9 @@ def main():
         return 0
     W, K, E = args.warmup, args.steps, args.e2e_steps
     R = min(K, 64)                 # instrumented steps for the attention-kernel timing
-    RL = min(K, 16)                # steps issued as per-layer calls
+    RL = min(K, 16)                # steps issued as per-layer calls (each of the two forms)
     assert W >= 3 and K >= 1
-    dw = DeviceWorkload(wl, W + K + R + RL + E, device=f"cuda:{local}")
+    dw = DeviceWorkload(wl, W + K + R + 2 * RL + E, device=f"cuda:{local}")
     compact_ms_layers = dw.prefill(timed=True)
     # median layer: the first call of each kernel also pays its module load
     compact_ms = float(np.median(compact_ms_layers)) * len(compact_ms_layers)
@@ -522,7 +522,7 @@ def main():
 
     # exact held tokens after each step: +1 per head, -1 per head whose token
     # t - w carried a flag (flags drawn by the same device generator)
-    NT = W + K + R + RL + E
+    NT = W + K + R + 2 * RL + E
     fl = dw.flags(0, L, P - w, NT) if P - w >= 0 else None
     retired = fl.sum(dim=(0, 1, 3)).cpu().numpy().astype(np.int64) if fl is not None else \
         np.zeros(NT, np.int64)
@@ -636,11 +636,36 @@ def main():
     torch.cuda.synchronize()
     pl_ms = pl0.elapsed_time(pl1) / RL
     del graph
+    # ---- the same decode step as L fused calls (dms_decode_step_layers: the
+    # append and the attention of one layer in one launch), layer after layer ----
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for j in range(RL):
+            s = W + K + R + RL + j
+            for layer in range(L):
+                dw.pool.decode_step_layers(layer, P + s, si["k"][s][layer:layer + 1], si["v"][s][layer:layer + 1],
+                                           si["evict"][s][layer:layer + 1], si["q"][s][layer:layer + 1],
+                                           dw.out[layer:layer + 1])
+    torch.cuda.synchronize()
+    pf0, pf1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pf0.record(stream)
+    graph.replay()
+    pf1.record(stream)
+    torch.cuda.synchronize()
+    pf_ms = pf0.elapsed_time(pf1) / RL
+    del graph
+    fused_bytes = float(bytes_step[W + K + R + RL:W + K + R + 2 * RL].mean())
     per_layer_calls = {"ms_per_step": pl_ms, "decode_steps_per_s": 1e3 / pl_ms,
                        "value": float(bytes_step[W + K + R:W + K + R + RL].mean()) / (pl_ms * 1e-3) / 1e9,
                        "unit": "GB/s", "launches_per_step": 2 * L, "steps": RL,
                        "timing": "CUDA events around one replay of a captured graph of the steps, "
-                                 "each step one append and one attention call per layer"}
+                                 "each step one append and one attention call per layer",
+                       "fused_step": {"ms_per_step": pf_ms, "decode_steps_per_s": 1e3 / pf_ms,
+                                      "value": fused_bytes / (pf_ms * 1e-3) / 1e9, "unit": "GB/s",
+                                      "frac": fused_bytes / (pf_ms * 1e-3) / 1e9 / measured_peaks()[0],
+                                      "launches_per_step": L, "steps": RL,
+                                      "call": "dms_decode_step_layers, one layer per call (append/evict and "
+                                              "attention in one launch: decode_cluster_kernel)"}}
     st = dw.pool.stats()
     if st.error_flags:
         raise SystemExit(f"device error word 0x{st.error_flags:x}")
@@ -650,6 +675,9 @@ def main():
     value = total_bytes / (ms_max * 1e-3) / 1e9
 
     # ---- roofline of the attention kernel ----
+    plan_kind, plan_c = dms.dms_decode_attn_plan(dw.pool.handle, L, B)
+    attn_kernel_name = (f"decode_cluster_kernel<{wl.kv_dtype},{D}> ({plan_c} CTAs per head)"
+                        if plan_kind == dms.ATTN_CLUSTER else f"decode_attn_kernel<{wl.kv_dtype},{D}> (stream-K)")
     peak, peak_kind = measured_peaks()
     rbytes = bytes_step[W + K:W + K + R]
     achieved = float(rbytes.sum() / (attn_ms.sum() * 1e-3) / 1e9)
@@ -657,7 +685,7 @@ def main():
     traffic = None if ratio is None else ratio * float(rbytes.mean())
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": f"decode_attn_kernel<{wl.kv_dtype},{D}>",
+                "kernel": attn_kernel_name,
                 "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "algorithmic_bytes_per_launch": float(rbytes.mean()),
                 "attn_us_per_launch": float(attn_ms.mean() * 1e3),
@@ -669,7 +697,7 @@ def main():
     # pinned host), copies inside the timed region ----
     e2e = None
     if E > 0:
-        e0s = W + K + R + RL
+        e0s = W + K + R + 2 * RL
         stp = dms.Stepper(dw.pool, 0, L, B, stream=stream)
         hin = stp.host_inputs(E)
         hout = torch.empty(E, stp.layout.out_bytes, dtype=torch.uint8).pin_memory()
@@ -744,7 +772,7 @@ def main():
             "prefill_attention": prefill, "kv_projection_append": projection,
             "gpu_launches": 2 * K, "clocks": clk.summary(),
             "kernels_per_step": ["append_evict_kernel (1 launch, all layers)",
-                                 "decode_attn_kernel (1 launch, all layers)"],
+                                 f"{attn_kernel_name} (1 launch, all layers)"],
             "pool": {"blocks_in_use": int(st.blocks_in_use), "kv_bytes_in_use": int(st.kv_bytes_in_use),
                      "retained_tokens": int(st.retained_tokens),
                      "min_retained": int(st.min_retained), "max_retained": int(st.max_retained)},

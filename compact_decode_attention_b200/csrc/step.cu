@@ -46,9 +46,9 @@
 // Every mbarrier wait is bounded by the pool's wait limit.  The one cluster
 // barrier is a hardware barrier that every thread of every CTA arrives at
 // with the same instruction at the same point (a warp never splits over two
-// arrive forms: two forms in one warp, one lane each way, hung a GPU in an
-// earlier build) and waits on exactly once, so it cannot wait for a missing
-// arrival.
+// arrive forms: a warp whose lanes arrived with two different forms left the
+// barrier's phase count wrong and the cluster waiting for good) and waits on
+// exactly once, so it cannot wait for a missing arrival.
 #include <mutex>
 
 #include "append_core.cuh"
@@ -655,6 +655,36 @@ dms_status cluster_attn(dms_pool* pool, int layer0, int n_layers, int batch, con
 }  // namespace dms
 
 using namespace dms;
+
+extern "C" dms_status dms_decode_attn_plan(dms_pool* pool, int n_layers, int batch, int* kernel,
+                                           int* cluster_size) {
+  if (!pool || !kernel || !cluster_size || n_layers < 1 || batch < 1) {
+    set_last_error("bad arguments");
+    return DMS_ERR_INVALID_ARG;
+  }
+  const PoolView& v = pool->view;
+  const int H = n_layers * batch * v.Hkv, g = v.Hq / v.Hkv;
+  *kernel = DMS_ATTN_STREAM_K;
+  *cluster_size = 0;
+  if (pool->attn_kernel == DMS_ATTN_STREAM_K) return DMS_OK;
+  int C = 0;
+  using bf = __nv_bfloat16;
+  dms_status st;
+  if (v.kv_dtype == DMS_BF16)
+    st = v.D == 128 ? cluster_setup<KV_BF16, 128, bf, false>(&C, H, g) : cluster_setup<KV_BF16, 64, bf, false>(&C, H, g);
+  else if (v.kv_dtype == DMS_FP8_E4M3)
+    st = cluster_setup<KV_FP8, 128, bf, false>(&C, H, g);
+  else if (v.kv_dtype == DMS_INT4)
+    st = cluster_setup<KV_INT4, 128, bf, false>(&C, H, g);
+  else
+    st = v.D == 128 ? cluster_setup<KV_F32, 128, float, false>(&C, H, g) : cluster_setup<KV_F32, 64, float, false>(&C, H, g);
+  if (st != DMS_OK) return st;
+  if (C >= 2 || pool->attn_kernel == DMS_ATTN_CLUSTER) {
+    *kernel = DMS_ATTN_CLUSTER;
+    *cluster_size = C;
+  }
+  return DMS_OK;
+}
 
 extern "C" dms_status dms_decode_step_layers(dms_pool* pool, int layer0, int n_layers, int batch,
                                              int64_t pos, const void* k, const void* v,

@@ -96,6 +96,7 @@ _SIGS = {
     "dms_pool_layout": (_I, [_P, ctypes.POINTER(PoolLayout)]),
     "dms_pool_set_wait_limit": (_I, [_P, ctypes.c_uint64]),
     "dms_pool_set_attn_kernel": (_I, [_P, _I]),
+    "dms_decode_attn_plan": (_I, [_P, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "dms_decode_step_layers": (_I, [_P, _I, _I, _I, _I64, _P, _P, _I, _P, _P, _I, _P, ctypes.c_float, _P,
                                     ctypes.c_size_t, _P]),
     "dms_stepper_inject_fault": (_I, [_P, _I]),
@@ -180,6 +181,14 @@ def dms_pool_set_wait_limit(pool: int, limit_ns: int):
 
 def dms_pool_set_attn_kernel(pool: int, kind: int):
     _check(lib().dms_pool_set_attn_kernel(pool, kind), "dms_pool_set_attn_kernel")
+
+
+def dms_decode_attn_plan(pool: int, n_layers: int, batch: int) -> tuple:
+    """(kernel, cluster_size) a decode attention call over n_layers x batch would use."""
+    k, c = _I(), _I()
+    _check(lib().dms_decode_attn_plan(pool, n_layers, batch, ctypes.byref(k), ctypes.byref(c)),
+           "dms_decode_attn_plan")
+    return k.value, c.value
 
 
 def dms_decode_step_layers(pool: int, layer0: int, n_layers: int, batch: int, pos: int, k: int, v: int,

@@ -205,6 +205,14 @@ dms_status dms_pool_set_wait_limit(dms_pool* pool, uint64_t limit_ns);
 #define DMS_ATTN_CLUSTER 2
 dms_status dms_pool_set_attn_kernel(dms_pool* pool, int kind);
 
+/* The kernel a decode attention call over n_layers x batch heads of this
+ * pool would use now (*kernel = DMS_ATTN_CLUSTER or DMS_ATTN_STREAM_K) and,
+ * for the cluster kernel, its CTAs per head (*cluster_size; 0 for stream-K).
+ * For the plain calls (dms_decode_attn_layers, dms_decode_step_layers); the
+ * current device must be the pool's.  Host query, nothing is launched. */
+dms_status dms_decode_attn_plan(dms_pool* pool, int n_layers, int batch, int* kernel,
+                                int* cluster_size);
+
 /* Region offsets of the pool buffer. */
 dms_status dms_pool_layout(const dms_pool* pool, dms_pool_layout_t* out);
 
