@@ -233,7 +233,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
                0x1: "gpu_idle"}
 
-    def __init__(self, index: int, period_s: float = 0.002):
+    def __init__(self, index: int, period_s: float = 0.0002):
         self.samples, self.reasons = [], 0
         self.ok = False
         try:
@@ -321,14 +321,18 @@ def cpu_baseline(wl, t0: int, n_heads: int, n_steps: int, bytes_per_step: float)
         for t in range(wl.prompt, t0):
             store.append(t, int(flags[t]))
         prep.append((flags, Kf, Vf, qs, store))
-    # timed: the oracle's decode step for each sampled head
+    # timed: the oracle's decode step for each sampled head, step by step
+    # (one step = every sampled head's step), and the bytes those heads hold
+    row_bytes = 2 * wl.kv_row_bytes()
+    sample_bytes = 0
     start = time.perf_counter()
-    for (flags, Kf, Vf, qs, store) in prep:
-        for s in range(n_steps):
-            t = t0 + s
+    for s in range(n_steps):
+        t = t0 + s
+        for (flags, Kf, Vf, qs, store) in prep:
             store.append(t, int(flags[t]))
             oatt.decode_attention(qs[s], Kf[:t + 1, None, :], Vf[:t + 1, None, :], flags[:t + 1, None],
                                   t, wl.window)
+            sample_bytes += store.n_retained * row_bytes
     elapsed = time.perf_counter() - start
     per_head_step = elapsed / (len(prep) * n_steps)
     step_time = per_head_step * H
@@ -338,6 +342,8 @@ def cpu_baseline(wl, t0: int, n_heads: int, n_steps: int, bytes_per_step: float)
                    f"t={t0}: slot bookkeeping + fp64 masked attention per head, {elapsed:.1f} s; "
                    f"per-step time = mean head-step time x {H} heads"),
         "seconds": elapsed, "step_seconds_extrapolated": step_time,
+        "sample_heads": len(prep), "sample_steps": n_steps, "sample_bytes": sample_bytes,
+        "sample_value": sample_bytes / elapsed / 1e9,
         "compaction": oracle_compaction(wl, picks[:4 if wl.prompt <= 32768 else 1]),
     }
 
@@ -440,27 +446,54 @@ def reduce_over_ranks(ms: float, nbytes: float, device="cpu"):
 # the benchmark
 # ---------------------------------------------------------------------------
 
+def needs_l2_flush(wl) -> bool:
+    """True when a step's held K/V (expected) fits in L2, so that timed steps
+    must start after an L2 flush."""
+    return expected_bytes_per_step(wl) <= L2_BYTES
+
+
+def bench_config(wl, world: int) -> dict:
+    """The `config` of a bench line (the same for both arms)."""
+    held = expected_bytes_per_step(wl)
+    l2 = (f"flush: {L2_FLUSH_BYTES >> 20} MB written then read before each timed step, outside its events "
+          f"({held / 1e6:.0f} MB of held K/V per step fits in the 126 MB L2)" if needs_l2_flush(wl) else
+          f"no flush: {held / 1e6:.0f} MB of held K/V read per step > 126 MB L2")
+    return {"workload": wl.name, "layers": wl.n_layers, "batch": wl.batch, "q_heads": wl.n_q_heads,
+            "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "prompt": wl.prompt, "window": wl.window,
+            "kv_dtype": wl.kv_dtype, "seed": wl.seed, "parallelism": f"replicas x{world}", "l2": l2}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     wl = with_kv_dtype(configs.BY_NAME[args.workload], args.kv_dtype)
     bps = expected_bytes_per_step(wl)
-    t0 = time.perf_counter()
     steps = max(1, args.steps)
-    per = max(1, args.cpu_steps // 3)
-    cb = cpu_baseline(wl, wl.prompt + args.warmup, max(8, args.cpu_heads // 3), per, bps)
+    n_heads = max(8, args.cpu_heads // 3)
+    H = wl.n_layers * wl.batch * wl.n_kv_heads
+    t0 = time.perf_counter()
+    if args.warmup > 0:   # untimed warm-up steps of the same sample
+        cpu_baseline(wl, wl.prompt, n_heads, min(args.warmup, 3), bps)
+    cb = cpu_baseline(wl, wl.prompt + args.warmup, n_heads, steps, bps)
     wall = time.perf_counter() - t0
     line = {
-        "impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
+        "impl": "reference", "metric": METRIC, "value": cb["sample_value"], "unit": "GB/s",
         "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
-        "ms_per_step": cb["step_seconds_extrapolated"] * 1e3, "higher_is_better": True,
+        "ms_per_step": cb["seconds"] / steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "bytes_per_step": bps},
-        "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "compaction")},
-        "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "note": ("the reference arm is the CPU oracle (the pages ship no code); each step is a bounded "
-                 "sample of the workload's decode step, extrapolated by head count"),
+        "config": bench_config(wl, args.gpus),
+        "timing": (f"host wall clock around the {steps} timed steps; each step is the oracle's decode step of "
+                   f"the same {cb['sample_heads']} sampled (layer, sequence, kv-head) heads of {H}, and the value "
+                   f"is the K/V those heads hold over that time"),
+        "sampled": {"heads": cb["sample_heads"], "of_heads": H, "steps": steps,
+                    "ms_per_full_step_extrapolated": cb["step_seconds_extrapolated"] * 1e3,
+                    "extrapolation": f"mean head-step time x {H} heads (not what was timed)"},
+        "cpu_baseline": {k: cb[k] for k in ("unit", "cores", "kind", "sample", "compaction")} |
+                        {"value": cb["sample_value"]},
+        "e2e": {"value": cb["sample_value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": ("the reference arm is the CPU oracle (the pages ship no code), timed on a bounded sample "
+                 "of each decode step"),
         "wall_s": wall,
     }
     print(json.dumps(line))
@@ -562,7 +595,7 @@ def main():
     # every timed step starts after an L2 flush (a write of L2_FLUSH_BYTES,
     # then a read of it, so that no dirty line is left for the step to write
     # back), outside the event pair that times it, and the step times are summed
-    flush = bool(bytes_step[W] <= L2_BYTES)
+    flush = needs_l2_flush(wl)
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=f"cuda:{local}") if flush else None
     flush_sink = torch.empty((), dtype=torch.int32, device=f"cuda:{local}")
 
@@ -758,14 +791,7 @@ def main():
                        "the K steps (an L2 flush between steps, outside the pairs)" if flush else
                        "CUDA events around one replay of a captured graph of the K steps"), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.kv_dtype == "bf16" else wl.kv_dtype, "data": "synthetic",
-            "config": {"workload": wl.name, "layers": L, "batch": B, "q_heads": wl.n_q_heads,
-                       "kv_heads": Hkv, "head_dim": D, "prompt": P, "window": w, "kv_dtype": wl.kv_dtype,
-                       "seed": wl.seed, "parallelism": f"replicas x{world}",
-                       "l2": (f"flush: {L2_FLUSH_BYTES >> 20} MB written then read before each timed step, outside "
-                              f"its events ({bytes_step[W] / 1e6:.0f} MB of held K/V per step fits in "
-                              f"the 126 MB L2)" if flush else
-                              f"no flush: {bytes_step[W] / 1e6:.0f} MB of held K/V read per step "
-                              f"> 126 MB L2")},
+            "config": bench_config(wl, world),
             "decode_steps_per_s": world * K / (ms_max * 1e-3),
             "per_layer_calls": per_layer_calls,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "compaction": compaction,
