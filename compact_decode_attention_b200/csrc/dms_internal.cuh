@@ -386,6 +386,12 @@ struct dms_pool;
 namespace dms {
 dms_status prefill_plan_launch(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
                                const uint8_t* evict, cudaStream_t stream);
+// prefill compaction of a copy store (bf16 / fp32) in one launch (csrc/prefill_cluster.cu),
+// for prompts of up to prefill_cluster_max_prompt() tokens
+int prefill_cluster_max_prompt();
+dms_status prefill_cluster_launch(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
+                                  const void* k, const void* v, dms_dtype in_dtype, const uint8_t* evict,
+                                  cudaStream_t stream);
 
 }  // namespace dms
 

@@ -12,7 +12,10 @@
 // eviction and the kept rows are quantised (FastDMS page, FP8 paragraph:
 // eviction is decided before FP8 quantisation).
 //
-// Two kernels, in stream order:
+// Copy stores (bf16, fp32) take one launch instead, a cluster per
+// (sequence, kv-head) (csrc/prefill_cluster.cu), for prompts up to 262144
+// tokens.  FP8 and 4-bit stores, and longer prompts, take two kernels, in
+// stream order:
 //   plan     one CTA per (256-token chunk, sequence): per-head kept counts by
 //            warp ballot + popcount (and, for an FP8 store, the per-head |x|
 //            maximum of every prompt row).  The last CTA of a sequence to
@@ -617,6 +620,8 @@ extern "C" dms_status dms_compact_prefill_seqs(dms_pool* pool, int layer, int se
     return DMS_ERR_UNSUPPORTED;
   }
   const bool bf16 = in_dtype == DMS_BF16;
+  if (!fp8 && !int4 && prompt_len <= prefill_cluster_max_prompt())   // copy stores: one launch
+    return prefill_cluster_launch(pool, layer, seq0, batch, prompt_len, k, v, in_dtype, evict, stream);
   dms_status st;
   if (fp8)
     st = bf16 ? launch_plan<__nv_bfloat16, true>(pool, layer, seq0, batch, prompt_len, evict, k, v, stream)
