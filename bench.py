@@ -69,6 +69,9 @@ def parse_args():
     ap.add_argument("--cpu-heads", type=int, default=72)
     ap.add_argument("--cpu-steps", type=int, default=90)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="run a short fixed case for kernel captures (prefill, 4 all-layer steps, "
+                         "2 steps as per-layer fused calls) and exit; prints no bench line")
     return ap.parse_args()
 
 
@@ -500,6 +503,28 @@ def run_reference(args):
     return 0
 
 
+def profile_case(wl, device):
+    """Prefill, then steps 0-3 as all-layer steps (attention in one launch
+    per step) and steps 4-5 as per-layer fused calls (append + attention in
+    one launch per layer): the case the kernel captures under profiles/ use."""
+    import torch
+    from compact_decode_attention_b200.workload import DeviceWorkload
+    dw = DeviceWorkload(wl, 6, device=device)
+    dw.prefill()
+    si, P, L = dw.step_inputs, wl.prompt, wl.n_layers
+    for s in range(4):
+        dw.step(s)
+    for s in range(4, 6):
+        for layer in range(L):
+            sl = slice(layer, layer + 1)
+            dw.pool.decode_step_layers(layer, P + s, si["k"][s][sl], si["v"][s][sl], si["evict"][s][sl],
+                                       si["q"][s][sl], dw.out[sl])
+    torch.cuda.synchronize()
+    flags = dw.pool.stats().error_flags
+    print(json.dumps({"profile_case": wl.name, "error_flags": flags}))
+    return 0 if flags == 0 else 1
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -539,6 +564,8 @@ def main():
         if rank == 0:
             print(json.dumps({"workload": wl.name, "prompt": wl.prompt, "prefill_attention": line}))
         return 0
+    if args.profile_case:          # a short case for profiler captures (one GPU)
+        return profile_case(wl, f"cuda:{local}")
     W, K, E = args.warmup, args.steps, args.e2e_steps
     R = min(K, 64)                 # instrumented steps for the attention-kernel timing
     RL = min(K, 16)                # steps issued as per-layer calls (each of the two forms)
@@ -575,9 +602,11 @@ def main():
                   "peak_kind": f"{hbm_kind} copy bandwidth",
                   "ms_per_layer": compact_ms / L, "algorithmic_bytes_per_layer": compact_bytes / L,
                   "full_read_value": full_read_bytes / (compact_ms * 1e-3) / 1e9,
-                  "timing": "CUDA events around each layer's dms_compact_prefill call (plan and "
-                            "scatter kernels), layers after the first captured in one CUDA graph "
-                            "replayed once; median layer"}
+                  "kernels": ("prefill_cluster_kernel (one launch a layer)"
+                              if wl.kv_dtype in ("bf16", "f32") and P <= 16 * 63 * 256 else
+                              "prefill_plan_kernel + prefill_scatter_kernel (two launches a layer)"),
+                  "timing": "CUDA events around each layer's dms_compact_prefill call, layers after "
+                            "the first captured in one CUDA graph replayed once; median layer"}
     held = base + np.cumsum(H - retired)                  # after step s
     bytes_step = held.astype(np.float64) * row_bytes
 
