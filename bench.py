@@ -185,48 +185,105 @@ def projection_line(wl, device, n_calls=8):
             "kernel": "project_append_kernel<128> (split-K over d_model, epilogue appends)"}
 
 
+def prefill_tiles(flags: np.ndarray, P: int, w: int, tile: int = 128):
+    """Key tiles per (sequence, kv-head) that the prefill attention kernel
+    computes, summed over its query tiles: (dense, sparse).  flags uint8
+    [B, P, Hkv].  Dense: every causal tile.  Sparse: a query tile
+    [i0, i0 + 128) reads the band of prompt tiles from the one holding
+    i0 - w + 1 to the diagonal, plus ceil(n_far / 128) tiles of older
+    unflagged keys from the store (n_far of them), unless those tiles' slots
+    run past the head's kept rows (then all causal tiles)."""
+    B, _, Hkv = flags.shape
+    n = (P + tile - 1) // tile
+    dense = n * (n + 1) // 2
+    sparse = np.zeros((B, Hkv), dtype=np.int64)
+    for b in range(B):
+        for h in range(Hkv):
+            f = flags[b, :, h]
+            unfl = np.concatenate([[0], np.cumsum(f == 0)])
+            kept = int(unfl[P]) + int(np.sum(f[max(0, P - w):] != 0))
+            tot = 0
+            for qt in range(n):
+                lo = qt * tile - w + 1
+                kl = lo // tile if lo > 0 else 0
+                nf = (int(unfl[kl * tile]) + tile - 1) // tile
+                if kl > 0 and nf * tile <= kept:
+                    tot += nf + qt - kl + 1
+                else:
+                    tot += qt + 1
+            sparse[b, h] = tot
+    return dense, sparse
+
+
 def prefill_attention_line(wl, device, n_layers=3):
     """dms_prefill_attn (prompt attention under the DMS mask on the tensor
-    cores, fused with compaction) at the workload's prompt shapes: one layer
-    per call, the median of n_layers calls, each into an empty layer of a
-    small pool.  FLOPs = the causal 128 x 128 tiles the kernel computes
-    (QK and PV, 2 flops per multiply-add)."""
+    cores, with compaction) at the workload's prompt shapes: one layer per
+    call, the median of n_layers calls, each into an empty layer of a small
+    pool; the default reading (old kept keys from the store) and the dense
+    one (every causal tile from the prompt).  FLOPs = 4 D 128^2 per key tile
+    computed (QK and PV, 2 flops per multiply-add); the visible (query, key)
+    pairs give the method's own count."""
     import torch
     from compact_decode_attention_b200 import dms
     from compact_decode_attention_b200.workload import DeviceWorkload, STREAM_K, STREAM_Q, STREAM_V
     if wl.kv_dtype != "bf16" or wl.head_dim not in (64, 128):
         return None
     P, B, Hq, Hkv, D = wl.prompt, wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    g = Hq // Hkv
     gen = DeviceWorkload(wl, 0, device=device, max_blocks=16)
     k = gen.normal(STREAM_K, 0, 1, 0, P, Hkv)[0]
     v = gen.normal(STREAM_V, 0, 1, 0, P, Hkv)[0]
     q = gen.normal(STREAM_Q, 0, 1, 0, P, Hq)[0]
     f = gen.flags(0, 1, 0, P)[0]
     out = torch.empty_like(q)
-    pool = dms.Pool(n_layers + 1, B, Hq, Hkv, D, wl.window, dms.DMS_BF16,
-                    (n_layers + 1) * B * Hkv * (P // 64 + 2), P + 1, device=device)
-    pool.prefill_attn(0, 0, q, k, v, f, out)          # warm-up (module load, attributes)
-    torch.cuda.synchronize()
-    ts = []
-    for layer in range(1, n_layers + 1):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        pool.prefill_attn(layer, 0, q, k, v, f, out)
-        e1.record()
+
+    def time_mode(mode):
+        pool = dms.Pool(n_layers + 1, B, Hq, Hkv, D, wl.window, dms.DMS_BF16,
+                        (n_layers + 1) * B * Hkv * (P // 64 + 2), P + 1, device=device)
+        pool.set_prefill_mode(mode)
+        pool.prefill_attn(0, 0, q, k, v, f, out)          # warm-up (module load, attributes)
         torch.cuda.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    if pool.stats(check=False).error_flags:
-        raise SystemExit("prefill attention set the device error word")
-    ms = float(np.median(ts))
-    n = (P + 127) // 128
-    flops = 4.0 * D * 128 * 128 * n * (n + 1) / 2 * Hq * B
+        ts = []
+        for layer in range(1, n_layers + 1):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            pool.prefill_attn(layer, 0, q, k, v, f, out)
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        if pool.stats(check=False).error_flags:
+            raise SystemExit("prefill attention set the device error word")
+        return float(np.median(ts))
+
+    ms = time_mode(dms.PREFILL_SPARSE)
+    ms_dense = time_mode(dms.PREFILL_DENSE)
+    fl = f.cpu().numpy()
+    dense_tiles, sparse_tiles = prefill_tiles(fl, P, wl.window)
+    tile_flops = 4.0 * D * 128 * 128
+    flops = tile_flops * float(sparse_tiles.sum()) * g
+    flops_dense = tile_flops * dense_tiles * Hq * B
+    # visible (query, key) pairs: min(i + 1, w) + unflagged keys older than the window
+    pairs = 0
+    for b in range(B):
+        for h in range(Hkv):
+            unfl = np.concatenate([[0], np.cumsum(fl[b, :, h] == 0)])
+            i = np.arange(P)
+            pairs += int(np.sum(np.minimum(i + 1, wl.window) + unfl[np.maximum(i - wl.window + 1, 0)])) * g
     peak, kind = measured_bf16_tflops()
     tf = flops / (ms * 1e-3) / 1e12
     return {"value": tf, "unit": "TFLOP/s", "ms_per_layer": ms, "prompt": P,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
                          "frac": tf / peak, "peak_kind": kind},
-            "flops_basis": "causal 128x128 tiles computed (QK^T and PV), per layer",
-            "kernel": f"prefill_attn_kernel<{D}> (tcgen05, fused compaction)"}
+            "flops_basis": "128x128 key tiles computed (QK^T and PV), per layer: prompt tiles from the "
+                           "window band to the diagonal plus tiles of older kept keys read from the store",
+            "tiles_per_layer": int(sparse_tiles.sum()) * g, "dense_tiles_per_layer": int(dense_tiles) * Hq * B,
+            "visible_pair_tflops": 4.0 * D * pairs / (ms * 1e-3) / 1e12,
+            "dense": {"ms_per_layer": ms_dense, "value": flops_dense / (ms_dense * 1e-3) / 1e12,
+                      "frac": flops_dense / (ms_dense * 1e-3) / 1e12 / peak,
+                      "mode": "every causal tile from the prompt, kept rows stored by the attention kernel"},
+            "speedup_vs_dense": ms_dense / ms,
+            "timing": "CUDA events around each layer's dms_prefill_attn call (compaction included), median",
+            "kernel": f"prefill_attn_kernel<{D}> (tcgen05), old kept keys from the store"}
 
 
 class ClockSampler:

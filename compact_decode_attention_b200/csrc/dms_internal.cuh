@@ -405,6 +405,7 @@ struct dms_pool {
   int device;
   int sm_count;
   int attn_kernel;  // DMS_ATTN_* (dms_pool_set_attn_kernel)
+  int prefill_mode; // DMS_PREFILL_* (dms_pool_set_prefill_mode)
 };
 
 namespace dms {

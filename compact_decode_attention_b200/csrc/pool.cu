@@ -346,6 +346,7 @@ dms_status dms_pool_create(const dms_pool_config* cfg, void* dev_buf, size_t byt
   p->device = dev;
   p->sm_count = device_sm_count(dev);
   p->attn_kernel = DMS_ATTN_AUTO;
+  p->prefill_mode = DMS_PREFILL_SPARSE;
   p->view = make_view(*cfg, lay, dev_buf);
   st = clear_pool(p, stream);
   if (st != DMS_OK) {
@@ -385,6 +386,15 @@ dms_status dms_pool_set_attn_kernel(dms_pool* pool, int kind) {
     return DMS_ERR_INVALID_ARG;
   }
   pool->attn_kernel = kind;
+  return DMS_OK;
+}
+
+dms_status dms_pool_set_prefill_mode(dms_pool* pool, int mode) {
+  if (!pool || (mode != DMS_PREFILL_SPARSE && mode != DMS_PREFILL_DENSE)) {
+    set_last_error("null pool or unknown prefill mode %d", mode);
+    return DMS_ERR_INVALID_ARG;
+  }
+  pool->prefill_mode = mode;
   return DMS_OK;
 }
 

@@ -26,12 +26,27 @@
 // filled by tensor-map (TMA) loads: the query tile once, then per key tile
 // its keys into the one tile buffer and, once S has read them, its values
 // into the same buffer while the softmax runs (about 100 KB a CTA, so that
-// two fit on an SM).  The CTA of the first query head of each kv-head group
-// writes, at its diagonal key tile, the tile's kept rows into the pool (slots
-// from the prefix counts of the count and plan kernels) and the window ring.
+// two fit on an SM).
+//
+// Which key tiles (bf16 store):
+//   sparse (default)  the layer is compacted before this kernel.  A key
+//       older than i0 - w + 1 is outside the window of every query of the
+//       tile [i0, i0 + 128), so it is seen exactly when it carries no flag,
+//       and the unflagged keys are what the store holds, in position order.
+//       Keys before the band of tiles that holds i0 - w + 1 are therefore
+//       read from the store as dense 128-key tiles (two 64-row blocks, masked
+//       only past the last one), and only the band and the diagonal come
+//       from the prompt with the full mask.  At a keep rate k and a prompt
+//       of P >> w the tiles computed fall from about P^2 / 2 to about
+//       k P^2 / 2 + P w.
+//   dense  every causal tile from the prompt; the CTA of the first query
+//       head of each kv-head group writes, at its diagonal key tile, the
+//       tile's kept rows into the pool (slots from the prefix counts of the
+//       plan kernel) and the window ring.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <string.h>
 
 #include "dms_internal.cuh"
 #include "umma.cuh"
@@ -57,7 +72,7 @@ struct PaSmem {
   static constexpr int FLAGS = P + kPaTile * kPaTile * 2;  // 2 x 4 words of evict-flag bits
   static constexpr int BARS = FLAGS + 2 * kPaTile;     // mbarriers: S, O, Q, K, V
   static constexpr int MISC = BARS + 64;               // tmem base, scan
-  static constexpr int RED = MISC + 64;                // [SPLIT parts][128 rows] floats
+  static constexpr int RED = MISC + 128;               // [SPLIT parts][128 rows] floats
   static constexpr int BYTES = RED + PaSplit<D>::SPLIT * kPaTile * 4 + 1024;  // + alignment slack
 };
 
@@ -70,8 +85,8 @@ template <int D>
 __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     prefill_attn_kernel(PoolView v, int layer, int seq0, int P, const __grid_constant__ CUtensorMap tq,
                         const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                        const uint8_t* evict, __nv_bfloat16* out, float scale_log2, int n_qtiles,
-                        int compact) {
+                        const __grid_constant__ CUtensorMap tpool, const uint8_t* evict,
+                        __nv_bfloat16* out, float scale_log2, int n_qtiles, int compact, int sparse) {
   using S = PaSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -95,7 +110,8 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
   uint64_t* bar_k = bar_s + 3;
   uint64_t* bar_v = bar_s + 4;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::MISC);
-  int* s_scan = reinterpret_cast<int*>(smem + S::MISC) + 4;
+  int* s_scan = reinterpret_cast<int*>(smem + S::MISC) + 4;   // [8]
+  int* s_cnt = reinterpret_cast<int*>(smem + S::MISC) + 12;   // [16]
 
   // tensor-map loads of one [128 x D] tile: boxes of 64 columns x 128 rows
   // with 128-byte swizzle (the operand image of umma.cuh); rows past the
@@ -105,6 +121,20 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
 #pragma unroll
     for (int kb = 0; kb < D / 64; ++kb)
       umma::tma_load_3d(dst + kb * kPaTile * 128, map, x0 + kb * 64, row0, b, bar);
+  };
+  // a far tile: the store's slots [128 k, 128 k + 128) of this head, two
+  // 64-row blocks; each block's K (kv = 0) or V (kv = 1) rows are copied per
+  // 64-column half into rows 0..63 / 64..127 of the tile.  The store's
+  // 16-byte chunks are already XOR-swizzled by row (chunk c of row r at
+  // c ^ (r & 7)), which is the operand image a 128-byte-swizzled box load
+  // makes, so the copies use no swizzle of their own.
+  auto load_far = [&](uint8_t* dst, int blk0, int blk1, int kv, uint64_t* bar) {
+    mbar_arrive_expect_tx(bar, S::TILE);
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb) {
+      umma::tma_load_4d(dst + kb * kPaTile * 128, &tpool, 0, kb, 0, 2 * blk0 + kv, bar);
+      umma::tma_load_4d(dst + kb * kPaTile * 128 + 64 * 128, &tpool, 0, kb, 0, 2 * blk1 + kv, bar);
+    }
   };
   // evict flag of key j0 + r of tile kt (loaded a tile ahead, packed later)
   auto flag_of = [&](int kt) -> uint8_t {
@@ -127,11 +157,74 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     umma::tmem_relinquish();
   }
   __syncthreads();  // barriers initialised before any thread waits on them
-  if (tid == 0) {
-    load_tile(smem + S::Q, &tq, hq * D, i0, bar_q);
-    load_tile(smem + S::KV, &tk, hkv * D, 0, bar_k);
+  if (tid == 0) load_tile(smem + S::Q, &tq, hq * D, i0, bar_q);
+
+  // ---- the key tiles of this query tile ----
+  // Every row i of the tile sees keys j < lo = i0 - w + 1 only when they carry
+  // no evict flag (i - j >= w for all of them).  With `sparse`, keys before
+  // the band [kt_lo * 128, i0 + 128) that holds lo are not read from the
+  // prompt: the unflagged ones among them are the store's first n_far slots
+  // (the store keeps them in position order), read as nf dense "far" tiles;
+  // the band is read from the prompt with the full mask.  The store must
+  // hold this head's prompt, which the counts check: its held count must
+  // equal the kept count of the flags, and the far tiles' slots must exist;
+  // otherwise every key tile comes from the prompt.
+  int kt_lo = 0, nf = 0, n_far = 0;
+  const int32_t* far_bt = v.bt + int64_t(v.head(layer, seq0 + b, hkv)) * v.mbh;
+  if (sparse) {
+    const int lo = i0 - v.w + 1;
+    const int kl = lo > 0 ? lo / kPaTile : 0;
+    if (kl > 0) {
+      const int bs = kl * kPaTile;
+      int cf = 0, ct = 0;
+      for (int j = tid; j < P; j += THREADS) {
+        const uint8_t f = evict[(int64_t(b) * P + j) * v.Hkv + hkv];
+        ct += (f == 0 || P - 1 - j < v.w) ? 1 : 0;
+        cf += (f == 0 && j < bs) ? 1 : 0;
+      }
+      cf = __reduce_add_sync(0xffffffffu, cf);
+      ct = __reduce_add_sync(0xffffffffu, ct);
+      if (lane == 0) {
+        s_cnt[warp] = cf;
+        s_cnt[8 + warp] = ct;
+      }
+      // a compaction that failed (this call's or an earlier one: the error
+      // word is sticky) may have left a head's old rows in place
+      if (tid == 0) s_scan[0] = *reinterpret_cast<volatile uint32_t*>(&v.hdr->error) != 0u;
+      __syncthreads();
+      int tf = 0, tt = 0;
+#pragma unroll
+      for (int x = 0; x < THREADS / 32; ++x) {
+        tf += s_cnt[x];
+        tt += s_cnt[8 + x];
+      }
+      const int held = v.n_slots[v.head(layer, seq0 + b, hkv)];
+      const int nft = (tf + kPaTile - 1) / kPaTile;
+      if (!s_scan[0] && held == tt && nft * kPaTile <= held && 2 * nft <= v.mbh) {
+        kt_lo = kl;
+        nf = nft;
+        n_far = tf;
+      }
+    }
   }
-  uint8_t f_cur = flag_of(0);
+  const int n_tiles = nf + (qt - kt_lo + 1);
+  // block ids of far tile k (thread 0; the next tile's are loaded a tile ahead)
+  int fb0 = 0, fb1 = 0, nb0 = 0, nb1 = 0;
+  if (tid == 0) {
+    if (nf > 0) {
+      fb0 = far_bt[0];
+      fb1 = far_bt[1];
+      if (nf > 1) {
+        nb0 = far_bt[2];
+        nb1 = far_bt[3];
+      }
+      load_far(smem + S::KV, fb0, fb1, 0, bar_k);
+    } else {
+      load_tile(smem + S::KV, &tk, hkv * D, kt_lo * kPaTile, bar_k);
+    }
+  }
+  auto flag_at = [&](int it) -> uint8_t { return it >= nf ? flag_of(kt_lo + it - nf) : 0; };
+  uint8_t f_cur = flag_at(0);
   umma::fence_before_sync();
   __syncthreads();
   umma::fence_after_sync();
@@ -147,22 +240,36 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
   volatile int never = 0;
   bool ok = true;
 
-  for (int kt = 0; kt <= qt; ++kt) {
-    const int cur = kt & 1, j0 = kt * kPaTile;
-    if (kt > 0) {  // P V of tile kt-1 is done: P and the tile buffer are free
-      ok &= mbar_wait_bounded(bar_o, (kt - 1) & 1, &never, v.wait_ns);
+  for (int it = 0; it < n_tiles; ++it) {
+    const bool far = it < nf;
+    const int kt = far ? -1 : kt_lo + it - nf;
+    const int cur = it & 1, j0 = kt * kPaTile;
+    if (it > 0) {  // P V of tile it-1 is done: P and the tile buffer are free
+      ok &= mbar_wait_bounded(bar_o, (it - 1) & 1, &never, v.wait_ns);
       __syncwarp();
       umma::fence_after_sync();
-      if (tid == 0) load_tile(smem + S::KV, &tk, hkv * D, j0, bar_k);
+      if (tid == 0) {
+        if (far) {
+          fb0 = nb0;
+          fb1 = nb1;
+          if (it + 1 < nf) {  // ids of the next far tile, used one tile later
+            nb0 = far_bt[2 * (it + 1)];
+            nb1 = far_bt[2 * (it + 1) + 1];
+          }
+          load_far(smem + S::KV, fb0, fb1, 0, bar_k);
+        } else {
+          load_tile(smem + S::KV, &tk, hkv * D, j0, bar_k);
+        }
+      }
       __syncwarp();
     }
     {  // this tile's flags as 4 words of bits (bit c = key j0 + c flagged)
       const unsigned fw = __ballot_sync(0xffffffffu, f_cur != 0);
       if (lane == 0 && h == 0) s_fbits[cur * 4 + warp] = fw;
     }
-    const uint8_t f_next = kt < qt ? flag_of(kt + 1) : 0;
-    if (kt == 0) ok &= mbar_wait_bounded(bar_q, 0, &never, v.wait_ns);
-    ok &= mbar_wait_bounded(bar_k, kt & 1, &never, v.wait_ns);  // K_kt landed
+    const uint8_t f_next = it + 1 < n_tiles ? flag_at(it + 1) : 0;
+    if (it == 0) ok &= mbar_wait_bounded(bar_q, 0, &never, v.wait_ns);
+    ok &= mbar_wait_bounded(bar_k, it & 1, &never, v.wait_ns);  // K of tile it landed
     __syncwarp();
     __syncthreads();
     const uint32_t aK = smem_u32(smem + S::KV), aV = aK;
@@ -174,19 +281,29 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
                        k0 > 0);
       umma::commit(bar_s);
     }
-    ok &= mbar_wait_bounded(bar_s, kt & 1, &never, v.wait_ns);
+    ok &= mbar_wait_bounded(bar_s, it & 1, &never, v.wait_ns);
     __syncwarp();  // lanes leave the wait loop independently; tcgen05.ld is warp-collective
     umma::fence_after_sync();
     // S read the keys: the values of the same tile stream into the buffer
     // while the softmax runs
-    if (tid == 0) load_tile(smem + S::KV, &tv, hkv * D, j0, bar_v);
+    if (tid == 0) {
+      if (far) load_far(smem + S::KV, fb0, fb1, 1, bar_v);
+      else load_tile(smem + S::KV, &tv, hkv * D, j0, bar_v);
+    }
     __syncwarp();
 
     // ---- masked online softmax on query row i (log2 domain) ----
     // visibility of key j0 + c as bits: flag clear or inside the window
     // (c >= i - w + 1 - j0), causal (c <= i - j0), inside the prompt (c < P - j0)
     uint32_t vis[HC / 32];
-    {
+    if (far) {  // every row sees the tile's first n_far - 128 it slots
+      const int lim = n_far - it * kPaTile;
+#pragma unroll
+      for (int x = 0; x < HC / 32; ++x) {
+        const int x_lt = lim - 32 * ((HC / 32) * h + x);
+        vis[x] = x_lt <= 0 ? 0u : x_lt >= 32 ? ~0u : (1u << x_lt) - 1u;
+      }
+    } else {
       const int hi = i - j0, lo = i - v.w + 1 - j0, end = P - j0;
 #pragma unroll
       for (int x = 0; x < HC / 32; ++x) {
@@ -245,7 +362,7 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
       *reinterpret_cast<uint4*>(smem + S::P + umma::sw128_offset(kPaTile, r, h * HC + ch * 8)) = w4;
     }
     // O row *= alpha when this warp has a row whose maximum moved
-    if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+    if (it > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
       for (int cb = 0; cb < OC / 32; ++cb) {
         float o[32];
@@ -263,16 +380,16 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     __syncthreads();
     if (tid == 0) {
       umma::fence_after_sync();
-      ok &= mbar_wait_bounded(bar_v, kt & 1, &never, v.wait_ns);  // V_kt landed
+      ok &= mbar_wait_bounded(bar_v, it & 1, &never, v.wait_ns);  // V of tile it landed
 #pragma unroll
       for (int k0 = 0; k0 < kPaTile; k0 += 16)
         umma::mma_bf16(t_o, umma::desc_k16(aP, kPaTile, k0), umma::desc_mn_k16(aV, kPaTile, k0), idO,
-                       kt > 0 || k0 > 0);
+                       it > 0 || k0 > 0);
       umma::commit(bar_o);
     }
     __syncwarp();
   }
-  ok &= mbar_wait_bounded(bar_o, qt & 1, &never, v.wait_ns);
+  ok &= mbar_wait_bounded(bar_o, (n_tiles - 1) & 1, &never, v.wait_ns);
   __syncwarp();
   umma::fence_after_sync();
 
@@ -415,6 +532,29 @@ static dms_status encode_bf16_map(CUtensorMap* m, const void* base, int batch, i
   return DMS_OK;
 }
 
+// Tensor map of the store's blocks as [2 * max_blocks tiles (block b's K
+// tile is 2b, its V tile 2b + 1)][64 rows][D / 64 halves][64 bf16]: boxes of
+// one 64-column half of 64 rows, no swizzle (the rows are stored swizzled).
+static dms_status encode_store_map(CUtensorMap* m, const PoolView& pv) {
+  auto enc = tensor_map_encoder();
+  if (!enc) {
+    set_last_error("cuTensorMapEncodeTiled is not available");
+    return DMS_ERR_CUDA;
+  }
+  const cuuint64_t dims[4] = {64, cuuint64_t(pv.D / 64), cuuint64_t(kBlockTokens), cuuint64_t(2 * pv.max_blocks)};
+  const cuuint64_t strides[3] = {128, cuuint64_t(pv.row_bytes), cuuint64_t(pv.tile_bytes)};
+  const cuuint32_t box[4] = {64, 1, cuuint32_t(kBlockTokens), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, pv.blocks, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_last_error("cuTensorMapEncodeTiled (store) failed (%d)", int(r));
+    return DMS_ERR_CUDA;
+  }
+  return DMS_OK;
+}
+
 extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,
                                        const void* q, const void* k, const void* v,
                                        dms_dtype in_dtype, const uint8_t* evict, void* out,
@@ -442,15 +582,23 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
     set_last_error("q, k, v and out must be 16-byte aligned");
     return DMS_ERR_INVALID_ARG;
   }
-  // A bf16 store takes the kept rows from the attention kernel's tiles, after
-  // the prefix counts and block tables of the count and plan kernels.  FP8
-  // and 4-bit stores quantise them: the layer is compacted first, as by
+  // bf16 store, sparse (default): the layer is compacted first and the
+  // attention kernel reads the old kept keys back from the store.  bf16
+  // store, dense: the kept rows come from the attention kernel's tiles, after
+  // the prefix counts and block tables of the plan kernel.  FP8 and 4-bit
+  // stores quantise the rows: the layer is compacted first, as by
   // dms_compact_prefill_seqs (scales, plan, scatter), and the attention
-  // kernel stores nothing.
-  const int fused = pv.kv_dtype == DMS_BF16 ? 1 : 0;
-  dms_status st = fused ? prefill_plan_launch(pool, layer, seq0, batch, prompt_len, evict, stream)
-                        : dms_compact_prefill_seqs(pool, layer, seq0, batch, prompt_len, k, v, in_dtype,
-                                                   evict, stream);
+  // kernel reads every key from the bf16 inputs.
+  const bool bf16_store = pv.kv_dtype == DMS_BF16;
+  const int sparse = bf16_store && pool->prefill_mode == DMS_PREFILL_SPARSE &&
+                     2 * pv.max_blocks <= int64_t(INT32_MAX) ? 1 : 0;
+  const int fused = bf16_store && !sparse ? 1 : 0;
+  CUtensorMap tpool;
+  memset(&tpool, 0, sizeof(tpool));
+  dms_status st = sparse ? encode_store_map(&tpool, pv) : DMS_OK;
+  if (st != DMS_OK) return st;
+  st = fused ? prefill_plan_launch(pool, layer, seq0, batch, prompt_len, evict, stream)
+             : dms_compact_prefill_seqs(pool, layer, seq0, batch, prompt_len, k, v, in_dtype, evict, stream);
   if (st != DMS_OK) return st;
   const int n_qtiles = (prompt_len + kPaTile - 1) / kPaTile;
   const dim3 grid(n_qtiles, pv.Hq, batch);
@@ -474,7 +622,7 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
                           carveout_attr, "prefill attn carveout");
     if (st != DMS_OK) return st;
     prefill_attn_kernel<128><<<grid, PaSplit<128>::THREADS, PaSmem<128>::BYTES, stream>>>(
-        pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, fused);
+        pv, layer, seq0, prompt_len, tq, tk, tv, tpool, evict, ko, scale_log2, n_qtiles, fused, sparse);
   } else {
     static FuncAttrCache smem_attr, carveout_attr;  // per device
     st = ensure_func_attr(reinterpret_cast<const void*>(prefill_attn_kernel<64>),
@@ -487,7 +635,7 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
                           carveout_attr, "prefill attn carveout");
     if (st != DMS_OK) return st;
     prefill_attn_kernel<64><<<grid, PaSplit<64>::THREADS, PaSmem<64>::BYTES, stream>>>(
-        pv, layer, seq0, prompt_len, tq, tk, tv, evict, ko, scale_log2, n_qtiles, fused);
+        pv, layer, seq0, prompt_len, tq, tk, tv, tpool, evict, ko, scale_log2, n_qtiles, fused, sparse);
   }
   return cuda_status(cudaGetLastError(), "prefill_attn_kernel");
 }

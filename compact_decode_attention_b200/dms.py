@@ -32,6 +32,7 @@ DEVERR_BAD_SEQUENCE = 0x40
 
 FAULT_DROP_INPUT_SIGNAL = 1
 ATTN_AUTO, ATTN_STREAM_K, ATTN_CLUSTER = 0, 1, 2
+PREFILL_SPARSE, PREFILL_DENSE = 0, 1
 
 BLOCK_TOKENS = 64
 
@@ -96,6 +97,7 @@ _SIGS = {
     "dms_pool_layout": (_I, [_P, ctypes.POINTER(PoolLayout)]),
     "dms_pool_set_wait_limit": (_I, [_P, ctypes.c_uint64]),
     "dms_pool_set_attn_kernel": (_I, [_P, _I]),
+    "dms_pool_set_prefill_mode": (_I, [_P, _I]),
     "dms_decode_attn_plan": (_I, [_P, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "dms_decode_step_layers": (_I, [_P, _I, _I, _I, _I64, _P, _P, _I, _P, _P, _I, _P, ctypes.c_float, _P,
                                     ctypes.c_size_t, _P]),
@@ -181,6 +183,10 @@ def dms_pool_set_wait_limit(pool: int, limit_ns: int):
 
 def dms_pool_set_attn_kernel(pool: int, kind: int):
     _check(lib().dms_pool_set_attn_kernel(pool, kind), "dms_pool_set_attn_kernel")
+
+
+def dms_pool_set_prefill_mode(pool: int, mode: int):
+    _check(lib().dms_pool_set_prefill_mode(pool, mode), "dms_pool_set_prefill_mode")
 
 
 def dms_decode_attn_plan(pool: int, n_layers: int, batch: int) -> tuple:
@@ -399,6 +405,9 @@ class Pool:
 
     def set_attn_kernel(self, kind: int):
         dms_pool_set_attn_kernel(self.handle, int(kind))
+
+    def set_prefill_mode(self, mode: int):
+        dms_pool_set_prefill_mode(self.handle, int(mode))
 
     def compact_prefill(self, layer, k, v, evict, stream=None):
         B, P = k.shape[0], k.shape[1]

@@ -205,6 +205,25 @@ dms_status dms_pool_set_wait_limit(dms_pool* pool, uint64_t limit_ns);
 #define DMS_ATTN_CLUSTER 2
 dms_status dms_pool_set_attn_kernel(dms_pool* pool, int kind);
 
+/* How dms_prefill_attn reads the keys of a bf16 pool (host setting of the
+ * handle, applied to calls made after it):
+ *   DMS_PREFILL_SPARSE  the layer is compacted first (as by
+ *                       dms_compact_prefill_seqs); then, for a tile of 128
+ *                       queries, keys older than every query's window are
+ *                       read from the compact store (only the unflagged ones
+ *                       exist there, in position order) as dense 128-key
+ *                       tiles, and only the tiles holding the window edge,
+ *                       the diagonal and the keys between are read from the
+ *                       prompt with the full mask.  The default.
+ *   DMS_PREFILL_DENSE   every causal key tile is read from the prompt and
+ *                       masked; the kernel stores each diagonal tile's kept
+ *                       rows itself.
+ * Both give the same attention (rounding order aside) and the same store.
+ * FP8 and 4-bit pools always use the dense form on the bf16 inputs. */
+#define DMS_PREFILL_SPARSE 0
+#define DMS_PREFILL_DENSE 1
+dms_status dms_pool_set_prefill_mode(dms_pool* pool, int mode);
+
 /* The kernel a decode attention call over n_layers x batch heads of this
  * pool would use now (*kernel = DMS_ATTN_CLUSTER or DMS_ATTN_STREAM_K) and,
  * for the cluster kernel, its CTAs per head (*cluster_size; 0 for stream-K).
@@ -291,8 +310,10 @@ dms_status dms_decode_attn_seqs(dms_pool* pool, int layer0, int n_layers, int n_
  *   q, out  [batch, P, Hq, D]  bf16      k, v  [batch, P, Hkv, D]  bf16
  *   evict   [batch, P, Hkv]    uint8     sm_scale <= 0 selects 1/sqrt(D)
  * Needs a bf16, FP8 or 4-bit pool with head_dim 64 or 128 (else
- * DMS_ERR_UNSUPPORTED).  A bf16 pool is filled by the attention kernel
- * itself; an FP8 or 4-bit pool is compacted first, as by
+ * DMS_ERR_UNSUPPORTED).  A bf16 pool is compacted first and its old kept
+ * keys are read back from the store (DMS_PREFILL_SPARSE, the default), or
+ * filled by the attention kernel itself (DMS_PREFILL_DENSE, see
+ * dms_pool_set_prefill_mode); an FP8 or 4-bit pool is compacted first, as by
  * dms_compact_prefill_seqs, and the attention reads the bf16 inputs.
  * The sequences must be empty in that layer (else DMS_DEVERR_LAYER_NOT_EMPTY
  * and nothing is stored; the outputs are still computed).  Runs on the

@@ -118,3 +118,62 @@ def test_unsupported_pools_are_refused():
     with pytest.raises(dms.DmsError) as e:
         pool.prefill_attn(0, 0, x, kv, kv, f, x)
     assert e.value.status == dms.DMS_ERR_UNSUPPORTED
+
+
+def _sampled_check(got, Q, K, V, F, w, idx, b=0):
+    for i in idx:
+        exp = oatt.decode_attention(Q[b, i].astype(np.float64), K[b, :i + 1], V[b, :i + 1], F[b, :i + 1], i, w)
+        err = np.abs(got[b, i] - exp).max()
+        assert err < TOL, (i, err)
+
+
+@pytest.mark.parametrize("D,w,p_keep", [(128, 128, 0.15), (64, 128, 0.15), (128, 256, 0.0),
+                                        (128, 128, 1.0), (64, 200, 0.4)])
+def test_sparse_and_dense_reading_agree_with_the_oracle(D, w, p_keep):
+    """Old kept keys read back from the store (default) against every key
+    tile read from the prompt: the same store bit for bit, outputs within
+    the bf16 bound of the oracle and of each other.  Keep rates 0 (far keys
+    all evicted: no far tile), 1 (every old key kept) and in between, ragged
+    far counts (not multiples of 128), a window that is not a tile multiple."""
+    B, P, Hq, Hkv = 2, 1500, 8, 2
+    Q, K, V, F = _inputs(300 + D + w, B, P, Hq, Hkv, D, p_keep)
+    outs, states = {}, {}
+    for mode in (dms.PREFILL_SPARSE, dms.PREFILL_DENSE):
+        pool = dms.Pool(1, B, Hq, Hkv, D, w, dms.DMS_BF16, B * Hkv * (P // 64 + 2), P + 1)
+        pool.set_prefill_mode(mode)
+        outs[mode] = _run(pool, 0, Q, K, V, F)
+        _check_store(pool, 0, K, V, F, P, w)
+        states[mode] = read_state(pool)
+    assert np.isfinite(outs[dms.PREFILL_SPARSE]).all()
+    for key in ("n_slots", "n_retained", "ring"):
+        assert np.array_equal(states[0][key], states[1][key]), key
+    assert np.abs(outs[0] - outs[1]).max() < TOL
+    idx = sorted(set(np.random.default_rng(D + w).integers(0, P, 24).tolist()) | {0, w, 383, 384, P - 1})
+    for b in range(B):
+        _sampled_check(outs[dms.PREFILL_SPARSE], Q, K, V, F, w, idx, b)
+
+
+def test_sparse_reading_falls_back_when_far_blocks_are_missing():
+    """A window shorter than a key tile with few kept keys: the far tiles'
+    second block may not exist, so those query tiles read the prompt."""
+    B, P, Hq, Hkv, D, w = 1, 700, 8, 2, 128, 16
+    Q, K, V, F = _inputs(55, B, P, Hq, Hkv, D, 0.05)
+    pool = dms.Pool(1, B, Hq, Hkv, D, w, dms.DMS_BF16, B * Hkv * (P // 64 + 2), P + 1)
+    got = _run(pool, 0, Q, K, V, F)
+    exp = oatt.prefill_attention(Q[0].astype(np.float64), K[0], V[0], F[0], w)
+    assert np.abs(got[0] - exp).max() < TOL
+    _check_store(pool, 0, K, V, F, P, w)
+
+
+def test_a_layer_that_is_not_empty_still_gets_correct_outputs():
+    """The second prompt into the same layer is refused by the compaction
+    (DMS_DEVERR_LAYER_NOT_EMPTY); the store still holds the first prompt,
+    so the attention must read every key from the second prompt."""
+    B, P, Hq, Hkv, D, w = 1, 900, 8, 2, 128, 128
+    Q, K, V, F = _inputs(61, B, P, Hq, Hkv, D, 0.2)
+    Q2, K2, V2, F2 = _inputs(62, B, P, Hq, Hkv, D, 0.2)
+    pool = dms.Pool(1, B, Hq, Hkv, D, w, dms.DMS_BF16, 2 * B * Hkv * (P // 64 + 2), P + 1)
+    _run(pool, 0, Q, K, V, F)
+    got = _run(pool, 0, Q2, K2, V2, F2)
+    assert read_state(pool)["error"] & dms.DEVERR_LAYER_NOT_EMPTY
+    _sampled_check(got, Q2, K2, V2, F2, w, [0, 200, 511, 512, 640, 777, P - 1])
