@@ -81,6 +81,32 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Paired fp32 arithmetic of sm_100 (one instruction for two lanes of
+// values, each rounded as the scalar operation would be) and the
+// three-input maximum.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
+      "mov.b64 rc, {%5, %6};\n\tfma.rn.f32x2 %0, ra, rb, rc;\n\t}"
+      : "=l"(d)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 ra, rb;\n\tmov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
+      "add.rn.f32x2 %0, ra, rb;\n\t}"
+      : "=l"(d)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 template <int D>
 __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     prefill_attn_kernel(PoolView v, int layer, int seq0, int P, const __grid_constant__ CUtensorMap tq,
@@ -492,6 +518,416 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
   if (warp == 0) umma::tmem_dealloc(tbase, 256);
 }
 
+// ---------------------------------------------------------------------------
+// Two query heads of one kv-head per CTA (sparse reading, an even group
+// size g).  The heads share every K and V tile; per key tile the MMA thread
+// issues S_A = Q_A K^T and S_B = Q_B K^T, and the softmax of head A runs
+// while S_B is computed, that of head B while P_A V is, so the tensor cores
+// and the softmax warps work at the same time inside one CTA.  K and V have
+// their own buffers: the next key tile loads as soon as both S products have
+// read the current one, during the softmax; the values of a tile load once
+// both P V products of the previous tile are done.  One CTA per SM (the four
+// accumulators take all 512 tensor-memory columns).
+//
+// Warps 0-7 run head A's softmax, 8-15 head B's (two threads per query row,
+// as above), warp 16 loads tiles and issues the MMAs (one thread).  The
+// hand-offs are mbarriers: S ready (commit), P ready (one arrival per
+// softmax warp), O done (commit), K and V buffers free (commit).
+constexpr int kPpThreads = 2 * 2 * kPaTile + 32;
+constexpr int kPpMaxFarIds = 2048;   // far-tile block ids cached in shared memory
+
+template <int D>
+struct PpSmem {
+  static constexpr int TILE = kPaTile * D * 2;
+  static constexpr int QA = 0, QB = TILE, K = 2 * TILE, V = 3 * TILE;
+  static constexpr int PA = 4 * TILE;                          // [128 queries x 128 keys] bf16
+  static constexpr int PB = PA + kPaTile * kPaTile * 2;
+  static constexpr int FLAGS = PB + kPaTile * kPaTile * 2;     // [2 heads][2][4] words
+  static constexpr int BARS = FLAGS + 64;                      // 16 mbarriers
+  static constexpr int MISC = BARS + 128;                      // tmem base, abort, counts
+  static constexpr int RED = MISC + 256;                       // [2 heads][2 parts][128] floats
+  static constexpr int IDS = RED + 2 * 2 * kPaTile * 4;        // far-tile block ids
+  static constexpr int USED = IDS + kPpMaxFarIds * 4;
+  // at least 116 KB, so that a second CTA never waits on an SM for tensor memory
+  static constexpr int BYTES = (USED > 116 * 1024 ? USED : 116 * 1024) + 1024;
+};
+
+__device__ __forceinline__ void pp_group_bar(int grp) {
+  asm volatile("bar.sync %0, 256;" ::"r"(1 + grp) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPpThreads, 1)
+    prefill_pair_kernel(PoolView v, int layer, int seq0, int P, const __grid_constant__ CUtensorMap tq,
+                        const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                        const __grid_constant__ CUtensorMap tpool, const uint8_t* evict,
+                        __nv_bfloat16* out, float scale_log2, int n_qtiles) {
+  using S = PpSmem<D>;
+  constexpr int SPLIT = 2, HC = kPaTile / SPLIT, OC = D / SPLIT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qt = n_qtiles - 1 - int(blockIdx.x);  // heaviest query tiles first
+  const int hq0 = 2 * int(blockIdx.y), b = blockIdx.z;
+  const int g = v.Hq / v.Hkv, hkv = hq0 / g;
+  const int i0 = qt * kPaTile;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BARS);
+  uint64_t* bar_q = bars + 0;
+  uint64_t* bar_k = bars + 1;
+  uint64_t* bar_v = bars + 2;
+  uint64_t* bar_kfree = bars + 3;
+  uint64_t* bar_vfree = bars + 4;
+  uint64_t* bar_s = bars + 5;    // [2] S of head A / B computed
+  uint64_t* bar_o = bars + 7;    // [2] P V of head A / B computed
+  uint64_t* bar_p = bars + 9;    // [2] P of head A / B in shared memory
+  uint64_t* bar_fin = bars + 11; // every MMA done (exit)
+  int* s_misc = reinterpret_cast<int*>(smem + S::MISC);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_misc);
+  volatile int* s_abort = s_misc + 1;
+  int* s_cnt = s_misc + 8;       // [17 warps][2]
+  int* s_ids = reinterpret_cast<int*>(smem + S::IDS);
+
+  if (tid == 0) {
+    for (int x = 0; x < 12; ++x) mbar_init(&bars[x], x == 9 || x == 10 ? 8 : 1);
+    s_misc[1] = 0;
+    s_misc[2] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 16) {
+    umma::tmem_alloc(s_tmem, 512);
+    umma::tmem_relinquish();
+  }
+
+  // ---- the key tiles of this query tile (as in prefill_attn_kernel) ----
+  int kt_lo = 0, nf = 0, n_far = 0;
+  const int32_t* far_bt = v.bt + int64_t(v.head(layer, seq0 + b, hkv)) * v.mbh;
+  {
+    const int lo = i0 - v.w + 1;
+    const int kl = lo > 0 ? lo / kPaTile : 0;
+    if (kl > 0) {
+      const int bs = kl * kPaTile;
+      int cf = 0, ct = 0;
+      for (int j = tid; j < P; j += kPpThreads) {
+        const uint8_t f = evict[(int64_t(b) * P + j) * v.Hkv + hkv];
+        ct += (f == 0 || P - 1 - j < v.w) ? 1 : 0;
+        cf += (f == 0 && j < bs) ? 1 : 0;
+      }
+      cf = __reduce_add_sync(0xffffffffu, cf);
+      ct = __reduce_add_sync(0xffffffffu, ct);
+      if (lane == 0) {
+        s_cnt[2 * warp] = cf;
+        s_cnt[2 * warp + 1] = ct;
+      }
+      if (tid == 0) s_misc[2] = *reinterpret_cast<volatile uint32_t*>(&v.hdr->error) != 0u;
+      __syncthreads();
+      int tf = 0, tt = 0;
+#pragma unroll
+      for (int x = 0; x < kPpThreads / 32; ++x) {
+        tf += s_cnt[2 * x];
+        tt += s_cnt[2 * x + 1];
+      }
+      const int held = v.n_slots[v.head(layer, seq0 + b, hkv)];
+      const int nft = (tf + kPaTile - 1) / kPaTile;
+      if (!s_misc[2] && held == tt && nft * kPaTile <= held && 2 * nft <= v.mbh) {
+        kt_lo = kl;
+        nf = nft;
+        n_far = tf;
+      }
+    }
+  }
+  const int n_tiles = nf + (qt - kt_lo + 1);
+  umma::fence_before_sync();
+  __syncthreads();  // barriers initialised, tensor memory allocated
+  umma::fence_after_sync();
+  const uint32_t tbase = *s_tmem;
+
+  if (warp == 16) {
+    // ======================= loads and MMAs (one thread) =======================
+    const bool cached = 2 * nf <= kPpMaxFarIds;
+    if (cached)
+      for (int x = lane; x < 2 * nf; x += 32) s_ids[x] = far_bt[x];
+    __syncwarp();
+    if (lane == 0) {
+      auto far_id = [&](int x) { return cached ? s_ids[x] : far_bt[x]; };
+      auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, int x0, int row0, uint64_t* bar) {
+        mbar_arrive_expect_tx(bar, S::TILE);
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb)
+          umma::tma_load_3d(dst + kb * kPaTile * 128, map, x0 + kb * 64, row0, b, bar);
+      };
+      // tile it's keys (kv = 0) or values (kv = 1) into dst
+      auto load_kv = [&](int it, int kv, uint64_t* bar) {
+        uint8_t* dst = smem + (kv ? S::V : S::K);
+        if (it < nf) {
+          const int blk0 = far_id(2 * it), blk1 = far_id(2 * it + 1);
+          mbar_arrive_expect_tx(bar, S::TILE);
+#pragma unroll
+          for (int kb = 0; kb < D / 64; ++kb) {
+            umma::tma_load_4d(dst + kb * kPaTile * 128, &tpool, 0, kb, 0, 2 * blk0 + kv, bar);
+            umma::tma_load_4d(dst + kb * kPaTile * 128 + 64 * 128, &tpool, 0, kb, 0, 2 * blk1 + kv, bar);
+          }
+        } else {
+          load_tile(dst, kv ? &tv : &tk, hkv * D, (kt_lo + it - nf) * kPaTile, bar);
+        }
+      };
+      constexpr uint32_t idS = umma::idesc_bf16_f32(kPaTile, kPaTile);
+      constexpr uint32_t idO = umma::idesc_bf16_f32_bmn(kPaTile, D);
+      const uint32_t aQ[2] = {smem_u32(smem + S::QA), smem_u32(smem + S::QB)};
+      const uint32_t aPb[2] = {smem_u32(smem + S::PA), smem_u32(smem + S::PB)};
+      const uint32_t aK = smem_u32(smem + S::K), aV = smem_u32(smem + S::V);
+      mbar_arrive_expect_tx(bar_q, 2 * S::TILE);
+#pragma unroll
+      for (int kb = 0; kb < D / 64; ++kb) {
+        umma::tma_load_3d(smem + S::QA + kb * kPaTile * 128, &tq, hq0 * D + kb * 64, i0, b, bar_q);
+        umma::tma_load_3d(smem + S::QB + kb * kPaTile * 128, &tq, (hq0 + 1) * D + kb * 64, i0, b, bar_q);
+      }
+      load_kv(0, 0, bar_k);
+      load_kv(0, 1, bar_v);
+      int nk = 1, nv = 1, wk = 0, wv = 0;   // loads issued / waited on
+      bool qdone = false, ok = true;
+      // S of head hh for tile it (its keys have landed)
+      auto mma_s = [&](int hh) {
+#pragma unroll
+        for (int k0 = 0; k0 < D; k0 += 16)
+          umma::mma_bf16(tbase + 256 * hh, umma::desc_k16(aQ[hh], kPaTile, k0), umma::desc_k16(aK, kPaTile, k0),
+                         idS, k0 > 0);
+        umma::commit(&bar_s[hh]);
+      };
+      auto mma_pv = [&](int hh, int it) {
+#pragma unroll
+        for (int k0 = 0; k0 < kPaTile; k0 += 16)
+          umma::mma_bf16(tbase + 256 * hh + 128, umma::desc_k16(aPb[hh], kPaTile, k0),
+                         umma::desc_mn_k16(aV, kPaTile, k0), idO, it > 0 || k0 > 0);
+        umma::commit(&bar_o[hh]);
+      };
+      // Issue order: S_A(0) S_B(0), then per tile it: P_A V(it), S_A(it+1),
+      // P_B V(it), S_B(it+1).  While head A's softmax of tile it + 1 runs, the
+      // tensor cores compute head B's P V of tile it and S of tile it + 1,
+      // and the other way round.
+      ok = mbar_wait_bounded(bar_q, 0, s_abort, v.wait_ns);
+      qdone = ok;
+      ok = ok && mbar_wait_bounded(bar_k, 0, s_abort, v.wait_ns);
+      if (ok) {
+        wk = 1;
+        umma::fence_after_sync();
+        mma_s(0);
+        mma_s(1);
+        umma::commit(bar_kfree);   // phase 0: both S of tile 0 read the keys
+        if (n_tiles > 1) {
+          ok = mbar_wait_bounded(bar_kfree, 0, s_abort, v.wait_ns);
+          if (ok) {
+            load_kv(1, 0, bar_k);
+            nk = 2;
+          }
+        }
+      }
+      for (int it = 0; it < n_tiles && ok; ++it) {
+        const bool more = it + 1 < n_tiles;
+        if (!(ok = mbar_wait_bounded(bar_v, it & 1, s_abort, v.wait_ns))) break;
+        wv = it + 1;
+        if (!(ok = mbar_wait_bounded(&bar_p[0], it & 1, s_abort, v.wait_ns))) break;
+        umma::fence_after_sync();
+        mma_pv(0, it);
+        if (more) {
+          if (!(ok = mbar_wait_bounded(bar_k, (it + 1) & 1, s_abort, v.wait_ns))) break;
+          wk = it + 2;
+          umma::fence_after_sync();
+          mma_s(0);
+        }
+        if (!(ok = mbar_wait_bounded(&bar_p[1], it & 1, s_abort, v.wait_ns))) break;
+        umma::fence_after_sync();
+        mma_pv(1, it);
+        umma::commit(bar_vfree);     // phase it: both P V of tile it read the values
+        if (more) {
+          mma_s(1);
+          umma::commit(bar_kfree);   // phase it + 1: both S of tile it + 1 read the keys
+          if (!(ok = mbar_wait_bounded(bar_vfree, it & 1, s_abort, v.wait_ns))) break;
+          load_kv(it + 1, 1, bar_v);
+          nv = it + 2;
+          if (it + 2 < n_tiles) {
+            if (!(ok = mbar_wait_bounded(bar_kfree, (it + 1) & 1, s_abort, v.wait_ns))) break;
+            load_kv(it + 2, 0, bar_k);
+            nk = it + 3;
+          }
+        }
+      }
+      if (!ok) {
+        *s_abort = 1;
+        report_error(v.hdr, DMS_DEVERR_TIMEOUT, layer, seq0 + b, hq0);
+      }
+      // drain: every MMA issued and every copy still landing, each wait bounded
+      volatile int never = 0;
+      umma::commit(bar_fin);
+      mbar_wait_bounded(bar_fin, 0, &never, v.wait_ns);
+      if (!qdone) mbar_wait_bounded(bar_q, 0, &never, v.wait_ns);
+      if (nk > wk) mbar_wait_bounded(bar_k, (nk - 1) & 1, &never, v.wait_ns);
+      if (nv > wv) mbar_wait_bounded(bar_v, (nv - 1) & 1, &never, v.wait_ns);
+    }
+    __syncwarp();
+  } else {
+    // ======================= softmax of head A (warps 0-7) or B (8-15) =======================
+    const int G = warp >> 3;
+    const int tg = tid & 255, r = tg & (kPaTile - 1), h = tg >> 7, wg = tg >> 5;
+    const int i = i0 + r;
+    const int hq = hq0 + G;
+    uint32_t* fbits = reinterpret_cast<uint32_t*>(smem + S::FLAGS) + 8 * G;   // [2][4]
+    float* red = reinterpret_cast<float*>(smem + S::RED) + 2 * kPaTile * G;   // [2 parts][128]
+    uint8_t* Pbuf = smem + (G ? S::PB : S::PA);
+    const uint32_t t_s = tbase + 256 * G, t_o = t_s + 128;
+    auto flag_at = [&](int it) -> uint8_t {
+      if (it < nf || h != 0) return 0;
+      const int j = (kt_lo + it - nf) * kPaTile + r;
+      return j < P ? evict[(int64_t(b) * P + j) * v.Hkv + hkv] : 0;
+    };
+    // a wait that gives up stops every other wait of the CTA at once
+    auto wait_g = [&](uint64_t* bar, uint32_t parity) {
+      if (mbar_wait_bounded(bar, parity, s_abort, v.wait_ns)) return true;
+      *s_abort = 1;
+      return false;
+    };
+    float m = -1e30f, l = 0.f;
+    bool ok = true;
+    uint8_t f_cur = flag_at(0);
+    for (int it = 0; it < n_tiles; ++it) {
+      const bool far = it < nf;
+      const int cur = it & 1, j0 = (kt_lo + it - nf) * kPaTile;
+      {
+        const unsigned fw = __ballot_sync(0xffffffffu, f_cur != 0);
+        if (lane == 0 && h == 0) fbits[cur * 4 + wg] = fw;
+      }
+      const uint8_t f_next = it + 1 < n_tiles ? flag_at(it + 1) : 0;
+      ok &= wait_g(&bar_s[G], it & 1);
+      __syncwarp();
+      umma::fence_after_sync();
+      pp_group_bar(G);   // the flag bits of every warp of the head
+      uint32_t vis[HC / 32];
+      if (far) {
+        const int lim = n_far - it * kPaTile;
+#pragma unroll
+        for (int x = 0; x < HC / 32; ++x) {
+          const int x_lt = lim - 32 * ((HC / 32) * h + x);
+          vis[x] = x_lt <= 0 ? 0u : x_lt >= 32 ? ~0u : (1u << x_lt) - 1u;
+        }
+      } else {
+        const int hi = i - j0, lo = i - v.w + 1 - j0, end = P - j0;
+#pragma unroll
+        for (int x = 0; x < HC / 32; ++x) {
+          const int wd = (HC / 32) * h + x, c0 = 32 * wd;
+          const int x_le = hi - c0, x_ge = lo - c0, x_lt = end - c0;
+          const uint32_t le = x_le < 0 ? 0u : x_le >= 31 ? ~0u : (2u << x_le) - 1u;
+          const uint32_t ge = x_ge <= 0 ? ~0u : x_ge >= 32 ? 0u : ~((1u << x_ge) - 1u);
+          const uint32_t lt = x_lt <= 0 ? 0u : x_lt >= 32 ? ~0u : (1u << x_lt) - 1u;
+          vis[x] = (~fbits[cur * 4 + wd] | ge) & le & lt;
+        }
+      }
+      float s[HC];
+#pragma unroll
+      for (int cb = 0; cb < HC / 32; ++cb) {
+        float x[32];
+        umma::ld32(umma::taddr_of(t_s, warp, h * HC + cb * 32), x);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[cb * 32 + e] = x[e];
+      }
+      umma::wait_ld();
+      // mask only the 32-key words that are not wholly visible
+#pragma unroll
+      for (int x = 0; x < HC / 32; ++x) {
+        if (vis[x] != ~0u) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[x * 32 + e] = ((vis[x] >> e) & 1u) ? s[x * 32 + e] : -INFINITY;
+        }
+      }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < HC; c += 2) mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], s[c], s[c + 1]);
+      red[h * kPaTile + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
+      pp_group_bar(G);
+      float mx = red[r];
+#pragma unroll
+      for (int x = 1; x < SPLIT; ++x) mx = fmaxf(mx, red[x * kPaTile + r]);
+      float alpha = 1.f;
+      if (mx > m + 8.f) {   // lazy rescaling, as in prefill_attn_kernel
+        alpha = fast_exp2(m - mx);
+        m = mx;
+      }
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < HC; c += 2) {
+        float a0, a1;
+        ffma2(a0, a1, s[c], s[c + 1], scale_log2, scale_log2, -m, -m);
+        s[c] = fast_exp2(a0);
+        s[c + 1] = fast_exp2(a1);
+        const int q = (c >> 1) & 1;
+        fadd2(sum4[2 * q], sum4[2 * q + 1], sum4[2 * q], sum4[2 * q + 1], s[c], s[c + 1]);
+      }
+      l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+      if (it > 0) {   // P V of the previous tile: P buffer free, O settled
+        ok &= wait_g(&bar_o[G], (it - 1) & 1);
+        __syncwarp();
+        umma::fence_after_sync();
+      }
+#pragma unroll
+      for (int ch = 0; ch < HC / 8; ++ch) {
+        uint4 w4;
+        w4.x = pack2_bf16(s[ch * 8 + 0], s[ch * 8 + 1]);
+        w4.y = pack2_bf16(s[ch * 8 + 2], s[ch * 8 + 3]);
+        w4.z = pack2_bf16(s[ch * 8 + 4], s[ch * 8 + 5]);
+        w4.w = pack2_bf16(s[ch * 8 + 6], s[ch * 8 + 7]);
+        *reinterpret_cast<uint4*>(Pbuf + umma::sw128_offset(kPaTile, r, h * HC + ch * 8)) = w4;
+      }
+      if (it > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int cb = 0; cb < OC / 32; ++cb) {
+          float o[32];
+          umma::ld32(umma::taddr_of(t_o, warp, h * OC + cb * 32), o);
+          umma::wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          umma::st32(umma::taddr_of(t_o, warp, h * OC + cb * 32), o);
+        }
+        umma::wait_st();
+      }
+      fence_proxy_async_smem();   // P before the tensor cores read it
+      umma::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_p[G]);
+      f_cur = f_next;
+    }
+    ok &= wait_g(&bar_o[G], (n_tiles - 1) & 1);
+    __syncwarp();
+    umma::fence_after_sync();
+    pp_group_bar(G);   // every thread has read the last row maxima
+    red[h * kPaTile + r] = l;
+    pp_group_bar(G);
+    float lsum = red[r];
+#pragma unroll
+    for (int x = 1; x < SPLIT; ++x) lsum += red[x * kPaTile + r];
+    const float inv = i < P ? 1.f / lsum : 0.f;
+    __nv_bfloat16* dst = out + (int64_t(b) * P + i) * (int64_t(v.Hq) * D) + int64_t(hq) * D + h * OC;
+#pragma unroll
+    for (int cb = 0; cb < OC / 32; ++cb) {
+      float o[32];
+      umma::ld32(umma::taddr_of(t_o, warp, h * OC + cb * 32), o);
+      umma::wait_ld();
+      if (i < P) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 w4;
+          w4.x = pack2_bf16(o[e + 0] * inv, o[e + 1] * inv);
+          w4.y = pack2_bf16(o[e + 2] * inv, o[e + 3] * inv);
+          w4.z = pack2_bf16(o[e + 4] * inv, o[e + 5] * inv);
+          w4.w = pack2_bf16(o[e + 6] * inv, o[e + 7] * inv);
+          *reinterpret_cast<uint4*>(dst + cb * 32 + e) = w4;
+        }
+      }
+    }
+    if (!ok && tg == 0) report_error(v.hdr, DMS_DEVERR_TIMEOUT, layer, seq0 + b, hq);
+  }
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == 16) umma::tmem_dealloc(tbase, 512);
+}
+
 }  // namespace dms
 
 using namespace dms;
@@ -610,6 +1046,27 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
   if (st == DMS_OK) st = encode_bf16_map(&tv, v, batch, prompt_len, pv.Hkv * pv.D);
   if (st != DMS_OK) return st;
   auto ko = static_cast<__nv_bfloat16*>(out);
+  if (sparse && (pv.Hq / pv.Hkv) % 2 == 0) {   // two query heads of a kv-head per CTA
+    const dim3 grid2(n_qtiles, pv.Hq / 2, batch);
+    if (pv.D == 128) {
+      static FuncAttrCache smem_attr;  // per device
+      st = ensure_func_attr(reinterpret_cast<const void*>(prefill_pair_kernel<128>),
+                            cudaFuncAttributeMaxDynamicSharedMemorySize, int(PpSmem<128>::BYTES), smem_attr,
+                            "prefill pair smem attribute");
+      if (st != DMS_OK) return st;
+      prefill_pair_kernel<128><<<grid2, kPpThreads, PpSmem<128>::BYTES, stream>>>(
+          pv, layer, seq0, prompt_len, tq, tk, tv, tpool, evict, ko, scale_log2, n_qtiles);
+    } else {
+      static FuncAttrCache smem_attr;  // per device
+      st = ensure_func_attr(reinterpret_cast<const void*>(prefill_pair_kernel<64>),
+                            cudaFuncAttributeMaxDynamicSharedMemorySize, int(PpSmem<64>::BYTES), smem_attr,
+                            "prefill pair smem attribute");
+      if (st != DMS_OK) return st;
+      prefill_pair_kernel<64><<<grid2, kPpThreads, PpSmem<64>::BYTES, stream>>>(
+          pv, layer, seq0, prompt_len, tq, tk, tv, tpool, evict, ko, scale_log2, n_qtiles);
+    }
+    return cuda_status(cudaGetLastError(), "prefill_pair_kernel");
+  }
   if (pv.D == 128) {
     static FuncAttrCache smem_attr, carveout_attr;  // per device
     st = ensure_func_attr(reinterpret_cast<const void*>(prefill_attn_kernel<128>),

@@ -127,15 +127,16 @@ def _sampled_check(got, Q, K, V, F, w, idx, b=0):
         assert err < TOL, (i, err)
 
 
-@pytest.mark.parametrize("D,w,p_keep", [(128, 128, 0.15), (64, 128, 0.15), (128, 256, 0.0),
-                                        (128, 128, 1.0), (64, 200, 0.4)])
-def test_sparse_and_dense_reading_agree_with_the_oracle(D, w, p_keep):
+@pytest.mark.parametrize("D,w,p_keep,Hq", [(128, 128, 0.15, 8), (64, 128, 0.15, 8), (128, 256, 0.0, 8),
+                                           (128, 128, 1.0, 8), (64, 200, 0.4, 8), (128, 128, 0.2, 6)])
+def test_sparse_and_dense_reading_agree_with_the_oracle(D, w, p_keep, Hq):
     """Old kept keys read back from the store (default) against every key
     tile read from the prompt: the same store bit for bit, outputs within
     the bf16 bound of the oracle and of each other.  Keep rates 0 (far keys
     all evicted: no far tile), 1 (every old key kept) and in between, ragged
-    far counts (not multiples of 128), a window that is not a tile multiple."""
-    B, P, Hq, Hkv = 2, 1500, 8, 2
+    far counts (not multiples of 128), a window that is not a tile multiple;
+    an even group size runs two query heads per CTA, an odd one (g = 3) one."""
+    B, P, Hkv = 2, 1500, 2
     Q, K, V, F = _inputs(300 + D + w, B, P, Hq, Hkv, D, p_keep)
     outs, states = {}, {}
     for mode in (dms.PREFILL_SPARSE, dms.PREFILL_DENSE):
