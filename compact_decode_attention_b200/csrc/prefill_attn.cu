@@ -796,10 +796,12 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         if (lane == 0 && h == 0) fbits[cur * 4 + wg] = fw;
       }
       const uint8_t f_next = it + 1 < n_tiles ? flag_at(it + 1) : 0;
-      ok &= wait_g(&bar_s[G], it & 1);
+      // one warp of the head polls the mbarrier; the named barrier holds the
+      // other seven without issuing (it also publishes the flag bits)
+      if (wg == 0) ok &= wait_g(&bar_s[G], it & 1);
       __syncwarp();
+      pp_group_bar(G);
       umma::fence_after_sync();
-      pp_group_bar(G);   // the flag bits of every warp of the head
       uint32_t vis[HC / 32];
       if (far) {
         const int lim = n_far - it * kPaTile;
@@ -893,10 +895,10 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       if (lane == 0) mbar_arrive(&bar_p[G]);
       f_cur = f_next;
     }
-    ok &= wait_g(&bar_o[G], (n_tiles - 1) & 1);
+    if (wg == 0) ok &= wait_g(&bar_o[G], (n_tiles - 1) & 1);
     __syncwarp();
+    pp_group_bar(G);   // the last P V is done; every thread has read the last row maxima
     umma::fence_after_sync();
-    pp_group_bar(G);   // every thread has read the last row maxima
     red[h * kPaTile + r] = l;
     pp_group_bar(G);
     float lsum = red[r];
