@@ -283,7 +283,8 @@ def prefill_attention_line(wl, device, n_layers=3):
                       "mode": "every causal tile from the prompt, kept rows stored by the attention kernel"},
             "speedup_vs_dense": ms_dense / ms,
             "timing": "CUDA events around each layer's dms_prefill_attn call (compaction included), median",
-            "kernel": f"prefill_attn_kernel<{D}> (tcgen05), old kept keys from the store"}
+            "kernel": (f"prefill_pair_kernel<{D}>" if g % 2 == 0 else f"prefill_attn_kernel<{D}>") +
+                      " (tcgen05), old kept keys from the store"}
 
 
 class ClockSampler:

@@ -1,7 +1,8 @@
 """Host logic of bench.py on CPU: the cross-rank reduction with two gloo
 ranks (max of device times, sum of bytes), the expected-bytes formula, the
 store-dtype override, the sysfs cpu-list parser, the lookup of a profiled
-traffic ratio and the reference arm's line."""
+traffic ratio, the reference arm's line and the prefill attention's tile
+count."""
 import json
 import os
 import subprocess
@@ -104,3 +105,33 @@ def test_reference_arm_prints_one_line():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["cpu_baseline"]["compaction"]["ms_per_layer"] > 0
+
+
+def test_prefill_tile_counts_reduce_to_closed_forms():
+    """bench.prefill_tiles (the FLOP count of the prefill attention line):
+    the dense count is the number of causal tiles n (n + 1) / 2; with no
+    evict flag every old key sits in the store, so the far tiles are the old
+    tiles themselves and the sparse count equals the dense one; with every
+    key flagged only the band is read (for w = 128: the diagonal tile and
+    the one before it); any flags give a count between the two."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    P, w = 1000, 128
+    n = (P + 127) // 128
+    none = np.zeros((2, P, 3), np.uint8)
+    dense, sparse = bench.prefill_tiles(none, P, w)
+    assert dense == n * (n + 1) // 2
+    assert (sparse == dense).all()
+    allf = np.ones((1, P, 2), np.uint8)
+    _, sp = bench.prefill_tiles(allf, P, w)
+    assert (sp == 1 + 2 * (n - 1)).all()
+    rng = np.random.default_rng(3)
+    f = (rng.random((1, P, 4)) < 0.8).astype(np.uint8)
+    _, sp = bench.prefill_tiles(f, P, w)
+    assert (sp >= 1 + 2 * (n - 1)).all() and (sp <= dense).all()
+    # a window shorter than a tile with few kept keys: far tiles whose slots
+    # would run past the head's kept rows fall back to the causal tiles
+    f = (rng.random((1, P, 1)) < 0.97).astype(np.uint8)
+    _, sp = bench.prefill_tiles(f, P, 16)
+    assert sp[0, 0] <= dense
