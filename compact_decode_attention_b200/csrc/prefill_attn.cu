@@ -518,6 +518,27 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
   if (warp == 0) umma::tmem_dealloc(tbase, 256);
 }
 
+// Unflagged keys of head (b, hkv) before position bs (a multiple of 128 below
+// P - w, so kept = unflagged there), from the kept-token prefix counts the
+// layer's compaction left per 256-token chunk, plus the first 128 tokens of
+// bs's chunk when bs is not a chunk start.  Every thread calls it (one block
+// barrier); s_tmp holds 4 ints.
+__device__ __forceinline__ int far_keys(const PoolView& v, const uint8_t* evict, int b, int hkv, int P, int bs,
+                                        int tid, int* s_tmp) {
+  const int c = bs >> 8;
+  const int base = v.chunk_counts[(int64_t(b) * v.Hkv + hkv) * v.n_chunks_max + c];
+  if (bs & 255) {
+    if (tid < kPaTile) {
+      const int j = (c << 8) + tid;
+      const unsigned m = __ballot_sync(0xffffffffu, evict[(int64_t(b) * P + j) * v.Hkv + hkv] == 0);
+      if ((tid & 31) == 0) s_tmp[tid >> 5] = __popc(m);
+    }
+    __syncthreads();
+    return base + s_tmp[0] + s_tmp[1] + s_tmp[2] + s_tmp[3];
+  }
+  return base;
+}
+
 // ---------------------------------------------------------------------------
 // Two query heads of one kv-head per CTA (sparse reading, an even group
 // size g).  The heads share every K and V tile; per key tile the MMA thread
@@ -590,8 +611,15 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   if (tid == 0) {
     for (int x = 0; x < 12; ++x) mbar_init(&bars[x], x == 9 || x == 10 ? 8 : 1);
     s_misc[1] = 0;
-    s_misc[2] = 0;
+    s_misc[2] = *reinterpret_cast<volatile uint32_t*>(&v.hdr->error) != 0u;
     fence_mbar_init();
+    // both query tiles, while the key schedule is worked out
+    mbar_arrive_expect_tx(bar_q, 2 * S::TILE);
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb) {
+      umma::tma_load_3d(smem + S::QA + kb * kPaTile * 128, &tq, hq0 * D + kb * 64, i0, b, bar_q);
+      umma::tma_load_3d(smem + S::QB + kb * kPaTile * 128, &tq, (hq0 + 1) * D + kb * 64, i0, b, bar_q);
+    }
   }
   if (warp == 16) {
     umma::tmem_alloc(s_tmem, 512);
@@ -599,36 +627,20 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   }
 
   // ---- the key tiles of this query tile (as in prefill_attn_kernel) ----
+  // The store holds this head's prompt when the layer's compaction (just
+  // before this kernel) succeeded for every head: the error word is clear
+  // (it is sticky, so an earlier error also sends every tile to the prompt).
   int kt_lo = 0, nf = 0, n_far = 0;
   const int32_t* far_bt = v.bt + int64_t(v.head(layer, seq0 + b, hkv)) * v.mbh;
   {
     const int lo = i0 - v.w + 1;
     const int kl = lo > 0 ? lo / kPaTile : 0;
     if (kl > 0) {
-      const int bs = kl * kPaTile;
-      int cf = 0, ct = 0;
-      for (int j = tid; j < P; j += kPpThreads) {
-        const uint8_t f = evict[(int64_t(b) * P + j) * v.Hkv + hkv];
-        ct += (f == 0 || P - 1 - j < v.w) ? 1 : 0;
-        cf += (f == 0 && j < bs) ? 1 : 0;
-      }
-      cf = __reduce_add_sync(0xffffffffu, cf);
-      ct = __reduce_add_sync(0xffffffffu, ct);
-      if (lane == 0) {
-        s_cnt[2 * warp] = cf;
-        s_cnt[2 * warp + 1] = ct;
-      }
-      if (tid == 0) s_misc[2] = *reinterpret_cast<volatile uint32_t*>(&v.hdr->error) != 0u;
-      __syncthreads();
-      int tf = 0, tt = 0;
-#pragma unroll
-      for (int x = 0; x < kPpThreads / 32; ++x) {
-        tf += s_cnt[2 * x];
-        tt += s_cnt[2 * x + 1];
-      }
       const int held = v.n_slots[v.head(layer, seq0 + b, hkv)];
+      __syncthreads();   // s_misc[2] (error word, read by thread 0)
+      const int tf = far_keys(v, evict, b, hkv, P, kl * kPaTile, tid, s_cnt);
       const int nft = (tf + kPaTile - 1) / kPaTile;
-      if (!s_misc[2] && held == tt && nft * kPaTile <= held && 2 * nft <= v.mbh) {
+      if (!s_misc[2] && nft * kPaTile <= held && 2 * nft <= v.mbh) {
         kt_lo = kl;
         nf = nft;
         n_far = tf;
@@ -675,12 +687,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       const uint32_t aQ[2] = {smem_u32(smem + S::QA), smem_u32(smem + S::QB)};
       const uint32_t aPb[2] = {smem_u32(smem + S::PA), smem_u32(smem + S::PB)};
       const uint32_t aK = smem_u32(smem + S::K), aV = smem_u32(smem + S::V);
-      mbar_arrive_expect_tx(bar_q, 2 * S::TILE);
-#pragma unroll
-      for (int kb = 0; kb < D / 64; ++kb) {
-        umma::tma_load_3d(smem + S::QA + kb * kPaTile * 128, &tq, hq0 * D + kb * 64, i0, b, bar_q);
-        umma::tma_load_3d(smem + S::QB + kb * kPaTile * 128, &tq, (hq0 + 1) * D + kb * 64, i0, b, bar_q);
-      }
       load_kv(0, 0, bar_k);
       load_kv(0, 1, bar_v);
       int nk = 1, nv = 1, wk = 0, wv = 0;   // loads issued / waited on

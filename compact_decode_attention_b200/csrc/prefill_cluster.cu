@@ -159,8 +159,15 @@ __global__ void __launch_bounds__(kPcThreads) prefill_cluster_kernel(PoolView v,
     s_cnt[0] = mine;
   }
   __syncthreads();
-  int total = 0;
-  for (int r = 0; r < C; ++r) total += s_cnt[r];
+  int total = 0, before = 0;
+  for (int r = 0; r < C; ++r) {
+    before += r < j ? s_cnt[r] : 0;
+    total += s_cnt[r];
+  }
+  // kept tokens before each 256-token chunk of the span (the prefill
+  // scratch the two-launch planner fills too; prompt attention reads it)
+  if (tid < iters)
+    v.chunk_counts[(int64_t(b) * v.Hkv + h) * v.n_chunks_max + p0 / kPcThreads + tid] = before + s_wc[tid][0];
   // The head's kept rows are spread evenly over the cluster's CTAs (a span
   // inside the window keeps every token, the others few): CTA j copies rows
   // [r0, r1).  Their positions are read from the owning CTAs' lists (valid
