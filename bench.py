@@ -661,7 +661,7 @@ def main():
                   "ms_per_layer": compact_ms / L, "algorithmic_bytes_per_layer": compact_bytes / L,
                   "full_read_value": full_read_bytes / (compact_ms * 1e-3) / 1e9,
                   "kernels": ("prefill_cluster_kernel (one launch a layer)"
-                              if wl.kv_dtype in ("bf16", "f32") and P <= 16 * 63 * 256 else
+                              if wl.kv_dtype in ("bf16", "f32") and P <= 16384 else
                               "prefill_plan_kernel + prefill_scatter_kernel (two launches a layer)"),
                   "timing": "CUDA events around each layer's dms_compact_prefill call, layers after "
                             "the first captured in one CUDA graph replayed once; median layer"}

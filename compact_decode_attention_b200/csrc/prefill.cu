@@ -13,7 +13,7 @@
 // eviction is decided before FP8 quantisation).
 //
 // Copy stores (bf16, fp32) take one launch instead, a cluster per
-// (sequence, kv-head) (csrc/prefill_cluster.cu), for prompts up to 262144
+// (sequence, kv-head) (csrc/prefill_cluster.cu), for prompts up to 16384
 // tokens.  FP8 and 4-bit stores, and longer prompts, take two kernels, in
 // stream order:
 //   plan     one CTA per (256-token chunk, sequence): per-head kept counts by

@@ -299,8 +299,13 @@ __global__ void __launch_bounds__(kPcThreads) prefill_cluster_kernel(PoolView v,
   }
 }
 
-// Longest prompt the one-launch compaction takes (16 CTAs x 63 x 256 tokens).
-int prefill_cluster_max_prompt() { return kPcMaxC * (kPcMaxIters - 1) * kPcThreads; }
+// Longest prompt the one-launch compaction takes.  The kernel could take 16
+// CTAs x 63 x 256 tokens, but one cluster per head is a latency design: a
+// long prompt's head (131072 tokens, possibly all kept) over 16 CTAs took
+// 1.27 ms a layer on the Qwen3-8B batch-16 workload against 0.6 ms in the
+// two launches, whose scatter spreads every head over many CTAs.
+int prefill_cluster_max_prompt() { return 16384; }
+static_assert(16384 <= kPcMaxC * (kPcMaxIters - 1) * kPcThreads, "spans of at most 63 iterations");
 
 // One launch for a copy store: clusters of C CTAs per (sequence, kv-head).
 dms_status prefill_cluster_launch(dms_pool* pool, int layer, int seq0, int batch, int prompt_len,

@@ -190,3 +190,27 @@ def test_refused_call_leaves_the_planner_clean():
                                  {j: Kx[b, j, h] for j in range(P)}, {j: Vx[b, j, h] for j in range(P)},
                                  "fp8", scales[h])
     check_block_invariants(pool, state)
+
+
+@pytest.mark.parametrize("kind,P", [("bf16", 16384), ("bf16", 16384 + 300), ("f32", 16384 + 300)])
+def test_copy_stores_either_side_of_the_one_launch_limit(kind, P):
+    """Copy stores (bf16, fp32) take one launch up to 16384 prompt tokens and
+    the plan + scatter launches past it: both give the oracle's store bit for
+    bit."""
+    B, Hq, Hkv, D, w, seed = 2, 4, 4, 64, 512, 93
+    thr = [synth.keep_threshold(p) for p in (0.2, 1.0, 0.0, 0.05)]
+    Kd, Vd, Fd = _device_inputs(seed, B, P, Hkv, D, thr, kind)
+    code = dms.DMS_F32 if kind == "f32" else dms.DMS_BF16
+    pool = dms.Pool(1, B, Hq, Hkv, D, w, code, B * Hkv * (P // BT + 3), P + 2)
+    pool.buffer[pool.layout.blocks:].fill_(0xFF)
+    pool.compact_prefill(0, Kd, Vd, Fd)
+    state = read_state(pool)
+    assert state["error"] == 0
+    check_block_invariants(pool, state)
+    F = Fd.cpu().numpy()
+    for b in range(B):
+        K, V, _ = _host_sequence(seed, b, P, Hkv, D, thr, kind)
+        for h in range(Hkv):
+            store = oracle_store(F[b, :, h], np.zeros(0, np.uint8), w, P)
+            check_head_store(pool, state, head_id(pool.cfg, 0, b, h), store,
+                             {j: K[j, h] for j in range(P)}, {j: V[j, h] for j in range(P)}, kind)

@@ -178,3 +178,20 @@ def test_a_layer_that_is_not_empty_still_gets_correct_outputs():
     got = _run(pool, 0, Q2, K2, V2, F2)
     assert read_state(pool)["error"] & dms.DEVERR_LAYER_NOT_EMPTY
     _sampled_check(got, Q2, K2, V2, F2, w, [0, 200, 511, 512, 640, 777, P - 1])
+
+
+@pytest.mark.parametrize("P", [16384, 16384 + 500])
+def test_store_reading_on_either_side_of_the_one_launch_compaction(P):
+    """Prompts up to 16384 tokens are compacted in one launch, longer ones by
+    the plan and scatter launches; the prompt attention takes the far-key
+    counts from either one's chunk prefix counts.  Sampled queries (every
+    query tile is a different far/band split) against the oracle."""
+    B, Hq, Hkv, D, w = 1, 4, 2, 64, 512
+    Q, K, V, F = _inputs(70 + P, B, P, Hq, Hkv, D, 0.2)
+    pool = dms.Pool(1, B, Hq, Hkv, D, w, dms.DMS_BF16, B * Hkv * (P // 64 + 2), P + 1)
+    got = _run(pool, 0, Q, K, V, F)
+    assert np.isfinite(got).all()
+    rng = np.random.default_rng(P)
+    idx = sorted(set(rng.integers(0, P, 10).tolist()) | {w + 127, 4096, P - 129, P - 1})
+    _sampled_check(got, Q, K, V, F, w, idx)
+    _check_store(pool, 0, K, V, F, P, w)
