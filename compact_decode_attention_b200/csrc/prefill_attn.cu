@@ -107,6 +107,27 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// Unflagged keys of head (b, hkv) before position bs (a multiple of 128 below
+// P - w, so kept = unflagged there), from the kept-token prefix counts the
+// layer's compaction left per 256-token chunk, plus the first 128 tokens of
+// bs's chunk when bs is not a chunk start.  Every thread calls it (one block
+// barrier); s_tmp holds 4 ints.
+__device__ __forceinline__ int far_keys(const PoolView& v, const uint8_t* evict, int b, int hkv, int P, int bs,
+                                        int tid, int* s_tmp) {
+  const int c = bs >> 8;
+  const int base = v.chunk_counts[(int64_t(b) * v.Hkv + hkv) * v.n_chunks_max + c];
+  if (bs & 255) {
+    if (tid < kPaTile) {
+      const int j = (c << 8) + tid;
+      const unsigned m = __ballot_sync(0xffffffffu, evict[(int64_t(b) * P + j) * v.Hkv + hkv] == 0);
+      if ((tid & 31) == 0) s_tmp[tid >> 5] = __popc(m);
+    }
+    __syncthreads();
+    return base + s_tmp[0] + s_tmp[1] + s_tmp[2] + s_tmp[3];
+  }
+  return base;
+}
+
 template <int D>
 __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     prefill_attn_kernel(PoolView v, int layer, int seq0, int P, const __grid_constant__ CUtensorMap tq,
@@ -137,7 +158,7 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
   uint64_t* bar_v = bar_s + 4;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::MISC);
   int* s_scan = reinterpret_cast<int*>(smem + S::MISC) + 4;   // [8]
-  int* s_cnt = reinterpret_cast<int*>(smem + S::MISC) + 12;   // [16]
+  int* s_cnt = reinterpret_cast<int*>(smem + S::MISC) + 12;   // [4] (far_keys)
 
   // tensor-map loads of one [128 x D] tile: boxes of 64 columns x 128 rows
   // with 128-byte swizzle (the operand image of umma.cuh); rows past the
@@ -201,32 +222,15 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
     const int lo = i0 - v.w + 1;
     const int kl = lo > 0 ? lo / kPaTile : 0;
     if (kl > 0) {
-      const int bs = kl * kPaTile;
-      int cf = 0, ct = 0;
-      for (int j = tid; j < P; j += THREADS) {
-        const uint8_t f = evict[(int64_t(b) * P + j) * v.Hkv + hkv];
-        ct += (f == 0 || P - 1 - j < v.w) ? 1 : 0;
-        cf += (f == 0 && j < bs) ? 1 : 0;
-      }
-      cf = __reduce_add_sync(0xffffffffu, cf);
-      ct = __reduce_add_sync(0xffffffffu, ct);
-      if (lane == 0) {
-        s_cnt[warp] = cf;
-        s_cnt[8 + warp] = ct;
-      }
       // a compaction that failed (this call's or an earlier one: the error
       // word is sticky) may have left a head's old rows in place
       if (tid == 0) s_scan[0] = *reinterpret_cast<volatile uint32_t*>(&v.hdr->error) != 0u;
-      __syncthreads();
-      int tf = 0, tt = 0;
-#pragma unroll
-      for (int x = 0; x < THREADS / 32; ++x) {
-        tf += s_cnt[x];
-        tt += s_cnt[8 + x];
-      }
       const int held = v.n_slots[v.head(layer, seq0 + b, hkv)];
+      __syncthreads();
+      const bool failed = s_scan[0] != 0;
+      const int tf = far_keys(v, evict, b, hkv, P, kl * kPaTile, tid, s_cnt);
       const int nft = (tf + kPaTile - 1) / kPaTile;
-      if (!s_scan[0] && held == tt && nft * kPaTile <= held && 2 * nft <= v.mbh) {
+      if (!failed && nft * kPaTile <= held && 2 * nft <= v.mbh) {
         kt_lo = kl;
         nf = nft;
         n_far = tf;
@@ -518,27 +522,6 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
   if (warp == 0) umma::tmem_dealloc(tbase, 256);
 }
 
-// Unflagged keys of head (b, hkv) before position bs (a multiple of 128 below
-// P - w, so kept = unflagged there), from the kept-token prefix counts the
-// layer's compaction left per 256-token chunk, plus the first 128 tokens of
-// bs's chunk when bs is not a chunk start.  Every thread calls it (one block
-// barrier); s_tmp holds 4 ints.
-__device__ __forceinline__ int far_keys(const PoolView& v, const uint8_t* evict, int b, int hkv, int P, int bs,
-                                        int tid, int* s_tmp) {
-  const int c = bs >> 8;
-  const int base = v.chunk_counts[(int64_t(b) * v.Hkv + hkv) * v.n_chunks_max + c];
-  if (bs & 255) {
-    if (tid < kPaTile) {
-      const int j = (c << 8) + tid;
-      const unsigned m = __ballot_sync(0xffffffffu, evict[(int64_t(b) * P + j) * v.Hkv + hkv] == 0);
-      if ((tid & 31) == 0) s_tmp[tid >> 5] = __popc(m);
-    }
-    __syncthreads();
-    return base + s_tmp[0] + s_tmp[1] + s_tmp[2] + s_tmp[3];
-  }
-  return base;
-}
-
 // ---------------------------------------------------------------------------
 // Two query heads of one kv-head per CTA (sparse reading, an even group
 // size g).  The heads share every K and V tile; per key tile the MMA thread
@@ -605,7 +588,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   int* s_misc = reinterpret_cast<int*>(smem + S::MISC);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_misc);
   volatile int* s_abort = s_misc + 1;
-  int* s_cnt = s_misc + 8;       // [17 warps][2]
+  int* s_cnt = s_misc + 8;       // [4] (far_keys)
   int* s_ids = reinterpret_cast<int*>(smem + S::IDS);
 
   if (tid == 0) {
