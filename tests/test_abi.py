@@ -79,6 +79,10 @@ def test_null_arguments_rejected_without_cuda(lib):
     assert lib.dms_compact_prefill(None, 0, 1, 1, None, None, 1, None, None) == dms.DMS_ERR_INVALID_ARG
     assert lib.dms_decode_attn(None, 0, 1, None, 1, None, 0.0, None, 0, None) == dms.DMS_ERR_INVALID_ARG
     assert lib.dms_synth_normal(0, 0, 0, 1, 1, 0, 1, 1, 64, 1, None, None) == dms.DMS_ERR_INVALID_ARG
+    # host settings of a pool handle
+    assert lib.dms_pool_set_prefill_mode(None, dms.PREFILL_SPARSE) == dms.DMS_ERR_INVALID_ARG
+    assert lib.dms_pool_set_attn_kernel(None, dms.ATTN_AUTO) == dms.DMS_ERR_INVALID_ARG
+    assert lib.dms_pool_set_wait_limit(None, 1000000) == dms.DMS_ERR_INVALID_ARG
     assert lib.dms_last_error().decode()
 
 
