@@ -152,9 +152,23 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   // ---- find this CTA's unit range: per-thread head ranges + block scan ----
   const int per = (Htot + kAttnThreads - 1) / kAttnThreads;
   const int hb = min(Htot, tid * per), he = min(Htot, hb + per);
+  // this thread's held counts, loaded once and together (kept in registers
+  // when it has at most kCache heads; the walks below reuse them)
+  constexpr int kCache = 4;
+  const bool cached = per <= kCache;
+  int ncache[kCache];
+#pragma unroll
+  for (int x = 0; x < kCache; ++x) ncache[x] = (cached && hb + x < he) ? n_of(p, hb + x) : 0;
+  auto n_mine = [&](int i) {   // held count of head i in [hb, he)
+    if (!cached) return n_of(p, i);
+    int n = 0;
+#pragma unroll
+    for (int x = 0; x < kCache; ++x) n = i == hb + x ? ncache[x] : n;
+    return n;
+  };
   int su = 0;
   for (int i = hb; i < he; ++i) {
-    const int n = n_of(p, i);
+    const int n = n_mine(i);
     su += units_of(n);
     if (n == 0 && i % G == c) {  // no key at all: define the output as 0
       const int64_t orow = int64_t(i / v.Hkv) * v.Hq + int64_t(i % v.Hkv) * g;
@@ -187,7 +201,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   if (u_beg < u_end && u_beg >= excl && u_beg < excl + su) {
     int pre = excl;
     for (int i = hb; i < he; ++i) {
-      const int nu = units_of(n_of(p, i));
+      const int nu = units_of(n_mine(i));
       if (u_beg < pre + nu) {
         s_misc[1] = i;
         s_misc[2] = pre;
@@ -200,7 +214,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   if (u_beg < u_end && u_end - 1 >= excl && u_end - 1 < excl + su) {
     int pre = excl;
     for (int i = hb; i < he; ++i) {
-      const int n = n_of(p, i);
+      const int n = n_mine(i);
       const int nu = units_of(n);
       if (u_end - 1 < pre + nu) {
         s_misc[4] = i;
@@ -224,7 +238,7 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   // held counts of heads i0 .. i0 + HEAD_WIN - 1 in shared memory, so that the
   // walks below need no dependent global loads (the scan just loaded them)
   int* s_nwin = s_misc + T::MISC_INTS;
-  for (int i = max(hb, i0); i < min(he, i0 + T::HEAD_WIN); ++i) s_nwin[i - i0] = n_of(p, i);
+  for (int i = max(hb, i0); i < min(he, i0 + T::HEAD_WIN); ++i) s_nwin[i - i0] = n_mine(i);
   __syncthreads();
   auto n_at = [&](int i) { return i - i0 < T::HEAD_WIN ? s_nwin[i - i0] : n_of(p, i); };
   const int qrow_bytes = g * D * T::QESZ;
