@@ -235,6 +235,14 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
   const int iL = s_misc[4], pL = s_misc[5], nL = s_misc[6];
   const int r = max(u_beg, pL);
   const int nA = u_end - r;
+  // producer: the block ids of segment A's first 32 units (below), loaded
+  // now so that their round trip overlaps the window fill and its barrier
+  int blkA = 0;
+  if (warp == kNCW && r + lane < u_end) {
+    const int bi = r + lane - pL;
+    if (DMS_CHECK(iL < Htot && bi >= 0 && bi < v.mbh, v.hdr, 304, iL, bi))
+      blkA = v.bt[int64_t(pool_head(p, iL)) * v.mbh + bi];
+  }
   // held counts of heads i0 .. i0 + HEAD_WIN - 1 in shared memory, so that the
   // walks below need no dependent global loads (the scan just loaded them)
   int* s_nwin = s_misc + T::MISC_INTS;
@@ -288,10 +296,10 @@ __global__ void __launch_bounds__(AttnTraits<KV, D>::THREADS, 1)
     // segment A: one head, units [r, u_end)
     for (int ub = r; ub < u_end; ub += 32) {
       const int u = ub + lane;
-      int blk = 0, rows = 0;
+      int blk = ub == r ? blkA : 0, rows = 0;
       if (u < u_end) {
         const int bi = u - pL;
-        if (DMS_CHECK(iL < Htot && bi >= 0 && bi < v.mbh, v.hdr, 304, iL, bi))
+        if (ub != r && DMS_CHECK(iL < Htot && bi >= 0 && bi < v.mbh, v.hdr, 304, iL, bi))
           blk = v.bt[int64_t(pool_head(p, iL)) * v.mbh + bi];
         rows = min(kBlockTokens, nL - bi * kBlockTokens);
       }
