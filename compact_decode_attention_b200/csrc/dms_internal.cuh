@@ -61,6 +61,8 @@ struct PoolView {
   int32_t* prefill_tickets; // prefill scratch [Bmax + 1] arrival counters (self-resetting)
   int32_t* pair_n;          // prefill scratch [Bmax][Hkv] kept tokens of each (sequence, head)
   int32_t* pair_base;       // prefill scratch [Bmax * Hkv + 1] first allocation index of each pair
+  int32_t* pos_of_slot;     // prefill scratch, FP8 and 4-bit stores only (else null):
+                            // [Bmax][Hkv][mbh * BT] prompt position of each kept slot
   void* stats;              // staging for dms_pool_stats
 
   __host__ __device__ __forceinline__ int head(int l, int b, int h) const {

@@ -132,6 +132,8 @@ static dms_status plan_layout(const dms_pool_config* c, dms_pool_layout_t* lay) 
   off = align256(off + uint64_t(c->max_batch + 1) * 4);                         // prefill tickets
   off = align256(off + uint64_t(c->max_batch) * c->n_kv_heads * 4);             // pair counts
   off = align256(off + (uint64_t(c->max_batch) * c->n_kv_heads + 1) * 4);       // pair bases
+  if (c->kv_dtype == DMS_FP8_E4M3 || c->kv_dtype == DMS_INT4)                     // slot positions
+    off = align256(off + uint64_t(c->max_batch) * c->n_kv_heads * mbh * kBlockTokens * 4);
   off = align256(off + sizeof(dms_pool_stats_t));                                // stats
   lay->blocks = off;
   lay->block_bytes = 2 * kBlockTokens * row_bytes;
@@ -190,6 +192,11 @@ static PoolView make_view(const dms_pool_config& c, const dms_pool_layout_t& lay
   s = align256(s + uint64_t(c.max_batch) * c.n_kv_heads * 4);
   v.pair_base = reinterpret_cast<int32_t*>(b + s);
   s = align256(s + (uint64_t(c.max_batch) * c.n_kv_heads + 1) * 4);
+  v.pos_of_slot = nullptr;
+  if (c.kv_dtype == DMS_FP8_E4M3 || c.kv_dtype == DMS_INT4) {
+    v.pos_of_slot = reinterpret_cast<int32_t*>(b + s);
+    s = align256(s + uint64_t(c.max_batch) * c.n_kv_heads * uint64_t(lay.max_blocks_per_head) * kBlockTokens * 4);
+  }
   v.stats = b + s;
   return v;
 }

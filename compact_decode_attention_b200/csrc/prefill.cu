@@ -421,6 +421,10 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(PoolView v, int la
   if (!go) return;
   const int hd = v.head(layer, seq0 + b, h);
   const int32_t* table = v.bt + int64_t(hd) * v.mbh;
+  // prompt position of each kept slot (quantised stores: the prompt
+  // attention gathers its old kept keys from the bf16 prompt by position)
+  if (STORE != 0 && v.pos_of_slot && mine && keep)
+    v.pos_of_slot[(int64_t(b) * v.Hkv + h) * (int64_t(v.mbh) * v.BT) + base + rank] = j;
   if (mine && keep && j >= P - v.w) {
     const int slot = base + rank;
     const int64_t ri = int64_t(hd) * v.w + (j % v.w);

@@ -537,7 +537,17 @@ __global__ void __launch_bounds__(PaSplit<D>::THREADS, 2)
 // as above), warp 16 loads tiles and issues the MMAs (one thread).  The
 // hand-offs are mbarriers: S ready (commit), P ready (one arrival per
 // softmax warp), O done (commit), K and V buffers free (commit).
-constexpr int kPpThreads = 2 * 2 * kPaTile + 32;
+//
+// FP8 and 4-bit stores hold quantised rows, while the prompt's attention runs
+// on the bf16 keys and values; for them warp 17 fetches each old-key tile
+// from the prompt instead: the compaction left the prompt position of every
+// kept slot in the pool's scratch, so tile t is the prompt rows of slots
+// [128 t, 128 t + 128), gathered 16 bytes at a time (cp.async) into the
+// swizzled operand image, the keys by warp 17 and the values by warp 18.
+// The MMA thread requests each tile (an mbarrier per K / V buffer) when it
+// would have loaded it; the gather warp waits for its copies, fences them
+// for the tensor cores and arrives on the buffer's full barrier.
+constexpr int kPpThreads = 2 * 2 * kPaTile + 96;
 constexpr int kPpMaxFarIds = 2048;   // far-tile block ids cached in shared memory
 
 template <int D>
@@ -560,12 +570,19 @@ __device__ __forceinline__ void pp_group_bar(int grp) {
   asm volatile("bar.sync %0, 256;" ::"r"(1 + grp) : "memory");
 }
 
+// 16 bytes global -> shared, bypassing L1; completion by cp_async_wait_all
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 template <int D>
 __global__ void __launch_bounds__(kPpThreads, 1)
     prefill_pair_kernel(PoolView v, int layer, int seq0, int P, const __grid_constant__ CUtensorMap tq,
                         const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                         const __grid_constant__ CUtensorMap tpool, const uint8_t* evict,
-                        __nv_bfloat16* out, float scale_log2, int n_qtiles) {
+                        __nv_bfloat16* out, float scale_log2, int n_qtiles, const __nv_bfloat16* kin,
+                        const __nv_bfloat16* vin, int far_in) {
   using S = PpSmem<D>;
   constexpr int SPLIT = 2, HC = kPaTile / SPLIT, OC = D / SPLIT;
   extern __shared__ uint8_t smem_raw[];
@@ -585,6 +602,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   uint64_t* bar_o = bars + 7;    // [2] P V of head A / B computed
   uint64_t* bar_p = bars + 9;    // [2] P of head A / B in shared memory
   uint64_t* bar_fin = bars + 11; // every MMA done (exit)
+  uint64_t* req_k = bars + 12;   // far_in: the MMA thread asks for the next old-key tile's keys
+  uint64_t* req_v = bars + 13;   // ... and values
   int* s_misc = reinterpret_cast<int*>(smem + S::MISC);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_misc);
   volatile int* s_abort = s_misc + 1;
@@ -592,7 +611,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   int* s_ids = reinterpret_cast<int*>(smem + S::IDS);
 
   if (tid == 0) {
-    for (int x = 0; x < 12; ++x) mbar_init(&bars[x], x == 9 || x == 10 ? 8 : 1);
+    for (int x = 0; x < 14; ++x) mbar_init(&bars[x], x == 9 || x == 10 ? 8 : 1);
     s_misc[1] = 0;
     s_misc[2] = *reinterpret_cast<volatile uint32_t*>(&v.hdr->error) != 0u;
     fence_mbar_init();
@@ -638,7 +657,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
 
   if (warp == 16) {
     // ======================= loads and MMAs (one thread) =======================
-    const bool cached = 2 * nf <= kPpMaxFarIds;
+    const bool cached = !far_in && 2 * nf <= kPpMaxFarIds;
     if (cached)
       for (int x = lane; x < 2 * nf; x += 32) s_ids[x] = far_bt[x];
     __syncwarp();
@@ -653,7 +672,9 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       // tile it's keys (kv = 0) or values (kv = 1) into dst
       auto load_kv = [&](int it, int kv, uint64_t* bar) {
         uint8_t* dst = smem + (kv ? S::V : S::K);
-        if (it < nf) {
+        if (it < nf && far_in) {
+          mbar_arrive(kv ? req_v : req_k);   // warp 17 gathers it from the prompt
+        } else if (it < nf) {
           const int blk0 = far_id(2 * it), blk1 = far_id(2 * it + 1);
           mbar_arrive_expect_tx(bar, S::TILE);
 #pragma unroll
@@ -751,6 +772,46 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       if (!qdone) mbar_wait_bounded(bar_q, 0, &never, v.wait_ns);
       if (nk > wk) mbar_wait_bounded(bar_k, (nk - 1) & 1, &never, v.wait_ns);
       if (nv > wv) mbar_wait_bounded(bar_v, (nv - 1) & 1, &never, v.wait_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 17) {
+    // ============ old-key tiles from the prompt (quantised stores) ============
+    // warp 17 gathers the keys, warp 18 the values
+    const int kv = warp - 17;
+    if (far_in && nf > 0) {
+      constexpr int NCH = D / 8, RPP = 32 / NCH;   // 16-byte chunks per row, rows per pass
+      const int32_t* pos = v.pos_of_slot + (int64_t(b) * v.Hkv + hkv) * (int64_t(v.mbh) * v.BT);
+      const int64_t tok_elems = int64_t(v.Hkv) * D;
+      bool ok = true;
+      for (int t = 0; t < nf && ok; ++t) {
+        int prow[4];   // prompt positions of the tile's rows lane, lane + 32, + 64, + 96
+#pragma unroll
+        for (int x = 0; x < 4; ++x) prow[x] = pos[int64_t(t) * kPaTile + 32 * x + lane];
+        {
+          if (lane == 0) {
+            ok = mbar_wait_bounded(kv ? req_v : req_k, t & 1, s_abort, v.wait_ns);
+            if (!ok) *s_abort = 1;
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          const __nv_bfloat16* src = (kv ? vin : kin) + int64_t(b) * P * tok_elems + int64_t(hkv) * D;
+          const uint32_t dst = smem_u32(smem + (kv ? S::V : S::K));
+          const int c = lane % NCH;
+#pragma unroll
+          for (int pss = 0; pss < 4 * NCH; ++pss) {   // RPP whole rows per pass, coalesced
+            const int rr = pss * RPP + lane / NCH;
+            const int x = (pss * RPP) >> 5;
+            const int mine = x == 0 ? prow[0] : x == 1 ? prow[1] : x == 2 ? prow[2] : prow[3];
+            const int prompt_row = __shfl_sync(0xffffffffu, mine, rr & 31);
+            cp_async16(dst + umma::sw128_offset(kPaTile, rr, c * 8), src + int64_t(prompt_row) * tok_elems + c * 8);
+          }
+          cp_async_wait_all();
+          fence_proxy_async_smem();   // the copies, before the tensor cores read them
+          __syncwarp();
+          if (lane == 0) mbar_arrive(kv ? bar_v : bar_k);
+        }
+      }
+      if (!ok && lane == 0) report_error(v.hdr, DMS_DEVERR_TIMEOUT, layer, seq0 + b, hq0);
     }
     __syncwarp();
   } else {
@@ -1017,8 +1078,12 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
   // dms_compact_prefill_seqs (scales, plan, scatter), and the attention
   // kernel reads every key from the bf16 inputs.
   const bool bf16_store = pv.kv_dtype == DMS_BF16;
+  const bool even_g = (pv.Hq / pv.Hkv) % 2 == 0;
   const int sparse = bf16_store && pool->prefill_mode == DMS_PREFILL_SPARSE &&
                      2 * pv.max_blocks <= int64_t(INT32_MAX) ? 1 : 0;
+  // quantised stores: old kept keys gathered from the prompt by position
+  // (two query heads per CTA only)
+  const int far_in = !bf16_store && pool->prefill_mode == DMS_PREFILL_SPARSE && even_g && pv.pos_of_slot ? 1 : 0;
   const int fused = bf16_store && !sparse ? 1 : 0;
   CUtensorMap tpool;
   memset(&tpool, 0, sizeof(tpool));
@@ -1037,7 +1102,7 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
   if (st == DMS_OK) st = encode_bf16_map(&tv, v, batch, prompt_len, pv.Hkv * pv.D);
   if (st != DMS_OK) return st;
   auto ko = static_cast<__nv_bfloat16*>(out);
-  if (sparse && (pv.Hq / pv.Hkv) % 2 == 0) {   // two query heads of a kv-head per CTA
+  if ((sparse && even_g) || far_in) {   // two query heads of a kv-head per CTA
     const dim3 grid2(n_qtiles, pv.Hq / 2, batch);
     if (pv.D == 128) {
       static FuncAttrCache smem_attr;  // per device
@@ -1046,7 +1111,8 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
                             "prefill pair smem attribute");
       if (st != DMS_OK) return st;
       prefill_pair_kernel<128><<<grid2, kPpThreads, PpSmem<128>::BYTES, stream>>>(
-          pv, layer, seq0, prompt_len, tq, tk, tv, tpool, evict, ko, scale_log2, n_qtiles);
+          pv, layer, seq0, prompt_len, tq, tk, tv, tpool, evict, ko, scale_log2, n_qtiles,
+          static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), far_in);
     } else {
       static FuncAttrCache smem_attr;  // per device
       st = ensure_func_attr(reinterpret_cast<const void*>(prefill_pair_kernel<64>),
@@ -1054,7 +1120,8 @@ extern "C" dms_status dms_prefill_attn(dms_pool* pool, int layer, int seq0, int 
                             "prefill pair smem attribute");
       if (st != DMS_OK) return st;
       prefill_pair_kernel<64><<<grid2, kPpThreads, PpSmem<64>::BYTES, stream>>>(
-          pv, layer, seq0, prompt_len, tq, tk, tv, tpool, evict, ko, scale_log2, n_qtiles);
+          pv, layer, seq0, prompt_len, tq, tk, tv, tpool, evict, ko, scale_log2, n_qtiles,
+          static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), far_in);
     }
     return cuda_status(cudaGetLastError(), "prefill_pair_kernel");
   }

@@ -219,7 +219,10 @@ dms_status dms_pool_set_attn_kernel(dms_pool* pool, int kind);
  *                       masked; the kernel stores each diagonal tile's kept
  *                       rows itself.
  * Both give the same attention (rounding order aside) and the same store.
- * FP8 and 4-bit pools always use the dense form on the bf16 inputs. */
+ * FP8 and 4-bit pools hold quantised rows, while the prompt's attention runs
+ * on the bf16 inputs: in sparse mode their old kept keys are gathered from
+ * the prompt by the positions their compaction records (an even group size
+ * g only; otherwise, and in dense mode, every causal tile is read). */
 #define DMS_PREFILL_SPARSE 0
 #define DMS_PREFILL_DENSE 1
 dms_status dms_pool_set_prefill_mode(dms_pool* pool, int mode);
@@ -314,7 +317,8 @@ dms_status dms_decode_attn_seqs(dms_pool* pool, int layer0, int n_layers, int n_
  * keys are read back from the store (DMS_PREFILL_SPARSE, the default), or
  * filled by the attention kernel itself (DMS_PREFILL_DENSE, see
  * dms_pool_set_prefill_mode); an FP8 or 4-bit pool is compacted first, as by
- * dms_compact_prefill_seqs, and the attention reads the bf16 inputs.
+ * dms_compact_prefill_seqs, and the attention reads the bf16 inputs (old kept
+ * keys gathered by position in sparse mode).
  * The sequences must be empty in that layer (else DMS_DEVERR_LAYER_NOT_EMPTY
  * and nothing is stored; the outputs are still computed).  Runs on the
  * tensor cores (tcgen05, accumulators in tensor memory).

@@ -75,12 +75,14 @@ def test_long_prompt_sampled_queries_and_sequence_offset():
     _check_store(pool, 2, K, V, F, P, w)
 
 
-@pytest.mark.parametrize("kind", ["fp8", "int4"])
-def test_quantised_pools_compact_first_then_attend(kind):
+@pytest.mark.parametrize("kind,P", [("fp8", 333), ("int4", 333), ("fp8", 1500), ("int4", 1500)])
+def test_quantised_pools_compact_first_then_attend(kind, P):
     """FP8 and 4-bit stores: the layer is compacted as by
     dms_compact_prefill_seqs (codes and scales bit-exact against the
-    oracle), and every query's output matches the oracle on the bf16 inputs."""
-    B, P, Hq, Hkv, D, w = 2, 333, 8, 2, 128, 64
+    oracle), and every query's output matches the oracle on the bf16 inputs
+    (the old kept keys are gathered from the prompt by the positions the
+    compaction recorded; at P = 1500 several such tiles per query tile)."""
+    B, Hq, Hkv, D, w = 2, 8, 2, 128, 64
     Q, K, V, F = _inputs(41, B, P, Hq, Hkv, D, 0.3)
     code = dms.DMS_FP8_E4M3 if kind == "fp8" else dms.DMS_INT4
     pool = dms.Pool(1, B, Hq, Hkv, D, w, code, B * Hkv * (P // 64 + 2), P + 1)
@@ -195,3 +197,24 @@ def test_store_reading_on_either_side_of_the_one_launch_compaction(P):
     idx = sorted(set(rng.integers(0, P, 10).tolist()) | {w + 127, 4096, P - 129, P - 1})
     _sampled_check(got, Q, K, V, F, w, idx)
     _check_store(pool, 0, K, V, F, P, w)
+
+
+@pytest.mark.parametrize("kind", ["fp8", "int4"])
+def test_quantised_pools_both_readings_agree(kind):
+    """The gathered old-key tiles against every causal tile from the prompt
+    (DMS_PREFILL_DENSE): the same store, outputs within the bf16 bound."""
+    B, P, Hq, Hkv, D, w = 1, 1200, 8, 2, 128, 128
+    Q, K, V, F = _inputs(83, B, P, Hq, Hkv, D, 0.2)
+    code = dms.DMS_FP8_E4M3 if kind == "fp8" else dms.DMS_INT4
+    outs, states = [], []
+    for mode in (dms.PREFILL_SPARSE, dms.PREFILL_DENSE):
+        pool = dms.Pool(1, B, Hq, Hkv, D, w, code, B * Hkv * (P // 64 + 2), P + 1)
+        pool.set_prefill_mode(mode)
+        outs.append(_run(pool, 0, Q, K, V, F))
+        states.append(read_state(pool))
+    assert states[0]["error"] == 0 and states[1]["error"] == 0
+    for key in ("n_slots", "n_retained", "ring"):
+        assert np.array_equal(states[0][key], states[1][key]), key
+    assert np.isfinite(outs[0]).all()
+    assert np.abs(outs[0] - outs[1]).max() < TOL
+    _sampled_check(outs[0], Q, K, V, F, w, [0, 127, 128, 300, 640, 900, P - 1])
